@@ -1,0 +1,433 @@
+"""Pins of the CPU oracle to things other than itself.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees with an
+external fact: published generator vectors, brute-force enumeration, closed forms,
+library routines (numpy, torch SDPA and autograd) or finite differences.  They are
+collected by ``test_oracle_pins.py`` and re-run against deliberately broken copies of
+the oracle by ``test_oracle_mutants.py`` (every planted mistake must trip a pin).
+
+Special cases used (from the method's statement on the pages):
+  * flat search scores every cluster centroid, so a hierarchical walk whose beam keeps
+    every node above the leaf level equals brute-force top-B over all leaves;
+  * sparse attention over every key is full softmax attention;
+  * a centroid is the mean of its members (k-means), and with balanced children a
+    parent centroid is the mean of its children's centroids.
+"""
+from __future__ import annotations
+
+import itertools
+import os
+
+import numpy as np
+import torch
+
+from oracle import oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+# ---------------------------------------------------------------------------
+# small deterministic fixtures
+# ---------------------------------------------------------------------------
+
+def _mixture(rng, n, d, comps, sigma=0.3):
+    c = rng.standard_normal((comps, d))
+    c /= np.linalg.norm(c, axis=1, keepdims=True)
+    return c[rng.integers(0, comps, n)] + sigma * rng.standard_normal((n, d))
+
+
+def tiny_tree_case(seed=0, n=1024, d=32, r=8, branching=(8, 8), leaf=16, iters=4):
+    rng = np.random.default_rng(seed)
+    K = _mixture(rng, n, d, 16)
+    W = rng.standard_normal((d, r)) / np.sqrt(d)
+    Z = K @ W
+    tree = orc.build_tree(orc.project(K, W), branching, leaf, iters, seed=seed, trace=True)
+    return K, W, Z, tree
+
+
+# ---------------------------------------------------------------------------
+# generator
+# ---------------------------------------------------------------------------
+
+def pin_splitmix64_published_vectors():
+    rows = [l.split() for l in open(os.path.join(GOLDEN, "splitmix64.txt")) if l[0] != "#"]
+    assert rows
+    for seed, i, val in rows:
+        assert orc.splitmix64_at(int(seed), int(i)) == int(val), (seed, i)
+
+
+def pin_init_rule():
+    """Child j of a segment starts at the member with the j-th smallest init hash."""
+    rng = np.random.default_rng(3)
+    pos = np.sort(rng.choice(5000, 40, replace=False))
+    Zs = rng.standard_normal((40, 5))
+    for level, seed in ((0, 0), (2, 77)):
+        h = np.array([orc.init_hash(seed, level, int(p)) for p in pos], dtype=np.uint64)
+        want = Zs[np.argsort(h, kind="stable")[:6]]
+        got = orc.level_init(Zs, pos, 6, seed, level)
+        np.testing.assert_array_equal(got, want)
+    # the hash of (seed, level, pos) is the generator output `pos` of the stream whose
+    # state is output `level` of the stream seeded with `seed`
+    assert orc.init_hash(0, 0, 0) == orc.splitmix64_at(orc.splitmix64_at(0, 0), 0)
+    assert orc.init_hash(5, 3, 11) == orc.splitmix64_at(orc.splitmix64_at(5, 3), 11)
+
+
+# ---------------------------------------------------------------------------
+# projection
+# ---------------------------------------------------------------------------
+
+def pin_projection_matches_numpy():
+    rng = np.random.default_rng(1)
+    X = rng.standard_normal((37, 24))
+    W = rng.standard_normal((24, 7))
+    np.testing.assert_allclose(orc.project(X, W), X @ W, rtol=1e-12, atol=1e-12)
+    Qg = rng.standard_normal((9, 4, 24))
+    np.testing.assert_allclose(orc.query_latent(Qg, W), Qg.mean(axis=1) @ W, rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# balanced assignment
+# ---------------------------------------------------------------------------
+
+def _pair_key(D, pos, i, c):
+    return (D[i, c], pos[i], c)
+
+
+def _is_stable(D, pos, a, b):
+    m = len(a)
+    for i in range(m):
+        for c in range(b):
+            if c == a[i]:
+                continue
+            if _pair_key(D, pos, i, c) >= _pair_key(D, pos, i, a[i]):
+                continue                          # i does not prefer c
+            members = [j for j in range(m) if a[j] == c]
+            if any((D[i, c], pos[i]) < (D[j, c], pos[j]) for j in members):
+                return False                      # (i, c) blocks
+    return True
+
+
+def _all_balanced(m, b):
+    cap = m // b
+    for lab in itertools.product(range(b), repeat=m):
+        if all(lab.count(c) == cap for c in range(b)):
+            yield np.array(lab)
+
+
+def pin_balanced_assign_bruteforce():
+    rng = np.random.default_rng(7)
+    for trial in range(24):
+        b = (2, 3, 4)[trial % 3]
+        m = b * (2 if b > 2 else 3 + trial % 2)
+        if trial % 4 == 0:  # coarse integer distances: many exact ties
+            D = rng.integers(0, 3, (m, b)).astype(float)
+        else:
+            D = rng.random((m, b))
+        pos = np.sort(rng.choice(100, m, replace=False))
+        stable = [a for a in _all_balanced(m, b) if _is_stable(D, pos, a, b)]
+        assert len(stable) == 1, (trial, len(stable))
+        np.testing.assert_array_equal(orc.balanced_assign(D, pos), stable[0])
+
+
+def _deferred_acceptance(D, pos, b):
+    """Key-proposing deferred acceptance, written independently of the oracle."""
+    m = D.shape[0]
+    cap = m // b
+    pref = [sorted(range(b), key=lambda c, i=i: (D[i, c], c)) for i in range(m)]
+    nxt = [0] * m
+    held = {c: [] for c in range(b)}
+    free = list(range(m))
+    while free:
+        i = free.pop()
+        c = pref[i][nxt[i]]
+        nxt[i] += 1
+        held[c].append(i)
+        if len(held[c]) > cap:
+            held[c].sort(key=lambda j: (D[j, c], pos[j]))
+            free.append(held[c].pop())
+    a = np.empty(m, int)
+    for c, js in held.items():
+        a[js] = c
+    return a
+
+
+def pin_balanced_assign_vs_deferred_acceptance():
+    rng = np.random.default_rng(11)
+    for m, b in ((64, 4), (240, 8), (256, 16)):
+        D = rng.random((m, b)) ** 2
+        pos = np.sort(rng.choice(10 * m, m, replace=False))
+        a = orc.balanced_assign(D, pos)
+        np.testing.assert_array_equal(np.bincount(a, minlength=b), np.full(b, m // b))
+        np.testing.assert_array_equal(a, _deferred_acceptance(D, pos, b))
+
+
+def pin_distances_closed_form():
+    rng = np.random.default_rng(5)
+    Z, mu = rng.standard_normal((20, 6)), rng.standard_normal((3, 6))
+    want = ((Z[:, None, :] - mu[None]) ** 2).sum(-1)
+    np.testing.assert_allclose(orc.distances(Z, mu), want, rtol=1e-12)
+    a = rng.integers(0, 3, 20)
+    a[:3] = [0, 1, 2]
+    want_mu = np.stack([Z[a == c].mean(0) for c in range(3)])
+    np.testing.assert_allclose(orc.means(Z, a, 3), want_mu, rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# tree build
+# ---------------------------------------------------------------------------
+
+def pin_tree_invariants():
+    K, W, Z, tree = tiny_tree_case()
+    n, L, leaf = Z.shape[0], len(tree.branching), tree.leaf_size
+    li = tree.leaf_index.astype(np.int64)
+    np.testing.assert_array_equal(np.sort(li), np.arange(n))            # permutation
+    leaves = li.reshape(-1, leaf)
+    assert np.all(np.diff(leaves, axis=1) > 0)                           # ascending in a leaf
+    # members of every node at every level, from the leaf partition
+    for l in range(L):
+        per_node = n // tree.nodes[l]
+        groups = li.reshape(tree.nodes[l], per_node)                     # node-major leaf order
+        mu = Z[groups].mean(axis=1)
+        np.testing.assert_allclose(tree.centroids[l], mu, rtol=1e-10, atol=1e-12)
+        np.testing.assert_array_equal(tree.min_pos[l], groups.min(axis=1))
+        if l > 0:
+            b = tree.branching[l]
+            parent = tree.centroids[l].reshape(-1, b, Z.shape[1]).mean(axis=1)
+            np.testing.assert_allclose(parent, tree.centroids[l - 1], rtol=1e-10, atol=1e-12)
+    # the trace's last assignment of each level is the partition above
+    for l in range(L):
+        per_node = n // tree.nodes[l]
+        node_of = np.empty(n, np.int64)
+        node_of[li] = np.repeat(np.arange(tree.nodes[l]), per_node)
+        np.testing.assert_array_equal(tree.trace[l, -1], node_of)
+
+
+def pin_tree_first_step_from_init():
+    """Level 0's first assignment uses the seeded start and the stable balanced rule."""
+    K, W, Z, tree = tiny_tree_case()
+    n = Z.shape[0]
+    b = tree.branching[0]
+    pos = np.arange(n)
+    h = np.array([orc.init_hash(0, 0, int(p)) for p in pos], dtype=np.uint64)
+    mu0 = Z[np.argsort(h)[:b]]
+    D = ((Z[:, None, :] - mu0[None]) ** 2).sum(-1)
+    a = _deferred_acceptance_fast(D, pos, b)
+    np.testing.assert_array_equal(tree.trace[0, 0], a)
+
+
+def _deferred_acceptance_fast(D, pos, b):
+    """Round-synchronous deferred acceptance (numpy), independent of the oracle."""
+    m = D.shape[0]
+    cap = m // b
+    order = np.lexsort((np.broadcast_to(np.arange(b), D.shape), D), axis=1)
+    ptr = np.zeros(m, np.int64)
+    rows = np.arange(m)
+    while True:
+        ch = order[rows, ptr]
+        moved = False
+        for c in range(b):
+            w = np.nonzero(ch == c)[0]
+            if len(w) > cap:
+                o = np.lexsort((pos[w], D[w, c]))
+                ptr[w[o[cap:]]] += 1
+                moved = True
+        if not moved:
+            return ch
+
+
+def pin_tree_deterministic_and_seeded():
+    _, _, Z, t1 = tiny_tree_case()
+    t2 = orc.build_tree(Z, t1.branching, t1.leaf_size, 4, seed=0)
+    np.testing.assert_array_equal(t1.leaf_index, t2.leaf_index)
+    t3 = orc.build_tree(Z, t1.branching, t1.leaf_size, 4, seed=1)
+    assert not np.array_equal(t1.leaf_index, t3.leaf_index)
+
+
+# ---------------------------------------------------------------------------
+# hierarchical search
+# ---------------------------------------------------------------------------
+
+def _flat_topB(qlat, tree, B, q_pos=None):
+    """Brute force: score every leaf centroid, keep the B best (score desc, id asc)."""
+    leafc = tree.centroids[-1]
+    T = qlat.shape[0]
+    out = np.full((T, B * tree.leaf_size), -1, np.int64)
+    for t in range(T):
+        s = leafc @ qlat[t]
+        ids = np.arange(len(s))
+        if q_pos is not None:
+            keep = tree.min_pos[-1] <= q_pos[t]
+            s, ids = s[keep], ids[keep]
+        o = np.lexsort((ids, -s))[:B]
+        keys = tree.leaf_index.reshape(-1, tree.leaf_size)[ids[o]].reshape(-1)
+        out[t, :len(keys)] = keys
+    return out
+
+
+def pin_select_full_beam_equals_flat():
+    K, W, Z, tree = tiny_tree_case()
+    rng = np.random.default_rng(2)
+    q = rng.standard_normal((20, 3, K.shape[1]))
+    qlat = q.mean(axis=1) @ W
+    full = [tree.nodes[l] for l in range(len(tree.nodes) - 1)]
+    for B in (1, 5, 12):
+        idx, bt, scored = orc.select(qlat, tree, full + [B], trace=True)
+        np.testing.assert_array_equal(idx, _flat_topB(qlat, tree, B))
+        assert np.all(scored == sum(tree.nodes))
+    # causal: a leaf is reachable with a full beam iff its smallest position is visible
+    q_pos = rng.integers(0, Z.shape[0], 20)
+    idx, bt, _ = orc.select(qlat, tree, full + [7], q_pos=q_pos, trace=True)
+    np.testing.assert_array_equal(idx, _flat_topB(qlat, tree, 7, q_pos))
+
+
+def pin_select_beam_walk():
+    """Narrow beams: counts, ranking and parent/child structure of every kept node."""
+    K, W, Z, tree = tiny_tree_case()
+    rng = np.random.default_rng(4)
+    qlat = rng.standard_normal((16, W.shape[1]))
+    beam = [3, 5]
+    idx, bt, scored = orc.select(qlat, tree, beam, trace=True)
+    b1 = tree.branching[1]
+    assert np.all(scored == tree.nodes[0] + beam[0] * b1)
+    for t in range(16):
+        s0 = tree.centroids[0] @ qlat[t]
+        top0 = np.lexsort((np.arange(len(s0)), -s0))[:beam[0]]
+        np.testing.assert_array_equal(bt[0, t, :beam[0]], top0)
+        cand = (top0[:, None] * b1 + np.arange(b1)).reshape(-1)
+        s1 = tree.centroids[1][cand] @ qlat[t]
+        top1 = cand[np.lexsort((cand, -s1))[:beam[1]]]
+        np.testing.assert_array_equal(bt[1, t, :beam[1]], top1)
+        want = tree.leaf_index.reshape(-1, tree.leaf_size)[top1].reshape(-1)
+        np.testing.assert_array_equal(idx[t], want)
+    # causal eligibility, brute force: every kept node's smallest position is visible,
+    # and no eligible child of a kept parent that scored higher was dropped
+    q_pos = rng.integers(0, Z.shape[0] // 3, 16)
+    idx, bt, _ = orc.select(qlat, tree, beam, q_pos=q_pos, trace=True)
+    for t in range(16):
+        for l in range(2):
+            kept = bt[l, t][bt[l, t] >= 0]
+            assert np.all(tree.min_pos[l][kept] <= q_pos[t])
+        elig0 = np.nonzero(tree.min_pos[0] <= q_pos[t])[0]
+        s0 = tree.centroids[0][elig0] @ qlat[t]
+        top0 = elig0[np.lexsort((elig0, -s0))[:beam[0]]]
+        np.testing.assert_array_equal(bt[0, t][bt[0, t] >= 0], top0)
+        valid = idx[t][idx[t] >= 0]
+        assert len(valid) % tree.leaf_size == 0 and len(valid) > 0
+
+
+# ---------------------------------------------------------------------------
+# attention
+# ---------------------------------------------------------------------------
+
+def _sdpa_dense(Qg, K, V, mask, scale):
+    """torch SDPA in float64 on CPU: Qg [T,G,d], K/V [n,d], mask [T,n] bool (True=visible)."""
+    q = torch.from_numpy(Qg).permute(1, 0, 2)[None]           # [1, G, T, d]
+    k = torch.from_numpy(K)[None, None].expand(1, Qg.shape[1], -1, -1)
+    v = torch.from_numpy(V)[None, None].expand(1, Qg.shape[1], -1, -1)
+    m = torch.from_numpy(mask)[None, None]
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=m, scale=scale)
+    return o[0].permute(1, 0, 2).numpy()
+
+
+def _attn_case(seed=0, T=6, G=3, d=16, n=40, K_sel=12):
+    rng = np.random.default_rng(seed)
+    Qg = rng.standard_normal((T, G, d))
+    K = rng.standard_normal((n, d))
+    V = rng.standard_normal((n, d))
+    idx = np.stack([rng.choice(n - 8, K_sel, replace=False) for _ in range(T)]).astype(np.int32)
+    idx[:, -2:] = -1
+    return rng, Qg, K, V, idx
+
+
+def _mask_from(idx, n, tail, q_pos, causal):
+    T = idx.shape[0]
+    mask = np.zeros((T, n), bool)
+    for t in range(T):
+        sel = idx[t][idx[t] >= 0]
+        mask[t, sel] = True
+        mask[t, tail[0]:tail[1]] = True
+        if causal:
+            mask[t, q_pos[t] + 1:] = False
+    return mask
+
+
+def pin_attention_equals_sdpa():
+    rng, Qg, K, V, idx = _attn_case()
+    n, d = K.shape
+    scale = 1 / np.sqrt(d)
+    # every key selected (through the index list and a tail) = full attention
+    all_idx = np.tile(np.arange(n - 8, dtype=np.int32), (Qg.shape[0], 1))
+    O, LSE = orc.attn_fwd(Qg, K, V, all_idx, tail=(n - 8, n), scale=scale)
+    full = _sdpa_dense(Qg, K, V, np.ones((Qg.shape[0], n), bool), scale)
+    np.testing.assert_allclose(O, full, rtol=1e-10, atol=1e-12)
+    lse_want = np.log(np.exp(scale * np.einsum("tgd,nd->tgn", Qg, K)).sum(-1))
+    np.testing.assert_allclose(LSE, lse_want, rtol=1e-10)
+    # sparse + tail + causal against a boolean mask
+    q_pos = rng.integers(n // 2, n, Qg.shape[0]).astype(np.int32)
+    for causal in (False, True):
+        O, _ = orc.attn_fwd(Qg, K, V, idx, q_pos=q_pos, causal=causal, tail=(n - 8, n), scale=scale)
+        mask = _mask_from(idx, n, (n - 8, n), q_pos, causal)
+        np.testing.assert_allclose(O, _sdpa_dense(Qg, K, V, mask, scale), rtol=1e-10, atol=1e-12)
+
+
+def pin_attention_special_cases():
+    rng, Qg, K, V, idx = _attn_case(1)
+    T = Qg.shape[0]
+    one = np.full((T, 3), -1, np.int32)
+    one[:, 1] = np.arange(T) * 2
+    O, LSE = orc.attn_fwd(Qg, K, V, one, scale=0.7)
+    for t in range(T):
+        np.testing.assert_allclose(O[t], np.broadcast_to(V[2 * t], O[t].shape), rtol=1e-12)
+        np.testing.assert_allclose(LSE[t], 0.7 * Qg[t] @ K[2 * t], rtol=1e-12)
+    perm = idx[:, rng.permutation(idx.shape[1])]
+    a, _ = orc.attn_fwd(Qg, K, V, idx)
+    b, _ = orc.attn_fwd(Qg, K, V, perm)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-14)
+    none = np.full((T, 4), -1, np.int32)
+    O, LSE = orc.attn_fwd(Qg, K, V, none)
+    assert np.all(O == 0) and np.all(np.isneginf(LSE))
+
+
+def pin_backward_autograd():
+    rng, Qg, K, V, idx = _attn_case(2)
+    n, d = K.shape
+    q_pos = rng.integers(n // 2, n, Qg.shape[0]).astype(np.int32)
+    dO = rng.standard_normal(Qg.shape)
+    scale = 0.3
+    dQ, dK, dV = orc.attn_bwd(Qg, K, V, idx, dO, q_pos=q_pos, causal=True, tail=(n - 8, n), scale=scale)
+    mask = torch.from_numpy(_mask_from(idx, n, (n - 8, n), q_pos, True))
+    q = torch.from_numpy(Qg).requires_grad_()
+    k = torch.from_numpy(K).requires_grad_()
+    v = torch.from_numpy(V).requires_grad_()
+    s = scale * torch.einsum("tgd,nd->tgn", q, k)
+    s = s.masked_fill(~mask[:, None, :], float("-inf"))
+    o = torch.einsum("tgn,nd->tgd", torch.softmax(s, -1), v)
+    o.backward(torch.from_numpy(dO))
+    np.testing.assert_allclose(dQ, q.grad.numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dK, k.grad.numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dV, v.grad.numpy(), rtol=1e-9, atol=1e-12)
+
+
+def pin_backward_finite_differences():
+    rng, Qg, K, V, idx = _attn_case(3, T=3, G=2, d=6, n=20, K_sel=6)
+    dO = rng.standard_normal(Qg.shape)
+    dQ, dK, dV = orc.attn_bwd(Qg, K, V, idx, dO)
+
+    def loss(Qx, Kx, Vx):
+        O, _ = orc.attn_fwd(Qx, Kx, Vx, idx)
+        return float((O * dO).sum())
+
+    eps = 1e-6
+    for arr, grad, pick in ((Qg, dQ, (1, 1, 2)), (K, dK, (int(idx[0, 0]), 3)), (V, dV, (int(idx[2, 1]), 0))):
+        plus, minus = arr.copy(), arr.copy()
+        plus[pick] += eps
+        minus[pick] -= eps
+        args_p = [Qg, K, V]
+        args_m = [Qg, K, V]
+        which = 0 if arr is Qg else (1 if arr is K else 2)
+        args_p[which], args_m[which] = plus, minus
+        fd = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        assert abs(fd - grad[pick]) < 1e-6 * max(1.0, abs(fd)), (which, fd, grad[pick])
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
