@@ -1,0 +1,354 @@
+// api.cu -- C ABI of the LSA library: argument validation, workspace layout and
+// dispatch to the kernels.  Every check runs on the host before any launch; no
+// call aborts, traps or throws.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "lsa_common.cuh"
+#include "lsa_internal.h"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int ok() {
+  g_err[0] = '\0';
+  return LSA_OK;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(LSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+uint64_t align256(uint64_t x) { return (x + 255) & ~uint64_t(255); }
+
+bool valid_dtype(int dt) { return dt == LSA_F32 || dt == LSA_BF16; }
+
+// Recompute a descriptor from its defining fields and compare, so a corrupted or
+// hand-made struct is rejected.
+int check_desc(const lsa_tree_desc* t) {
+  if (!t) return fail(LSA_ERR_INVALID_ARG, "tree descriptor is NULL");
+  lsa_tree_desc ref;
+  int rc = lsa_tree_describe(t->n_heads, t->r, t->branching, t->levels, t->leaf_size, &ref);
+  if (rc != LSA_OK) return rc;
+  if (memcmp(&ref, t, sizeof(ref)) != 0)
+    return fail(LSA_ERR_INVALID_ARG, "tree descriptor was not produced by lsa_tree_describe");
+  return LSA_OK;
+}
+
+}  // namespace
+
+namespace lsa {
+
+size_t build_workspace_layout(const lsa_tree_desc& t, char* base, BuildPlan* P) {
+  const int64_t H = t.n_heads, n = t.n_tree, R = t.r, nslots = H * n;
+  int bmax = 0;
+  int64_t max_tiles = 0, max_partial = 0, max_grid_segc = 0, S = 1;
+  for (int l = 0; l < t.levels; ++l) {
+    const int b = t.branching[l];
+    bmax = b > bmax ? b : bmax;
+    const int64_t m = n / S, cap = m / b, nseg = H * S;
+    const int64_t tiles = nseg * ceil_div(m, kTile);
+    max_tiles = tiles > max_tiles ? tiles : max_tiles;
+    const int64_t cpn = ceil_div(cap, kMeanChunk);
+    const int64_t part = cpn > 1 ? nseg * b * cpn * R : 0;
+    max_partial = part > max_partial ? part : max_partial;
+    if (m > kCtaMaxSeg) max_grid_segc = nseg * b > max_grid_segc ? nseg * b : max_grid_segc;
+    S *= b;
+  }
+  const int64_t max_nodes = H * t.nodes[t.levels - 1];
+  uint64_t off = 0;
+  auto take = [&](uint64_t bytes) {
+    uint64_t at = off;
+    off = align256(off + (bytes ? bytes : 1));
+    return base ? base + at : nullptr;
+  };
+  char* p;
+  p = take(nslots * R * 4);              if (P) P->Za = reinterpret_cast<float*>(p);
+  p = take(nslots * R * 4);              if (P) P->Zb = reinterpret_cast<float*>(p);
+  p = take(nslots * 4);                  if (P) P->pa = reinterpret_cast<int32_t*>(p);
+  p = take(nslots * 4);                  if (P) P->pb = reinterpret_cast<int32_t*>(p);
+  p = take(nslots * 4);                  if (P) P->order = reinterpret_cast<int32_t*>(p);
+  p = take(nslots * bmax * 4);           if (P) P->D = reinterpret_cast<float*>(p);
+  p = take(nslots * 8);                  if (P) P->pref = reinterpret_cast<uint64_t*>(p);
+  p = take(nslots * 4);                  if (P) P->dbits = reinterpret_cast<uint32_t*>(p);
+  p = take(nslots);                      if (P) P->choice = reinterpret_cast<uint8_t*>(p);
+  p = take(nslots);                      if (P) P->ptr = reinterpret_cast<uint8_t*>(p);
+  p = take(max_nodes * R * 4);           if (P) P->mu = reinterpret_cast<float*>(p);
+  p = take(max_tiles * bmax * 4);        if (P) P->tcnt = reinterpret_cast<int32_t*>(p);
+  p = take(max_tiles * bmax * 8);        if (P) P->toff = reinterpret_cast<int64_t*>(p);
+  p = take(max_tiles * bmax * 8);        if (P) P->cand_h = reinterpret_cast<uint64_t*>(p);
+  p = take(max_tiles * bmax * 8);        if (P) P->cand_slot = reinterpret_cast<int64_t*>(p);
+  p = take(max_partial * 4);             if (P) P->partial = reinterpret_cast<float*>(p);
+  p = take(max_grid_segc * 2048 * 4);    if (P) P->hist = reinterpret_cast<uint32_t*>(p);
+  p = take(max_grid_segc * 8);           if (P) P->thr = reinterpret_cast<unsigned long long*>(p);
+  p = take(max_grid_segc * 8);           if (P) P->prefix = reinterpret_cast<unsigned long long*>(p);
+  p = take(max_grid_segc * 4);           if (P) P->need = reinterpret_cast<uint32_t*>(p);
+  p = take(max_grid_segc * 4);           if (P) P->active = reinterpret_cast<int32_t*>(p);
+  p = take(24 * 4);                      if (P) P->flags = reinterpret_cast<int32_t*>(p);
+  p = take(sizeof(GridBarrier));         if (P) P->bar = reinterpret_cast<GridBarrier*>(p);
+  return off;
+}
+
+}  // namespace lsa
+
+extern "C" {
+
+int lsa_version(void) { return LSA_VERSION; }
+
+const char* lsa_strerror(int status) {
+  switch (status) {
+    case LSA_OK: return "ok";
+    case LSA_ERR_INVALID_ARG: return "invalid argument";
+    case LSA_ERR_SHAPE: return "unsupported or inconsistent shape";
+    case LSA_ERR_CUDA: return "CUDA error";
+    case LSA_ERR_TIMEOUT: return "device loop hit its iteration cap";
+    case LSA_ERR_NONFINITE: return "NaN in an ordering decision";
+    case LSA_ERR_WORKSPACE: return "workspace missing or too small";
+    default: return "unknown status";
+  }
+}
+
+const char* lsa_last_error(void) { return g_err; }
+
+int lsa_tree_describe(int32_t n_heads, int32_t r, const int32_t* branching, int32_t levels, int32_t leaf_size,
+                      lsa_tree_desc* out) {
+  if (!branching || !out) return fail(LSA_ERR_INVALID_ARG, "branching and out must be non-NULL");
+  if (n_heads < 1) return fail(LSA_ERR_SHAPE, "n_heads must be >= 1 (got %d)", n_heads);
+  if (r != 16 && r != 32 && r != 64) return fail(LSA_ERR_SHAPE, "r must be 16, 32 or 64 (got %d)", r);
+  if (levels < 1 || levels > LSA_MAX_LEVELS) return fail(LSA_ERR_SHAPE, "levels must be in [1, 8] (got %d)", levels);
+  if (leaf_size < 8 || leaf_size > 4096) return fail(LSA_ERR_SHAPE, "leaf_size must be in [8, 4096] (got %d)", leaf_size);
+  lsa_tree_desc t;
+  memset(&t, 0, sizeof(t));
+  t.n_heads = n_heads;
+  t.r = r;
+  t.levels = levels;
+  t.leaf_size = leaf_size;
+  int64_t nodes = 1;
+  for (int l = 0; l < levels; ++l) {
+    if (branching[l] < 2 || branching[l] > LSA_MAX_BRANCHING)
+      return fail(LSA_ERR_SHAPE, "branching[%d] must be in [2, 16] (got %d)", l, branching[l]);
+    nodes *= branching[l];
+    if (nodes * leaf_size > (int64_t(1) << 30)) return fail(LSA_ERR_SHAPE, "tree larger than 2^30 keys");
+    t.branching[l] = branching[l];
+    t.nodes[l] = nodes;
+  }
+  t.n_tree = nodes * leaf_size;
+  if ((int64_t)n_heads * t.n_tree >= (int64_t(1) << 31))
+    return fail(LSA_ERR_SHAPE, "n_heads * n_tree must stay below 2^31 (got %lld)", (long long)n_heads * t.n_tree);
+  uint64_t off = 0;
+  for (int l = 0; l < levels; ++l) {
+    t.off_centroids[l] = off;
+    off = align256(off + (uint64_t)n_heads * t.nodes[l] * r * sizeof(float));
+  }
+  for (int l = 0; l < levels; ++l) {
+    t.off_min_pos[l] = off;
+    off = align256(off + (uint64_t)n_heads * t.nodes[l] * sizeof(int32_t));
+  }
+  t.off_leaf_index = off;
+  off = align256(off + (uint64_t)n_heads * t.n_tree * sizeof(int32_t));
+  t.bytes = off;
+  *out = t;
+  return ok();
+}
+
+int lsa_build_workspace_bytes(const lsa_tree_desc* tree, int32_t d, size_t* bytes) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  *bytes = lsa::build_workspace_layout(*tree, nullptr, nullptr);
+  return ok();
+}
+
+int lsa_build_tree(const lsa_tree_desc* tree, void* tree_mem, const void* K, int64_t n_cap, int32_t d,
+                   int32_t dtype, const void* W, int32_t iters, uint64_t seed, void* workspace,
+                   size_t workspace_bytes, int32_t* trace, int32_t* status, void* stream) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (!tree_mem || !K || !W) return fail(LSA_ERR_INVALID_ARG, "tree_mem, K and W must be non-NULL");
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  if (n_cap < tree->n_tree) return fail(LSA_ERR_SHAPE, "n_cap (%lld) < n_tree (%lld)", (long long)n_cap, (long long)tree->n_tree);
+  if (iters < 1 || iters > 1000) return fail(LSA_ERR_INVALID_ARG, "iters must be in [1, 1000] (got %d)", iters);
+  const size_t need = lsa::build_workspace_layout(*tree, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need)
+    return fail(LSA_ERR_WORKSPACE, "build needs %zu workspace bytes (got %zu)", need, workspace ? workspace_bytes : (size_t)0);
+  lsa::BuildPlan P;
+  lsa::build_workspace_layout(*tree, static_cast<char*>(workspace), &P);
+  P.iters = iters;
+  P.seed = seed;
+  P.coop_blocks = lsa::da_grid_blocks();
+  if (P.coop_blocks <= 0) return fail(LSA_ERR_CUDA, "cannot size the cooperative assignment grid");
+  cudaError_t e = lsa::run_build(P, *tree, tree_mem, K, n_cap, d, dtype, W, trace, status,
+                                 static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_build_tree");
+  return ok();
+}
+
+int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq, int32_t d,
+               int32_t dtype, const void* W, const int32_t* beam, const int32_t* q_pos, int32_t* idx_out,
+               float* qlat_out, int32_t* beam_out, int32_t* status, void* stream) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (!beam) return fail(LSA_ERR_INVALID_ARG, "beam must be non-NULL");
+  if (T < 0) return fail(LSA_ERR_SHAPE, "T must be >= 0");
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  if (Hq < tree->n_heads || Hq % tree->n_heads) return fail(LSA_ERR_SHAPE, "Hq (%d) must be a multiple of n_heads (%d)", Hq, tree->n_heads);
+  if (Hq / tree->n_heads > 64) return fail(LSA_ERR_SHAPE, "more than 64 query heads per group");
+  lsa::SelectArgs a;
+  memset(&a, 0, sizeof(a));
+  int beam_max = 0;
+  for (int l = 0; l < tree->levels; ++l) {
+    const int64_t avail = l == 0 ? tree->nodes[0] : (int64_t)beam[l - 1] * tree->branching[l];
+    if (beam[l] < 1 || beam[l] > LSA_MAX_BEAM || beam[l] > avail)
+      return fail(LSA_ERR_SHAPE, "beam[%d] = %d must be in [1, min(64, %lld)]", l, beam[l], (long long)avail);
+    beam_max = beam[l] > beam_max ? beam[l] : beam_max;
+    a.beam[l] = beam[l];
+    a.branching[l] = tree->branching[l];
+    a.nodes[l] = tree->nodes[l];
+    a.off_c[l] = tree->off_centroids[l];
+    a.off_m[l] = tree->off_min_pos[l];
+  }
+  if (T == 0) return ok();
+  if (!tree_mem || !Q || !W || !idx_out) return fail(LSA_ERR_INVALID_ARG, "tree_mem, Q, W and idx_out must be non-NULL");
+  a.Q = Q; a.W = W; a.tree = static_cast<const char*>(tree_mem); a.q_pos = q_pos; a.idx_out = idx_out;
+  a.qlat_out = qlat_out; a.beam_out = beam_out; a.status = status;
+  a.T = T; a.Hq = Hq; a.Hkv = tree->n_heads; a.G = Hq / tree->n_heads; a.d = d; a.r = tree->r;
+  a.levels = tree->levels; a.leaf = tree->leaf_size; a.beam_max = beam_max; a.n_tree = tree->n_tree;
+  a.off_leaf = tree->off_leaf_index;
+  cudaError_t e = lsa::run_select(a, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_select");
+  return ok();
+}
+
+static int attn_common_checks(const void* Q, int32_t T, int32_t Hq, const void* K, const void* V, int32_t n_heads,
+                              int64_t n_cap, int32_t d, int32_t dtype, const int32_t* idx, int32_t K_sel,
+                              const int32_t* q_pos, int32_t causal, int64_t tail_begin, int64_t tail_end) {
+  if (T < 0 || n_heads < 1 || Hq < n_heads || Hq % n_heads) return fail(LSA_ERR_SHAPE, "need T >= 0 and Hq a multiple of n_heads");
+  const int G = Hq / n_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(LSA_ERR_SHAPE, "query heads per group must be 1, 2, 4 or 8 (got %d)", G);
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  if (n_cap < 1) return fail(LSA_ERR_SHAPE, "n_cap must be >= 1");
+  if (K_sel < 0) return fail(LSA_ERR_SHAPE, "K_sel must be >= 0");
+  if (tail_begin < 0 || tail_end < tail_begin || tail_end > n_cap)
+    return fail(LSA_ERR_SHAPE, "tail range [%lld, %lld) must lie in [0, n_cap)", (long long)tail_begin, (long long)tail_end);
+  if (T > 0) {
+    if (!Q || !K || !V) return fail(LSA_ERR_INVALID_ARG, "Q, K and V must be non-NULL");
+    if (K_sel > 0 && !idx) return fail(LSA_ERR_INVALID_ARG, "idx must be non-NULL when K_sel > 0");
+    if (causal && !q_pos) return fail(LSA_ERR_INVALID_ARG, "q_pos is required when causal");
+  }
+  return LSA_OK;
+}
+
+int lsa_attn_workspace_bytes(int32_t T, int32_t Hq, int32_t n_heads, int32_t d, int32_t K_sel, int64_t tail_len,
+                             size_t* bytes) {
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
+  if (T < 0 || n_heads < 1 || Hq < 1 || K_sel < 0 || tail_len < 0 || (d != 64 && d != 128))
+    return fail(LSA_ERR_SHAPE, "bad sizes");
+  const int ns = lsa::attn_splits(T, n_heads, K_sel + tail_len);
+  *bytes = ns > 1 ? (size_t)T * Hq * ns * (d + 2) * sizeof(float) : 0;
+  return ok();
+}
+
+static void fill_attn(lsa::AttnArgs& a, const void* Q, int32_t T, int32_t Hq, const void* K, const void* V,
+                      int32_t n_heads, int64_t n_cap, int32_t d, const int32_t* idx, int32_t K_sel,
+                      const int32_t* q_pos, int32_t causal, int64_t tail_begin, int64_t tail_end, float scale,
+                      int32_t* status) {
+  memset(&a, 0, sizeof(a));
+  a.Q = Q; a.K = K; a.V = V; a.idx = K_sel > 0 ? idx : nullptr; a.q_pos = q_pos; a.status = status;
+  a.T = T; a.n_cap = n_cap; a.tail_begin = tail_begin; a.tail_end = tail_end;
+  a.Hq = Hq; a.Hkv = n_heads; a.G = Hq / n_heads; a.d = d; a.K_sel = K_sel; a.causal = causal ? 1 : 0;
+  const int64_t keys = K_sel + (tail_end - tail_begin);
+  a.nsplit = lsa::attn_splits(T, n_heads, keys);
+  int64_t kps = (keys + a.nsplit - 1) / a.nsplit;
+  kps = (kps + 15) / 16 * 16;
+  a.keys_per_split = (int32_t)(kps > 0 ? kps : 16);
+  a.scale = scale;
+  a.scale_log2 = scale * 1.44269504088896340736f;
+}
+
+int lsa_sparse_attn(const void* Q, int32_t T, int32_t Hq, const void* K, const void* V, int32_t n_heads,
+                    int64_t n_cap, int32_t d, int32_t dtype, const int32_t* idx, int32_t K_sel, const int32_t* q_pos,
+                    int32_t causal, int64_t tail_begin, int64_t tail_end, float scale, void* O, float* LSE,
+                    void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  int rc = attn_common_checks(Q, T, Hq, K, V, n_heads, n_cap, d, dtype, idx, K_sel, q_pos, causal, tail_begin, tail_end);
+  if (rc != LSA_OK) return rc;
+  if (!std::isfinite(scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite");
+  if (T == 0) return ok();
+  if (!O || !LSE) return fail(LSA_ERR_INVALID_ARG, "O and LSE must be non-NULL");
+  lsa::AttnArgs a;
+  fill_attn(a, Q, T, Hq, K, V, n_heads, n_cap, d, idx, K_sel, q_pos, causal, tail_begin, tail_end, scale, status);
+  a.O = O;
+  a.LSE = LSE;
+  if (a.nsplit > 1) {
+    const size_t need = (size_t)T * Hq * a.nsplit * (d + 2) * sizeof(float);
+    if (!workspace || workspace_bytes < need)
+      return fail(LSA_ERR_WORKSPACE, "attention needs %zu workspace bytes (got %zu)", need, workspace ? workspace_bytes : (size_t)0);
+    a.part = static_cast<float*>(workspace);
+  }
+  cudaError_t e = lsa::run_attn_fwd(a, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn");
+  return ok();
+}
+
+int lsa_sparse_attn_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, const void* V, int32_t n_heads,
+                        int64_t n_cap, int32_t d, int32_t dtype, const void* O, const float* LSE, const void* dO,
+                        const int32_t* idx, int32_t K_sel, const int32_t* q_pos, int32_t causal, int64_t tail_begin,
+                        int64_t tail_end, float scale, float* dQ, float* dK, float* dV, int32_t* status,
+                        void* stream) {
+  int rc = attn_common_checks(Q, T, Hq, K, V, n_heads, n_cap, d, dtype, idx, K_sel, q_pos, causal, tail_begin, tail_end);
+  if (rc != LSA_OK) return rc;
+  if (!std::isfinite(scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite");
+  if (!dK || !dV) return fail(LSA_ERR_INVALID_ARG, "dK and dV must be non-NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t kv_bytes = (size_t)n_heads * n_cap * d * sizeof(float);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(dK, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_bwd");
+  if ((e = cudaMemsetAsync(dV, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_bwd");
+  if (T == 0) return ok();
+  if (!O || !LSE || !dO || !dQ) return fail(LSA_ERR_INVALID_ARG, "O, LSE, dO and dQ must be non-NULL");
+  lsa::AttnArgs a;
+  fill_attn(a, Q, T, Hq, K, V, n_heads, n_cap, d, idx, K_sel, q_pos, causal, tail_begin, tail_end, scale, status);
+  a.O = const_cast<void*>(O);
+  a.LSE = const_cast<float*>(LSE);
+  a.dO = dO;
+  a.dQ = dQ;
+  a.dK = dK;
+  a.dV = dV;
+  if (a.nsplit > 1 && (e = cudaMemsetAsync(dQ, 0, (size_t)T * Hq * d * sizeof(float), st)) != cudaSuccess)
+    return cuda_fail(e, "lsa_sparse_attn_bwd");
+  e = lsa::run_attn_bwd(a, dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_bwd");
+  return ok();
+}
+
+int lsa_status_clear(int32_t* status, void* stream) {
+  if (!status) return fail(LSA_ERR_INVALID_ARG, "status is NULL");
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_status_clear");
+  return ok();
+}
+
+int lsa_status_check(const int32_t* status, void* stream, int32_t* host_out) {
+  if (!status || !host_out) return fail(LSA_ERR_INVALID_ARG, "status and host_out must be non-NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(host_out, status, sizeof(int32_t), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_status_check");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+// lsa_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/lsa.h"
+
+namespace lsa {
+
+constexpr int kTile = 1024;           // keys per tile in partition / init passes
+constexpr int64_t kCtaMaxSeg = 8192;  // segments up to this size: one CTA runs the whole assignment
+constexpr int kMeanChunk = 256;       // keys summed by one warp before a second-stage sum
+constexpr int kMaxRounds = 4096;      // proposal-round cap of the balanced assignment
+constexpr uint64_t kBarrierTimeoutNs = 2000000000ull;  // grid-barrier wait cap (2 s)
+
+struct GridBarrier {
+  unsigned arrive;
+  unsigned gen;
+  int abort;
+  int pad;
+};
+
+// Device workspace of one tree build, carved out of the caller's buffer.
+struct BuildPlan {
+  float* Za;
+  float* Zb;
+  int32_t* pa;
+  int32_t* pb;
+  int32_t* order;
+  float* D;
+  uint64_t* pref;
+  uint32_t* dbits;
+  uint8_t* choice;
+  uint8_t* ptr;
+  float* mu;
+  int32_t* tcnt;
+  int64_t* toff;
+  uint64_t* cand_h;
+  int64_t* cand_slot;
+  float* partial;
+  uint32_t* hist;
+  unsigned long long* thr;
+  unsigned long long* prefix;
+  uint32_t* need;
+  int32_t* active;
+  int32_t* flags;
+  GridBarrier* bar;
+  int iters;
+  uint64_t seed;
+  int coop_blocks;
+};
+
+// Byte sizes of every region of a build workspace (layout shared by the size
+// query and the carving of a caller buffer).
+size_t build_workspace_layout(const lsa_tree_desc& t, char* base, BuildPlan* plan);
+
+cudaError_t run_build(const BuildPlan& P, const lsa_tree_desc& t, void* tree_mem, const void* K, int64_t n_cap,
+                      int d, int dtype, const void* W, int32_t* trace, int32_t* status, cudaStream_t st);
+int da_grid_blocks();
+
+struct SelectArgs {
+  const void* Q;
+  const void* W;
+  const char* tree;
+  const int32_t* q_pos;
+  int32_t* idx_out;
+  float* qlat_out;
+  int32_t* beam_out;
+  int32_t* status;
+  int64_t T;
+  int32_t Hq, Hkv, G, d, r, levels, leaf, beam_max;
+  int64_t n_tree;
+  int32_t branching[LSA_MAX_LEVELS];
+  int32_t beam[LSA_MAX_LEVELS];
+  int64_t nodes[LSA_MAX_LEVELS];
+  uint64_t off_c[LSA_MAX_LEVELS];
+  uint64_t off_m[LSA_MAX_LEVELS];
+  uint64_t off_leaf;
+};
+cudaError_t run_select(const SelectArgs& a, int dtype, cudaStream_t st);
+
+struct AttnArgs {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int32_t* idx;
+  const int32_t* q_pos;
+  void* O;
+  float* LSE;
+  float* part;        // split partials [T][Hq][nsplit][d + 2]
+  const void* dO;
+  float* dQ;
+  float* dK;
+  float* dV;
+  int32_t* status;
+  int64_t T, n_cap, tail_begin, tail_end;
+  int32_t Hq, Hkv, G, d, K_sel, causal, nsplit, keys_per_split;
+  float scale_log2;   // scale * log2(e)
+  float scale;
+};
+int attn_splits(int64_t T, int Hkv, int64_t keys);
+cudaError_t run_attn_fwd(const AttnArgs& a, int dtype, cudaStream_t st);
+cudaError_t run_attn_bwd(const AttnArgs& a, int dtype, cudaStream_t st);
+
+}  // namespace lsa

@@ -1,0 +1,295 @@
+"""Thin Python binding of the C ABI in ``include/lsa.h`` (``liblsa.so``).
+
+The ``lsa_*`` functions keep the C names and only marshal arguments: torch
+tensors become device pointers and sizes, the current torch stream becomes the
+``cudaStream_t``.  Every step of the computation runs in the CUDA library; if the
+library cannot be loaded, importing this module raises.  A few helpers below
+(``build_tree``, ``select``, ``sparse_attn``, ``sparse_attn_bwd``) allocate
+outputs and workspace with torch and then call the same entry points.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from dataclasses import dataclass
+
+import torch
+
+from . import build_ext
+
+LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_SHAPE, LSA_ERR_CUDA, LSA_ERR_TIMEOUT, LSA_ERR_NONFINITE, LSA_ERR_WORKSPACE = range(7)
+LSA_F32, LSA_BF16 = 0, 1
+MAX_LEVELS = 8
+_DTYPE = {torch.float32: LSA_F32, torch.bfloat16: LSA_BF16}
+
+
+class LsaError(RuntimeError):
+    def __init__(self, code: int, what: str, detail: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {lsa_strerror(code)} ({code}){': ' + detail if detail else ''}")
+
+
+class lsa_tree_desc(ctypes.Structure):
+    _fields_ = [
+        ("n_heads", ctypes.c_int32), ("r", ctypes.c_int32), ("levels", ctypes.c_int32),
+        ("leaf_size", ctypes.c_int32), ("n_tree", ctypes.c_int64),
+        ("branching", ctypes.c_int32 * MAX_LEVELS), ("nodes", ctypes.c_int64 * MAX_LEVELS),
+        ("off_centroids", ctypes.c_uint64 * MAX_LEVELS), ("off_min_pos", ctypes.c_uint64 * MAX_LEVELS),
+        ("off_leaf_index", ctypes.c_uint64), ("bytes", ctypes.c_uint64),
+    ]
+
+
+def _load():
+    path = os.environ.get("LSA_LIBRARY") or build_ext.LIB
+    if not os.path.exists(path):
+        raise ImportError(f"CUDA library {path} is missing; build it with "
+                          f"`python -m hierarchical_latent_key_b200.build_ext`")
+    lib = ctypes.CDLL(path)
+    P, i32, i64, u64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+    D = ctypes.POINTER(lsa_tree_desc)
+    f32 = ctypes.c_float
+    sig = {
+        "lsa_version": (ctypes.c_int, []),
+        "lsa_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+        "lsa_last_error": (ctypes.c_char_p, []),
+        "lsa_tree_describe": (ctypes.c_int, [i32, i32, P, i32, i32, D]),
+        "lsa_build_workspace_bytes": (ctypes.c_int, [D, i32, ctypes.POINTER(sz)]),
+        "lsa_build_tree": (ctypes.c_int, [D, P, P, i64, i32, i32, P, i32, u64, P, sz, P, P, P]),
+        "lsa_select": (ctypes.c_int, [D, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, P]),
+        "lsa_attn_workspace_bytes": (ctypes.c_int, [i32, i32, i32, i32, i32, i64, ctypes.POINTER(sz)]),
+        "lsa_sparse_attn": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i64, i64,
+                                           f32, P, P, P, sz, P, P]),
+        "lsa_sparse_attn_bwd": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, P, P, P, i32, P, i32,
+                                               i64, i64, f32, P, P, P, P, P]),
+        "lsa_status_clear": (ctypes.c_int, [P, P]),
+        "lsa_status_check": (ctypes.c_int, [P, P, ctypes.POINTER(i32)]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+LIBRARY_PATH = _lib._name
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch tensor")
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to the LSA library must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream, ref: torch.Tensor | None = None):
+    if stream is None:
+        dev = ref.device if ref is not None and ref.is_cuda else torch.device("cuda", torch.cuda.current_device())
+        stream = torch.cuda.current_stream(dev)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype(t: torch.Tensor) -> int:
+    try:
+        return _DTYPE[t.dtype]
+    except KeyError:
+        raise TypeError(f"unsupported dtype {t.dtype}") from None
+
+
+def _raise(rc: int, what: str):
+    if rc != LSA_OK:
+        raise LsaError(rc, what, _lib.lsa_last_error().decode())
+
+
+# --- C ABI, same names ------------------------------------------------------------
+
+def lsa_version() -> int:
+    return int(_lib.lsa_version())
+
+
+def lsa_strerror(code: int) -> str:
+    return _lib.lsa_strerror(int(code)).decode()
+
+
+def lsa_tree_describe(n_heads: int, r: int, branching, leaf_size: int) -> lsa_tree_desc:
+    br = (ctypes.c_int32 * max(MAX_LEVELS, len(branching)))(*branching)
+    out = lsa_tree_desc()
+    _raise(_lib.lsa_tree_describe(n_heads, r, ctypes.cast(br, ctypes.c_void_p), len(branching), leaf_size,
+                                  ctypes.byref(out)), "lsa_tree_describe")
+    return out
+
+
+def lsa_build_workspace_bytes(desc: lsa_tree_desc, d: int) -> int:
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_build_workspace_bytes(ctypes.byref(desc), d, ctypes.byref(n)), "lsa_build_workspace_bytes")
+    return int(n.value)
+
+
+def lsa_build_tree(desc, tree_mem, K, W, iters, seed, workspace, trace=None, status=None, stream=None):
+    """K: [n_heads, n_cap, d]; W: [n_heads, d, r]; tree_mem/workspace: uint8 device tensors."""
+    _raise(_lib.lsa_build_tree(ctypes.byref(desc), _ptr(tree_mem), _ptr(K), K.shape[1], K.shape[2], _dtype(K),
+                               _ptr(W), iters, seed & ((1 << 64) - 1), _ptr(workspace), workspace.numel(),
+                               _ptr(trace), _ptr(status), _stream(stream, K)), "lsa_build_tree")
+
+
+def lsa_select(desc, tree_mem, Q, W, beam, q_pos, idx_out, qlat_out=None, beam_out=None, status=None,
+               stream=None):
+    """Q: [T, Hq, d]; beam: host sequence of ints; q_pos: int32 [T] or None."""
+    bm = (ctypes.c_int32 * max(MAX_LEVELS, len(beam)))(*beam)
+    T, Hq, d = Q.shape
+    _raise(_lib.lsa_select(ctypes.byref(desc), _ptr(tree_mem), _ptr(Q), T, Hq, d, _dtype(Q), _ptr(W),
+                           ctypes.cast(bm, ctypes.c_void_p), _ptr(q_pos), _ptr(idx_out), _ptr(qlat_out),
+                           _ptr(beam_out), _ptr(status), _stream(stream, Q)), "lsa_select")
+
+
+def lsa_attn_workspace_bytes(T, Hq, n_heads, d, K_sel, tail_len) -> int:
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_attn_workspace_bytes(T, Hq, n_heads, d, K_sel, tail_len, ctypes.byref(n)),
+           "lsa_attn_workspace_bytes")
+    return int(n.value)
+
+
+def lsa_sparse_attn(Q, K, V, idx, q_pos, causal, tail_begin, tail_end, scale, O, LSE, workspace=None,
+                    status=None, stream=None):
+    T, Hq, d = Q.shape
+    K_sel = 0 if idx is None else idx.shape[-1]
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _raise(_lib.lsa_sparse_attn(_ptr(Q), T, Hq, _ptr(K), _ptr(V), K.shape[0], K.shape[1], d, _dtype(Q), _ptr(idx),
+                                K_sel, _ptr(q_pos), int(bool(causal)), tail_begin, tail_end, float(scale), _ptr(O),
+                                _ptr(LSE), _ptr(workspace), ws_n, _ptr(status), _stream(stream, Q)),
+           "lsa_sparse_attn")
+
+
+def lsa_sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos, causal, tail_begin, tail_end, scale, dQ, dK, dV,
+                        status=None, stream=None):
+    T, Hq, d = Q.shape
+    K_sel = 0 if idx is None else idx.shape[-1]
+    _raise(_lib.lsa_sparse_attn_bwd(_ptr(Q), T, Hq, _ptr(K), _ptr(V), K.shape[0], K.shape[1], d, _dtype(Q),
+                                    _ptr(O), _ptr(LSE), _ptr(dO), _ptr(idx), K_sel, _ptr(q_pos),
+                                    int(bool(causal)), tail_begin, tail_end, float(scale), _ptr(dQ), _ptr(dK),
+                                    _ptr(dV), _ptr(status), _stream(stream, Q)), "lsa_sparse_attn_bwd")
+
+
+def lsa_status_clear(status, stream=None):
+    _raise(_lib.lsa_status_clear(_ptr(status), _stream(stream, status)), "lsa_status_clear")
+
+
+def lsa_status_check(status, stream=None) -> int:
+    out = ctypes.c_int32()
+    _raise(_lib.lsa_status_check(_ptr(status), _stream(stream, status), ctypes.byref(out)), "lsa_status_check")
+    return int(out.value)
+
+
+# --- helpers: torch-allocated outputs around the same entry points -----------------
+
+def _new_status(device):
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def check_status(status, what: str):
+    code = lsa_status_check(status)
+    if code != LSA_OK:
+        raise LsaError(code, what, "reported by a kernel")
+
+
+@dataclass
+class Tree:
+    desc: lsa_tree_desc
+    mem: torch.Tensor          # uint8 [desc.bytes] on the device
+
+    @property
+    def levels(self) -> int:
+        return self.desc.levels
+
+    @property
+    def branching(self):
+        return tuple(self.desc.branching[l] for l in range(self.desc.levels))
+
+    def centroids(self, level: int) -> torch.Tensor:
+        d = self.desc
+        n = d.n_heads * d.nodes[level] * d.r
+        off = d.off_centroids[level]
+        return self.mem[off:off + 4 * n].view(torch.float32).view(d.n_heads, d.nodes[level], d.r)
+
+    def min_pos(self, level: int) -> torch.Tensor:
+        d = self.desc
+        n = d.n_heads * d.nodes[level]
+        off = d.off_min_pos[level]
+        return self.mem[off:off + 4 * n].view(torch.int32).view(d.n_heads, d.nodes[level])
+
+    def leaf_index(self) -> torch.Tensor:
+        d = self.desc
+        n = d.n_heads * d.n_tree
+        off = d.off_leaf_index
+        return self.mem[off:off + 4 * n].view(torch.int32).view(d.n_heads, d.n_tree)
+
+
+def build_tree(K, W, branching, leaf_size, iters, seed, trace=False, workspace=None, status=None, check=True):
+    """Build the index over positions [0, leaf_size * prod(branching)) of K."""
+    Hkv, n_cap, d = K.shape
+    desc = lsa_tree_describe(Hkv, W.shape[2], branching, leaf_size)
+    mem = torch.empty(desc.bytes, dtype=torch.uint8, device=K.device)
+    need = lsa_build_workspace_bytes(desc, d)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=K.device)
+    tr = torch.empty(len(branching), iters, Hkv, desc.n_tree, dtype=torch.int32, device=K.device) if trace else None
+    st = _new_status(K.device) if status is None else status
+    lsa_build_tree(desc, mem, K, W, iters, seed, workspace, tr, st)
+    if check:
+        check_status(st, "lsa_build_tree")
+    tree = Tree(desc, mem)
+    return (tree, tr) if trace else tree
+
+
+def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, status=None, check=True):
+    T = Q.shape[0]
+    d = tree.desc
+    K_sel = beam[-1] * d.leaf_size
+    idx = torch.empty(d.n_heads, T, K_sel, dtype=torch.int32, device=Q.device)
+    ql = torch.empty(T, d.n_heads, d.r, dtype=torch.float32, device=Q.device) if qlat else None
+    bo = torch.empty(d.levels, d.n_heads, T, max(beam), dtype=torch.int32, device=Q.device) if beams else None
+    st = _new_status(Q.device) if status is None else status
+    lsa_select(d, tree.mem, Q, W, beam, q_pos, idx, ql, bo, st)
+    if check:
+        check_status(st, "lsa_select")
+    out = [idx]
+    if qlat:
+        out.append(ql)
+    if beams:
+        out.append(bo)
+    return out[0] if len(out) == 1 else tuple(out)
+
+
+def sparse_attn(Q, K, V, idx, q_pos=None, causal=False, tail=(0, 0), scale=None, workspace=None, status=None,
+                check=True):
+    T, Hq, d = Q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    K_sel = 0 if idx is None else idx.shape[-1]
+    need = lsa_attn_workspace_bytes(T, Hq, K.shape[0], d, K_sel, tail[1] - tail[0])
+    if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
+        workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
+    O = torch.empty_like(Q)
+    LSE = torch.empty(T, Hq, dtype=torch.float32, device=Q.device)
+    st = _new_status(Q.device) if status is None else status
+    lsa_sparse_attn(Q, K, V, idx, q_pos, causal, tail[0], tail[1], scale, O, LSE, workspace if need else None, st)
+    if check:
+        check_status(st, "lsa_sparse_attn")
+    return O, LSE
+
+
+def sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos=None, causal=False, tail=(0, 0), scale=None, status=None,
+                    check=True):
+    T, Hq, d = Q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dQ = torch.empty(T, Hq, d, dtype=torch.float32, device=Q.device)
+    dK = torch.empty(K.shape, dtype=torch.float32, device=Q.device)
+    dV = torch.empty(V.shape, dtype=torch.float32, device=Q.device)
+    st = _new_status(Q.device) if status is None else status
+    lsa_sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos, causal, tail[0], tail[1], scale, dQ, dK, dV, st)
+    if check:
+        check_status(st, "lsa_sparse_attn_bwd")
+    return dQ, dK, dV

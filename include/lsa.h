@@ -1,0 +1,206 @@
+/*
+ * lsa.h -- C ABI of the B200 (sm_100a) library for the hot path of Latent Sparse
+ * Attention (LSA) with a hierarchical latent-key index.
+ *
+ * What the path computes (pages about "Latent Sparse Attention"):
+ *  - kongchang.com, "Latent Sparse Attention Breaks Through the Million-Token
+ *    Context Bottleneck", section "How LSA Sidesteps Per-Key Scoring with
+ *    Hierarchical Clustering": keys are projected into a low-dimensional latent
+ *    space and grouped level by level into a tree whose root holds all keys;
+ *    a query starts at the root, scores a few candidate clusters per level and
+ *    descends into a few branches until it reaches leaf key subsets.
+ *  - bdtechtalks.com, "Latent sparse attention", section "How latent sparse
+ *    attention works": each cluster keeps a centroid next to references to its
+ *    original keys; the query is compared with centroids, a fixed number of
+ *    original keys is taken from the chosen clusters and attention runs over
+ *    them (plus a window of recent tokens); hierarchical search keeps a fixed
+ *    budget per level.
+ *  - kongchang.com, section "The Accuracy-Efficiency Dilemma": sparse attention
+ *    where each query interacts with only k keys.
+ *
+ * Conventions shared by every entry point
+ *  - Device pointers are plain CUDA device addresses allocated by the caller;
+ *    the library never allocates device memory.  Host pointers are marked "host".
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued asynchronously on it; a call returns once its launches are
+ *    queued.  Only lsa_status_check synchronises.
+ *  - Every call validates its arguments on the host first and returns an
+ *    lsa_status; on a validation error nothing is launched.  lsa_last_error()
+ *    then holds a one-line explanation (thread-local).
+ *  - `status` is a caller-allocated device int32 (zero it before use, e.g. with
+ *    lsa_status_clear).  Kernels that detect a problem while running (a NaN score,
+ *    a device loop that hit its round cap) write a nonzero lsa_status code there;
+ *    the first code written wins.  Read it with lsa_status_check.
+ *  - dtype: LSA_F32 or LSA_BF16; Q, K, V, W, O and dO of one call share it.
+ *    Accumulation is fp32 throughout; gradients are fp32.
+ *  - No call aborts, traps or throws.
+ */
+#ifndef LSA_H
+#define LSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LSA_VERSION 1
+#define LSA_MAX_LEVELS 8
+#define LSA_MAX_BRANCHING 16
+#define LSA_MAX_BEAM 64
+
+typedef enum lsa_status {
+  LSA_OK = 0,
+  LSA_ERR_INVALID_ARG = 1, /* null pointer, unknown dtype, bad scalar            */
+  LSA_ERR_SHAPE = 2,       /* sizes inconsistent or outside supported limits     */
+  LSA_ERR_CUDA = 3,        /* a CUDA runtime call or launch failed               */
+  LSA_ERR_TIMEOUT = 4,     /* a device loop or barrier hit its iteration cap     */
+  LSA_ERR_NONFINITE = 5,   /* NaN met where an ordering decision was needed      */
+  LSA_ERR_WORKSPACE = 6    /* workspace missing or smaller than required         */
+} lsa_status;
+
+typedef enum lsa_dtype { LSA_F32 = 0, LSA_BF16 = 1 } lsa_dtype;
+
+/* Geometry and memory layout of a tree (one tree per KV head, all heads in one
+ * buffer).  Filled by lsa_tree_describe; treat as read-only afterwards.
+ * Layout of the tree buffer (byte offsets, every region 256-byte aligned):
+ *   centroids of level l : float [n_heads][nodes[l]][r]   at off_centroids[l]
+ *   min_pos of level l   : int32 [n_heads][nodes[l]]      at off_min_pos[l]
+ *                          (smallest key position under the node)
+ *   leaf_index           : int32 [n_heads][n_tree]        at off_leaf_index
+ *                          (keys of leaf 0 in ascending position, then leaf 1, ...)
+ * Node ids: level l has nodes[l] = b_0*...*b_l nodes; the children of node p of
+ * level l-1 are p*b_l + j, j < b_l.  Leaves are the nodes of the last level and
+ * each holds exactly leaf_size keys. */
+typedef struct lsa_tree_desc {
+  int32_t n_heads;
+  int32_t r;
+  int32_t levels;
+  int32_t leaf_size;
+  int64_t n_tree;                         /* = leaf_size * prod(branching)     */
+  int32_t branching[LSA_MAX_LEVELS];
+  int64_t nodes[LSA_MAX_LEVELS];
+  uint64_t off_centroids[LSA_MAX_LEVELS];
+  uint64_t off_min_pos[LSA_MAX_LEVELS];
+  uint64_t off_leaf_index;
+  uint64_t bytes;                         /* size of the tree buffer           */
+} lsa_tree_desc;
+
+/* Library version (LSA_VERSION). */
+int lsa_version(void);
+
+/* Static text for a status code; never NULL. */
+const char *lsa_strerror(int status);
+
+/* Detail of the last error returned on this thread ("" if none). */
+const char *lsa_last_error(void);
+
+/* Host only.  Fills *out for n_heads trees with latent dim r, `levels` levels of
+ * fan-out branching[0..levels) (root to leaves, each in [2, 16]) and leaves of
+ * leaf_size keys.  Limits: 1 <= levels <= 8, r in {16, 32, 64}, leaf_size in [8, 4096],
+ * n_tree <= 2^30 and n_heads * n_tree < 2^31.
+ * Returns LSA_ERR_SHAPE / LSA_ERR_INVALID_ARG on violations. */
+int lsa_tree_describe(int32_t n_heads, int32_t r, const int32_t *branching /* host */,
+                      int32_t levels, int32_t leaf_size, lsa_tree_desc *out /* host */);
+
+/* Host only.  Device workspace bytes lsa_build_tree needs for keys of width d. */
+int lsa_build_workspace_bytes(const lsa_tree_desc *tree, int32_t d, size_t *bytes /* host */);
+
+/* Build the index (kongchang.com, "How LSA Sidesteps Per-Key Scoring with
+ * Hierarchical Clustering": latent projection, then clustering level by level
+ * from the root "similar to hierarchical k-means").
+ *  K        : [n_heads][n_cap][d] keys; positions [0, n_tree) are indexed, the
+ *             rest (decode appends) are left for the dense tail.
+ *  W        : [n_heads][d][r] latent projection (same dtype as K).
+ *  iters    : k-means rounds per level (>= 1).  Each round assigns every key of a
+ *             parent node to one of its b_l children with exactly
+ *             (parent size / b_l) keys per child -- the unique stable assignment
+ *             under the pair order (squared distance asc, key position asc,
+ *             child asc) -- then moves each child centroid to its members' mean.
+ *             Round 1 starts from the members with the b_l smallest SplitMix64
+ *             hashes of (seed, level, position).  Stored centroids are the means
+ *             of the last round's assignment.
+ *  trace    : optional (NULL) int32 [levels][iters][n_heads][n_tree]: node id of
+ *             every key (indexed by position) after each round's assignment.
+ *  tree_mem : tree->bytes of device memory, written completely.
+ * Limits: d in {64, 128}; n_cap >= n_tree.  Writes LSA_ERR_TIMEOUT to *status if
+ * an assignment needs more than 4096 proposal rounds (never seen in practice),
+ * LSA_ERR_NONFINITE if a distance is NaN. */
+int lsa_build_tree(const lsa_tree_desc *tree, void *tree_mem, const void *K, int64_t n_cap,
+                   int32_t d, int32_t dtype, const void *W, int32_t iters, uint64_t seed,
+                   void *workspace, size_t workspace_bytes, int32_t *trace, int32_t *status,
+                   void *stream);
+
+/* Hierarchical search (kongchang.com, "How LSA Sidesteps ..."; bdtechtalks.com,
+ * "How latent sparse attention works": fixed budget per level, a fixed number
+ * of original keys from the chosen clusters).
+ *  Q       : [T][Hq][d] queries; Hq = G * n_heads, query head h belongs to group
+ *            h / G and the G heads of a group share one selection.
+ *  W       : the [n_heads][d][r] projection the tree was built with.
+ *  beam    : host int32[levels]; beam[0] <= nodes[0], beam[l] <= beam[l-1]*b_l,
+ *            every beam[l] in [1, 64].
+ *  q_pos   : NULL (non-causal) or device int32[T] query positions; a node is a
+ *            candidate only if its min_pos <= q_pos.
+ * Per (group g, query t): q = (mean of the group's G query rows) . W[g] (fp32);
+ * level-0 candidates are all top nodes, level-l candidates the children of the
+ * nodes kept at level l-1; score = <q, centroid> (fp32); keep the beam[l] best by
+ * (score desc, node id asc).
+ *  idx_out : [n_heads][T][beam[levels-1] * leaf_size] int32 key positions of the
+ *            kept leaves, leaf by leaf in rank order, ascending inside a leaf,
+ *            -1 where fewer leaves were eligible.
+ *  qlat_out: optional [T][n_heads][r] float query latents.
+ *  beam_out: optional [levels][n_heads][T][max beam] int32 kept node ids per level
+ *            in rank order, -1 padded.
+ * Writes LSA_ERR_NONFINITE to *status if a score is NaN. */
+int lsa_select(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, int32_t T,
+               int32_t Hq, int32_t d, int32_t dtype, const void *W, const int32_t *beam,
+               const int32_t *q_pos, int32_t *idx_out, float *qlat_out, int32_t *beam_out,
+               int32_t *status, void *stream);
+
+/* Host only.  Workspace bytes lsa_sparse_attn needs for these sizes (0 when the
+ * call runs without key splitting). */
+int lsa_attn_workspace_bytes(int32_t T, int32_t Hq, int32_t n_heads, int32_t d, int32_t K_sel,
+                             int64_t tail_len, size_t *bytes);
+
+/* Sparse attention forward (kongchang.com, "The Accuracy-Efficiency Dilemma";
+ * bdtechtalks.com, "How latent sparse attention works").
+ *  Q [T][Hq][d];  K, V [n_heads][n_cap][d];  idx [n_heads][T][K_sel] key positions
+ *  (-1 = none) shared by the G query heads of a group; the dense range
+ *  [tail_begin, tail_end) of positions is attended by every query as well.
+ *  causal: key j is visible to query t only if j <= q_pos[t] (q_pos device
+ *  int32[T], required when causal).  logits = scale * <q, k>.
+ *  O   [T][Hq][d] (dtype of Q) = softmax-weighted sum of V rows;
+ *  LSE [T][Hq] float = natural log of the softmax denominator (-inf and O = 0 when
+ *  a query sees no key).  Indices must lie in [0, n_cap) or be -1, and must not
+ *  repeat within a row or fall inside the tail range. */
+int lsa_sparse_attn(const void *Q, int32_t T, int32_t Hq, const void *K, const void *V,
+                    int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, const int32_t *idx,
+                    int32_t K_sel, const int32_t *q_pos, int32_t causal, int64_t tail_begin,
+                    int64_t tail_end, float scale, void *O, float *LSE, void *workspace,
+                    size_t workspace_bytes, int32_t *status, void *stream);
+
+/* Backward of lsa_sparse_attn for a fixed selection (same arguments), given the
+ * forward's O and LSE and the upstream gradient dO ([T][Hq][d], dtype of Q).
+ * Outputs (float): dQ [T][Hq][d]; dK, dV [n_heads][n_cap][d], overwritten (zero
+ * where no query sees the key); dK/dV sum over the G heads of a group and over
+ * every query that sees the key.  Needs no workspace. */
+int lsa_sparse_attn_bwd(const void *Q, int32_t T, int32_t Hq, const void *K, const void *V,
+                        int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, const void *O,
+                        const float *LSE, const void *dO, const int32_t *idx, int32_t K_sel,
+                        const int32_t *q_pos, int32_t causal, int64_t tail_begin,
+                        int64_t tail_end, float scale, float *dQ, float *dK, float *dV,
+                        int32_t *status, void *stream);
+
+/* Zero the device status word on `stream`. */
+int lsa_status_clear(int32_t *status, void *stream);
+
+/* Synchronise `stream`, copy the device status word to *host_out and return
+ * LSA_OK, or LSA_ERR_CUDA if the stream reported an error. */
+int lsa_status_check(const int32_t *status, void *stream, int32_t *host_out /* host */);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H */

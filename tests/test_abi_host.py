@@ -1,0 +1,120 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every
+declared symbol, and rejects bad arguments with status codes before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hierarchical_latent_key_b200 import build_ext, configs
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lsa():
+    build_ext.build()
+    from hierarchical_latent_key_b200 import lsa as mod
+    return mod
+
+
+def declared_symbols():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names |= set(re.findall(r"\b(lsa_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lsa):
+    lib = ctypes.CDLL(lsa.LIBRARY_PATH)
+    syms = declared_symbols()
+    assert len(syms) >= 12
+    for s in syms:
+        assert hasattr(lib, s), s
+
+
+def test_version_and_strerror(lsa):
+    assert lsa.lsa_version() == 1
+    for code in range(7):
+        assert lsa.lsa_strerror(code)
+    assert lsa.lsa_strerror(99) == "unknown status"
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(n_heads=0), 2), (dict(r=48), 2), (dict(branching=(16, 1)), 2), (dict(branching=(17,)), 2),
+    (dict(leaf_size=4), 2), (dict(branching=(16,) * 9), 2), (dict(branching=(16,) * 7, leaf_size=64), 2), (dict(n_heads=4, branching=(16,) * 6), 2),
+])
+def test_describe_rejects(lsa, kw, code):
+    args = dict(n_heads=2, r=64, branching=(16, 16), leaf_size=64)
+    args.update(kw)
+    with pytest.raises(lsa.LsaError) as e:
+        lsa.lsa_tree_describe(args["n_heads"], args["r"], args["branching"], args["leaf_size"])
+    assert e.value.code == code
+
+
+def test_describe_layout(lsa):
+    d = lsa.lsa_tree_describe(8, 64, (8, 16, 16, 16, 5), 64)
+    assert d.n_tree == 10485760
+    assert [d.nodes[l] for l in range(5)] == [8, 128, 2048, 32768, 163840]
+    offs = [d.off_centroids[l] for l in range(5)] + [d.off_min_pos[l] for l in range(5)] + [d.off_leaf_index]
+    assert all(o % 256 == 0 for o in offs) and offs == sorted(offs)
+    assert d.bytes >= d.off_leaf_index + 8 * d.n_tree * 4
+
+
+@pytest.mark.parametrize("name", ["decode_128k", "prefill_1m", "decode_10m"])
+def test_index_is_about_two_percent_of_kv(lsa, name):
+    """The pages put the index at about 2% of the KV cache; the layout here lands near it."""
+    c = configs.get(name)
+    d = lsa.lsa_tree_describe(c.Hkv, c.r, c.branching, c.leaf)
+    kv_bytes = 2 * c.Hkv * c.n * c.d * 2
+    assert 0.005 <= d.bytes / kv_bytes <= 0.03, d.bytes / kv_bytes
+
+
+def test_workspace_queries(lsa):
+    d = lsa.lsa_tree_describe(2, 64, (16, 16, 8), 64)
+    assert lsa.lsa_build_workspace_bytes(d, 128) > 2 * 2 * 131072 * 64 * 4
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_build_workspace_bytes(d, 96)
+    assert lsa.lsa_attn_workspace_bytes(4096, 32, 8, 128, 2048, 0) == 0     # enough units: no split
+    assert lsa.lsa_attn_workspace_bytes(1, 32, 8, 128, 2048, 64) > 0       # decode: split partials
+
+
+def test_calls_validate_before_launch(lsa):
+    """Bad arguments come back as status codes; no device is needed to see them."""
+    import torch
+    L = lsa._lib
+    d = lsa.lsa_tree_describe(1, 16, (16, 16), 16)
+    bm = (ctypes.c_int32 * 8)(4, 65)
+    rc = L.lsa_select(ctypes.byref(d), None, None, 4, 1, 64, 0, None, ctypes.cast(bm, ctypes.c_void_p),
+                      None, None, None, None, None, None)
+    assert rc == lsa.LSA_ERR_SHAPE and b"beam[1]" in L.lsa_last_error()
+    bm = (ctypes.c_int32 * 8)(4, 8)
+    rc = L.lsa_select(ctypes.byref(d), None, None, 4, 1, 64, 0, None, ctypes.cast(bm, ctypes.c_void_p),
+                      None, None, None, None, None, None)
+    assert rc == lsa.LSA_ERR_INVALID_ARG
+    d2 = lsa.lsa_tree_describe(2, 16, (16, 16), 16)
+    rc = L.lsa_select(ctypes.byref(d2), None, None, 4, 3, 64, 0, None, ctypes.cast(bm, ctypes.c_void_p),
+                      None, None, None, None, None, None)
+    assert rc == lsa.LSA_ERR_SHAPE
+    bad = lsa.lsa_tree_desc.from_buffer_copy(d)
+    bad.off_leaf_index += 256
+    n = ctypes.c_size_t()
+    assert L.lsa_build_workspace_bytes(ctypes.byref(bad), 64, ctypes.byref(n)) == lsa.LSA_ERR_INVALID_ARG
+    # attention: 3 query heads per group, bad tail, causal without positions, missing workspace
+    args = lambda **kw: dict(dict(Q=1, T=2, Hq=8, K=1, V=1, H=2, n_cap=100, d=128, dt=1, idx=1, K_sel=16,
+                                  qp=None, causal=0, tb=0, te=0), **kw)
+    def call(a):
+        P = lambda v: ctypes.c_void_p(16) if v else None
+        return L.lsa_sparse_attn(P(a["Q"]), a["T"], a["Hq"], P(a["K"]), P(a["V"]), a["H"], a["n_cap"], a["d"],
+                                 a["dt"], P(a["idx"]), a["K_sel"], P(a["qp"]), a["causal"], a["tb"], a["te"],
+                                 0.1, ctypes.c_void_p(16), ctypes.c_void_p(16), None, 0, None, None)
+    assert call(args(Hq=6)) == lsa.LSA_ERR_SHAPE
+    assert call(args(tb=50, te=120)) == lsa.LSA_ERR_SHAPE
+    assert call(args(causal=1)) == lsa.LSA_ERR_INVALID_ARG
+    assert call(args(dt=7)) == lsa.LSA_ERR_INVALID_ARG
+    assert call(args(d=96)) == lsa.LSA_ERR_SHAPE
+    assert call(args(T=1, K_sel=2048)) == lsa.LSA_ERR_WORKSPACE
+    assert call(args(T=0)) == lsa.LSA_OK
