@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the LSA hot path (hierarchical latent-key select + sparse attention).
+
+Default workload: last-chunk prefill at 1M context (4096 new query tokens, 32 query
+/ 8 KV heads, d=128, tree 16/16/16/4 with leaf 64, beam 8/32/32/32 -> 2048 keys per
+query).  A step = select + sparse attention for the whole chunk; the index over the
+cached keys is built once before timing (its time is reported as build_ms).
+``--workload decode_10m`` times single-token decode steps at 10,485,760 tokens
+(append one key/value row per KV head, select, attend to selection + tail).
+
+Launch: ``python bench.py [--gpus N] [--steps K] [--warmup W]``; for N > 1 under
+torchrun, every rank runs its own independent request (weak scaling) and rank 0
+prints one JSON line.  ``--impl reference`` times the CPU oracle instead.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from hierarchical_latent_key_b200 import configs  # noqa: E402
+
+METRIC = "LSA layer queries/sec (select+attn) at 1M/10M ctx; HBM GB/s and tensor % of peak"
+L2_FLUSH_BYTES = 512 << 20   # > 126 MB L2
+
+
+# ---------------------------------------------------------------------------
+# host helpers (also exercised by the multi-process CPU tests)
+# ---------------------------------------------------------------------------
+
+def rank_seed(base: int, rank: int) -> int:
+    """Each rank serves its own request: independent synthetic inputs per rank."""
+    return int(base) + 7919 * int(rank)
+
+
+def aggregate(local_s: float, units_per_rank: int, world: int, reduce_max=None):
+    """Whole-job throughput: all ranks' units over the slowest rank's device time."""
+    t = reduce_max(local_s) if reduce_max is not None else local_s
+    return world * units_per_rank / t, t
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return dict(hbm_gbs=j.get("hbm_gbs", 6650.0), bf16_tflops=j.get("bf16_tflops", 1590.0),
+                    bf16_tflops_sustained=j.get("bf16_tflops_sustained", 1400.0), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=self.file, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        self.file.flush()
+
+    def summary(self):
+        rows = []
+        try:
+            with open(self.file.name) as f:
+                for line in f:
+                    p = [x.strip() for x in line.split(",")]
+                    if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                        rows.append(p)
+        finally:
+            os.unlink(self.file.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def cores_used() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------------------
+# CUDA arm
+# ---------------------------------------------------------------------------
+
+class Prefill:
+    """Last-chunk prefill: one step = select + attention for the whole chunk."""
+
+    def __init__(self, cfg, dev, seed):
+        from hierarchical_latent_key_b200 import lsa
+        self.lsa, self.cfg, self.dev = lsa, cfg, dev
+        c = cfg.case(dev, seed)
+        self.K, self.V, self.W, self.Q, self.q_pos = c.K, c.V, c.W, c.Q, c.q_pos
+        del c
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        self.tree = lsa.build_tree(self.K, self.W, cfg.branching, cfg.leaf, cfg.iters, seed)
+        torch.cuda.synchronize(dev)
+        self.build_ms = 1e3 * (time.perf_counter() - t0)
+        T, Hq, d = self.Q.shape
+        self.idx = torch.empty(cfg.Hkv, T, cfg.K_sel, dtype=torch.int32, device=dev)
+        self.O = torch.empty_like(self.Q)
+        self.LSE = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        need = lsa.lsa_attn_workspace_bytes(T, Hq, cfg.Hkv, d, cfg.K_sel, 0)
+        self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        self.scale = 1.0 / math.sqrt(d)
+        self.units = T
+        self.launches_per_step = 1 + 1 + (1 if need else 0)
+
+    def select(self, Q=None):
+        self.lsa.lsa_select(self.tree.desc, self.tree.mem, self.Q if Q is None else Q, self.W, self.cfg.beam,
+                            self.q_pos, self.idx, status=self.status)
+
+    def attend(self, Q=None, O=None, LSE=None):
+        self.lsa.lsa_sparse_attn(self.Q if Q is None else Q, self.K, self.V, self.idx, self.q_pos, True, 0, 0,
+                                 self.scale, self.O if O is None else O, self.LSE if LSE is None else LSE,
+                                 self.ws, self.status)
+
+    def attn_algorithmic_bytes(self):
+        """Bytes the attention must move at least: every distinct selected K/V row once,
+        plus queries, outputs, LSE and the index lists."""
+        d = self.Q.shape[2]
+        rows = 0
+        for g in range(self.cfg.Hkv):
+            v = self.idx[g]
+            rows += int(torch.unique(v[v >= 0]).numel())
+        esz = self.Q.element_size()
+        return (rows * 2 * d * esz + 2 * self.Q.numel() * esz + self.LSE.numel() * 4 + self.idx.numel() * 4,
+                rows)
+
+    def attn_flops(self):
+        T, Hq, d = self.Q.shape
+        return 4.0 * T * Hq * self.cfg.K_sel * d
+
+
+def time_steps(w, steps, warmup, flush, stream):
+    """Device time of `steps` steps (select + attention), L2 flushed between steps."""
+    for _ in range(warmup):
+        flush.zero_()
+        w.select()
+        w.attend()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        w.select()
+        ev[k][1].record(stream)
+        w.attend()
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    sel = [ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)]
+    att = [ev[k][1].elapsed_time(ev[k][2]) for k in range(steps)]
+    return sel, att
+
+
+def time_e2e(w, steps, flush, stream):
+    """Same step through the public API with pinned host buffers: H2D of the chunk's
+    queries, select + attention, D2H of the outputs, all inside the timed region."""
+    Qh = w.Q.cpu().pin_memory()
+    Oh = torch.empty(w.O.shape, dtype=w.O.dtype).pin_memory()
+    Lh = torch.empty(w.LSE.shape, dtype=torch.float32).pin_memory()
+    Qd = torch.empty_like(w.Q)
+    times = []
+    for k in range(steps + 1):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Qd.copy_(Qh, non_blocking=True)
+        w.select(Qd)
+        w.attend(Qd)
+        Oh.copy_(w.O, non_blocking=True)
+        Lh.copy_(w.LSE, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if k:  # first pass warms the pinned-copy path
+            times.append(a.elapsed_time(b))
+    h2d = Qh.numel() * Qh.element_size()
+    d2h = Oh.numel() * Oh.element_size() + Lh.numel() * 4
+    return times, h2d, d2h
+
+
+def cpu_baseline_prefill(w, n_queries=4096):
+    """The oracle as it stands on this host: select + attention for a sample of the chunk's
+    queries on KV head 0 (of 8), on the index the GPU built (exported to float64)."""
+    from oracle import oracle as orc
+    cfg = w.cfg
+    h = 0
+    tree = orc.Tree.from_levels(cfg.branching, cfg.leaf,
+                                [w.tree.centroids(l)[h].cpu() for l in range(len(cfg.branching))],
+                                [w.tree.min_pos(l)[h].cpu() for l in range(len(cfg.branching))],
+                                w.tree.leaf_index()[h].cpu())
+    Kh = orc._f64(w.K[h].cpu())
+    Vh = orc._f64(w.V[h].cpu())
+    sel = slice(cfg.T - n_queries, cfg.T)
+    Qg = w.Q[sel, h * cfg.G:(h + 1) * cfg.G].cpu()
+    Wh = w.W[h].cpu()
+    qp = w.q_pos[sel].cpu().numpy()
+    t0 = time.perf_counter()
+    qlat = orc.query_latent(Qg, Wh)
+    idx, _, _ = orc.select(qlat, tree, cfg.beam, q_pos=qp)
+    orc.attn_fwd(Qg, Kh, Vh, idx, q_pos=qp, causal=True)
+    dt = time.perf_counter() - t0
+    qps = n_queries / (dt * cfg.Hkv)
+    return {"value": qps, "unit": "queries/s", "cores": cores_used(), "kind": "oracle",
+            "sample": f"{n_queries} of {cfg.T} chunk queries on KV head 0 of {cfg.Hkv} (select + attention, "
+                      f"float64 C oracle, OpenMP), scaled x{cfg.Hkv} heads; index built on the GPU"}
+
+
+def bench_config(args):
+    if args.workload != "prefill_1m":
+        raise SystemExit(f"workload {args.workload} is not wired into the benchmark yet")
+    cfg = configs.get(args.workload)
+    if args.small:
+        cfg = cfg.scaled(name="prefill_1m_geometry_131k", n=131072, branching=(8, 8, 8, 4), comps=1024)
+    return cfg
+
+
+def run_cuda(args, rank, world, local_rank):
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = bench_config(args)
+    seed = rank_seed(cfg.seed, rank)
+    w = Prefill(cfg, dev, seed)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    pg = world > 1
+    if pg:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        sel, att = time_steps(w, args.steps, args.warmup, flush, stream)
+        if pg:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+    code = w.lsa.lsa_status_check(w.status)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code}: {w.lsa.lsa_strerror(code)}")
+    total_s = (sum(sel) + sum(att)) / 1e3
+
+    def reduce_max(x):
+        if not pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    value, t_max = aggregate(total_s, w.units * args.steps, world, reduce_max)
+    e2e_t, h2d, d2h = time_e2e(w, args.steps, flush, stream)
+    e2e_value, _ = aggregate(sum(e2e_t) / 1e3, w.units * args.steps, world, reduce_max)
+    alg_bytes, rows = w.attn_algorithmic_bytes()
+    att_s = statistics.mean(att) / 1e3
+    peaks = measured_peaks()
+    achieved = alg_bytes / att_s / 1e9
+    line = None
+    if rank == 0:
+        clocks = clk.summary()
+        cpu = None if args.no_cpu_baseline else cpu_baseline_prefill(w)
+        line = {
+            "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * t_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{cfg.name}: {cfg.T} query tokens over {cfg.n:,} cached keys, "
+                                   f"{cfg.Hq}/{cfg.Hkv} heads, d={cfg.d}, r={cfg.r}, tree "
+                                   f"{'/'.join(map(str, cfg.branching))} leaf {cfg.leaf}, beam "
+                                   f"{'/'.join(map(str, cfg.beam))} ({cfg.K_sel} keys/query), causal",
+                       "global_batch": cfg.T * world, "seq_len": cfg.n, "parallelism": f"dp{world}",
+                       "l2": "flushed between timed steps (512 MiB write outside the events)"},
+            "breakdown_ms": {"select": statistics.mean(sel), "attention": statistics.mean(att),
+                             "build_once": w.build_ms},
+            "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "roofline": {"kernel": "k_attn_fwd", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": peaks["source"],
+                         "algorithmic_bytes": alg_bytes, "distinct_kv_rows": rows,
+                         "tensor_tflops": w.attn_flops() / att_s / 1e12},
+            "gpu_launches": w.launches_per_step * args.steps,
+            "clocks": clocks,
+            "cpu_baseline": cpu,
+        }
+    return line
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle on this host
+# ---------------------------------------------------------------------------
+
+def run_reference(args):
+    from oracle import oracle as orc
+    cfg = bench_config(args)
+    one = cfg.scaled(Hkv=1, Hq=cfg.G)
+    c = one.case("cpu")
+    t0 = time.perf_counter()
+    Z = orc.project(c.K[0, :cfg.n], c.W[0])
+    tree = orc.build_tree(Z, cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    build_s = time.perf_counter() - t0
+    Kh, Vh = orc._f64(c.K[0]), orc._f64(c.V[0])
+    n_q = 256
+    times = []
+    for k in range(args.warmup + args.steps):
+        sel = slice((k * n_q) % cfg.T, (k * n_q) % cfg.T + n_q)
+        Qg = c.Q[sel]
+        qp = c.q_pos[sel].numpy()
+        t0 = time.perf_counter()
+        qlat = orc.query_latent(Qg, c.W[0])
+        idx, _, _ = orc.select(qlat, tree, cfg.beam, q_pos=qp)
+        orc.attn_fwd(Qg, Kh, Vh, idx, q_pos=qp, causal=True)
+        if k >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    per_q = sum(times) / (len(times) * n_q) * cfg.Hkv
+    value = 1.0 / per_q
+    sample = (f"{n_q} chunk queries per step on one KV head (of {cfg.Hkv}), scaled x{cfg.Hkv}; "
+              f"oracle-built index over {cfg.n:,} keys (build {build_s:.0f} s, untimed)")
+    return {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": cfg.name, "global_batch": n_q, "seq_len": cfg.n, "parallelism": "none"},
+            "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores_used(), "kind": "oracle",
+                             "sample": sample}}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["lsa", "reference"], default="lsa")
+    ap.add_argument("--workload", default="prefill_1m", choices=sorted(configs.CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--small", action="store_true",
+                    help="profiling case: the prefill geometry (4096 queries x 2048 keys) over 131,072 cached "
+                         "keys, tree 8/8/8/4, so a kernel capture stays small")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_cuda(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

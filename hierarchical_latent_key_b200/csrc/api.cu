@@ -190,8 +190,9 @@ int lsa_build_tree(const lsa_tree_desc* tree, void* tree_mem, const void* K, int
   P.seed = seed;
   P.coop_blocks = lsa::da_grid_blocks();
   if (P.coop_blocks <= 0) return fail(LSA_ERR_CUDA, "cannot size the cooperative assignment grid");
-  cudaError_t e = lsa::run_build(P, *tree, tree_mem, K, n_cap, d, dtype, W, trace, status,
-                                 static_cast<cudaStream_t>(stream));
+  cudaError_t e = cudaMemsetAsync(tree_mem, 0, tree->bytes, static_cast<cudaStream_t>(stream));
+  if (e == cudaSuccess)
+    e = lsa::run_build(P, *tree, tree_mem, K, n_cap, d, dtype, W, trace, status, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lsa_build_tree");
   return ok();
 }

@@ -123,7 +123,7 @@ int lsa_build_workspace_bytes(const lsa_tree_desc *tree, int32_t d, size_t *byte
  *             of the last round's assignment.
  *  trace    : optional (NULL) int32 [levels][iters][n_heads][n_tree]: node id of
  *             every key (indexed by position) after each round's assignment.
- *  tree_mem : tree->bytes of device memory, written completely.
+ *  tree_mem : tree->bytes of device memory, written completely (alignment gaps are zeroed).
  * Limits: d in {64, 128}; n_cap >= n_tree.  Writes LSA_ERR_TIMEOUT to *status if
  * an assignment needs more than 4096 proposal rounds (never seen in practice),
  * LSA_ERR_NONFINITE if a distance is NaN. */

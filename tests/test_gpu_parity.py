@@ -24,6 +24,16 @@ def lsa():
     return mod
 
 
+def _check_grad(name, got, want):
+    """Gradient tolerance: the forward thresholds (2e-2 max-abs, 2e-3 mean-abs at |O| ~ 1)
+    applied relative to the reference gradient's own scale (max |ref| and mean |ref|).  The
+    dominant deviation is the bf16 rounding (2^-9 relative) of the stored forward output that
+    enters the row term sum_j P_j dP_j = dO . O, as in any backward that reuses O."""
+    err = np.abs(got - want)
+    assert err.max() <= 2e-2 * np.abs(want).max(), (name, err.max(), np.abs(want).max())
+    assert err.mean() <= 2e-3 * np.abs(want).mean(), (name, err.mean(), np.abs(want).mean())
+
+
 def _tol(dtype):
     return (1e-4, 1e-4) if dtype == "f32" else (2e-2, 2e-3)
 
@@ -119,10 +129,7 @@ def test_train_shape_small_fwd_bwd(lsa):
         oQ, oK, oV = orc.attn_bwd(case.Q[:, sl], case.K[h], case.V[h], idx[h].cpu(), case.dO[:, sl],
                                   q_pos=qp, causal=True)
         for name, got, want in (("dQ", dQ[:, sl], oQ), ("dK", dK[h], oK), ("dV", dV[h], oV)):
-            err = np.abs(got.cpu().numpy() - want)
-            rms = np.sqrt((want ** 2).mean())
-            assert err.max() <= 2e-2 * rms and err.mean() <= 2e-3 * rms, \
-                (h, name, err.max(), err.mean(), rms)
+            _check_grad(name, got.cpu().numpy(), want)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
