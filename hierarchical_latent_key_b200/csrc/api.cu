@@ -50,6 +50,9 @@ int check_desc(const lsa_tree_desc* t) {
 
 namespace lsa {
 
+// Record a message for lsa_last_error() on this thread and return `code`.
+int report_error(int code, const char* msg) { return fail(code, "%s", msg); }
+
 size_t build_workspace_layout(const lsa_tree_desc& t, char* base, BuildPlan* P) {
   const int64_t H = t.n_heads, n = t.n_tree, R = t.r, nslots = H * n;
   int bmax = 0;

@@ -101,6 +101,7 @@ struct AttnArgs {
   float scale;
 };
 int attn_splits(int64_t T, int Hkv, int64_t keys);
+int report_error(int code, const char* msg);
 cudaError_t run_attn_fwd(const AttnArgs& a, int dtype, cudaStream_t st);
 cudaError_t run_attn_bwd(const AttnArgs& a, int dtype, cudaStream_t st);
 

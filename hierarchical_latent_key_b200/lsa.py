@@ -62,6 +62,8 @@ def _load():
                                            f32, P, P, P, sz, P, P]),
         "lsa_sparse_attn_bwd": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, P, P, P, i32, P, i32,
                                                i64, i64, f32, P, P, P, P, P]),
+        "lsa_sparse_attn_noalloc": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i64,
+                                                   i64, f32, P, P, P, P]),
         "lsa_status_clear": (ctypes.c_int, [P, P]),
         "lsa_status_check": (ctypes.c_int, [P, P, ctypes.POINTER(i32)]),
     }
@@ -162,6 +164,17 @@ def lsa_sparse_attn(Q, K, V, idx, q_pos, causal, tail_begin, tail_end, scale, O,
                                 K_sel, _ptr(q_pos), int(bool(causal)), tail_begin, tail_end, float(scale), _ptr(O),
                                 _ptr(LSE), _ptr(workspace), ws_n, _ptr(status), _stream(stream, Q)),
            "lsa_sparse_attn")
+
+
+def lsa_sparse_attn_noalloc(Q, K, V, idx, q_pos, causal, tail_begin, tail_end, scale, O, LSE, status=None,
+                            stream=None):
+    """lsa_sparse_attn without a workspace argument (split partials in the library's built-in array)."""
+    T, Hq, d = Q.shape
+    K_sel = 0 if idx is None else idx.shape[-1]
+    _raise(_lib.lsa_sparse_attn_noalloc(_ptr(Q), T, Hq, _ptr(K), _ptr(V), K.shape[0], K.shape[1], d, _dtype(Q),
+                                        _ptr(idx), K_sel, _ptr(q_pos), int(bool(causal)), tail_begin, tail_end,
+                                        float(scale), _ptr(O), _ptr(LSE), _ptr(status), _stream(stream, Q)),
+           "lsa_sparse_attn_noalloc")
 
 
 def lsa_sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos, causal, tail_begin, tail_end, scale, dQ, dK, dV,

@@ -192,6 +192,33 @@ int lsa_sparse_attn_bwd(const void *Q, int32_t T, int32_t Hq, const void *K, con
                         int64_t tail_end, float scale, float *dQ, float *dK, float *dV,
                         int32_t *status, void *stream);
 
+/* Same computation and arguments as lsa_sparse_attn, for callers that cannot
+ * allocate device memory: a plugin whose host framework passes it only its input
+ * and output buffers, or a decode loop that must not call cudaMalloc (which can
+ * synchronise the whole device) once serving has started.  The pages have no
+ * counterpart of this call; it only changes where the split partials live.
+ *  - Nothing is allocated: when the keys of a query are split over several CTAs
+ *    (few queries, long key lists: decode), the partial results go to a built-in
+ *    device array of LSA_NOALLOC_SCRATCH_BYTES (4 MiB).  Every GPU that loads the
+ *    library holds that array until the process exits.  A call needing more
+ *    (lsa_attn_workspace_bytes reports the need) returns LSA_ERR_WORKSPACE with
+ *    nothing launched.  At d = 128 a call needs at most about G * 0.62 MB (G =
+ *    query heads per KV head), so every call with G <= 4 fits, e.g. any number of
+ *    decode tokens with 32 query heads over 8 KV heads; G = 8 can need up to about
+ *    4.9 MB.  Calls that need no split use no scratch at all.
+ *  - The first call on a device looks up that device's address of the array (once
+ *    per device, with the device current); make that first call before any stream
+ *    capture.
+ *  - All calls share the one array and it keeps the last call's contents; every
+ *    call overwrites the partials it reads, so nothing needs clearing, but calls
+ *    that overlap on the GPU (other streams, other host threads) race on it. */
+#define LSA_NOALLOC_SCRATCH_BYTES (4u << 20)
+int lsa_sparse_attn_noalloc(const void *Q, int32_t T, int32_t Hq, const void *K, const void *V,
+                            int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype,
+                            const int32_t *idx, int32_t K_sel, const int32_t *q_pos, int32_t causal,
+                            int64_t tail_begin, int64_t tail_end, float scale, void *O, float *LSE,
+                            int32_t *status, void *stream);
+
 /* Zero the device status word on `stream`. */
 int lsa_status_clear(int32_t *status, void *stream);
 
