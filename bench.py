@@ -175,6 +175,168 @@ class Prefill:
         return 4.0 * T * Hq * self.cfg.K_sel * d
 
 
+class Decode:
+    """Single-request decode: step s appends one key and one value row per KV head at
+    position n + s, selects for the new token and attends to the selection plus the dense
+    tail of appended rows [n, n + s] (causal by position)."""
+
+    def __init__(self, cfg, dev, seed, steps):
+        from hierarchical_latent_key_b200 import lsa
+        cfg = cfg.scaled(T=steps)
+        self.lsa, self.cfg, self.dev = lsa, cfg, dev
+        c = cfg.case(dev, seed)
+        self.K, self.V, self.W, self.Q, self.q_pos = c.K, c.V, c.W, c.Q, c.q_pos
+        del c
+        n = cfg.n
+        self.Knew = self.K[:, n:].clone()          # rows the steps append, staged apart
+        self.Vnew = self.V[:, n:].clone()
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        self.tree = lsa.build_tree(self.K, self.W, cfg.branching, cfg.leaf, cfg.iters, seed)
+        torch.cuda.synchronize(dev)
+        self.build_ms = 1e3 * (time.perf_counter() - t0)
+        _, Hq, d = self.Q.shape
+        self.idx = torch.empty(cfg.Hkv, 1, cfg.K_sel, dtype=torch.int32, device=dev)
+        self.O = torch.empty(1, Hq, d, dtype=self.Q.dtype, device=dev)
+        self.LSE = torch.empty(1, Hq, dtype=torch.float32, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        need = lsa.lsa_attn_workspace_bytes(1, Hq, cfg.Hkv, d, cfg.K_sel, steps)
+        self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        self.scale = 1.0 / math.sqrt(d)
+        self.launches_per_step = 1 + 1 + (1 if need else 0)
+
+    def append(self, s, K_row=None, V_row=None):
+        p = self.cfg.n + s
+        self.K[:, p].copy_(self.Knew[:, s] if K_row is None else K_row, non_blocking=True)
+        self.V[:, p].copy_(self.Vnew[:, s] if V_row is None else V_row, non_blocking=True)
+
+    def select(self, s, Q=None):
+        self.lsa.lsa_select(self.tree.desc, self.tree.mem, self.Q[s:s + 1] if Q is None else Q, self.W,
+                            self.cfg.beam, self.q_pos[s:s + 1], self.idx, status=self.status)
+
+    def attend(self, s, Q=None):
+        n = self.cfg.n
+        self.lsa.lsa_sparse_attn(self.Q[s:s + 1] if Q is None else Q, self.K, self.V, self.idx,
+                                 self.q_pos[s:s + 1], True, n, n + s + 1, self.scale, self.O, self.LSE, self.ws,
+                                 self.status)
+
+    def bytes_per_step(self, s):
+        """Algorithmic bytes of one step: gathered K/V rows of the selection and the tail,
+        centroid rows scored, projection, query/output, key lists."""
+        cfg, d = self.cfg, self.Q.shape[2]
+        esz = self.Q.element_size()
+        attn = cfg.Hkv * (cfg.K_sel + s + 1) * 2 * d * esz + 2 * cfg.Hq * d * esz + cfg.Hkv * cfg.K_sel * 4
+        cand = cfg.nodes[0] + sum(cfg.beam[l - 1] * cfg.branching[l] for l in range(1, len(cfg.branching)))
+        sel = (cfg.Hkv * cand * (cfg.r * 4 + 4) + cfg.Hkv * d * cfg.r * esz + cfg.Hq * d * esz
+               + 2 * cfg.Hkv * cfg.K_sel * 4)
+        return attn, sel
+
+
+def time_decode(w, steps, warmup, flush, stream):
+    """Per step: events around append, select and attention; L2 flushed between steps."""
+    for s in range(warmup):
+        w.append(s)
+        w.select(s)
+        w.attend(s)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for k in range(steps):
+        s = warmup + k
+        flush.zero_()
+        ev[k][0].record(stream)
+        w.append(s)
+        ev[k][1].record(stream)
+        w.select(s)
+        ev[k][2].record(stream)
+        w.attend(s)
+        ev[k][3].record(stream)
+    torch.cuda.synchronize()
+    app = [ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)]
+    sel = [ev[k][1].elapsed_time(ev[k][2]) for k in range(steps)]
+    att = [ev[k][2].elapsed_time(ev[k][3]) for k in range(steps)]
+    return app, sel, att
+
+
+def time_decode_e2e(w, steps, warmup, flush, stream):
+    """Decode steps through the public API from pinned host buffers: H2D of the token's
+    query and its new key/value rows, append + select + attention, D2H of O and LSE."""
+    first = warmup
+    Qh = w.Q[first:first + steps].cpu().pin_memory()
+    Kh = w.Knew[:, first:first + steps].transpose(0, 1).contiguous().cpu().pin_memory()
+    Vh = w.Vnew[:, first:first + steps].transpose(0, 1).contiguous().cpu().pin_memory()
+    Oh = torch.empty((steps,) + tuple(w.O.shape[1:]), dtype=w.O.dtype).pin_memory()
+    Lh = torch.empty((steps,) + tuple(w.LSE.shape[1:]), dtype=torch.float32).pin_memory()
+    Qd = torch.empty_like(w.Q[:1])
+    Kd = torch.empty_like(Kh[0], device=w.dev)
+    Vd = torch.empty_like(Vh[0], device=w.dev)
+    times = []
+    for k in range(steps):
+        s = first + k
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        Qd.copy_(Qh[k:k + 1], non_blocking=True)
+        Kd.copy_(Kh[k], non_blocking=True)
+        Vd.copy_(Vh[k], non_blocking=True)
+        w.append(s, Kd, Vd)
+        w.select(s, Qd)
+        w.attend(s, Qd)
+        Oh[k].copy_(w.O[0], non_blocking=True)
+        Lh[k].copy_(w.LSE[0], non_blocking=True)
+        b.record(stream)
+        times.append((a, b))
+    torch.cuda.synchronize()
+    t = [a.elapsed_time(b) for a, b in times]
+    h2d = Qh[0].numel() * Qh.element_size() + 2 * Kh[0].numel() * Kh.element_size()
+    d2h = Oh[0].numel() * Oh.element_size() + Lh[0].numel() * 4
+    return t, h2d, d2h
+
+
+def run_decode(args, dev, rank, world, reduce_max):
+    cfg = configs.get("decode_10m")
+    steps, warmup = cfg.T, args.warmup
+    w = Decode(cfg, dev, rank_seed(cfg.seed, rank), warmup + steps)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    torch.cuda.synchronize()
+    app, sel, att = time_decode(w, steps, warmup, flush, stream)
+    code = w.lsa.lsa_status_check(w.status)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code}: {w.lsa.lsa_strerror(code)}")
+    total_s = (sum(app) + sum(sel) + sum(att)) / 1e3
+    value, t_max = aggregate(total_s, steps, world, reduce_max)
+    e2e_t, h2d, d2h = time_decode_e2e(w, steps, warmup, flush, stream)
+    e2e_value, _ = aggregate(sum(e2e_t) / 1e3, steps, world, reduce_max)
+    peaks = measured_peaks()
+    att_b = statistics.mean(w.bytes_per_step(warmup + k)[0] for k in range(steps))
+    sel_b = w.bytes_per_step(0)[1]
+    a_s, s_s = statistics.mean(att) / 1e3, statistics.mean(sel) / 1e3
+    step_s = total_s / steps
+    out = {
+        "value": value, "unit": "queries/s", "steps": steps, "ms_per_step": 1e3 * t_max / steps,
+        "config": {"workload": f"{cfg.name}: single-request decode over {cfg.n:,} indexed keys, {cfg.Hq}/{cfg.Hkv} "
+                               f"heads, d={cfg.d}, r={cfg.r}, tree {'/'.join(map(str, cfg.branching))} leaf "
+                               f"{cfg.leaf}, beam {'/'.join(map(str, cfg.beam))} ({cfg.K_sel} keys) + dense tail "
+                               f"of appended keys", "seq_len": cfg.n,
+                   "l2": "flushed between timed steps (512 MiB write outside the events)"},
+        "breakdown_us": {"append": 1e3 * statistics.mean(app), "select": 1e3 * statistics.mean(sel),
+                         "attention": 1e3 * statistics.mean(att), "build_once_ms": w.build_ms},
+        "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
+                     "step": {"achieved": (att_b + sel_b) / step_s / 1e9,
+                              "frac": (att_b + sel_b) / step_s / 1e9 / peaks["hbm_gbs"],
+                              "algorithmic_bytes": att_b + sel_b},
+                     "k_attn_fwd": {"achieved": att_b / a_s / 1e9, "frac": att_b / a_s / 1e9 / peaks["hbm_gbs"],
+                                    "algorithmic_bytes": att_b},
+                     "k_select": {"achieved": sel_b / s_s / 1e9, "frac": sel_b / s_s / 1e9 / peaks["hbm_gbs"],
+                                  "algorithmic_bytes": sel_b}, "traffic": None},
+        "gpu_launches": w.launches_per_step * steps,
+    }
+    del w
+    torch.cuda.empty_cache()
+    return out
+
+
 def time_steps(w, steps, warmup, flush, stream):
     """Device time of `steps` steps (select + attention), L2 flushed between steps."""
     for _ in range(warmup):
@@ -291,13 +453,23 @@ def run_cuda(args, rank, world, local_rank):
     e2e_t, h2d, d2h = time_e2e(w, args.steps, flush, stream)
     e2e_value, _ = aggregate(sum(e2e_t) / 1e3, w.units * args.steps, world, reduce_max)
     alg_bytes, rows = w.attn_algorithmic_bytes()
+    cpu = cpu_baseline_prefill(w) if (rank == 0 and not args.no_cpu_baseline) else None
+    att_flops = w.attn_flops()
+    build_ms = w.build_ms
     att_s = statistics.mean(att) / 1e3
     peaks = measured_peaks()
     achieved = alg_bytes / att_s / 1e9
+    launches = w.launches_per_step * args.steps
+    decode = None
+    if not args.no_decode and not args.small:
+        del w
+        torch.cuda.empty_cache()
+        with ClockSampler(local_rank) as clk_dec:
+            decode = run_decode(args, dev, rank, world, reduce_max)
+        decode["clocks"] = clk_dec.summary()
     line = None
     if rank == 0:
         clocks = clk.summary()
-        cpu = None if args.no_cpu_baseline else cpu_baseline_prefill(w)
         line = {
             "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * t_max / args.steps, "higher_is_better": True,
@@ -309,16 +481,17 @@ def run_cuda(args, rank, world, local_rank):
                        "global_batch": cfg.T * world, "seq_len": cfg.n, "parallelism": f"dp{world}",
                        "l2": "flushed between timed steps (512 MiB write outside the events)"},
             "breakdown_ms": {"select": statistics.mean(sel), "attention": statistics.mean(att),
-                             "build_once": w.build_ms},
+                             "build_once": build_ms},
             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "roofline": {"kernel": "k_attn_fwd", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                          "peak_source": peaks["source"],
                          "algorithmic_bytes": alg_bytes, "distinct_kv_rows": rows,
-                         "tensor_tflops": w.attn_flops() / att_s / 1e12},
-            "gpu_launches": w.launches_per_step * args.steps,
+                         "tensor_tflops": att_flops / att_s / 1e12},
+            "gpu_launches": launches,
             "clocks": clocks,
             "cpu_baseline": cpu,
+            "decode_10m": decode,
         }
     return line
 
@@ -370,6 +543,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["lsa", "reference"], default="lsa")
     ap.add_argument("--workload", default="prefill_1m", choices=sorted(configs.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the 10M-token decode measurement")
     ap.add_argument("--small", action="store_true",
                     help="profiling case: the prefill geometry (4096 queries x 2048 keys) over 131,072 cached "
                          "keys, tree 8/8/8/4, so a kernel capture stays small")

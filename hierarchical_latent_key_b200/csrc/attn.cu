@@ -8,12 +8,12 @@
 //
 // Work unit: one (query t, KV group g); the G query heads of the group share
 // the key list, so every gathered K/V row serves G heads.  Inside a CTA each
-// warp is split into four 8-lane groups; a group owns one key at a time, each
-// lane holding d/8 consecutive elements of the K and V rows (16-byte loads), so
-// a group reads a row with fully used sectors and the dot products reduce over
-// 8 lanes only.  Every 8-lane group keeps its own online-softmax state (base-2
-// exponent, scale folded into the query); states are merged at the end of the
-// CTA and, when the keys are split over CTAs (decode), by a combine kernel.
+// warp is split into groups of LPK = d/8 lanes; a group owns one key at a time,
+// each lane holding 8 consecutive elements of the K and V rows (16-byte loads for
+// bf16), so a group reads a row with fully used sectors and the dot products
+// reduce over the group only.  Every group keeps its own online-softmax state
+// (base-2 exponent, scale folded into the query); states are merged at the end
+// of the CTA and, when the keys are split over CTAs (decode), by a combine kernel.
 
 #include <cmath>
 
@@ -24,7 +24,6 @@ namespace lsa {
 
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = kAttnWarps * 32;
-constexpr int kKeysPerIter = kAttnWarps * 4;
 constexpr float kLn2 = 0.69314718055994530942f;
 
 template <int N>
@@ -49,10 +48,11 @@ __device__ __forceinline__ void load_row(const __nv_bfloat16* p, float (&v)[N]) 
   }
 }
 
-__device__ __forceinline__ float group8_sum(float v) {
-  v += __shfl_xor_sync(0xffffffffu, v, 4);
-  v += __shfl_xor_sync(0xffffffffu, v, 2);
-  v += __shfl_xor_sync(0xffffffffu, v, 1);
+// Sum over the LPK lanes that share a key (xor offsets stay inside the group).
+template <int LPK>
+__device__ __forceinline__ float group_sum(float v) {
+#pragma unroll
+  for (int o = LPK / 2; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
 }
 
@@ -61,12 +61,35 @@ __device__ __forceinline__ int64_t unit_key(const AttnArgs& a, const int32_t* ix
   return i < a.K_sel ? (int64_t)__ldg(&ix[i]) : a.tail_begin + (i - a.K_sel);
 }
 
-template <typename T, int DK, int G>
+// Fetch K and V slices of the key at virtual position i of the unit (zeros and
+// ok = false when the key is absent, out of range or in the causal future).
+template <typename T, int EPL>
+__device__ __forceinline__ bool fetch_kv(const AttnArgs& a, const int32_t* ix, const T* Kh, const T* Vh,
+                                         int64_t i, int64_t k_end, int64_t qpos, int off,
+                                         float (&kv)[EPL], float (&vv)[EPL]) {
+  const int64_t j = i < k_end ? unit_key(a, ix, i) : -1;
+  const bool ok = j >= 0 && j < a.n_cap && j <= qpos;
+  if (ok) {
+    load_row<EPL>(Kh + j * a.d + off, kv);
+    load_row<EPL>(Vh + j * a.d + off, vv);
+  } else {
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) { kv[e] = 0.f; vv[e] = 0.f; }
+  }
+  return ok;
+}
+
+// LPK lanes own one key at a time (EPL = d / LPK elements each); a warp holds
+// 32 / LPK keys per step, and the next step's rows are loaded before the current
+// ones are used, so two rows per lane group are in flight.
+template <typename T, int DK, int G, int LPK>
 __global__ void __launch_bounds__(kAttnThreads) k_attn_fwd(AttnArgs a) {
-  constexpr int EPL = DK / 8;
+  constexpr int EPL = DK / LPK;
+  constexpr int KPW = 32 / LPK;                 // keys per warp per step
+  constexpr int KPI = KPW * kAttnWarps;         // keys per CTA per step
   __shared__ float s_m[kAttnWarps][G], s_l[kAttnWarps][G];
   __shared__ float s_acc[kAttnWarps][G][DK];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane >> 3, sl = lane & 7;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane / LPK, sl = lane % LPK;
   const int64_t t = blockIdx.x / a.nsplit;
   const int split = blockIdx.x % a.nsplit;
   const int g = blockIdx.y;
@@ -78,11 +101,12 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_fwd(AttnArgs a) {
   const int64_t k_begin = (int64_t)split * a.keys_per_split;
   const int64_t k_end = min64(nkeys, k_begin + a.keys_per_split);
   const int64_t qpos = a.causal ? (int64_t)a.q_pos[t] : INT64_MAX;
+  const int off = sl * EPL;
 
   float q[G][EPL];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
-    load_row<EPL>(Q + (t * a.Hq + (int64_t)g * G + h) * DK + sl * EPL, q[h]);
+    load_row<EPL>(Q + (t * a.Hq + (int64_t)g * G + h) * DK + off, q[h]);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) q[h][e] *= a.scale_log2;
   }
@@ -93,25 +117,19 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_fwd(AttnArgs a) {
 #pragma unroll
     for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
   }
-  for (int64_t base = k_begin + warp * 4; base < k_end; base += kKeysPerIter) {
-    const int64_t i = base + sub;
-    const int64_t j = i < k_end ? unit_key(a, ix, i) : -1;
-    const bool ok = j >= 0 && j < a.n_cap && j <= qpos;
-    float kv[EPL], vv[EPL];
-    if (ok) {
-      load_row<EPL>(Kh + j * DK + sl * EPL, kv);
-      load_row<EPL>(Vh + j * DK + sl * EPL, vv);
-    } else {
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) { kv[e] = 0.f; vv[e] = 0.f; }
-    }
+  int64_t base = k_begin + warp * KPW;
+  float kv[EPL], vv[EPL];
+  bool ok = fetch_kv<T, EPL>(a, ix, Kh, Vh, base + sub, k_end, qpos, off, kv, vv);
+  for (; base < k_end; base += KPI) {
+    float kn[EPL], vn[EPL];
+    const bool okn = fetch_kv<T, EPL>(a, ix, Kh, Vh, base + KPI + sub, k_end, qpos, off, kn, vn);
     float s[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
       float x = 0.f;
 #pragma unroll
       for (int e = 0; e < EPL; ++e) x = fmaf(q[h][e], kv[e], x);
-      s[h] = group8_sum(x);
+      s[h] = group_sum<LPK>(x);
     }
     if (ok) {
 #pragma unroll
@@ -125,28 +143,31 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_fwd(AttnArgs a) {
         m[h] = mn;
       }
     }
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) { kv[e] = kn[e]; vv[e] = vn[e]; }
+    ok = okn;
   }
-  // merge the four 8-lane groups of the warp
+  // merge the key groups of the warp
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     float M = m[h];
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 8));
-    M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, 16));
+#pragma unroll
+    for (int o = LPK; o < 32; o <<= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     const float f = M == -INFINITY ? 0.f : exp2f(m[h] - M);
     float L = l[h] * f;
-    L += __shfl_xor_sync(0xffffffffu, L, 8);
-    L += __shfl_xor_sync(0xffffffffu, L, 16);
+#pragma unroll
+    for (int o = LPK; o < 32; o <<= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
       float v = acc[h][e] * f;
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 16);
+#pragma unroll
+      for (int o = LPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
       acc[h][e] = v;
     }
     if (lane == 0) { s_m[warp][h] = M; s_l[warp][h] = L; }
     if (sub == 0) {
 #pragma unroll
-      for (int e = 0; e < EPL; ++e) s_acc[warp][h][sl * EPL + e] = acc[h][e];
+      for (int e = 0; e < EPL; ++e) s_acc[warp][h][off + e] = acc[h][e];
     }
   }
   __syncthreads();
@@ -202,11 +223,13 @@ __device__ __forceinline__ void red_add4(float* p, float a, float b, float c, fl
   atomicAdd(reinterpret_cast<float4*>(p), make_float4(a, b, c, d));
 }
 
-template <typename T, int DK, int G>
+template <typename T, int DK, int G, int LPK>
 __global__ void __launch_bounds__(kAttnThreads) k_attn_bwd(AttnArgs a) {
-  constexpr int EPL = DK / 8;
+  constexpr int EPL = DK / LPK;
+  constexpr int KPW = 32 / LPK;
+  constexpr int KPI = KPW * kAttnWarps;
   __shared__ float s_dq[kAttnWarps][G][DK];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane >> 3, sl = lane & 7;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, sub = lane / LPK, sl = lane % LPK;
   const int64_t t = blockIdx.x / a.nsplit;
   const int split = blockIdx.x % a.nsplit;
   const int g = blockIdx.y;
@@ -222,36 +245,30 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_bwd(AttnArgs a) {
   const int64_t k_begin = (int64_t)split * a.keys_per_split;
   const int64_t k_end = min64(nkeys, k_begin + a.keys_per_split);
   const int64_t qpos = a.causal ? (int64_t)a.q_pos[t] : INT64_MAX;
+  const int off = sl * EPL;
   constexpr float kLog2e = 1.44269504088896340736f;
 
   float q[G][EPL], go[G][EPL], lse2[G], delta[G], dq[G][EPL];
 #pragma unroll
   for (int h = 0; h < G; ++h) {
     const int64_t row = t * a.Hq + (int64_t)g * G + h;
-    load_row<EPL>(Q + row * DK + sl * EPL, q[h]);
-    load_row<EPL>(dO + row * DK + sl * EPL, go[h]);
+    load_row<EPL>(Q + row * DK + off, q[h]);
+    load_row<EPL>(dO + row * DK + off, go[h]);
     float ov[EPL];
-    load_row<EPL>(O + row * DK + sl * EPL, ov);
+    load_row<EPL>(O + row * DK + off, ov);
     float x = 0.f;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) x = fmaf(go[h][e], ov[e], x);
-    delta[h] = group8_sum(x);
+    delta[h] = group_sum<LPK>(x);
     lse2[h] = a.LSE[row] * kLog2e;
 #pragma unroll
     for (int e = 0; e < EPL; ++e) dq[h][e] = 0.f;
   }
-  for (int64_t base = k_begin + warp * 4; base < k_end; base += kKeysPerIter) {
+  for (int64_t base = k_begin + warp * KPW; base < k_end; base += KPI) {
     const int64_t i = base + sub;
     const int64_t j = i < k_end ? unit_key(a, ix, i) : -1;
-    const bool ok = j >= 0 && j < a.n_cap && j <= qpos;
     float kv[EPL], vv[EPL];
-    if (ok) {
-      load_row<EPL>(Kh + j * DK + sl * EPL, kv);
-      load_row<EPL>(Vh + j * DK + sl * EPL, vv);
-    } else {
-#pragma unroll
-      for (int e = 0; e < EPL; ++e) { kv[e] = 0.f; vv[e] = 0.f; }
-    }
+    const bool ok = fetch_kv<T, EPL>(a, ix, Kh, Vh, i, k_end, qpos, off, kv, vv);
     float p[G], ds[G];
 #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -261,8 +278,8 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_bwd(AttnArgs a) {
         x = fmaf(q[h][e], kv[e], x);
         y = fmaf(go[h][e], vv[e], y);
       }
-      x = group8_sum(x);
-      y = group8_sum(y);
+      x = group_sum<LPK>(x);
+      y = group_sum<LPK>(y);
       p[h] = ok ? exp2f(x * a.scale_log2 - lse2[h]) : 0.f;
       ds[h] = p[h] * (y - delta[h]);
 #pragma unroll
@@ -283,8 +300,8 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_bwd(AttnArgs a) {
           gk[c] = xk * a.scale;
           gv[c] = xv;
         }
-        red_add4(dKh + j * DK + sl * EPL + e, gk[0], gk[1], gk[2], gk[3]);
-        red_add4(dVh + j * DK + sl * EPL + e, gv[0], gv[1], gv[2], gv[3]);
+        red_add4(dKh + j * DK + off + e, gk[0], gk[1], gk[2], gk[3]);
+        red_add4(dVh + j * DK + off + e, gv[0], gv[1], gv[2], gv[3]);
       }
     }
   }
@@ -293,9 +310,9 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_bwd(AttnArgs a) {
 #pragma unroll
     for (int e = 0; e < EPL; ++e) {
       float v = dq[h][e];
-      v += __shfl_xor_sync(0xffffffffu, v, 8);
-      v += __shfl_xor_sync(0xffffffffu, v, 16);
-      if (sub == 0) s_dq[warp][h][sl * EPL + e] = v;
+#pragma unroll
+      for (int o = LPK; o < 32; o <<= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (sub == 0) s_dq[warp][h][off + e] = v;
     }
   __syncthreads();
   for (int x = threadIdx.x; x < G * DK; x += kAttnThreads) {
@@ -324,7 +341,7 @@ static cudaError_t launch_fwd(const AttnArgs& a, cudaStream_t st) {
   dim3 grid((unsigned)(a.T * a.nsplit), (unsigned)a.Hkv);
 #define LSA_FWD(DD, GG)                                                               \
   if (a.d == DD && a.G == GG) {                                                       \
-    k_attn_fwd<T, DD, GG><<<grid, kAttnThreads, 0, st>>>(a);                          \
+    k_attn_fwd<T, DD, GG, DD / 8><<<grid, kAttnThreads, 0, st>>>(a);                  \
     if (a.nsplit > 1) k_attn_combine<T, DD><<<(unsigned)(a.T * a.Hq), DD, 0, st>>>(a); \
     return cudaGetLastError();                                                        \
   }
@@ -339,7 +356,7 @@ static cudaError_t launch_bwd(const AttnArgs& a, cudaStream_t st) {
   dim3 grid((unsigned)(a.T * a.nsplit), (unsigned)a.Hkv);
 #define LSA_BWD(DD, GG)                                            \
   if (a.d == DD && a.G == GG) {                                    \
-    k_attn_bwd<T, DD, GG><<<grid, kAttnThreads, 0, st>>>(a);       \
+    k_attn_bwd<T, DD, GG, DD / 8><<<grid, kAttnThreads, 0, st>>>(a); \
     return cudaGetLastError();                                     \
   }
   LSA_BWD(64, 1) LSA_BWD(64, 2) LSA_BWD(64, 4) LSA_BWD(64, 8)
