@@ -139,35 +139,35 @@ class Prefill:
         torch.cuda.synchronize(dev)
         self.build_ms = 1e3 * (time.perf_counter() - t0)
         T, Hq, d = self.Q.shape
-        self.idx = torch.empty(cfg.Hkv, T, cfg.K_sel, dtype=torch.int32, device=dev)
+        self.leaves = torch.empty(cfg.Hkv, T, cfg.beam[-1], dtype=torch.int32, device=dev)
         self.O = torch.empty_like(self.Q)
         self.LSE = torch.empty(T, Hq, dtype=torch.float32, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        need = lsa.lsa_attn_workspace_bytes(T, Hq, cfg.Hkv, d, cfg.K_sel, 0)
+        need = lsa.lsa_tree_attn_workspace_bytes(self.tree.desc, T, Hq, d, self.Q.dtype, cfg.beam[-1])
         self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
         self.scale = 1.0 / math.sqrt(d)
         self.units = T
-        self.launches_per_step = 1 + 1 + (1 if need else 0)
+        self.launches_per_step = 1 + 7      # select; tree attention: 3 list + 2 tensor-core passes + 2
 
     def select(self, Q=None):
         self.lsa.lsa_select(self.tree.desc, self.tree.mem, self.Q if Q is None else Q, self.W, self.cfg.beam,
-                            self.q_pos, self.idx, status=self.status)
+                            self.q_pos, None, self.leaves, status=self.status)
 
     def attend(self, Q=None, O=None, LSE=None):
-        self.lsa.lsa_sparse_attn(self.Q if Q is None else Q, self.K, self.V, self.idx, self.q_pos, True, 0, 0,
-                                 self.scale, self.O if O is None else O, self.LSE if LSE is None else LSE,
-                                 self.ws, self.status)
+        self.lsa.lsa_tree_attn(self.tree.desc, self.tree.mem, self.Q if Q is None else Q, self.K, self.V,
+                               self.leaves, self.q_pos, True, self.scale, self.O if O is None else O,
+                               self.LSE if LSE is None else LSE, self.ws, self.status)
 
     def attn_algorithmic_bytes(self):
-        """Bytes the attention must move at least: every distinct selected K/V row once,
-        plus queries, outputs, LSE and the index lists."""
+        """Bytes the attention must move at least: the K/V rows of every distinct selected
+        leaf once, plus queries, outputs, LSE and the leaf lists."""
         d = self.Q.shape[2]
         rows = 0
         for g in range(self.cfg.Hkv):
-            v = self.idx[g]
-            rows += int(torch.unique(v[v >= 0]).numel())
+            v = self.leaves[g]
+            rows += int(torch.unique(v[v >= 0]).numel()) * self.cfg.leaf
         esz = self.Q.element_size()
-        return (rows * 2 * d * esz + 2 * self.Q.numel() * esz + self.LSE.numel() * 4 + self.idx.numel() * 4,
+        return (rows * 2 * d * esz + 2 * self.Q.numel() * esz + self.LSE.numel() * 4 + self.leaves.numel() * 4,
                 rows)
 
     def attn_flops(self):
@@ -188,8 +188,8 @@ class Decode:
         self.K, self.V, self.W, self.Q, self.q_pos = c.K, c.V, c.W, c.Q, c.q_pos
         del c
         n = cfg.n
-        self.Knew = self.K[:, n:].clone()          # rows the steps append, staged apart
-        self.Vnew = self.V[:, n:].clone()
+        self.Knew = self.K[:, n:].transpose(0, 1).contiguous()   # [steps, Hkv, d]: rows the steps append
+        self.Vnew = self.V[:, n:].transpose(0, 1).contiguous()
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
         self.tree = lsa.build_tree(self.K, self.W, cfg.branching, cfg.leaf, cfg.iters, seed)
@@ -203,12 +203,26 @@ class Decode:
         need = lsa.lsa_attn_workspace_bytes(1, Hq, cfg.Hkv, d, cfg.K_sel, steps)
         self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
         self.scale = 1.0 / math.sqrt(d)
-        self.launches_per_step = 1 + 1 + (1 if need else 0)
+        self.launches_per_step = 1 + 1 + 1 + (1 if need else 0)
 
-    def append(self, s, K_row=None, V_row=None):
-        p = self.cfg.n + s
-        self.K[:, p].copy_(self.Knew[:, s] if K_row is None else K_row, non_blocking=True)
-        self.V[:, p].copy_(self.Vnew[:, s] if V_row is None else V_row, non_blocking=True)
+    def append(self, s):
+        self.lsa.lsa_kv_append(self.K, self.V, self.cfg.n + s, self.Knew[s], self.Vnew[s])
+
+    def step(self, s):
+        self.append(s)
+        self.select(s)
+        self.attend(s)
+
+    def capture(self, steps):
+        """One CUDA graph per decode step (append, select, attention): a step is then
+        one launch, so host launch latency does not separate its kernels."""
+        self.graphs = []
+        for s in range(steps):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                self.step(s)
+            self.graphs.append(g)
+        torch.cuda.synchronize()
 
     def select(self, s, Q=None):
         self.lsa.lsa_select(self.tree.desc, self.tree.mem, self.Q[s:s + 1] if Q is None else Q, self.W,
@@ -233,54 +247,58 @@ class Decode:
 
 
 def time_decode(w, steps, warmup, flush, stream):
-    """Per step: events around append, select and attention; L2 flushed between steps."""
+    """Per step: one graph replay (append + select + attention), L2 flushed between
+    steps; a second pass with events between the kernels gives the breakdown."""
     for s in range(warmup):
-        w.append(s)
-        w.select(s)
-        w.attend(s)
+        w.graphs[s].replay()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
     for k in range(steps):
-        s = warmup + k
         flush.zero_()
         ev[k][0].record(stream)
-        w.append(s)
+        w.graphs[warmup + k].replay()
         ev[k][1].record(stream)
-        w.select(s)
-        ev[k][2].record(stream)
-        w.attend(s)
-        ev[k][3].record(stream)
     torch.cuda.synchronize()
-    app = [ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)]
-    sel = [ev[k][1].elapsed_time(ev[k][2]) for k in range(steps)]
-    att = [ev[k][2].elapsed_time(ev[k][3]) for k in range(steps)]
-    return app, sel, att
+    total = [ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)]
+    # breakdown (eager launches, host gaps included): append / select / attention
+    parts = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(8)]
+    for k in range(8):
+        s = warmup + k
+        flush.zero_()
+        torch.cuda.synchronize()
+        parts[k][0].record(stream)
+        w.append(s)
+        parts[k][1].record(stream)
+        w.select(s)
+        parts[k][2].record(stream)
+        w.attend(s)
+        parts[k][3].record(stream)
+    torch.cuda.synchronize()
+    br = {name: statistics.median(parts[k][i].elapsed_time(parts[k][i + 1]) for k in range(8)) * 1e3
+          for i, name in enumerate(("append", "select", "attention"))}
+    return total, br
 
 
 def time_decode_e2e(w, steps, warmup, flush, stream):
     """Decode steps through the public API from pinned host buffers: H2D of the token's
-    query and its new key/value rows, append + select + attention, D2H of O and LSE."""
+    query and its new key/value rows into the step's input slots, the step's graph
+    (append + select + attention), D2H of O and LSE."""
     first = warmup
     Qh = w.Q[first:first + steps].cpu().pin_memory()
-    Kh = w.Knew[:, first:first + steps].transpose(0, 1).contiguous().cpu().pin_memory()
-    Vh = w.Vnew[:, first:first + steps].transpose(0, 1).contiguous().cpu().pin_memory()
+    Kh = w.Knew[first:first + steps].cpu().pin_memory()
+    Vh = w.Vnew[first:first + steps].cpu().pin_memory()
     Oh = torch.empty((steps,) + tuple(w.O.shape[1:]), dtype=w.O.dtype).pin_memory()
     Lh = torch.empty((steps,) + tuple(w.LSE.shape[1:]), dtype=torch.float32).pin_memory()
-    Qd = torch.empty_like(w.Q[:1])
-    Kd = torch.empty_like(Kh[0], device=w.dev)
-    Vd = torch.empty_like(Vh[0], device=w.dev)
     times = []
     for k in range(steps):
         s = first + k
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        Qd.copy_(Qh[k:k + 1], non_blocking=True)
-        Kd.copy_(Kh[k], non_blocking=True)
-        Vd.copy_(Vh[k], non_blocking=True)
-        w.append(s, Kd, Vd)
-        w.select(s, Qd)
-        w.attend(s, Qd)
+        w.Q[s:s + 1].copy_(Qh[k:k + 1], non_blocking=True)
+        w.Knew[s].copy_(Kh[k], non_blocking=True)
+        w.Vnew[s].copy_(Vh[k], non_blocking=True)
+        w.graphs[s].replay()
         Oh[k].copy_(w.O[0], non_blocking=True)
         Lh[k].copy_(w.LSE[0], non_blocking=True)
         b.record(stream)
@@ -292,25 +310,108 @@ def time_decode_e2e(w, steps, warmup, flush, stream):
     return t, h2d, d2h
 
 
+class Train:
+    """Training-shaped layer at 128k: every step rebuilds the index from the step's keys,
+    selects for all 131072 causal queries, runs the tree attention forward and the
+    backward (dQ, dK, dV) for that selection."""
+
+    def __init__(self, cfg, dev, seed):
+        from hierarchical_latent_key_b200 import lsa
+        self.lsa, self.cfg, self.dev = lsa, cfg, dev
+        c = cfg.case(dev, seed)
+        self.K, self.V, self.W, self.Q, self.q_pos, self.dO = c.K, c.V, c.W, c.Q, c.q_pos, c.dO
+        del c
+        T, Hq, d = self.Q.shape
+        self.desc = lsa.lsa_tree_describe(cfg.Hkv, cfg.r, cfg.branching, cfg.leaf)
+        self.tree_mem = torch.empty(self.desc.bytes, dtype=torch.uint8, device=dev)
+        self.build_ws = torch.empty(lsa.lsa_build_workspace_bytes(self.desc, d), dtype=torch.uint8, device=dev)
+        self.idx = torch.empty(cfg.Hkv, T, cfg.K_sel, dtype=torch.int32, device=dev)
+        self.leaves = torch.empty(cfg.Hkv, T, cfg.beam[-1], dtype=torch.int32, device=dev)
+        self.O = torch.empty_like(self.Q)
+        self.LSE = torch.empty(T, Hq, dtype=torch.float32, device=dev)
+        self.dQ = torch.empty(T, Hq, d, dtype=torch.float32, device=dev)
+        self.dK = torch.empty(self.K.shape, dtype=torch.float32, device=dev)
+        self.dV = torch.empty(self.V.shape, dtype=torch.float32, device=dev)
+        need = lsa.lsa_tree_attn_workspace_bytes(self.desc, T, Hq, d, self.Q.dtype, cfg.beam[-1])
+        self.attn_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+        self.scale = 1.0 / math.sqrt(d)
+        self.seed = seed
+
+    def phases(self):
+        L, c = self.lsa, self.cfg
+        return (
+            ("build", lambda: L.lsa_build_tree(self.desc, self.tree_mem, self.K, self.W, c.iters, self.seed,
+                                              self.build_ws, None, self.status)),
+            ("select", lambda: L.lsa_select(self.desc, self.tree_mem, self.Q, self.W, c.beam, self.q_pos, self.idx,
+                                            self.leaves, status=self.status)),
+            ("forward", lambda: L.lsa_tree_attn(self.desc, self.tree_mem, self.Q, self.K, self.V, self.leaves,
+                                                self.q_pos, True, self.scale, self.O, self.LSE, self.attn_ws,
+                                                self.status)),
+            ("backward", lambda: L.lsa_sparse_attn_bwd(self.Q, self.K, self.V, self.O, self.LSE, self.dO,
+                                                       self.idx, self.q_pos, True, 0, 0, self.scale, self.dQ,
+                                                       self.dK, self.dV, self.status)),
+        )
+
+
+def run_train(args, dev, rank, world, reduce_max, steps=3, warmup=2):
+    cfg = configs.get("train_128k")
+    w = Train(cfg, dev, rank_seed(cfg.seed, rank))
+    stream = torch.cuda.current_stream(dev)
+    ph = w.phases()
+    for _ in range(warmup):
+        for _, f in ph:
+            f()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(ph) + 1)] for _ in range(steps)]
+    for k in range(steps):
+        ev[k][0].record(stream)
+        for i, (_, f) in enumerate(ph):
+            f()
+            ev[k][i + 1].record(stream)
+    torch.cuda.synchronize()
+    code = w.lsa.lsa_status_check(w.status)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code}: {w.lsa.lsa_strerror(code)}")
+    total_s = sum(ev[k][0].elapsed_time(ev[k][-1]) for k in range(steps)) / 1e3
+    value, t_max = aggregate(total_s, cfg.T * steps, world, reduce_max)
+    br = {name: statistics.mean(ev[k][i].elapsed_time(ev[k][i + 1]) for k in range(steps))
+          for i, (name, _) in enumerate(ph)}
+    flops_fwd = 4.0 * cfg.T * cfg.Hq * cfg.K_sel * cfg.d
+    out = {"value": value, "unit": "tokens/s (index build + select + attention forward + backward)",
+           "steps": steps, "warmup": warmup, "ms_per_step": 1e3 * t_max / steps,
+           "config": {"workload": f"{cfg.name}: causal layer over {cfg.T:,} tokens, {cfg.Hq}/{cfg.Hkv} heads, "
+                                  f"d={cfg.d}, r={cfg.r}, tree {'/'.join(map(str, cfg.branching))} leaf {cfg.leaf}, "
+                                  f"beam {'/'.join(map(str, cfg.beam))} ({cfg.K_sel} keys/query), index rebuilt "
+                                  f"every step", "seq_len": cfg.T},
+           "breakdown_ms": br,
+           "forward_tflops": flops_fwd / (br["forward"] / 1e3) / 1e12,
+           "backward_tflops": 2.5 * flops_fwd / (br["backward"] / 1e3) / 1e12,
+           "gpu_launches_per_step": None}
+    del w
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_decode(args, dev, rank, world, reduce_max):
     cfg = configs.get("decode_10m")
     steps, warmup = cfg.T, args.warmup
     w = Decode(cfg, dev, rank_seed(cfg.seed, rank), warmup + steps)
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-    torch.cuda.synchronize()
-    app, sel, att = time_decode(w, steps, warmup, flush, stream)
+    w.capture(warmup + steps)
+    total, br = time_decode(w, steps, warmup, flush, stream)
     code = w.lsa.lsa_status_check(w.status)
     if code != 0:
         raise RuntimeError(f"kernel status {code}: {w.lsa.lsa_strerror(code)}")
-    total_s = (sum(app) + sum(sel) + sum(att)) / 1e3
+    total_s = sum(total) / 1e3
     value, t_max = aggregate(total_s, steps, world, reduce_max)
     e2e_t, h2d, d2h = time_decode_e2e(w, steps, warmup, flush, stream)
     e2e_value, _ = aggregate(sum(e2e_t) / 1e3, steps, world, reduce_max)
     peaks = measured_peaks()
     att_b = statistics.mean(w.bytes_per_step(warmup + k)[0] for k in range(steps))
     sel_b = w.bytes_per_step(0)[1]
-    a_s, s_s = statistics.mean(att) / 1e3, statistics.mean(sel) / 1e3
+    a_s, s_s = br["attention"] / 1e6, br["select"] / 1e6
     step_s = total_s / steps
     out = {
         "value": value, "unit": "queries/s", "steps": steps, "ms_per_step": 1e3 * t_max / steps,
@@ -319,8 +420,9 @@ def run_decode(args, dev, rank, world, reduce_max):
                                f"{cfg.leaf}, beam {'/'.join(map(str, cfg.beam))} ({cfg.K_sel} keys) + dense tail "
                                f"of appended keys", "seq_len": cfg.n,
                    "l2": "flushed between timed steps (512 MiB write outside the events)"},
-        "breakdown_us": {"append": 1e3 * statistics.mean(app), "select": 1e3 * statistics.mean(sel),
-                         "attention": 1e3 * statistics.mean(att), "build_once_ms": w.build_ms},
+        "breakdown_us": {"step_graph": 1e3 * statistics.mean(total), "eager_append": br["append"],
+                         "eager_select": br["select"], "eager_attention": br["attention"],
+                         "build_once_ms": w.build_ms},
         "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
                      "step": {"achieved": (att_b + sel_b) / step_s / 1e9,
@@ -331,7 +433,9 @@ def run_decode(args, dev, rank, world, reduce_max):
                      "k_select": {"achieved": sel_b / s_s / 1e9, "frac": sel_b / s_s / 1e9 / peaks["hbm_gbs"],
                                   "algorithmic_bytes": sel_b}, "traffic": None},
         "gpu_launches": w.launches_per_step * steps,
+        "cuda_graph": "one graph per decode step (append, select, attention)",
     }
+    w.graphs = None
     del w
     torch.cuda.empty_cache()
     return out
@@ -460,13 +564,24 @@ def run_cuda(args, rank, world, local_rank):
     peaks = measured_peaks()
     achieved = alg_bytes / att_s / 1e9
     launches = w.launches_per_step * args.steps
-    decode = None
+    decode = train = None
+    del w
+    torch.cuda.empty_cache()
+    # secondary workloads: a failure is reported in the line instead of losing the headline
     if not args.no_decode and not args.small:
-        del w
+        try:
+            with ClockSampler(local_rank) as clk_dec:
+                decode = run_decode(args, dev, rank, world, reduce_max)
+            decode["clocks"] = clk_dec.summary()
+        except Exception as e:  # noqa: BLE001
+            decode = {"error": f"{type(e).__name__}: {e}"}
         torch.cuda.empty_cache()
-        with ClockSampler(local_rank) as clk_dec:
-            decode = run_decode(args, dev, rank, world, reduce_max)
-        decode["clocks"] = clk_dec.summary()
+    if not args.no_train and not args.small:
+        try:
+            train = run_train(args, dev, rank, world, reduce_max)
+        except Exception as e:  # noqa: BLE001
+            train = {"error": f"{type(e).__name__}: {e}"}
+        torch.cuda.empty_cache()
     line = None
     if rank == 0:
         clocks = clk.summary()
@@ -483,7 +598,7 @@ def run_cuda(args, rank, world, local_rank):
             "breakdown_ms": {"select": statistics.mean(sel), "attention": statistics.mean(att),
                              "build_once": build_ms},
             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "roofline": {"kernel": "k_attn_fwd", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+            "roofline": {"kernel": "lsa_tree_attn (k_tl_stats + k_tl_out + list/finish kernels)", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                          "peak_source": peaks["source"],
                          "algorithmic_bytes": alg_bytes, "distinct_kv_rows": rows,
@@ -492,6 +607,7 @@ def run_cuda(args, rank, world, local_rank):
             "clocks": clocks,
             "cpu_baseline": cpu,
             "decode_10m": decode,
+            "train_128k": train,
         }
     return line
 
@@ -544,6 +660,7 @@ def main(argv=None):
     ap.add_argument("--workload", default="prefill_1m", choices=sorted(configs.CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true", help="skip the 10M-token decode measurement")
+    ap.add_argument("--no-train", action="store_true", help="skip the training-shaped 128k layer step")
     ap.add_argument("--small", action="store_true",
                     help="profiling case: the prefill geometry (4096 queries x 2048 keys) over 131,072 cached "
                          "keys, tree 8/8/8/4, so a kernel capture stays small")

@@ -202,7 +202,7 @@ int lsa_build_tree(const lsa_tree_desc* tree, void* tree_mem, const void* K, int
 
 int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq, int32_t d,
                int32_t dtype, const void* W, const int32_t* beam, const int32_t* q_pos, int32_t* idx_out,
-               float* qlat_out, int32_t* beam_out, int32_t* status, void* stream) {
+               int32_t* leaves_out, float* qlat_out, int32_t* beam_out, int32_t* status, void* stream) {
   int rc = check_desc(tree);
   if (rc != LSA_OK) return rc;
   if (!beam) return fail(LSA_ERR_INVALID_ARG, "beam must be non-NULL");
@@ -226,8 +226,10 @@ int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, i
     a.off_m[l] = tree->off_min_pos[l];
   }
   if (T == 0) return ok();
-  if (!tree_mem || !Q || !W || !idx_out) return fail(LSA_ERR_INVALID_ARG, "tree_mem, Q, W and idx_out must be non-NULL");
+  if (!tree_mem || !Q || !W) return fail(LSA_ERR_INVALID_ARG, "tree_mem, Q and W must be non-NULL");
+  if (!idx_out && !leaves_out) return fail(LSA_ERR_INVALID_ARG, "give idx_out, leaves_out or both");
   a.Q = Q; a.W = W; a.tree = static_cast<const char*>(tree_mem); a.q_pos = q_pos; a.idx_out = idx_out;
+  a.leaves_out = leaves_out;
   a.qlat_out = qlat_out; a.beam_out = beam_out; a.status = status;
   a.T = T; a.Hq = Hq; a.Hkv = tree->n_heads; a.G = Hq / tree->n_heads; a.d = d; a.r = tree->r;
   a.levels = tree->levels; a.leaf = tree->leaf_size; a.beam_max = beam_max; a.n_tree = tree->n_tree;
@@ -308,6 +310,53 @@ int lsa_sparse_attn(const void* Q, int32_t T, int32_t Hq, const void* K, const v
   return ok();
 }
 
+int lsa_tree_attn_workspace_bytes(const lsa_tree_desc* tree, int32_t T, int32_t Hq, int32_t d, int32_t dtype,
+                                  int32_t n_leaves, size_t* bytes) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
+  if (T < 0 || Hq < tree->n_heads || Hq % tree->n_heads || n_leaves < 1 || n_leaves > LSA_MAX_BEAM ||
+      (d != 64 && d != 128))
+    return fail(LSA_ERR_SHAPE, "bad sizes");
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  const int G = Hq / tree->n_heads;
+  const bool fast = lsa::tree_attn_fast_path(dtype, d, G, tree->leaf_size);
+  *bytes = lsa::tree_attn_workspace(tree->n_heads, tree->nodes[tree->levels - 1], T, Hq, d, n_leaves,
+                                    tree->leaf_size, fast);
+  return ok();
+}
+
+int lsa_tree_attn(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
+                  const void* K, const void* V, int64_t n_cap, int32_t d, int32_t dtype, const int32_t* leaves,
+                  int32_t n_leaves, const int32_t* q_pos, int32_t causal, float scale, void* O, float* LSE,
+                  void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  size_t need = 0;
+  int rc = lsa_tree_attn_workspace_bytes(tree, T, Hq, d, dtype, n_leaves, &need);
+  if (rc != LSA_OK) return rc;
+  const int G = Hq / tree->n_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(LSA_ERR_SHAPE, "query heads per group must be 1, 2, 4 or 8");
+  if (n_cap < tree->n_tree) return fail(LSA_ERR_SHAPE, "n_cap (%lld) < n_tree", (long long)n_cap);
+  if (!std::isfinite(scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite");
+  if (T == 0) return ok();
+  if (!tree_mem || !Q || !K || !V || !leaves || !O || !LSE)
+    return fail(LSA_ERR_INVALID_ARG, "tree_mem, Q, K, V, leaves, O and LSE must be non-NULL");
+  if (causal && !q_pos) return fail(LSA_ERR_INVALID_ARG, "q_pos is required when causal");
+  if (!workspace || workspace_bytes < need)
+    return fail(LSA_ERR_WORKSPACE, "tree attention needs %zu workspace bytes (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  lsa::TreeAttnCall c;
+  memset(&c, 0, sizeof(c));
+  c.Q = Q; c.K = K; c.V = V;
+  c.leaf_index = reinterpret_cast<const int32_t*>(static_cast<const char*>(tree_mem) + tree->off_leaf_index);
+  c.leaves = leaves; c.q_pos = q_pos; c.O = O; c.LSE = LSE; c.workspace = workspace; c.status = status;
+  c.T = T; c.n_cap = n_cap; c.n_tree = tree->n_tree; c.NL = tree->nodes[tree->levels - 1];
+  c.Hq = Hq; c.H = tree->n_heads; c.d = d; c.dtype = dtype; c.B = n_leaves; c.leaf = tree->leaf_size;
+  c.causal = causal ? 1 : 0; c.scale = scale;
+  cudaError_t e = lsa::run_tree_attn(c, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_tree_attn");
+  return ok();
+}
+
 int lsa_sparse_attn_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, const void* V, int32_t n_heads,
                         int64_t n_cap, int32_t d, int32_t dtype, const void* O, const float* LSE, const void* dO,
                         const int32_t* idx, int32_t K_sel, const int32_t* q_pos, int32_t causal, int64_t tail_begin,
@@ -336,6 +385,19 @@ int lsa_sparse_attn_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, con
     return cuda_fail(e, "lsa_sparse_attn_bwd");
   e = lsa::run_attn_bwd(a, dtype, st);
   if (e != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_bwd");
+  return ok();
+}
+
+int lsa_kv_append(void* K, void* V, int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, int64_t pos,
+                  const void* K_rows, const void* V_rows, void* stream) {
+  if (!K || !V || !K_rows || !V_rows) return fail(LSA_ERR_INVALID_ARG, "K, V, K_rows and V_rows must be non-NULL");
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (n_heads < 1 || (d != 64 && d != 128)) return fail(LSA_ERR_SHAPE, "need n_heads >= 1 and d in {64, 128}");
+  if (pos < 0 || pos >= n_cap) return fail(LSA_ERR_SHAPE, "pos %lld outside [0, n_cap)", (long long)pos);
+  const int64_t row_bytes = (int64_t)d * (dtype == LSA_BF16 ? 2 : 4);
+  cudaError_t e = lsa::run_kv_append(K, V, n_heads, n_cap, row_bytes, pos, K_rows, V_rows,
+                                     static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_kv_append");
   return ok();
 }
 

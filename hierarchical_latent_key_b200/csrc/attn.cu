@@ -327,6 +327,28 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_bwd(AttnArgs a) {
   }
 }
 
+// one 16-byte chunk per thread: rows of every head for K, then for V
+__global__ void k_kv_append(char* K, char* V, int64_t n_cap, int64_t row_bytes, int64_t pos, const char* Kr,
+                            const char* Vr, int64_t n_heads) {
+  const int64_t chunks = row_bytes / 16;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 2 * n_heads * chunks) return;
+  const int64_t which = i / (n_heads * chunks), rem = i % (n_heads * chunks);
+  const int64_t h = rem / chunks, c = rem % chunks;
+  char* dst = (which ? V : K) + (h * n_cap + pos) * row_bytes + c * 16;
+  const char* src = (which ? Vr : Kr) + h * row_bytes + c * 16;
+  *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+}
+
+cudaError_t run_kv_append(void* K, void* V, int64_t n_heads, int64_t n_cap, int64_t row_bytes, int64_t pos,
+                          const void* Kr, const void* Vr, cudaStream_t st) {
+  const int64_t n = 2 * n_heads * (row_bytes / 16);
+  k_kv_append<<<(unsigned)ceil_div(n, 256), 256, 0, st>>>(static_cast<char*>(K), static_cast<char*>(V), n_cap,
+                                                          row_bytes, pos, static_cast<const char*>(Kr),
+                                                          static_cast<const char*>(Vr), n_heads);
+  return cudaGetLastError();
+}
+
 int attn_splits(int64_t T, int Hkv, int64_t keys) {
   const int64_t units = T * Hkv;
   const int64_t target = 4 * 148;

@@ -66,6 +66,7 @@ struct SelectArgs {
   const char* tree;
   const int32_t* q_pos;
   int32_t* idx_out;
+  int32_t* leaves_out;
   float* qlat_out;
   int32_t* beam_out;
   int32_t* status;
@@ -100,8 +101,28 @@ struct AttnArgs {
   float scale_log2;   // scale * log2(e)
   float scale;
 };
+struct TreeAttnCall {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int32_t* leaf_index;
+  const int32_t* leaves;
+  const int32_t* q_pos;
+  void* O;
+  float* LSE;
+  void* workspace;
+  int32_t* status;
+  int64_t T, n_cap, n_tree, NL;
+  int32_t Hq, H, d, dtype, B, leaf, causal;
+  float scale;
+};
+size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast);
+bool tree_attn_fast_path(int dtype, int d, int G, int leaf);
+cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st);
 int attn_splits(int64_t T, int Hkv, int64_t keys);
 int report_error(int code, const char* msg);
+cudaError_t run_kv_append(void* K, void* V, int64_t n_heads, int64_t n_cap, int64_t row_bytes, int64_t pos,
+                          const void* Kr, const void* Vr, cudaStream_t st);
 cudaError_t run_attn_fwd(const AttnArgs& a, int dtype, cudaStream_t st);
 cudaError_t run_attn_bwd(const AttnArgs& a, int dtype, cudaStream_t st);
 

@@ -1,0 +1,594 @@
+// tree_attn.cu -- sparse attention over tree-structured selections, leaf by leaf.
+//
+// Method (kongchang.com, "Latent Sparse Attention Breaks Through the
+// Million-Token Context Bottleneck", sections "How LSA Sidesteps Per-Key
+// Scoring with Hierarchical Clustering" and "The Accuracy-Efficiency Dilemma";
+// bdtechtalks.com, "Latent sparse attention", section "How latent sparse
+// attention works"): each query attends to the original keys of the leaves its
+// walk kept.  The result equals lsa_sparse_attn on the expanded key lists.
+//
+// Schedule: instead of gathering every query's 2048 keys (each selected leaf is
+// re-read by every query that chose it), work is grouped by leaf: one CTA loads a
+// leaf's 64 K and V rows once and serves every (query, head) row that selected
+// it, with the products on the 5th-generation tensor cores (tcgen05.mma, bf16
+// operands in 128B-swizzled shared memory, fp32 accumulators in tensor memory).
+//   pass A: S = Q_rows . K_leaf^T -> per row, max and sum of exp over the leaf
+//   combine: per (query, head) the softmax denominator over all its leaves
+//   pass B: S again, P = exp(S - LSE) (bf16), O_rows += P . V_leaf (fp32 red-adds)
+// Rows of one CTA chunk: up to 128 (query, head) pairs of queries that chose the
+// leaf.  Shapes served here: bf16, d = 128, leaf size 64, G in {1, 2, 4, 8};
+// other shapes expand the leaves into key lists and use the generic kernels.
+#include <cstring>
+
+#include "lsa_common.cuh"
+#include "lsa_internal.h"
+
+namespace lsa {
+
+namespace {
+
+constexpr int kTL = 128;            // threads per CTA (one TMEM lane / row each)
+constexpr int kLeafKeys = 64;
+constexpr int kDim = 128;
+constexpr uint64_t kWaitNs = 1000000000ull;   // bounded wait on MMA completion (1 s)
+
+// ---- tcgen05 / shared-memory descriptor helpers (PTX ISA: tcgen05) ----------
+
+// Instruction descriptor, kind::f16: D fp32, A and B bf16, shapes M x N.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn_major ? 1u : 0u) << 15) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Shared-memory matrix descriptor for the 128-byte swizzled canonical layout
+// (atoms of 8 rows x 128 B at 1024-B aligned addresses).
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;   // descriptor version for sm_100
+  d |= (uint64_t)2 << 61;   // SWIZZLE_128B
+  return d;
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// Byte offset of 16-byte chunk c (0..15) of row r in a [rows x 128 bf16] tile
+// stored as two 64-element halves, each [rows x 128 B] with 8-row atoms.
+__device__ __forceinline__ uint32_t sw128_off(int r, int c, int half_bytes) {
+  return (uint32_t)((c >> 3) * half_bytes + (r >> 3) * 1024 + (r & 7) * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %6, %7, %8}, p;\n}\n" ::"r"(tmem_d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc), "r"(0u), "r"(0u), "r"(0u), "r"(0u));
+}
+__device__ __forceinline__ void tc_commit(uint32_t mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar)
+               : "memory");
+}
+
+__device__ __forceinline__ uint64_t now_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Wait for phase `parity` of an mbarrier, giving up after kWaitNs.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+  const uint64_t t0 = now_ns();
+  while (true) {
+    uint32_t done;
+    asm volatile(
+        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(mbar), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if (now_ns() - t0 > kWaitNs) return false;
+  }
+}
+
+// 32 consecutive fp32 columns of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      "tcgen05.wait::ld.sync.aligned;\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
+  atomicAdd(reinterpret_cast<float4*>(p), make_float4(a, b, c, d));
+}
+
+struct TreeAttnArgs {
+  const __nv_bfloat16* Q;
+  const __nv_bfloat16* K;
+  const __nv_bfloat16* V;
+  const int32_t* leaf_index;   // [H][n_tree]
+  const int32_t* leaves;       // [H][T][B]
+  const int32_t* q_pos;
+  int32_t* cnt;                // [H][NL]
+  int32_t* off;                // [H][NL + 1]
+  int32_t* ent;                // [H][T * B] (query << 6 | rank), grouped by leaf
+  float2* stats;               // [T][Hq][B] (max, sum) in base 2
+  float* lse2;                 // [T][Hq]
+  float* oacc;                 // [T][Hq][d]
+  __nv_bfloat16* O;
+  float* LSE;
+  int32_t* status;
+  int64_t T, n_cap, n_tree, NL;
+  int32_t Hq, H, G, B, causal;
+  float scale_log2;
+};
+
+// ---- leaf lists (counting sort of (query, rank) by leaf) ---------------------
+
+__global__ void k_tl_count(TreeAttnArgs a) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)a.H * a.T * a.B) return;
+  const int64_t g = i / (a.T * a.B);
+  const int32_t leaf = a.leaves[i];
+  if (leaf >= 0 && leaf < a.NL) atomicAdd(&a.cnt[g * a.NL + leaf], 1);
+}
+
+__global__ void __launch_bounds__(1024) k_tl_scan(TreeAttnArgs a) {
+  __shared__ int32_t s_warp[32];
+  const int64_t g = blockIdx.x;
+  int32_t* c = a.cnt + g * a.NL;
+  int32_t* o = a.off + g * (a.NL + 1);
+  const int64_t per = ceil_div(a.NL, 1024);
+  const int64_t lo = threadIdx.x * per, hi = min64(a.NL, lo + per);
+  int32_t s = 0;
+  for (int64_t i = lo; i < hi; ++i) s += c[i];
+  // block exclusive scan of the per-thread sums
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t inc = s;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    int32_t y = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += y;
+  }
+  if (lane == 31) s_warp[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = s_warp[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int32_t y = __shfl_up_sync(0xffffffffu, w, d);
+      if (lane >= d) w += y;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  int32_t run = inc - s + (warp ? s_warp[warp - 1] : 0);
+  for (int64_t i = lo; i < hi; ++i) {
+    o[i] = run;
+    run += c[i];
+    c[i] = 0;  // becomes the fill cursor
+  }
+  if (threadIdx.x == 1023) o[a.NL] = run;
+}
+
+__global__ void k_tl_fill(TreeAttnArgs a) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)a.H * a.T * a.B) return;
+  const int64_t g = i / (a.T * a.B), rem = i % (a.T * a.B);
+  const int64_t t = rem / a.B, k = rem % a.B;
+  const int32_t leaf = a.leaves[i];
+  if (leaf < 0 || leaf >= a.NL) return;
+  const int32_t pos = a.off[g * (a.NL + 1) + leaf] + atomicAdd(&a.cnt[g * a.NL + leaf], 1);
+  a.ent[g * a.T * a.B + pos] = (int32_t)((t << 6) | k);
+}
+
+// ---- shared pieces of the two passes ----------------------------------------
+
+struct LeafSmem {
+  uint32_t sA, sK, sV, sP;       // shared addresses (1024-B aligned)
+  int32_t* pos;                  // [64] key positions of the leaf
+  uint32_t mbar;
+  uint32_t* taddr_slot;
+};
+
+// Load the leaf's K (and V) rows into the swizzled tiles; positions to smem.
+__device__ __forceinline__ void load_leaf(const TreeAttnArgs& a, int64_t g, int64_t leaf, const LeafSmem& s,
+                                          bool with_v) {
+  const int t = threadIdx.x;
+  if (t < kLeafKeys) s.pos[t] = a.leaf_index[g * a.n_tree + leaf * kLeafKeys + t];
+  __syncthreads();
+  const __nv_bfloat16* Kh = a.K + g * a.n_cap * kDim;
+  const __nv_bfloat16* Vh = a.V + g * a.n_cap * kDim;
+  // 64 rows x 16 chunks; thread t takes row t / 2, chunks (t % 2) * 8 .. + 8
+  const int r = t >> 1, c0 = (t & 1) * 8;
+  const int64_t j = s.pos[r];
+#pragma unroll
+  for (int c = c0; c < c0 + 8; ++c) {
+    cp_async16(s.sK + sw128_off(r, c, kLeafKeys * 128), Kh + j * kDim + c * 8);
+    if (with_v) cp_async16(s.sV + sw128_off(r, c, kLeafKeys * 128), Vh + j * kDim + c * 8);
+  }
+}
+
+// Load up to 128 (query, head) rows of a chunk into the A tile; returns this
+// thread's row: query index (or -1) and rank.
+__device__ __forceinline__ void load_rows(const TreeAttnArgs& a, int64_t g, const int32_t* ent, int64_t n_ent,
+                                          int64_t e0, const LeafSmem& s, int64_t& tq, int& rank, int& h) {
+  const int t = threadIdx.x;
+  const int64_t e = e0 + t / a.G;
+  h = t % a.G;
+  tq = -1;
+  rank = 0;
+  if (e < n_ent) {
+    const int32_t v = ent[e];
+    tq = v >> 6;
+    rank = v & 63;
+    const __nv_bfloat16* q = a.Q + (tq * a.Hq + g * a.G + h) * kDim;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) cp_async16(s.sA + sw128_off(t, c, kTL * 128), q + c * 8);
+  }
+}
+
+// S[128 rows x 64 keys] = A . K_leaf^T into TMEM columns [col, col + 64).
+__device__ __forceinline__ void issue_qk(const LeafSmem& s, uint32_t tmem, int col) {
+  constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
+#pragma unroll
+  for (int kk = 0; kk < 8; ++kk) {
+    const uint32_t koff = (uint32_t)((kk & 3) * 32);
+    const uint64_t da = sdesc_sw128(s.sA + (kk >> 2) * (kTL * 128) + koff, 16, 1024);
+    const uint64_t db = sdesc_sw128(s.sK + (kk >> 2) * (kLeafKeys * 128) + koff, 16, 1024);
+    tc_mma(tmem + col, da, db, idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// This thread's 64 scores (base-2 scaled, causally masked) from TMEM.
+__device__ __forceinline__ void read_scores(const TreeAttnArgs& a, const LeafSmem& s, uint32_t tmem, int64_t tq,
+                                            float (&sc)[64]) {
+  const int warp = threadIdx.x >> 5;
+  float v[32];
+  const int64_t qp = (a.causal && tq >= 0) ? (int64_t)a.q_pos[tq] : INT64_MAX;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + half * 32, v);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+      const int key = half * 32 + i;
+      sc[key] = (int64_t)s.pos[key] <= qp ? v[i] * a.scale_log2 : -INFINITY;
+    }
+  }
+}
+
+__device__ __forceinline__ void alloc_tmem(uint32_t* slot, uint32_t ncols) {
+  if ((threadIdx.x >> 5) == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
+                 "r"(ncols));
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+  }
+}
+__device__ __forceinline__ void free_tmem(uint32_t taddr, uint32_t ncols) {
+  if ((threadIdx.x >> 5) == 0)
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols));
+}
+
+__device__ __forceinline__ char* align1024(char* p) {
+  return reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// ---- pass A: per-row max and exp-sum over each selected leaf -----------------
+
+__global__ void __launch_bounds__(kTL) k_tl_stats(TreeAttnArgs a) {
+  extern __shared__ char smem_raw[];
+  __shared__ int32_t s_pos[kLeafKeys];
+  __shared__ __align__(8) uint64_t s_mbar;
+  __shared__ uint32_t s_taddr;
+  const int64_t g = blockIdx.y, leaf = blockIdx.x;
+  const int32_t* offg = a.off + g * (a.NL + 1);
+  const int64_t e_lo = offg[leaf], n_ent = offg[leaf + 1] - e_lo;
+  if (n_ent == 0) return;
+  const int32_t* ent = a.ent + g * a.T * a.B + e_lo;
+  char* base = align1024(smem_raw);
+  LeafSmem s;
+  s.sA = smem_u32(base);
+  s.sK = s.sA + kTL * 256;
+  s.sV = 0;
+  s.sP = 0;
+  s.pos = s_pos;
+  s.mbar = smem_u32(&s_mbar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
+    asm volatile("fence.mbarrier_init.release.cluster;");
+  }
+  alloc_tmem(&s_taddr, 64);
+  load_leaf(a, g, leaf, s, false);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_taddr;
+  uint32_t phase = 0;
+  bool ok = true;
+  for (int64_t e0 = 0; e0 < n_ent && ok; e0 += kTL / a.G) {
+    int64_t tq;
+    int rank, h;
+    load_rows(a, g, ent, n_ent, e0, s, tq, rank, h);
+    cp_async_wait_all();
+    fence_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue_qk(s, tmem, 0);
+      tc_commit(s.mbar);
+    }
+    ok = __syncthreads_and(mbar_wait(s.mbar, phase));
+    phase ^= 1;
+    tc_fence_after();
+    if (ok) {
+      float sc[64];
+      read_scores(a, s, tmem, tq, sc);
+      if (tq >= 0) {
+        float m = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) m = fmaxf(m, sc[i]);
+        float l = 0.f;
+        if (m != -INFINITY) {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) l += exp2f(sc[i] - m);
+        }
+        a.stats[(tq * a.Hq + g * a.G + h) * a.B + rank] = make_float2(m, l);
+      }
+    } else {
+      set_status(a.status, LSA_ERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  free_tmem(tmem, 64);
+}
+
+// ---- combine: softmax denominator of every (query, head) over its leaves -----
+
+__global__ void k_tl_lse(TreeAttnArgs a) {
+  const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // t * Hq + head
+  if (row >= a.T * a.Hq) return;
+  const int64_t t = row / a.Hq, head = row % a.Hq, g = head / a.G;
+  const int32_t* lv = a.leaves + (g * a.T + t) * a.B;
+  const float2* st = a.stats + row * a.B;
+  float M = -INFINITY;
+  for (int k = 0; k < a.B; ++k)
+    if (lv[k] >= 0) M = fmaxf(M, st[k].x);
+  float L = 0.f;
+  if (M != -INFINITY)
+    for (int k = 0; k < a.B; ++k)
+      if (lv[k] >= 0 && st[k].y > 0.f) L += st[k].y * exp2f(st[k].x - M);
+  a.lse2[row] = L > 0.f ? M + log2f(L) : INFINITY;   // +inf: no visible key, P = 0
+  a.LSE[row] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+}
+
+// ---- pass B: O_rows += softmax(S) . V_leaf ------------------------------------
+
+__global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
+  extern __shared__ char smem_raw[];
+  __shared__ int32_t s_pos[kLeafKeys];
+  __shared__ __align__(8) uint64_t s_mbar;
+  __shared__ uint32_t s_taddr;
+  const int64_t g = blockIdx.y, leaf = blockIdx.x;
+  const int32_t* offg = a.off + g * (a.NL + 1);
+  const int64_t e_lo = offg[leaf], n_ent = offg[leaf + 1] - e_lo;
+  if (n_ent == 0) return;
+  const int32_t* ent = a.ent + g * a.T * a.B + e_lo;
+  char* base = align1024(smem_raw);
+  LeafSmem s;
+  s.sA = smem_u32(base);                       // 32 KB: rows x d
+  s.sK = s.sA + kTL * 256;                     // 16 KB
+  s.sV = s.sK + kLeafKeys * 256;               // 16 KB
+  s.sP = s.sV + kLeafKeys * 256;               // 16 KB: rows x 64 keys
+  s.pos = s_pos;
+  s.mbar = smem_u32(&s_mbar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
+    asm volatile("fence.mbarrier_init.release.cluster;");
+  }
+  alloc_tmem(&s_taddr, 256);
+  load_leaf(a, g, leaf, s, true);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_taddr;
+  const int warp = threadIdx.x >> 5;
+  uint32_t phase = 0;
+  bool ok = true;
+  char* sP_gen = base + (s.sP - s.sA);
+  for (int64_t e0 = 0; e0 < n_ent && ok; e0 += kTL / a.G) {
+    int64_t tq;
+    int rank, h;
+    load_rows(a, g, ent, n_ent, e0, s, tq, rank, h);
+    cp_async_wait_all();
+    fence_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue_qk(s, tmem, 0);
+      tc_commit(s.mbar);
+    }
+    ok = __syncthreads_and(mbar_wait(s.mbar, phase));
+    phase ^= 1;
+    tc_fence_after();
+    if (ok) {
+      float sc[64];
+      read_scores(a, s, tmem, tq, sc);
+      const float lse = tq >= 0 ? a.lse2[tq * a.Hq + g * a.G + h] : INFINITY;
+      // P row (bf16) into the K-major A tile of the second product
+      const int r = threadIdx.x;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float p0 = exp2f(sc[c * 8 + 2 * q] - lse), p1 = exp2f(sc[c * 8 + 2 * q + 1] - lse);
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          w[q] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        *reinterpret_cast<uint4*>(sP_gen + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (ok && threadIdx.x == 0) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t da = sdesc_sw128(s.sP + kk * 32, 16, 1024);
+        const uint64_t db = sdesc_sw128(s.sV + kk * 2048, kLeafKeys * 128, 1024);
+        tc_mma(tmem + 64, da, db, idesc, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(s.mbar);
+    }
+    if (ok) {
+      ok = __syncthreads_and(mbar_wait(s.mbar, phase));
+      phase ^= 1;
+    }
+    tc_fence_after();
+    if (ok) {
+      // every lane takes part in the (warp-collective) TMEM loads; only rows of
+      // real queries are added to the output
+      float* dst = tq >= 0 ? a.oacc + (tq * a.Hq + g * a.G + h) * kDim : nullptr;
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 64 + part * 32, v);
+        if (dst) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) red_add_v4(dst + part * 32 + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+      }
+    } else {
+      set_status(a.status, LSA_ERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  free_tmem(tmem, 256);
+}
+
+__global__ void k_tl_finish(TreeAttnArgs a) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= a.T * a.Hq * (kDim / 4)) return;
+  const float4 v = reinterpret_cast<const float4*>(a.oacc)[i];
+  __nv_bfloat162 lo = __floats2bfloat162_rn(v.x, v.y), hi = __floats2bfloat162_rn(v.z, v.w);
+  uint2 w;
+  w.x = *reinterpret_cast<uint32_t*>(&lo);
+  w.y = *reinterpret_cast<uint32_t*>(&hi);
+  reinterpret_cast<uint2*>(a.O)[i] = w;
+}
+
+// expand leaves into key lists (fallback shapes)
+__global__ void k_tl_expand(const int32_t* leaves, const int32_t* leaf_index, int64_t H, int64_t T, int B, int leaf,
+                            int64_t n_tree, int32_t* idx) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int64_t K_sel = (int64_t)B * leaf;
+  if (i >= H * T * K_sel) return;
+  const int64_t g = i / (T * K_sel), rem = i % (T * K_sel), t = rem / K_sel, k = rem % K_sel;
+  const int32_t lf = leaves[(g * T + t) * B + k / leaf];
+  idx[i] = lf >= 0 ? leaf_index[g * n_tree + (int64_t)lf * leaf + k % leaf] : -1;
+}
+
+constexpr size_t kStatsSmem = 1024 + kTL * 256 + kLeafKeys * 256;
+constexpr size_t kOutSmem = 1024 + kTL * 256 + 3 * kLeafKeys * 256;
+
+}  // namespace
+
+size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  if (!fast) return al((size_t)H * T * B * leaf * 4);
+  return al(H * NL * 4) + al(H * (NL + 1) * 4) + al((size_t)H * T * B * 4) + al((size_t)T * Hq * B * 8) +
+         al((size_t)T * Hq * 4) + al((size_t)T * Hq * d * 4);
+}
+
+bool tree_attn_fast_path(int dtype, int d, int G, int leaf) {
+  return dtype == LSA_BF16 && d == kDim && leaf == kLeafKeys && (G == 1 || G == 2 || G == 4 || G == 8);
+}
+
+cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
+  if (c.T == 0) return cudaSuccess;
+  const int G = c.Hq / c.H;
+  const bool fast = tree_attn_fast_path(c.dtype, c.d, G, c.leaf);
+  char* ws = static_cast<char*>(c.workspace);
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  cudaError_t e;
+  if (!fast) {
+    int32_t* idx = reinterpret_cast<int32_t*>(ws);
+    const int64_t total = (int64_t)c.H * c.T * c.B * c.leaf;
+    k_tl_expand<<<(unsigned)ceil_div(total, 256), 256, 0, st>>>(c.leaves, c.leaf_index, c.H, c.T, c.B, c.leaf,
+                                                                c.n_tree, idx);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.Q = c.Q; a.K = c.K; a.V = c.V; a.idx = idx; a.q_pos = c.q_pos; a.O = c.O; a.LSE = c.LSE;
+    a.status = c.status; a.T = c.T; a.n_cap = c.n_cap; a.Hq = c.Hq; a.Hkv = c.H; a.G = G; a.d = c.d;
+    a.K_sel = c.B * c.leaf; a.causal = c.causal; a.nsplit = 1;
+    a.keys_per_split = (int32_t)((a.K_sel + 15) / 16 * 16);
+    a.scale = c.scale; a.scale_log2 = c.scale * 1.44269504088896340736f;
+    return run_attn_fwd(a, c.dtype, st);   // one CTA per (query, group): needs no split workspace
+  }
+  TreeAttnArgs a;
+  a.Q = static_cast<const __nv_bfloat16*>(c.Q);
+  a.K = static_cast<const __nv_bfloat16*>(c.K);
+  a.V = static_cast<const __nv_bfloat16*>(c.V);
+  a.leaf_index = c.leaf_index;
+  a.leaves = c.leaves;
+  a.q_pos = c.q_pos;
+  size_t o = 0;
+  a.cnt = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.NL * 4);
+  a.off = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * (c.NL + 1) * 4);
+  a.ent = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * c.B * 4);
+  a.stats = reinterpret_cast<float2*>(ws + o); o += al((size_t)c.T * c.Hq * c.B * 8);
+  a.lse2 = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);
+  a.oacc = reinterpret_cast<float*>(ws + o);
+  a.O = static_cast<__nv_bfloat16*>(c.O);
+  a.LSE = c.LSE;
+  a.status = c.status;
+  a.T = c.T; a.n_cap = c.n_cap; a.n_tree = c.n_tree; a.NL = c.NL;
+  a.Hq = c.Hq; a.H = c.H; a.G = G; a.B = c.B; a.causal = c.causal;
+  a.scale_log2 = c.scale * 1.44269504088896340736f;
+  const int64_t n_sel = (int64_t)c.H * c.T * c.B;
+  if ((e = cudaMemsetAsync(a.cnt, 0, (size_t)c.H * c.NL * 4, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(a.oacc, 0, (size_t)c.T * c.Hq * kDim * 4, st)) != cudaSuccess) return e;
+  k_tl_count<<<(unsigned)ceil_div(n_sel, 256), 256, 0, st>>>(a);
+  k_tl_scan<<<(unsigned)c.H, 1024, 0, st>>>(a);
+  k_tl_fill<<<(unsigned)ceil_div(n_sel, 256), 256, 0, st>>>(a);
+  cudaFuncSetAttribute(k_tl_stats, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStatsSmem);
+  cudaFuncSetAttribute(k_tl_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOutSmem);
+  dim3 grid((unsigned)c.NL, (unsigned)c.H);
+  k_tl_stats<<<grid, kTL, kStatsSmem, st>>>(a);
+  k_tl_lse<<<(unsigned)ceil_div(c.T * c.Hq, 256), 256, 0, st>>>(a);
+  k_tl_out<<<grid, kTL, kOutSmem, st>>>(a);
+  k_tl_finish<<<(unsigned)ceil_div(c.T * c.Hq * (kDim / 4), 256), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace lsa

@@ -56,7 +56,10 @@ def _load():
         "lsa_tree_describe": (ctypes.c_int, [i32, i32, P, i32, i32, D]),
         "lsa_build_workspace_bytes": (ctypes.c_int, [D, i32, ctypes.POINTER(sz)]),
         "lsa_build_tree": (ctypes.c_int, [D, P, P, i64, i32, i32, P, i32, u64, P, sz, P, P, P]),
-        "lsa_select": (ctypes.c_int, [D, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, P]),
+        "lsa_select": (ctypes.c_int, [D, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]),
+        "lsa_tree_attn_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
+        "lsa_tree_attn": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, i32, P, i32, f32, P, P, P, sz,
+                                         P, P]),
         "lsa_attn_workspace_bytes": (ctypes.c_int, [i32, i32, i32, i32, i32, i64, ctypes.POINTER(sz)]),
         "lsa_sparse_attn": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i64, i64,
                                            f32, P, P, P, sz, P, P]),
@@ -64,6 +67,7 @@ def _load():
                                                i64, i64, f32, P, P, P, P, P]),
         "lsa_sparse_attn_noalloc": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i64,
                                                    i64, f32, P, P, P, P]),
+        "lsa_kv_append": (ctypes.c_int, [P, P, i32, i64, i32, i32, i64, P, P, P]),
         "lsa_status_clear": (ctypes.c_int, [P, P]),
         "lsa_status_check": (ctypes.c_int, [P, P, ctypes.POINTER(i32)]),
     }
@@ -138,14 +142,32 @@ def lsa_build_tree(desc, tree_mem, K, W, iters, seed, workspace, trace=None, sta
                                _ptr(trace), _ptr(status), _stream(stream, K)), "lsa_build_tree")
 
 
-def lsa_select(desc, tree_mem, Q, W, beam, q_pos, idx_out, qlat_out=None, beam_out=None, status=None,
-               stream=None):
+def lsa_select(desc, tree_mem, Q, W, beam, q_pos, idx_out, leaves_out=None, qlat_out=None, beam_out=None,
+               status=None, stream=None):
     """Q: [T, Hq, d]; beam: host sequence of ints; q_pos: int32 [T] or None."""
     bm = (ctypes.c_int32 * max(MAX_LEVELS, len(beam)))(*beam)
     T, Hq, d = Q.shape
     _raise(_lib.lsa_select(ctypes.byref(desc), _ptr(tree_mem), _ptr(Q), T, Hq, d, _dtype(Q), _ptr(W),
-                           ctypes.cast(bm, ctypes.c_void_p), _ptr(q_pos), _ptr(idx_out), _ptr(qlat_out),
-                           _ptr(beam_out), _ptr(status), _stream(stream, Q)), "lsa_select")
+                           ctypes.cast(bm, ctypes.c_void_p), _ptr(q_pos), _ptr(idx_out), _ptr(leaves_out),
+                           _ptr(qlat_out), _ptr(beam_out), _ptr(status), _stream(stream, Q)), "lsa_select")
+
+
+def lsa_tree_attn_workspace_bytes(desc, T, Hq, d, dtype, n_leaves) -> int:
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_tree_attn_workspace_bytes(ctypes.byref(desc), T, Hq, d, _DTYPE[dtype], n_leaves,
+                                              ctypes.byref(n)), "lsa_tree_attn_workspace_bytes")
+    return int(n.value)
+
+
+def lsa_tree_attn(desc, tree_mem, Q, K, V, leaves, q_pos, causal, scale, O, LSE, workspace, status=None,
+                  stream=None):
+    """leaves: int32 [n_heads, T, n_leaves] (kept leaf ids, -1 = none)."""
+    T, Hq, d = Q.shape
+    ws_n = workspace.numel() * workspace.element_size()
+    _raise(_lib.lsa_tree_attn(ctypes.byref(desc), _ptr(tree_mem), _ptr(Q), T, Hq, _ptr(K), _ptr(V), K.shape[1], d,
+                              _dtype(Q), _ptr(leaves), leaves.shape[-1], _ptr(q_pos), int(bool(causal)),
+                              float(scale), _ptr(O), _ptr(LSE), _ptr(workspace), ws_n, _ptr(status),
+                              _stream(stream, Q)), "lsa_tree_attn")
 
 
 def lsa_attn_workspace_bytes(T, Hq, n_heads, d, K_sel, tail_len) -> int:
@@ -185,6 +207,12 @@ def lsa_sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos, causal, tail_begin, tai
                                     _ptr(O), _ptr(LSE), _ptr(dO), _ptr(idx), K_sel, _ptr(q_pos),
                                     int(bool(causal)), tail_begin, tail_end, float(scale), _ptr(dQ), _ptr(dK),
                                     _ptr(dV), _ptr(status), _stream(stream, Q)), "lsa_sparse_attn_bwd")
+
+
+def lsa_kv_append(K, V, pos, K_rows, V_rows, stream=None):
+    """K, V: [n_heads, n_cap, d] caches; K_rows, V_rows: [n_heads, d] rows written at `pos`."""
+    _raise(_lib.lsa_kv_append(_ptr(K), _ptr(V), K.shape[0], K.shape[1], K.shape[2], _dtype(K), int(pos),
+                              _ptr(K_rows), _ptr(V_rows), _stream(stream, K)), "lsa_kv_append")
 
 
 def lsa_status_clear(status, stream=None):
@@ -258,18 +286,22 @@ def build_tree(K, W, branching, leaf_size, iters, seed, trace=False, workspace=N
     return (tree, tr) if trace else tree
 
 
-def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, status=None, check=True):
+def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, leaves=False, status=None, check=True):
+    """Returns idx (and, when asked, leaves, query latents, per-level beams, in that order)."""
     T = Q.shape[0]
     d = tree.desc
     K_sel = beam[-1] * d.leaf_size
     idx = torch.empty(d.n_heads, T, K_sel, dtype=torch.int32, device=Q.device)
+    lv = torch.empty(d.n_heads, T, beam[-1], dtype=torch.int32, device=Q.device) if leaves else None
     ql = torch.empty(T, d.n_heads, d.r, dtype=torch.float32, device=Q.device) if qlat else None
     bo = torch.empty(d.levels, d.n_heads, T, max(beam), dtype=torch.int32, device=Q.device) if beams else None
     st = _new_status(Q.device) if status is None else status
-    lsa_select(d, tree.mem, Q, W, beam, q_pos, idx, ql, bo, st)
+    lsa_select(d, tree.mem, Q, W, beam, q_pos, idx, lv, ql, bo, st)
     if check:
         check_status(st, "lsa_select")
     out = [idx]
+    if leaves:
+        out.append(lv)
     if qlat:
         out.append(ql)
     if beams:
@@ -291,6 +323,22 @@ def sparse_attn(Q, K, V, idx, q_pos=None, causal=False, tail=(0, 0), scale=None,
     lsa_sparse_attn(Q, K, V, idx, q_pos, causal, tail[0], tail[1], scale, O, LSE, workspace if need else None, st)
     if check:
         check_status(st, "lsa_sparse_attn")
+    return O, LSE
+
+
+def tree_attn(tree: Tree, Q, K, V, leaves, q_pos=None, causal=False, scale=None, workspace=None, status=None,
+              check=True):
+    T, Hq, d = Q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = lsa_tree_attn_workspace_bytes(tree.desc, T, Hq, d, Q.dtype, leaves.shape[-1])
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    O = torch.empty_like(Q)
+    LSE = torch.empty(T, Hq, dtype=torch.float32, device=Q.device)
+    st = _new_status(Q.device) if status is None else status
+    lsa_tree_attn(tree.desc, tree.mem, Q, K, V, leaves, q_pos, causal, scale, O, LSE, workspace, st)
+    if check:
+        check_status(st, "lsa_tree_attn")
     return O, LSE
 
 

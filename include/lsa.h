@@ -48,7 +48,7 @@ extern "C" {
 #define LSA_VERSION 1
 #define LSA_MAX_LEVELS 8
 #define LSA_MAX_BRANCHING 16
-#define LSA_MAX_BEAM 64
+#define LSA_MAX_BEAM 32
 
 typedef enum lsa_status {
   LSA_OK = 0,
@@ -139,24 +139,27 @@ int lsa_build_tree(const lsa_tree_desc *tree, void *tree_mem, const void *K, int
  *            h / G and the G heads of a group share one selection.
  *  W       : the [n_heads][d][r] projection the tree was built with.
  *  beam    : host int32[levels]; beam[0] <= nodes[0], beam[l] <= beam[l-1]*b_l,
- *            every beam[l] in [1, 64].
+ *            every beam[l] in [1, 32].
  *  q_pos   : NULL (non-causal) or device int32[T] query positions; a node is a
  *            candidate only if its min_pos <= q_pos.
  * Per (group g, query t): q = (mean of the group's G query rows) . W[g] (fp32);
  * level-0 candidates are all top nodes, level-l candidates the children of the
  * nodes kept at level l-1; score = <q, centroid> (fp32); keep the beam[l] best by
  * (score desc, node id asc).
- *  idx_out : [n_heads][T][beam[levels-1] * leaf_size] int32 key positions of the
- *            kept leaves, leaf by leaf in rank order, ascending inside a leaf,
- *            -1 where fewer leaves were eligible.
+ *  idx_out : optional [n_heads][T][beam[levels-1] * leaf_size] int32 key positions
+ *            of the kept leaves, leaf by leaf in rank order, ascending inside a
+ *            leaf, -1 where fewer leaves were eligible.
+ *  leaves_out: optional [n_heads][T][beam[levels-1]] int32 kept leaf ids in rank
+ *            order, -1 padded (the input of lsa_tree_attn).  At least one of
+ *            idx_out and leaves_out must be given.
  *  qlat_out: optional [T][n_heads][r] float query latents.
  *  beam_out: optional [levels][n_heads][T][max beam] int32 kept node ids per level
  *            in rank order, -1 padded.
  * Writes LSA_ERR_NONFINITE to *status if a score is NaN. */
 int lsa_select(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, int32_t T,
                int32_t Hq, int32_t d, int32_t dtype, const void *W, const int32_t *beam,
-               const int32_t *q_pos, int32_t *idx_out, float *qlat_out, int32_t *beam_out,
-               int32_t *status, void *stream);
+               const int32_t *q_pos, int32_t *idx_out, int32_t *leaves_out, float *qlat_out,
+               int32_t *beam_out, int32_t *status, void *stream);
 
 /* Host only.  Workspace bytes lsa_sparse_attn needs for these sizes (0 when the
  * call runs without key splitting). */
@@ -179,6 +182,26 @@ int lsa_sparse_attn(const void *Q, int32_t T, int32_t Hq, const void *K, const v
                     int32_t K_sel, const int32_t *q_pos, int32_t causal, int64_t tail_begin,
                     int64_t tail_end, float scale, void *O, float *LSE, void *workspace,
                     size_t workspace_bytes, int32_t *status, void *stream);
+
+/* Host only.  Workspace bytes lsa_tree_attn needs. */
+int lsa_tree_attn_workspace_bytes(const lsa_tree_desc *tree, int32_t T, int32_t Hq, int32_t d,
+                                  int32_t dtype, int32_t n_leaves, size_t *bytes);
+
+/* Sparse attention over tree-structured selections (the same sources as
+ * lsa_sparse_attn): query t of group g attends to the keys of the leaves
+ * leaves[g][t][0..n_leaves) (-1 = none) of the index built by lsa_build_tree,
+ * i.e. exactly lsa_sparse_attn with the expanded key lists and no tail.
+ * Computed leaf by leaf: every selected leaf's K/V rows are read once per pass
+ * and shared by all (query, head) rows that chose the leaf, with the products on
+ * the tensor cores (bf16, d = 128, leaf size 64; other shapes run the generic
+ * kernels on the expanded lists).  Outputs as lsa_sparse_attn.  The summation
+ * order over leaves is not fixed (fp32 atomic adds), so results may differ from
+ * run to run in the last bits.  n_leaves in [1, 32]. */
+int lsa_tree_attn(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, int32_t T,
+                  int32_t Hq, const void *K, const void *V, int64_t n_cap, int32_t d,
+                  int32_t dtype, const int32_t *leaves, int32_t n_leaves, const int32_t *q_pos,
+                  int32_t causal, float scale, void *O, float *LSE, void *workspace,
+                  size_t workspace_bytes, int32_t *status, void *stream);
 
 /* Backward of lsa_sparse_attn for a fixed selection (same arguments), given the
  * forward's O and LSE and the upstream gradient dO ([T][Hq][d], dtype of Q).
@@ -218,6 +241,13 @@ int lsa_sparse_attn_noalloc(const void *Q, int32_t T, int32_t Hq, const void *K,
                             const int32_t *idx, int32_t K_sel, const int32_t *q_pos, int32_t causal,
                             int64_t tail_begin, int64_t tail_end, float scale, void *O, float *LSE,
                             int32_t *status, void *stream);
+
+/* Decode append (bdtechtalks.com, "How latent sparse attention works": the
+ * recent tokens join the attended keys): write the new key row and value row of
+ * every KV head at position `pos` of the caches K, V [n_heads][n_cap][d].
+ * K_rows, V_rows: [n_heads][d] in the caches' dtype.  One kernel launch. */
+int lsa_kv_append(void *K, void *V, int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype,
+                  int64_t pos, const void *K_rows, const void *V_rows, void *stream);
 
 /* Zero the device status word on `stream`. */
 int lsa_status_clear(int32_t *status, void *stream);

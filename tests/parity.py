@@ -32,9 +32,11 @@ def _eps_stable(D, a, Zs, mu, rel=STABLE_EPS_REL):
     return not block.any()
 
 
-def check_build_stagewise(Z, trace, branching, leaf, iters, seed, max_segments=None, rng=None):
+def check_build_stagewise(Z, trace, branching, leaf, iters, seed, max_segments=None, rng=None, check=None):
     """Z: [n, r] float64 latents of one head (oracle projection); trace: [L, iters, n]
-    GPU node ids by position.  Returns (rounds that differed, keys that differed)."""
+    GPU node ids by position; check(level, round, segment_size) -> bool selects which
+    rounds are recomputed (all by default).  Returns (rounds that differed, keys that
+    differed)."""
     Z = np.asarray(Z, np.float64)
     trace = np.asarray(trace)
     n = Z.shape[0]
@@ -56,6 +58,8 @@ def check_build_stagewise(Z, trace, branching, leaf, iters, seed, max_segments=N
             pos = order[s]
             Zs = Z[pos]
             for t in range(iters):
+                if check is not None and not check(l, t, m):
+                    continue
                 if t == 0:
                     mu = orc.level_init(Zs, pos, b, seed, l)
                 else:

@@ -89,15 +89,15 @@ def test_calls_validate_before_launch(lsa):
     d = lsa.lsa_tree_describe(1, 16, (16, 16), 16)
     bm = (ctypes.c_int32 * 8)(4, 65)
     rc = L.lsa_select(ctypes.byref(d), None, None, 4, 1, 64, 0, None, ctypes.cast(bm, ctypes.c_void_p),
-                      None, None, None, None, None, None)
+                      None, None, None, None, None, None, None)
     assert rc == lsa.LSA_ERR_SHAPE and b"beam[1]" in L.lsa_last_error()
     bm = (ctypes.c_int32 * 8)(4, 8)
     rc = L.lsa_select(ctypes.byref(d), None, None, 4, 1, 64, 0, None, ctypes.cast(bm, ctypes.c_void_p),
-                      None, None, None, None, None, None)
+                      None, None, None, None, None, None, None)
     assert rc == lsa.LSA_ERR_INVALID_ARG
     d2 = lsa.lsa_tree_describe(2, 16, (16, 16), 16)
     rc = L.lsa_select(ctypes.byref(d2), None, None, 4, 3, 64, 0, None, ctypes.cast(bm, ctypes.c_void_p),
-                      None, None, None, None, None, None)
+                      None, None, None, None, None, None, None)
     assert rc == lsa.LSA_ERR_SHAPE
     bad = lsa.lsa_tree_desc.from_buffer_copy(d)
     bad.off_leaf_index += 256

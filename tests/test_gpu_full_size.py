@@ -1,0 +1,199 @@
+"""Full-size workloads on the GPU, checked against the oracle on sampled outputs.
+
+Each test runs the CUDA path in the launch configuration bench.py times (tree build,
+select, tree or key-list attention; decode with the dense tail) at the workload's full
+size, then checks (a) properties that hold at any size (balanced leaves, permutation,
+centroid = mean of members on sampled nodes) and (b) sampled outputs the oracle computes
+one by one: k-means rounds of sampled parent nodes (stage-wise), the beam walk of sampled
+queries (stage-wise, near-tie band), and attention of sampled queries on the GPU's keys.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from hierarchical_latent_key_b200 import configs
+from oracle import oracle as orc
+from tests import parity
+
+pytestmark = [pytest.mark.gpu, pytest.mark.slow]
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def lsa():
+    from hierarchical_latent_key_b200 import lsa as mod
+    return mod
+
+
+def _rows(K, h, ids):
+    """Float64 copies of rows `ids` of head h of a (device) key/value tensor."""
+    t = torch.as_tensor(np.asarray(ids), dtype=torch.int64, device=K.device)
+    return K[h].index_select(0, t).double().cpu().numpy()
+
+
+def _tree_props(tree, h, K, W_h, n, leaf, rng, n_nodes=24):
+    """Permutation, ascending leaves, and centroid = mean of members for sampled nodes."""
+    li = tree.leaf_index()[h].cpu().numpy().astype(np.int64)
+    assert np.array_equal(np.sort(li), np.arange(n))
+    assert np.all(np.diff(li.reshape(-1, leaf), axis=1) > 0)
+    for l in range(tree.levels):
+        nodes = tree.desc.nodes[l]
+        per = n // nodes
+        pick = rng.choice(nodes, min(n_nodes, nodes), replace=False)
+        cent = tree.centroids(l)[h].cpu().numpy()
+        mpos = tree.min_pos(l)[h].cpu().numpy()
+        for node in pick:
+            members = li[node * per:(node + 1) * per]
+            Z = orc.project(_rows(K, h, members), W_h)
+            mu = Z.mean(axis=0)
+            assert np.abs(cent[node] - mu).max() <= 1e-5 * np.abs(mu).max() + 1e-6, (l, node)
+            assert mpos[node] == members.min()
+
+
+def _check_queries(case, cfg, tree, h, rows, q_pos, beams, idx, O, LSE, tail=(0, 0)):
+    """Stage-wise select and attention for query rows `rows` of head h (CPU case)."""
+    th = parity.export_tree(tree, h)
+    Qg = case.Q[rows][:, h * cfg.G:(h + 1) * cfg.G]
+    oq = orc.query_latent(Qg, case.W[h].cpu())
+    qp = None if q_pos is None else q_pos[rows]
+    near = parity.check_select_stagewise(oq, th, cfg.branching, cfg.leaf, cfg.beam, qp,
+                                         beams[:, h][:, rows].cpu().numpy(), idx[h][rows].cpu().numpy())
+    Oo, Lo = orc.attn_fwd(Qg, case.K[h].cpu(), case.V[h].cpu(), idx[h][rows].cpu(), q_pos=qp,
+                          causal=q_pos is not None, tail=tail)
+    mx, mean = parity.attn_errors(O[rows][:, h * cfg.G:(h + 1) * cfg.G].float().cpu(), Oo)
+    assert mx <= 2e-2 and mean <= 2e-3, (h, mx, mean)
+    assert np.abs(LSE[rows][:, h * cfg.G:(h + 1) * cfg.G].cpu().numpy() - Lo).max() <= 1e-3
+    return near
+
+
+def test_decode_128k_all_heads(lsa):
+    """All 8 KV heads, n = 131072, 256 decode steps (batched: causal by position, tail of
+    appended keys).  Build checked stage-wise on two heads (sampled deep nodes)."""
+    cfg = configs.get("decode_128k")
+    case = cfg.case("cpu")
+    g = {k: getattr(case, k).to(DEV) for k in ("Q", "K", "V", "W", "q_pos")}
+    tree, trace = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed, trace=True)
+    idx, beams = lsa.select(tree, g["Q"], g["W"], cfg.beam, g["q_pos"], beams=True)
+    O, LSE = lsa.sparse_attn(g["Q"], g["K"], g["V"], idx, g["q_pos"], True, (cfg.n, cfg.n_cap))
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(0)
+    qp = case.q_pos.numpy()
+    for h in (0, 5):
+        Z = orc.project(case.K[h, :cfg.n], case.W[h])
+        parity.check_build_stagewise(Z, trace[:, :, h].cpu().numpy(), cfg.branching, cfg.leaf, cfg.iters,
+                                     cfg.seed, max_segments=8, rng=rng,
+                                     check=lambda l, t, m: l > 0 or t in (0, cfg.iters - 1))
+    near = 0
+    for h in range(cfg.Hkv):
+        _tree_props(tree, h, case.K, case.W[h].float().numpy(), cfg.n, cfg.leaf, rng, n_nodes=6)
+        near += _check_queries(case, cfg, tree, h, np.arange(cfg.T), qp, beams, idx, O, LSE,
+                               tail=(cfg.n, cfg.n_cap))
+    print("decode_128k near-ties", near)
+
+
+def test_prefill_1m_full(lsa):
+    """1,048,576 cached keys, 4096-query causal chunk through select + tree attention."""
+    cfg = configs.get("prefill_1m")
+    case = cfg.case(DEV)
+    tree, trace = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed, trace=True)
+    idx, leaves, beams = lsa.select(tree, case.Q, case.W, cfg.beam, case.q_pos, beams=True, leaves=True)
+    O, LSE = lsa.tree_attn(tree, case.Q, case.K, case.V, leaves, case.q_pos, causal=True)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    qp = case.q_pos.cpu().numpy()
+    rows = np.sort(rng.choice(cfg.T, 48, replace=False))
+    near = 0
+    for h in (0, 3, 7):
+        Kh = case.K[h].double().cpu().numpy()
+        Vh = case.V[h].double().cpu().numpy()
+        Wh = case.W[h].double().cpu().numpy()
+        if h == 3:
+            Z = orc.project(Kh[:cfg.n], Wh)
+            parity.check_build_stagewise(Z, trace[:, :, h].cpu().numpy(), cfg.branching, cfg.leaf, cfg.iters,
+                                         cfg.seed, max_segments=4, rng=rng,
+                                         check=lambda l, t, m: m <= 65536 and t in (0, 4, 9))
+            del Z
+        _tree_props(tree, h, case.K, Wh, cfg.n, cfg.leaf, rng, n_nodes=8)
+        th = parity.export_tree(tree, h)
+        Qg = case.Q[rows][:, h * cfg.G:(h + 1) * cfg.G].double().cpu().numpy()
+        oq = orc.query_latent(Qg, Wh)
+        near += parity.check_select_stagewise(oq, th, cfg.branching, cfg.leaf, cfg.beam, qp[rows],
+                                              beams[:, h][:, rows].cpu().numpy(), idx[h][rows].cpu().numpy())
+        Oo, Lo = orc.attn_fwd(Qg, Kh, Vh, idx[h][rows].cpu(), q_pos=qp[rows], causal=True)
+        mx, mean = parity.attn_errors(O[rows][:, h * cfg.G:(h + 1) * cfg.G].float().cpu(), Oo)
+        assert mx <= 2e-2 and mean <= 2e-3, (h, mx, mean)
+        assert np.abs(LSE[rows][:, h * cfg.G:(h + 1) * cfg.G].cpu().numpy() - Lo).max() <= 1e-3
+        del Kh, Vh
+    print("prefill_1m near-ties", near)
+
+
+def test_decode_10m_full(lsa):
+    """10,485,760 indexed keys, decode steps through select + key-list attention with tail."""
+    cfg = configs.get("decode_10m").scaled(T=8)
+    case = cfg.case(DEV)
+    tree = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    rng = np.random.default_rng(2)
+    h = 6
+    _tree_props(tree, h, case.K, case.W[h].double().cpu().numpy(), cfg.n, cfg.leaf, rng, n_nodes=4)
+    # one decode step at a time, as bench.py runs them
+    th = parity.export_tree(tree, h)
+    W_h = case.W[h].double().cpu().numpy()
+    for s in range(cfg.T):
+        p = cfg.n + s
+        Qs = case.Q[s:s + 1]
+        idx, beams = lsa.select(tree, Qs, case.W, cfg.beam, case.q_pos[s:s + 1], beams=True)
+        O, LSE = lsa.sparse_attn(Qs, case.K, case.V, idx, case.q_pos[s:s + 1], True, (cfg.n, p + 1))
+        Qg = Qs[:, h * cfg.G:(h + 1) * cfg.G].double().cpu().numpy()
+        oq = orc.query_latent(Qg, W_h)
+        parity.check_select_stagewise(oq, th, cfg.branching, cfg.leaf, cfg.beam, np.array([p]),
+                                      beams[:, h].cpu().numpy(), idx[h].cpu().numpy())
+        # every selected key and every tail key precedes the query: compact them (non-causal)
+        sel = idx[h, 0].cpu().numpy()
+        keys = np.concatenate([sel[sel >= 0], np.arange(cfg.n, p + 1)])
+        Kc, Vc = _rows(case.K, h, keys), _rows(case.V, h, keys)
+        n_sel = int((sel >= 0).sum())
+        Oo, Lo = orc.attn_fwd(Qg, Kc, Vc, np.arange(n_sel, dtype=np.int32)[None], tail=(n_sel, len(keys)))
+        mx, mean = parity.attn_errors(O[:, h * cfg.G:(h + 1) * cfg.G].float().cpu(), Oo)
+        assert mx <= 2e-2 and mean <= 2e-3, (s, mx, mean)
+        assert np.abs(LSE[:, h * cfg.G:(h + 1) * cfg.G].cpu().numpy() - Lo).max() <= 1e-3
+
+
+def test_train_128k_full(lsa):
+    """131072-token causal layer: build, select, tree-attention forward, backward; oracle on
+    sampled queries (dQ, O) and sampled keys (dK, dV from every query that selected them)."""
+    cfg = configs.get("train_128k")
+    case = cfg.case(DEV)
+    tree = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select(tree, case.Q, case.W, cfg.beam, case.q_pos, leaves=True)
+    O, LSE = lsa.tree_attn(tree, case.Q, case.K, case.V, leaves, case.q_pos, causal=True)
+    dQ, dK, dV = lsa.sparse_attn_bwd(case.Q, case.K, case.V, O, LSE, case.dO, idx, case.q_pos, True)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(3)
+    h = 1
+    sl = slice(h * cfg.G, (h + 1) * cfg.G)
+    Qh = case.Q[:, sl].float().cpu().numpy()
+    Kh = case.K[h].float().cpu().numpy()
+    Vh = case.V[h].float().cpu().numpy()
+    dOh = case.dO[:, sl].float().cpu().numpy()
+    qp = case.q_pos.cpu().numpy()
+    ih = idx[h].cpu().numpy()
+    rows = np.sort(rng.choice(cfg.T, 64, replace=False))
+    Oo, Lo = orc.attn_fwd(Qh[rows], Kh, Vh, ih[rows], q_pos=qp[rows], causal=True)
+    mx, mean = parity.attn_errors(O[rows][:, sl].float().cpu(), Oo)
+    assert mx <= 2e-2 and mean <= 2e-3, (mx, mean)
+    oQ, _, _ = orc.attn_bwd(Qh[rows], Kh, Vh, ih[rows], dOh[rows], q_pos=qp[rows], causal=True)
+    got = dQ[rows][:, sl].cpu().numpy()
+    err = np.abs(got - oQ)
+    assert err.max() <= 2e-2 * np.abs(oQ).max() and err.mean() <= 2e-3 * np.abs(oQ).mean()
+    # a few keys: every query that selected them contributes to dK, dV
+    keys = rng.choice(cfg.n // 2, 3, replace=False)
+    for j in keys:
+        users = np.nonzero((ih == j).any(axis=1) & (qp >= j))[0]
+        if len(users) == 0:
+            continue
+        _, oK, oV = orc.attn_bwd(Qh[users], Kh, Vh, ih[users], dOh[users], q_pos=qp[users], causal=True)
+        for name, got, want in (("dK", dK[h, j].cpu().numpy(), oK[j]), ("dV", dV[h, j].cpu().numpy(), oV[j])):
+            e = np.abs(got - want)
+            assert e.max() <= 2e-2 * np.abs(want).max() + 1e-6, (name, j, e.max(), np.abs(want).max())

@@ -213,3 +213,76 @@ def test_nonfinite_score_reports_status(lsa):
     with pytest.raises(lsa.LsaError) as e:
         lsa.select(tree, Q, g["W"], cfg.beam)
     assert e.value.code == lsa.LSA_ERR_NONFINITE
+
+
+@pytest.mark.parametrize("G,n_q", [(4, 384), (1, 200), (2, 256), (8, 128)])
+def test_tree_attention_matches_oracle(lsa, G, n_q):
+    """Leaf-by-leaf tensor-core attention = attention over the expanded key lists."""
+    cfg = configs.get("prefill_1m").scaled(n=8 * 8 * 4 * 2 * 64, branching=(8, 8, 4, 2), beam=(4, 16, 16, 8),
+                                           Hkv=2, Hq=2 * G, T=n_q, comps=256)
+    case = cfg.case("cpu", seed=11 + G)
+    g = _to(case)
+    tree = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select(tree, g["Q"], g["W"], cfg.beam, g["q_pos"], leaves=True)
+    O, LSE = lsa.tree_attn(tree, g["Q"], g["K"], g["V"], leaves, g["q_pos"], causal=True)
+    O2, L2 = lsa.sparse_attn(g["Q"], g["K"], g["V"], idx, g["q_pos"], True)
+    torch.cuda.synchronize()
+    qp = case.q_pos.numpy()
+    for h in range(cfg.Hkv):
+        sl = slice(h * G, (h + 1) * G)
+        Oo, Lo = orc.attn_fwd(case.Q[:, sl], case.K[h], case.V[h], idx[h].cpu(), q_pos=qp, causal=True)
+        mx, mean = parity.attn_errors(O[:, sl].float().cpu(), Oo)
+        assert mx <= 2e-2 and mean <= 2e-3, (h, mx, mean)
+        assert np.abs(LSE[:, sl].cpu().numpy() - Lo).max() <= 1e-3
+    assert (O.float() - O2.float()).abs().max().item() <= 2e-2
+
+
+def test_tree_attention_many_queries_per_leaf(lsa):
+    """Training geometry, scaled: causal, every leaf chosen by hundreds of queries (several
+    128-row chunks per leaf)."""
+    cfg = configs.get("train_128k").scaled(n=8192, T=8192, branching=(8, 4, 4), beam=(4, 8, 8), Hkv=2, Hq=8,
+                                           comps=64)
+    case = cfg.case("cpu")
+    g = _to(case)
+    tree = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select(tree, g["Q"], g["W"], cfg.beam, g["q_pos"], leaves=True)
+    O, LSE = lsa.tree_attn(tree, g["Q"], g["K"], g["V"], leaves, g["q_pos"], causal=True)
+    torch.cuda.synchronize()
+    qp = case.q_pos.numpy()
+    rows = np.random.default_rng(0).choice(cfg.T, 512, replace=False)
+    for h in range(cfg.Hkv):
+        sl = slice(h * cfg.G, (h + 1) * cfg.G)
+        Oo, Lo = orc.attn_fwd(case.Q[rows][:, sl], case.K[h], case.V[h], idx[h].cpu()[rows], q_pos=qp[rows],
+                              causal=True)
+        mx, mean = parity.attn_errors(O[rows][:, sl].float().cpu(), Oo)
+        assert mx <= 2e-2 and mean <= 2e-3, (h, mx, mean)
+        assert np.abs(LSE[rows][:, sl].cpu().numpy() - Lo).max() <= 1e-3
+
+
+def test_tree_attention_fallback_shapes(lsa):
+    """fp32 (tiny workload): the entry point expands the leaves and runs the generic kernels."""
+    cfg = configs.get("tiny")
+    case = cfg.case("cpu")
+    g = _to(case)
+    tree = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select(tree, g["Q"], g["W"], cfg.beam, None, leaves=True)
+    O, LSE = lsa.tree_attn(tree, g["Q"], g["K"], g["V"], leaves)
+    torch.cuda.synchronize()
+    Oo, Lo = orc.attn_fwd(case.Q, case.K[0], case.V[0], idx[0].cpu())
+    assert np.abs(O.cpu().numpy() - Oo).max() <= 1e-4
+
+
+def test_kv_append_writes_rows(lsa):
+    for dt in (torch.bfloat16, torch.float32):
+        K = torch.randn(3, 50, 128, device=DEV).to(dt)
+        V = torch.randn(3, 50, 128, device=DEV).to(dt)
+        K0, V0 = K.clone(), V.clone()
+        kr = torch.randn(3, 128, device=DEV).to(dt)
+        vr = torch.randn(3, 128, device=DEV).to(dt)
+        lsa.lsa_kv_append(K, V, 17, kr, vr)
+        torch.cuda.synchronize()
+        assert torch.equal(K[:, 17], kr) and torch.equal(V[:, 17], vr)
+        K[:, 17], V[:, 17] = K0[:, 17], V0[:, 17]
+        assert torch.equal(K, K0) and torch.equal(V, V0)
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_kv_append(K, V, 50, kr, vr)
