@@ -216,7 +216,8 @@ int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, i
   int beam_max = 0;
   for (int l = 0; l < tree->levels; ++l) {
     const int64_t avail = l == 0 ? tree->nodes[0] : (int64_t)beam[l - 1] * tree->branching[l];
-    if (beam[l] < 1 || beam[l] > LSA_MAX_BEAM || beam[l] > avail)
+    if (beam[l] < 1 || beam[l] > LSA_MAX_BEAM || beam[l] > avail ||
+        (l + 1 < tree->levels && (int64_t)beam[l] * tree->branching[l + 1] > 512))
       return fail(LSA_ERR_SHAPE, "beam[%d] = %d must be in [1, min(64, %lld)]", l, beam[l], (long long)avail);
     beam_max = beam[l] > beam_max ? beam[l] : beam_max;
     a.beam[l] = beam[l];

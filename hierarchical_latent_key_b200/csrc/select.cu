@@ -8,7 +8,7 @@
 // attention works": hierarchical search with a fixed budget per level, then a
 // fixed number of original keys taken from the chosen clusters.
 //
-// One CTA (8 warps) per (query t, KV group g).  Scores are fp32 inner products
+// One CTA (4 warps) per (query t, KV group g).  Scores are fp32 inner products
 // of the group's latent query with fp32 centroids (exact enough that ordering
 // decisions only differ from an fp64 evaluation inside a ~1e-6 relative band).
 // Candidates are ranked by a packed 64-bit key (orderable score, ~node id) so a
@@ -24,7 +24,7 @@
 
 namespace lsa {
 
-constexpr int kSelThreads = 256;
+constexpr int kSelThreads = 128;   // 4 warps x 128 candidates >= beam * branching (32 * 16)
 
 // Bitonic sort (descending) of 32*E keys held in registers, E per lane; element
 // index i = lane * E + e.  Pairs closer than E sit in one lane; farther pairs are
@@ -98,12 +98,12 @@ __device__ __forceinline__ int merge_sorted(const unsigned long long* src, int m
 }
 
 template <typename T, int R, int DK>
-__global__ void __launch_bounds__(kSelThreads, 2) k_select(SelectArgs a) {
+__global__ void __launch_bounds__(kSelThreads, 4) k_select(SelectArgs a) {
   __shared__ float s_q[DK];
   __shared__ float s_part[kSelThreads];
   __shared__ __align__(16) float s_lat[R];
-  __shared__ unsigned long long s_cand[8 * 128];
-  __shared__ unsigned long long s_merge[8 * LSA_MAX_BEAM];
+  __shared__ unsigned long long s_cand[(kSelThreads / 32) * 128];
+  __shared__ unsigned long long s_merge[(kSelThreads / 32) * LSA_MAX_BEAM];
   __shared__ int32_t s_kept[LSA_MAX_BEAM];
   __shared__ int32_t s_next[LSA_MAX_BEAM];
   __shared__ int s_nkept;
@@ -190,8 +190,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_select(SelectArgs a) {
     __syncthreads();
     if (nw_act > 1 && warp == 0) {
       const int m = nw_act * KW;
-      const int cnt = m <= 128 ? merge_sorted<4>(s_merge, m, a.beam[l], s_next)
-                               : merge_sorted<8>(s_merge, m, a.beam[l], s_next);
+      const int cnt = merge_sorted<4>(s_merge, m, a.beam[l], s_next);   // m <= 4 * 32
       if (lane == 0) s_nkept = cnt;
     }
     __syncthreads();

@@ -321,8 +321,8 @@ __global__ void __launch_bounds__(kTL) k_tl_stats(TreeAttnArgs a) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
     asm volatile("fence.mbarrier_init.release.cluster;");
   }
+  load_leaf(a, g, leaf, s, false);             // loads in flight while TMEM is allocated
   alloc_tmem(&s_taddr, 64);
-  load_leaf(a, g, leaf, s, false);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -403,15 +403,15 @@ __global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
   s.sA = smem_u32(base);                       // 32 KB: rows x d
   s.sK = s.sA + kTL * 256;                     // 16 KB
   s.sV = s.sK + kLeafKeys * 256;               // 16 KB
-  s.sP = s.sV + kLeafKeys * 256;               // 16 KB: rows x 64 keys
+  s.sP = s.sA;                                 // P (rows x 64 keys) overwrites the consumed Q tile
   s.pos = s_pos;
   s.mbar = smem_u32(&s_mbar);
   if (threadIdx.x == 0) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
     asm volatile("fence.mbarrier_init.release.cluster;");
   }
-  alloc_tmem(&s_taddr, 256);
-  load_leaf(a, g, leaf, s, true);
+  load_leaf(a, g, leaf, s, true);              // loads in flight while TMEM is allocated
+  alloc_tmem(&s_taddr, 128);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -419,7 +419,7 @@ __global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
   const int warp = threadIdx.x >> 5;
   uint32_t phase = 0;
   bool ok = true;
-  char* sP_gen = base + (s.sP - s.sA);
+  char* sP_gen = base;
   for (int64_t e0 = 0; e0 < n_ent && ok; e0 += kTL / a.G) {
     int64_t tq;
     int rank, h;
@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
       for (int kk = 0; kk < 4; ++kk) {
         const uint64_t da = sdesc_sw128(s.sP + kk * 32, 16, 1024);
         const uint64_t db = sdesc_sw128(s.sV + kk * 2048, kLeafKeys * 128, 1024);
-        tc_mma(tmem + 64, da, db, idesc, kk > 0 ? 1u : 0u);
+        tc_mma(tmem, da, db, idesc, kk > 0 ? 1u : 0u);   // O over S's columns: S is in P now
       }
       tc_commit(s.mbar);
     }
@@ -480,7 +480,7 @@ __global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
 #pragma unroll
       for (int part = 0; part < 4; ++part) {
         float v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 64 + part * 32, v);
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + part * 32, v);
         if (dst) {
 #pragma unroll
           for (int i = 0; i < 32; i += 4) red_add_v4(dst + part * 32 + i, v[i], v[i + 1], v[i + 2], v[i + 3]);
@@ -492,7 +492,7 @@ __global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
     tc_fence_before();
     __syncthreads();
   }
-  free_tmem(tmem, 256);
+  free_tmem(tmem, 128);
 }
 
 __global__ void k_tl_finish(TreeAttnArgs a) {
@@ -518,7 +518,7 @@ __global__ void k_tl_expand(const int32_t* leaves, const int32_t* leaf_index, in
 }
 
 constexpr size_t kStatsSmem = 1024 + kTL * 256 + kLeafKeys * 256;
-constexpr size_t kOutSmem = 1024 + kTL * 256 + 3 * kLeafKeys * 256;
+constexpr size_t kOutSmem = 1024 + kTL * 256 + 2 * kLeafKeys * 256;
 
 }  // namespace
 
