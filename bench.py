@@ -325,7 +325,6 @@ class Train:
         self.desc = lsa.lsa_tree_describe(cfg.Hkv, cfg.r, cfg.branching, cfg.leaf)
         self.tree_mem = torch.empty(self.desc.bytes, dtype=torch.uint8, device=dev)
         self.build_ws = torch.empty(lsa.lsa_build_workspace_bytes(self.desc, d), dtype=torch.uint8, device=dev)
-        self.idx = torch.empty(cfg.Hkv, T, cfg.K_sel, dtype=torch.int32, device=dev)
         self.leaves = torch.empty(cfg.Hkv, T, cfg.beam[-1], dtype=torch.int32, device=dev)
         self.O = torch.empty_like(self.Q)
         self.LSE = torch.empty(T, Hq, dtype=torch.float32, device=dev)
@@ -334,6 +333,8 @@ class Train:
         self.dV = torch.empty(self.V.shape, dtype=torch.float32, device=dev)
         need = lsa.lsa_tree_attn_workspace_bytes(self.desc, T, Hq, d, self.Q.dtype, cfg.beam[-1])
         self.attn_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        need = lsa.lsa_tree_attn_bwd_workspace_bytes(self.desc, T, Hq, d, self.Q.dtype, cfg.beam[-1])
+        self.bwd_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.scale = 1.0 / math.sqrt(d)
         self.seed = seed
@@ -343,14 +344,14 @@ class Train:
         return (
             ("build", lambda: L.lsa_build_tree(self.desc, self.tree_mem, self.K, self.W, c.iters, self.seed,
                                               self.build_ws, None, self.status)),
-            ("select", lambda: L.lsa_select(self.desc, self.tree_mem, self.Q, self.W, c.beam, self.q_pos, self.idx,
+            ("select", lambda: L.lsa_select(self.desc, self.tree_mem, self.Q, self.W, c.beam, self.q_pos, None,
                                             self.leaves, status=self.status)),
             ("forward", lambda: L.lsa_tree_attn(self.desc, self.tree_mem, self.Q, self.K, self.V, self.leaves,
                                                 self.q_pos, True, self.scale, self.O, self.LSE, self.attn_ws,
                                                 self.status)),
-            ("backward", lambda: L.lsa_sparse_attn_bwd(self.Q, self.K, self.V, self.O, self.LSE, self.dO,
-                                                       self.idx, self.q_pos, True, 0, 0, self.scale, self.dQ,
-                                                       self.dK, self.dV, self.status)),
+            ("backward", lambda: L.lsa_tree_attn_bwd(self.desc, self.tree_mem, self.Q, self.K, self.V, self.O,
+                                                     self.LSE, self.dO, self.leaves, self.q_pos, True, self.scale,
+                                                     self.dQ, self.dK, self.dV, self.bwd_ws, self.status)),
         )
 
 
@@ -516,15 +517,51 @@ def cpu_baseline_prefill(w, n_queries=4096):
 
 
 def bench_config(args):
-    if args.workload != "prefill_1m":
-        raise SystemExit(f"workload {args.workload} is not wired into the benchmark yet")
-    cfg = configs.get(args.workload)
+    cfg = configs.get("prefill_1m")
     if args.small:
         cfg = cfg.scaled(name="prefill_1m_geometry_131k", n=131072, branching=(8, 8, 8, 4), comps=1024)
     return cfg
 
 
+def run_single(args, rank, world, local_rank):
+    """Headline = one of the secondary workloads alone (decode_10m or train_128k)."""
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    pg = world > 1
+
+    def reduce_max(x):
+        if not pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    if pg:
+        torch.distributed.barrier()
+    with ClockSampler(local_rank) as clk:
+        if args.workload == "decode_10m":
+            r = run_decode(args, dev, rank, world, reduce_max)
+        else:
+            r = run_train(args, dev, rank, world, reduce_max, steps=args.steps, warmup=args.warmup)
+        if pg:
+            torch.distributed.barrier()
+    if rank != 0:
+        return None
+    unit = r.pop("unit")
+    line = {"metric": METRIC, "value": r.pop("value"), "unit": unit, "n_gpus": world,
+            "steps": r.pop("steps"), "warmup": r.pop("warmup", args.warmup), "ms_per_step": r.pop("ms_per_step"),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "clocks": clk.summary()}
+    line["config"] = dict(r.pop("config"), parallelism=f"dp{world}")
+    line.update(r)
+    return line
+
+
 def run_cuda(args, rank, world, local_rank):
+    if args.workload in ("decode_10m", "train_128k"):
+        return run_single(args, rank, world, local_rank)
+    if args.workload != "prefill_1m":
+        raise SystemExit(f"workload {args.workload} has no benchmark (parity tests only)")
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     cfg = bench_config(args)

@@ -358,6 +358,56 @@ int lsa_tree_attn(const lsa_tree_desc* tree, const void* tree_mem, const void* Q
   return ok();
 }
 
+int lsa_tree_attn_bwd_workspace_bytes(const lsa_tree_desc* tree, int32_t T, int32_t Hq, int32_t d, int32_t dtype,
+                                      int32_t n_leaves, size_t* bytes) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
+  if (T < 0 || Hq < tree->n_heads || Hq % tree->n_heads || n_leaves < 1 || n_leaves > LSA_MAX_BEAM ||
+      (d != 64 && d != 128))
+    return fail(LSA_ERR_SHAPE, "bad sizes");
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  const bool fast = lsa::tree_attn_fast_path(dtype, d, Hq / tree->n_heads, tree->leaf_size);
+  *bytes = lsa::tree_attn_bwd_workspace(tree->n_heads, tree->nodes[tree->levels - 1], T, Hq, d, n_leaves,
+                                        tree->leaf_size, fast);
+  return ok();
+}
+
+int lsa_tree_attn_bwd(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
+                      const void* K, const void* V, int64_t n_cap, int32_t d, int32_t dtype, const void* O,
+                      const float* LSE, const void* dO, const int32_t* leaves, int32_t n_leaves,
+                      const int32_t* q_pos, int32_t causal, float scale, float* dQ, float* dK, float* dV,
+                      void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  size_t need = 0;
+  int rc = lsa_tree_attn_bwd_workspace_bytes(tree, T, Hq, d, dtype, n_leaves, &need);
+  if (rc != LSA_OK) return rc;
+  const int G = Hq / tree->n_heads;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(LSA_ERR_SHAPE, "query heads per group must be 1, 2, 4 or 8");
+  if (n_cap < tree->n_tree) return fail(LSA_ERR_SHAPE, "n_cap (%lld) < n_tree", (long long)n_cap);
+  if (!std::isfinite(scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite");
+  if (!dK || !dV) return fail(LSA_ERR_INVALID_ARG, "dK and dV must be non-NULL");
+  if (T > 0) {
+    if (!tree_mem || !Q || !K || !V || !O || !LSE || !dO || !leaves || !dQ)
+      return fail(LSA_ERR_INVALID_ARG, "tree_mem, Q, K, V, O, LSE, dO, leaves and dQ must be non-NULL");
+    if (causal && !q_pos) return fail(LSA_ERR_INVALID_ARG, "q_pos is required when causal");
+    if (!workspace || workspace_bytes < need)
+      return fail(LSA_ERR_WORKSPACE, "tree attention backward needs %zu workspace bytes (got %zu)", need,
+                  workspace ? workspace_bytes : (size_t)0);
+  }
+  lsa::TreeAttnCall c;
+  memset(&c, 0, sizeof(c));
+  c.Q = Q; c.K = K; c.V = V;
+  c.leaf_index = tree_mem ? reinterpret_cast<const int32_t*>(static_cast<const char*>(tree_mem) + tree->off_leaf_index)
+                          : nullptr;
+  c.leaves = leaves; c.q_pos = q_pos; c.workspace = workspace; c.status = status;
+  c.T = T; c.n_cap = n_cap; c.n_tree = tree->n_tree; c.NL = tree->nodes[tree->levels - 1];
+  c.Hq = Hq; c.H = tree->n_heads; c.d = d; c.dtype = dtype; c.B = n_leaves; c.leaf = tree->leaf_size;
+  c.causal = causal ? 1 : 0; c.scale = scale;
+  cudaError_t e = lsa::run_tree_attn_bwd(c, O, LSE, dO, dQ, dK, dV, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_tree_attn_bwd");
+  return ok();
+}
+
 int lsa_sparse_attn_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, const void* V, int32_t n_heads,
                         int64_t n_cap, int32_t d, int32_t dtype, const void* O, const float* LSE, const void* dO,
                         const int32_t* idx, int32_t K_sel, const int32_t* q_pos, int32_t causal, int64_t tail_begin,

@@ -199,21 +199,51 @@ __global__ void __launch_bounds__(kAttnThreads) k_attn_fwd(AttnArgs a) {
   }
 }
 
+// Merge the split partials of one (query, head) row: the splits' maxima and sums
+// are read by one thread each, the d outputs by one thread each with all split
+// loads issued together.
 template <typename T, int DK>
-__global__ void k_attn_combine(AttnArgs a) {
+__global__ void __launch_bounds__(DK) k_attn_combine(AttnArgs a) {
+  __shared__ float s_f[1024];
+  __shared__ float s_M, s_L;
   const int64_t row = blockIdx.x;  // t * Hq + head
   const int dim = threadIdx.x;
-  const float* p = a.part + row * a.nsplit * (DK + 2);
-  float M = -INFINITY;
-  for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, p[s * (DK + 2) + DK]);
-  float L = 0.f, o = 0.f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < a.nsplit; ++s) {
-      const float f = exp2f(p[s * (DK + 2) + DK] - M);
-      L += p[s * (DK + 2) + DK + 1] * f;
-      o += p[s * (DK + 2) + dim] * f;
-    }
+  const int ns = a.nsplit;
+  const float* p = a.part + row * ns * (DK + 2);
+  float m = -INFINITY;
+  for (int s = dim; s < ns; s += DK) m = fmaxf(m, p[s * (DK + 2) + DK]);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if ((dim & 31) == 0) s_f[dim >> 5] = m;
+  __syncthreads();
+  if (dim == 0) {
+    float M = -INFINITY;
+    for (int w = 0; w < DK / 32; ++w) M = fmaxf(M, s_f[w]);
+    s_M = M;
   }
+  __syncthreads();
+  const float M = s_M;
+  float l = 0.f;
+  for (int s = dim; s < ns; s += DK) {
+    const float f = M == -INFINITY ? 0.f : exp2f(p[s * (DK + 2) + DK] - M);
+    s_f[32 + s] = f;
+    l += p[s * (DK + 2) + DK + 1] * f;
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  __syncthreads();
+  if ((dim & 31) == 0) s_f[dim >> 5] = l;
+  __syncthreads();
+  if (dim == 0) {
+    float L = 0.f;
+    for (int w = 0; w < DK / 32; ++w) L += s_f[w];
+    s_L = L;
+  }
+  __syncthreads();
+  const float L = s_L;
+  float o = 0.f;
+#pragma unroll 8
+  for (int s = 0; s < ns; ++s) o += p[s * (DK + 2) + dim] * s_f[32 + s];
   T* O = static_cast<T*>(a.O);
   O[row * DK + dim] = from_f32<T>(L > 0.f ? o / L : 0.f);
   if (dim == 0) a.LSE[row] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;

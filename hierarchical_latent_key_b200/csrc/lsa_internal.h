@@ -119,6 +119,9 @@ struct TreeAttnCall {
 size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast);
 bool tree_attn_fast_path(int dtype, int d, int G, int leaf);
 cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st);
+size_t tree_attn_bwd_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast);
+cudaError_t run_tree_attn_bwd(const TreeAttnCall& c, const void* O, const float* LSE, const void* dO, float* dQ,
+                              float* dK, float* dV, cudaStream_t st);
 int attn_splits(int64_t T, int Hkv, int64_t keys);
 int report_error(int code, const char* msg);
 cudaError_t run_kv_append(void* K, void* V, int64_t n_heads, int64_t n_cap, int64_t row_bytes, int64_t pos,

@@ -101,6 +101,7 @@ template <typename T, int R, int DK>
 __global__ void __launch_bounds__(kSelThreads, 4) k_select(SelectArgs a) {
   __shared__ float s_q[DK];
   __shared__ float s_part[kSelThreads];
+  __shared__ __align__(16) T s_w[DK * R];
   __shared__ __align__(16) float s_lat[R];
   __shared__ unsigned long long s_cand[(kSelThreads / 32) * 128];
   __shared__ unsigned long long s_merge[(kSelThreads / 32) * LSA_MAX_BEAM];
@@ -118,14 +119,21 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_select(SelectArgs a) {
     s_q[j] = s / (float)a.G;
   }
   __syncthreads();
-  // latent query = group query . W[g]; thread (k, part) sums a slice of d
+  // latent query = group query . W[g]: W[g] is staged in shared memory with
+  // 16-byte loads (one memory round trip), then thread (k, part) sums a slice of d
   {
     constexpr int PARTS = kSelThreads / R;
     constexpr int SPAN = DK / PARTS;
-    const int k = tid % R, p = tid / R;
+    constexpr int VEC = 16 / sizeof(T);
     const T* W = static_cast<const T*>(a.W) + (int64_t)g * DK * R;
+#pragma unroll
+    for (int i = tid * VEC; i < DK * R; i += kSelThreads * VEC)
+      *reinterpret_cast<uint4*>(&s_w[i]) = __ldg(reinterpret_cast<const uint4*>(W + i));
+    __syncthreads();
+    const int k = tid % R, p = tid / R;
     float acc = 0.f;
-    for (int j = p * SPAN; j < (p + 1) * SPAN; ++j) acc = fmaf(s_q[j], to_f32(W[j * R + k]), acc);
+#pragma unroll 16
+    for (int j = p * SPAN; j < (p + 1) * SPAN; ++j) acc = fmaf(s_q[j], to_f32(s_w[j * R + k]), acc);
     s_part[tid] = acc;
     __syncthreads();
     if (tid < R) {
@@ -137,6 +145,9 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_select(SelectArgs a) {
     __syncthreads();
   }
   const int64_t qpos = a.q_pos ? (int64_t)a.q_pos[t] : (int64_t)LLONG_MAX;
+  // a query at or past the last indexed position sees every node (decode): no
+  // per-node eligibility load is needed
+  const bool all_eligible = qpos >= a.n_tree - 1;
   int ncand = (int)a.nodes[0];
   int n_kept = 0;
   for (int l = 0; l < a.levels; ++l) {
@@ -152,7 +163,7 @@ __global__ void __launch_bounds__(kSelThreads, 4) k_select(SelectArgs a) {
       unsigned long long key = 0ull;
       if (i < ncand) {
         const int64_t id = l == 0 ? i : (int64_t)s_kept[i / b] * b + (i % b);
-        if ((int64_t)__ldg(&mpos[id]) <= qpos) {
+        if (all_eligible || (int64_t)__ldg(&mpos[id]) <= qpos) {
           const float4* cr = reinterpret_cast<const float4*>(cent + id * R);
           float sc = 0.f;
 #pragma unroll

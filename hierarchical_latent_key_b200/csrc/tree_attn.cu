@@ -215,40 +215,39 @@ struct LeafSmem {
   uint32_t* taddr_slot;
 };
 
-// Load the leaf's K (and V) rows into the swizzled tiles; positions to smem.
-__device__ __forceinline__ void load_leaf(const TreeAttnArgs& a, int64_t g, int64_t leaf, const LeafSmem& s,
-                                          bool with_v) {
-  const int t = threadIdx.x;
-  if (t < kLeafKeys) s.pos[t] = a.leaf_index[g * a.n_tree + leaf * kLeafKeys + t];
-  __syncthreads();
-  const __nv_bfloat16* Kh = a.K + g * a.n_cap * kDim;
-  const __nv_bfloat16* Vh = a.V + g * a.n_cap * kDim;
-  // 64 rows x 16 chunks; thread t takes row t / 2, chunks (t % 2) * 8 .. + 8
-  const int r = t >> 1, c0 = (t & 1) * 8;
-  const int64_t j = s.pos[r];
-#pragma unroll
-  for (int c = c0; c < c0 + 8; ++c) {
-    cp_async16(s.sK + sw128_off(r, c, kLeafKeys * 128), Kh + j * kDim + c * 8);
-    if (with_v) cp_async16(s.sV + sw128_off(r, c, kLeafKeys * 128), Vh + j * kDim + c * 8);
-  }
-}
-
-// Load up to 128 (query, head) rows of a chunk into the A tile; returns this
-// thread's row: query index (or -1) and rank.
-__device__ __forceinline__ void load_rows(const TreeAttnArgs& a, int64_t g, const int32_t* ent, int64_t n_ent,
-                                          int64_t e0, const LeafSmem& s, int64_t& tq, int& rank, int& h) {
-  const int t = threadIdx.x;
-  const int64_t e = e0 + t / a.G;
-  h = t % a.G;
+// This thread's row of a chunk: query index (or -1), rank of the leaf in that
+// query's list, and head within the group.
+__device__ __forceinline__ void row_of(const TreeAttnArgs& a, const int32_t* ent, int64_t n_ent, int64_t e0,
+                                       int64_t& tq, int& rank, int& h) {
+  const int64_t e = e0 + threadIdx.x / a.G;
+  h = threadIdx.x % a.G;
   tq = -1;
   rank = 0;
   if (e < n_ent) {
     const int32_t v = ent[e];
     tq = v >> 6;
     rank = v & 63;
-    const __nv_bfloat16* q = a.Q + (tq * a.Hq + g * a.G + h) * kDim;
+  }
+}
+
+// Copy this thread's query row into row threadIdx.x of the A tile.
+__device__ __forceinline__ void copy_row(const TreeAttnArgs& a, int64_t g, int64_t tq, int h, uint32_t sA) {
+  if (tq < 0) return;
+  const __nv_bfloat16* q = a.Q + (tq * a.Hq + g * a.G + h) * kDim;
 #pragma unroll
-    for (int c = 0; c < 16; ++c) cp_async16(s.sA + sw128_off(t, c, kTL * 128), q + c * 8);
+  for (int c = 0; c < 16; ++c) cp_async16(sA + sw128_off(threadIdx.x, c, kTL * 128), q + c * 8);
+}
+
+// Copy the leaf's K (and V) rows (positions already in smem) into the tiles.
+__device__ __forceinline__ void copy_leaf(const TreeAttnArgs& a, int64_t g, const LeafSmem& s, bool with_v) {
+  const __nv_bfloat16* Kh = a.K + g * a.n_cap * kDim;
+  const __nv_bfloat16* Vh = a.V + g * a.n_cap * kDim;
+  const int r = threadIdx.x >> 1, c0 = (threadIdx.x & 1) * 8;
+  const int64_t j = s.pos[r];
+#pragma unroll
+  for (int c = c0; c < c0 + 8; ++c) {
+    cp_async16(s.sK + sw128_off(r, c, kLeafKeys * 128), Kh + j * kDim + c * 8);
+    if (with_v) cp_async16(s.sV + sw128_off(r, c, kLeafKeys * 128), Vh + j * kDim + c * 8);
   }
 }
 
@@ -321,7 +320,13 @@ __global__ void __launch_bounds__(kTL) k_tl_stats(TreeAttnArgs a) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
     asm volatile("fence.mbarrier_init.release.cluster;");
   }
-  load_leaf(a, g, leaf, s, false);             // loads in flight while TMEM is allocated
+  // first chunk's row and the leaf's key positions: independent loads in flight together
+  int64_t tq;
+  int rank, h;
+  row_of(a, ent, n_ent, 0, tq, rank, h);
+  if (threadIdx.x < kLeafKeys) s_pos[threadIdx.x] = a.leaf_index[g * a.n_tree + leaf * kLeafKeys + threadIdx.x];
+  __syncthreads();
+  copy_leaf(a, g, s, false);
   alloc_tmem(&s_taddr, 64);
   tc_fence_before();
   __syncthreads();
@@ -330,9 +335,8 @@ __global__ void __launch_bounds__(kTL) k_tl_stats(TreeAttnArgs a) {
   uint32_t phase = 0;
   bool ok = true;
   for (int64_t e0 = 0; e0 < n_ent && ok; e0 += kTL / a.G) {
-    int64_t tq;
-    int rank, h;
-    load_rows(a, g, ent, n_ent, e0, s, tq, rank, h);
+    if (e0 > 0) row_of(a, ent, n_ent, e0, tq, rank, h);
+    copy_row(a, g, tq, h, s.sA);
     cp_async_wait_all();
     fence_async_smem();
     __syncthreads();
@@ -410,7 +414,14 @@ __global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
     asm volatile("fence.mbarrier_init.release.cluster;");
   }
-  load_leaf(a, g, leaf, s, true);              // loads in flight while TMEM is allocated
+  // first chunk's row (and its LSE) and the leaf's key positions in flight together
+  int64_t tq;
+  int rank, h;
+  row_of(a, ent, n_ent, 0, tq, rank, h);
+  float lse = tq >= 0 ? a.lse2[tq * a.Hq + g * a.G + h] : INFINITY;
+  if (threadIdx.x < kLeafKeys) s_pos[threadIdx.x] = a.leaf_index[g * a.n_tree + leaf * kLeafKeys + threadIdx.x];
+  __syncthreads();
+  copy_leaf(a, g, s, true);
   alloc_tmem(&s_taddr, 128);
   tc_fence_before();
   __syncthreads();
@@ -421,9 +432,11 @@ __global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
   bool ok = true;
   char* sP_gen = base;
   for (int64_t e0 = 0; e0 < n_ent && ok; e0 += kTL / a.G) {
-    int64_t tq;
-    int rank, h;
-    load_rows(a, g, ent, n_ent, e0, s, tq, rank, h);
+    if (e0 > 0) {
+      row_of(a, ent, n_ent, e0, tq, rank, h);
+      lse = tq >= 0 ? a.lse2[tq * a.Hq + g * a.G + h] : INFINITY;
+    }
+    copy_row(a, g, tq, h, s.sA);
     cp_async_wait_all();
     fence_async_smem();
     __syncthreads();
@@ -438,7 +451,6 @@ __global__ void __launch_bounds__(kTL) k_tl_out(TreeAttnArgs a) {
     if (ok) {
       float sc[64];
       read_scores(a, s, tmem, tq, sc);
-      const float lse = tq >= 0 ? a.lse2[tq * a.Hq + g * a.G + h] : INFINITY;
       // P row (bf16) into the K-major A tile of the second product
       const int r = threadIdx.x;
 #pragma unroll
@@ -506,6 +518,246 @@ __global__ void k_tl_finish(TreeAttnArgs a) {
   reinterpret_cast<uint2*>(a.O)[i] = w;
 }
 
+// ---- backward, leaf by leaf -------------------------------------------------
+//
+// Same leaf lists as the forward.  Per leaf CTA and chunk of up to 128 rows:
+//   S = Q . K_leaf^T, dP = dO . V_leaf^T                   (tcgen05, TMEM cols 0..127)
+//   P = exp(S - LSE), dS = P * (dP - delta)                (bf16 tiles in smem)
+//   dV_leaf^T += dO^T . P,  dK_leaf^T += Q^T . dS          (TMEM accumulators, all chunks)
+//   dQ_rows = dS . K_leaf                                  (TMEM cols 0..127, fp32 red-adds)
+// A leaf owns its keys, so dK/dV of the leaf are stored once, without atomics.
+// delta = rowsum(dO * O) and the base-2 LSE come from k_tlb_rows.
+
+struct TreeBwdArgs {
+  TreeAttnArgs f;              // lists, Q/K/V, positions, sizes
+  const __nv_bfloat16* O;
+  const __nv_bfloat16* dO;
+  const float* LSE;
+  float* delta;                // [T][Hq]
+  float* lse2b;                // [T][Hq]
+  float* dQ;
+  float* dK;
+  float* dV;
+  float scale;
+};
+
+__global__ void k_tlb_rows(TreeBwdArgs b) {
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // one warp per row
+  const int lane = threadIdx.x & 31;
+  if (row >= b.f.T * b.f.Hq) return;
+  float v[4], o[4];
+  load4(b.dO + row * kDim + lane * 4, v);
+  load4(b.O + row * kDim + lane * 4, o);
+  float x = v[0] * o[0] + v[1] * o[1] + v[2] * o[2] + v[3] * o[3];
+#pragma unroll
+  for (int s = 16; s; s >>= 1) x += __shfl_xor_sync(0xffffffffu, x, s);
+  if (lane == 0) {
+    b.delta[row] = x;
+    const float L = b.LSE[row];
+    b.lse2b[row] = L == -INFINITY ? INFINITY : L * 1.44269504088896340736f;
+  }
+}
+
+__global__ void __launch_bounds__(kTL) k_tlb_leaf(TreeBwdArgs b) {
+  extern __shared__ char smem_raw[];
+  __shared__ int32_t s_pos[kLeafKeys];
+  __shared__ __align__(8) uint64_t s_mbar;
+  __shared__ uint32_t s_taddr;
+  const TreeAttnArgs& a = b.f;
+  const int64_t g = blockIdx.y, leaf = blockIdx.x;
+  const int32_t* offg = a.off + g * (a.NL + 1);
+  const int64_t e_lo = offg[leaf], n_ent = offg[leaf + 1] - e_lo;
+  if (n_ent == 0) return;
+  const int32_t* ent = a.ent + g * a.T * a.B + e_lo;
+  char* base = align1024(smem_raw);
+  const uint32_t sQ = smem_u32(base);            // 32 KB  rows x d
+  const uint32_t sdO = sQ + kTL * 256;           // 32 KB  rows x d
+  const uint32_t sK = sdO + kTL * 256;           // 16 KB  keys x d
+  const uint32_t sV = sK + kLeafKeys * 256;      // 16 KB  keys x d
+  const uint32_t sP = sV + kLeafKeys * 256;      // 16 KB  rows x keys
+  const uint32_t sdS = sP + kTL * 128;           // 16 KB  rows x keys
+  char* gP = base + (sP - sQ);
+  char* gdS = base + (sdS - sQ);
+  const uint32_t mbar = smem_u32(&s_mbar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(mbar));
+    asm volatile("fence.mbarrier_init.release.cluster;");
+  }
+  int64_t tq;
+  int rank, h;
+  row_of(a, ent, n_ent, 0, tq, rank, h);
+  int64_t row = tq >= 0 ? tq * a.Hq + g * a.G + h : -1;
+  float dlt = row >= 0 ? b.delta[row] : 0.f, lse = row >= 0 ? b.lse2b[row] : INFINITY;
+  if (threadIdx.x < kLeafKeys) s_pos[threadIdx.x] = a.leaf_index[g * a.n_tree + leaf * kLeafKeys + threadIdx.x];
+  __syncthreads();
+  {
+    LeafSmem ls;
+    ls.sK = sK;
+    ls.sV = sV;
+    ls.pos = s_pos;
+    copy_leaf(a, g, ls, true);
+  }
+  alloc_tmem(&s_taddr, 256);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_taddr;
+  const int warp = threadIdx.x >> 5;
+  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  uint32_t phase = 0;
+  bool ok = true;
+  bool first = true;
+  const int64_t qp = 0;
+  (void)qp;
+  for (int64_t e0 = 0; e0 < n_ent && ok; e0 += kTL / a.G) {
+    if (e0 > 0) {
+      row_of(a, ent, n_ent, e0, tq, rank, h);
+      row = tq >= 0 ? tq * a.Hq + g * a.G + h : -1;
+      dlt = row >= 0 ? b.delta[row] : 0.f;
+      lse = row >= 0 ? b.lse2b[row] : INFINITY;
+    }
+    if (row >= 0) {
+      const __nv_bfloat16* q = a.Q + row * kDim;
+      const __nv_bfloat16* go = b.dO + row * kDim;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) {
+        cp_async16(sQ + sw128_off(threadIdx.x, c, kTL * 128), q + c * 8);
+        cp_async16(sdO + sw128_off(threadIdx.x, c, kTL * 128), go + c * 8);
+      }
+    }
+    cp_async_wait_all();
+    fence_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      constexpr uint32_t id_s = idesc_bf16(128, 64, false, false);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ko = (uint32_t)(kk & 3) * 32;
+        tc_mma(tmem, sdesc_sw128(sQ + (kk >> 2) * (kTL * 128) + ko, 16, 1024),
+               sdesc_sw128(sK + (kk >> 2) * (kLeafKeys * 128) + ko, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t ko = (uint32_t)(kk & 3) * 32;
+        tc_mma(tmem + 64, sdesc_sw128(sdO + (kk >> 2) * (kTL * 128) + ko, 16, 1024),
+               sdesc_sw128(sV + (kk >> 2) * (kLeafKeys * 128) + ko, 16, 1024), id_s, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(mbar);
+    }
+    ok = __syncthreads_and(mbar_wait(mbar, phase));
+    phase ^= 1;
+    tc_fence_after();
+    if (!ok) {
+      set_status(a.status, LSA_ERR_TIMEOUT);
+      break;
+    }
+    {
+      const int64_t qpos = (a.causal && tq >= 0) ? (int64_t)a.q_pos[tq] : INT64_MAX;
+      const int r = threadIdx.x;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float sv[32], dv[32];
+        tmem_ld32(tmem + lane_base + half * 32, sv);
+        tmem_ld32(tmem + lane_base + 64 + half * 32, dv);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t wp[4], wd[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float p2[2], d2[2];
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+              const int i = c * 8 + 2 * q + u, key = half * 32 + i;
+              const bool vis = row >= 0 && (int64_t)s_pos[key] <= qpos;
+              const float p = vis ? exp2f(sv[i] * a.scale_log2 - lse) : 0.f;
+              p2[u] = p;
+              d2[u] = p * (dv[i] - dlt);
+            }
+            __nv_bfloat162 bp = __floats2bfloat162_rn(p2[0], p2[1]);
+            __nv_bfloat162 bd = __floats2bfloat162_rn(d2[0], d2[1]);
+            wp[q] = *reinterpret_cast<uint32_t*>(&bp);
+            wd[q] = *reinterpret_cast<uint32_t*>(&bd);
+          }
+          const int chunk = half * 4 + c;
+          const uint32_t off = (r >> 3) * 1024 + (r & 7) * 128 + ((chunk ^ (r & 7)) << 4);
+          *reinterpret_cast<uint4*>(gP + off) = make_uint4(wp[0], wp[1], wp[2], wp[3]);
+          *reinterpret_cast<uint4*>(gdS + off) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        }
+      }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      // dV^T (d x keys) += dO^T . P ; dK^T += Q^T . dS   (both operands MN-major)
+      constexpr uint32_t id_t = idesc_bf16(128, 64, true, true);
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t acc = (first && kk == 0) ? 0u : 1u;
+        tc_mma(tmem + 128, sdesc_sw128(sdO + kk * 2048, kTL * 128, 1024), sdesc_sw128(sP + kk * 2048, kTL * 128, 1024),
+               id_t, acc);
+        tc_mma(tmem + 192, sdesc_sw128(sQ + kk * 2048, kTL * 128, 1024), sdesc_sw128(sdS + kk * 2048, kTL * 128, 1024),
+               id_t, acc);
+      }
+      // dQ rows (rows x d) = dS . K_leaf   (dS K-major, K_leaf as MN-major B)
+      constexpr uint32_t id_q = idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        tc_mma(tmem, sdesc_sw128(sdS + kk * 32, 16, 1024), sdesc_sw128(sK + kk * 2048, kLeafKeys * 128, 1024),
+               id_q, kk > 0 ? 1u : 0u);
+      tc_commit(mbar);
+    }
+    first = false;
+    ok = __syncthreads_and(mbar_wait(mbar, phase));
+    phase ^= 1;
+    tc_fence_after();
+    if (!ok) {
+      set_status(a.status, LSA_ERR_TIMEOUT);
+      break;
+    }
+    {
+      float* dst = row >= 0 ? b.dQ + row * kDim : nullptr;
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        float v[32];
+        tmem_ld32(tmem + lane_base + part * 32, v);
+        if (dst) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            red_add_v4(dst + part * 32 + i, v[i] * b.scale, v[i + 1] * b.scale, v[i + 2] * b.scale,
+                       v[i + 3] * b.scale);
+        }
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  if (ok) {
+    // lane t holds dimension t of every key's gradient: store the leaf's rows once
+    tc_fence_after();
+    float* dKh = b.dK + g * a.n_cap * kDim;
+    float* dVh = b.dV + g * a.n_cap * kDim;
+    const int t = threadIdx.x;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float vv[32], kv[32];
+      tmem_ld32(tmem + lane_base + 128 + half * 32, vv);
+      tmem_ld32(tmem + lane_base + 192 + half * 32, kv);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int64_t j = s_pos[half * 32 + i];
+        dVh[j * kDim + t] = vv[i];
+        dKh[j * kDim + t] = kv[i] * b.scale;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  free_tmem(tmem, 256);
+}
+
 // expand leaves into key lists (fallback shapes)
 __global__ void k_tl_expand(const int32_t* leaves, const int32_t* leaf_index, int64_t H, int64_t T, int B, int leaf,
                             int64_t n_tree, int32_t* idx) {
@@ -519,6 +771,7 @@ __global__ void k_tl_expand(const int32_t* leaves, const int32_t* leaf_index, in
 
 constexpr size_t kStatsSmem = 1024 + kTL * 256 + kLeafKeys * 256;
 constexpr size_t kOutSmem = 1024 + kTL * 256 + 2 * kLeafKeys * 256;
+constexpr size_t kBwdSmem = 1024 + 2 * kTL * 256 + 2 * kLeafKeys * 256 + 2 * kTL * 128;
 
 }  // namespace
 
@@ -527,6 +780,12 @@ size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, 
   if (!fast) return al((size_t)H * T * B * leaf * 4);
   return al(H * NL * 4) + al(H * (NL + 1) * 4) + al((size_t)H * T * B * 4) + al((size_t)T * Hq * B * 8) +
          al((size_t)T * Hq * 4) + al((size_t)T * Hq * d * 4);
+}
+
+size_t tree_attn_bwd_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast) {
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  if (!fast) return al((size_t)H * T * B * leaf * 4);
+  return al(H * NL * 4) + al(H * (NL + 1) * 4) + al((size_t)H * T * B * 4) + 2 * al((size_t)T * Hq * 4);
 }
 
 bool tree_attn_fast_path(int dtype, int d, int G, int leaf) {
@@ -588,6 +847,67 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
   k_tl_lse<<<(unsigned)ceil_div(c.T * c.Hq, 256), 256, 0, st>>>(a);
   k_tl_out<<<grid, kTL, kOutSmem, st>>>(a);
   k_tl_finish<<<(unsigned)ceil_div(c.T * c.Hq * (kDim / 4), 256), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t run_tree_attn_bwd(const TreeAttnCall& c, const void* O, const float* LSE, const void* dO, float* dQ,
+                              float* dK, float* dV, cudaStream_t st) {
+  const int G = c.Hq / c.H;
+  const bool fast = tree_attn_fast_path(c.dtype, c.d, G, c.leaf);
+  char* ws = static_cast<char*>(c.workspace);
+  auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
+  cudaError_t e;
+  const size_t kv_bytes = (size_t)c.H * c.n_cap * c.d * sizeof(float);
+  if ((e = cudaMemsetAsync(dK, 0, kv_bytes, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(dV, 0, kv_bytes, st)) != cudaSuccess) return e;
+  if (c.T == 0) return cudaSuccess;
+  if (!fast) {
+    int32_t* idx = reinterpret_cast<int32_t*>(ws);
+    const int64_t total = (int64_t)c.H * c.T * c.B * c.leaf;
+    k_tl_expand<<<(unsigned)ceil_div(total, 256), 256, 0, st>>>(c.leaves, c.leaf_index, c.H, c.T, c.B, c.leaf,
+                                                                c.n_tree, idx);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.Q = c.Q; a.K = c.K; a.V = c.V; a.idx = idx; a.q_pos = c.q_pos; a.O = const_cast<void*>(O);
+    a.LSE = const_cast<float*>(LSE); a.dO = dO; a.dQ = dQ; a.dK = dK; a.dV = dV; a.status = c.status;
+    a.T = c.T; a.n_cap = c.n_cap; a.Hq = c.Hq; a.Hkv = c.H; a.G = G; a.d = c.d; a.K_sel = c.B * c.leaf;
+    a.causal = c.causal; a.nsplit = 1; a.keys_per_split = (int32_t)((a.K_sel + 15) / 16 * 16);
+    a.scale = c.scale; a.scale_log2 = c.scale * 1.44269504088896340736f;
+    return run_attn_bwd(a, c.dtype, st);
+  }
+  TreeBwdArgs b;
+  memset(&b, 0, sizeof(b));
+  TreeAttnArgs& a = b.f;
+  a.Q = static_cast<const __nv_bfloat16*>(c.Q);
+  a.K = static_cast<const __nv_bfloat16*>(c.K);
+  a.V = static_cast<const __nv_bfloat16*>(c.V);
+  a.leaf_index = c.leaf_index;
+  a.leaves = c.leaves;
+  a.q_pos = c.q_pos;
+  size_t o = 0;
+  a.cnt = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.NL * 4);
+  a.off = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * (c.NL + 1) * 4);
+  a.ent = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * c.B * 4);
+  b.delta = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);
+  b.lse2b = reinterpret_cast<float*>(ws + o);
+  a.status = c.status;
+  a.T = c.T; a.n_cap = c.n_cap; a.n_tree = c.n_tree; a.NL = c.NL;
+  a.Hq = c.Hq; a.H = c.H; a.G = G; a.B = c.B; a.causal = c.causal;
+  a.scale_log2 = c.scale * 1.44269504088896340736f;
+  b.O = static_cast<const __nv_bfloat16*>(O);
+  b.dO = static_cast<const __nv_bfloat16*>(dO);
+  b.LSE = LSE;
+  b.dQ = dQ; b.dK = dK; b.dV = dV; b.scale = c.scale;
+  const int64_t n_sel = (int64_t)c.H * c.T * c.B;
+  if ((e = cudaMemsetAsync(a.cnt, 0, (size_t)c.H * c.NL * 4, st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(dQ, 0, (size_t)c.T * c.Hq * kDim * 4, st)) != cudaSuccess) return e;
+  k_tl_count<<<(unsigned)ceil_div(n_sel, 256), 256, 0, st>>>(a);
+  k_tl_scan<<<(unsigned)c.H, 1024, 0, st>>>(a);
+  k_tl_fill<<<(unsigned)ceil_div(n_sel, 256), 256, 0, st>>>(a);
+  k_tlb_rows<<<(unsigned)ceil_div(c.T * c.Hq * 32, 256), 256, 0, st>>>(b);
+  cudaFuncSetAttribute(k_tlb_leaf, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem);
+  k_tlb_leaf<<<dim3((unsigned)c.NL, (unsigned)c.H), kTL, kBwdSmem, st>>>(b);
   return cudaGetLastError();
 }
 

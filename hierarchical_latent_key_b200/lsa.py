@@ -68,6 +68,9 @@ def _load():
         "lsa_sparse_attn_noalloc": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i64,
                                                    i64, f32, P, P, P, P]),
         "lsa_kv_append": (ctypes.c_int, [P, P, i32, i64, i32, i32, i64, P, P, P]),
+        "lsa_tree_attn_bwd_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
+        "lsa_tree_attn_bwd": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, P, P, P, i32, P, i32, f32,
+                                             P, P, P, P, sz, P, P]),
         "lsa_status_clear": (ctypes.c_int, [P, P]),
         "lsa_status_check": (ctypes.c_int, [P, P, ctypes.POINTER(i32)]),
     }
@@ -340,6 +343,41 @@ def tree_attn(tree: Tree, Q, K, V, leaves, q_pos=None, causal=False, scale=None,
     if check:
         check_status(st, "lsa_tree_attn")
     return O, LSE
+
+
+def lsa_tree_attn_bwd_workspace_bytes(desc, T, Hq, d, dtype, n_leaves) -> int:
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_tree_attn_bwd_workspace_bytes(ctypes.byref(desc), T, Hq, d, _DTYPE[dtype], n_leaves,
+                                                  ctypes.byref(n)), "lsa_tree_attn_bwd_workspace_bytes")
+    return int(n.value)
+
+
+def lsa_tree_attn_bwd(desc, tree_mem, Q, K, V, O, LSE, dO, leaves, q_pos, causal, scale, dQ, dK, dV, workspace,
+                      status=None, stream=None):
+    T, Hq, d = Q.shape
+    ws_n = workspace.numel() * workspace.element_size()
+    _raise(_lib.lsa_tree_attn_bwd(ctypes.byref(desc), _ptr(tree_mem), _ptr(Q), T, Hq, _ptr(K), _ptr(V), K.shape[1],
+                                  d, _dtype(Q), _ptr(O), _ptr(LSE), _ptr(dO), _ptr(leaves), leaves.shape[-1],
+                                  _ptr(q_pos), int(bool(causal)), float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                  _ptr(workspace), ws_n, _ptr(status), _stream(stream, Q)), "lsa_tree_attn_bwd")
+
+
+def tree_attn_bwd(tree: Tree, Q, K, V, O, LSE, dO, leaves, q_pos=None, causal=False, scale=None, workspace=None,
+                  status=None, check=True):
+    T, Hq, d = Q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    need = lsa_tree_attn_bwd_workspace_bytes(tree.desc, T, Hq, d, Q.dtype, leaves.shape[-1])
+    if workspace is None or workspace.numel() * workspace.element_size() < need:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+    dQ = torch.empty(T, Hq, d, dtype=torch.float32, device=Q.device)
+    dK = torch.empty(K.shape, dtype=torch.float32, device=Q.device)
+    dV = torch.empty(V.shape, dtype=torch.float32, device=Q.device)
+    st = _new_status(Q.device) if status is None else status
+    lsa_tree_attn_bwd(tree.desc, tree.mem, Q, K, V, O, LSE, dO, leaves, q_pos, causal, scale, dQ, dK, dV,
+                      workspace, st)
+    if check:
+        check_status(st, "lsa_tree_attn_bwd")
+    return dQ, dK, dV
 
 
 def sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos=None, causal=False, tail=(0, 0), scale=None, status=None,

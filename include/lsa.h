@@ -203,6 +203,23 @@ int lsa_tree_attn(const lsa_tree_desc *tree, const void *tree_mem, const void *Q
                   int32_t causal, float scale, void *O, float *LSE, void *workspace,
                   size_t workspace_bytes, int32_t *status, void *stream);
 
+/* Host only.  Workspace bytes lsa_tree_attn_bwd needs. */
+int lsa_tree_attn_bwd_workspace_bytes(const lsa_tree_desc *tree, int32_t T, int32_t Hq, int32_t d,
+                                      int32_t dtype, int32_t n_leaves, size_t *bytes);
+
+/* Backward of lsa_tree_attn for a fixed selection (the gradient of the same
+ * attention as lsa_sparse_attn_bwd, with the same outputs and conventions):
+ * computed leaf by leaf on the tensor cores, P and dS = P * (dP - rowsum(dO * O))
+ * rounded to bf16 for the products; each leaf's dK and dV rows are written once
+ * (a leaf owns its keys), dQ accumulates with fp32 red-adds (summation order not
+ * fixed).  dQ, dK, dV are overwritten. */
+int lsa_tree_attn_bwd(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, int32_t T,
+                      int32_t Hq, const void *K, const void *V, int64_t n_cap, int32_t d,
+                      int32_t dtype, const void *O, const float *LSE, const void *dO,
+                      const int32_t *leaves, int32_t n_leaves, const int32_t *q_pos, int32_t causal,
+                      float scale, float *dQ, float *dK, float *dV, void *workspace,
+                      size_t workspace_bytes, int32_t *status, void *stream);
+
 /* Backward of lsa_sparse_attn for a fixed selection (same arguments), given the
  * forward's O and LSE and the upstream gradient dO ([T][Hq][d], dtype of Q).
  * Outputs (float): dQ [T][Hq][d]; dK, dV [n_heads][n_cap][d], overwritten (zero

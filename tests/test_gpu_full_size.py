@@ -161,14 +161,14 @@ def test_decode_10m_full(lsa):
 
 
 def test_train_128k_full(lsa):
-    """131072-token causal layer: build, select, tree-attention forward, backward; oracle on
+    """131072-token causal layer: build, select, tree-attention forward and backward; oracle on
     sampled queries (dQ, O) and sampled keys (dK, dV from every query that selected them)."""
     cfg = configs.get("train_128k")
     case = cfg.case(DEV)
     tree = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
     idx, leaves = lsa.select(tree, case.Q, case.W, cfg.beam, case.q_pos, leaves=True)
     O, LSE = lsa.tree_attn(tree, case.Q, case.K, case.V, leaves, case.q_pos, causal=True)
-    dQ, dK, dV = lsa.sparse_attn_bwd(case.Q, case.K, case.V, O, LSE, case.dO, idx, case.q_pos, True)
+    dQ, dK, dV = lsa.tree_attn_bwd(tree, case.Q, case.K, case.V, O, LSE, case.dO, leaves, case.q_pos, causal=True)
     torch.cuda.synchronize()
     rng = np.random.default_rng(3)
     h = 1

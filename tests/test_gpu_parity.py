@@ -286,3 +286,28 @@ def test_kv_append_writes_rows(lsa):
         assert torch.equal(K, K0) and torch.equal(V, V0)
     with pytest.raises(lsa.LsaError):
         lsa.lsa_kv_append(K, V, 50, kr, vr)
+
+
+@pytest.mark.parametrize("G", [4, 1])
+def test_tree_attention_backward(lsa, G):
+    """Leaf-by-leaf tensor-core backward = oracle gradient (and = the key-list backward)."""
+    cfg = configs.get("train_128k").scaled(n=8192, T=8192, branching=(8, 4, 4), beam=(4, 8, 8), Hkv=2, Hq=2 * G,
+                                           comps=64)
+    case = cfg.case("cpu", seed=21 + G)
+    g = _to(case)
+    tree = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select(tree, g["Q"], g["W"], cfg.beam, g["q_pos"], leaves=True)
+    O, LSE = lsa.tree_attn(tree, g["Q"], g["K"], g["V"], leaves, g["q_pos"], causal=True)
+    dQ, dK, dV = lsa.tree_attn_bwd(tree, g["Q"], g["K"], g["V"], O, LSE, g["dO"], leaves, g["q_pos"], causal=True)
+    dQ2, dK2, dV2 = lsa.sparse_attn_bwd(g["Q"], g["K"], g["V"], O, LSE, g["dO"], idx, g["q_pos"], True)
+    torch.cuda.synchronize()
+    qp = case.q_pos.numpy()
+    for h in range(cfg.Hkv):
+        sl = slice(h * G, (h + 1) * G)
+        oQ, oK, oV = orc.attn_bwd(case.Q[:, sl], case.K[h], case.V[h], idx[h].cpu(), case.dO[:, sl],
+                                  q_pos=qp, causal=True)
+        for name, got, want in (("dQ", dQ[:, sl], oQ), ("dK", dK[h], oK), ("dV", dV[h], oV)):
+            _check_grad(name, got.cpu().numpy(), want)
+    for a, b in ((dQ, dQ2), (dK, dK2), (dV, dV2)):
+        ref = b.abs().max().item()
+        assert (a - b).abs().max().item() <= 2e-2 * ref
