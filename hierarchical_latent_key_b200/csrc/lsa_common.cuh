@@ -49,6 +49,16 @@ __device__ __forceinline__ void load2(const __nv_bfloat16* p, float (&v)[2]) {
   v[0] = f.x; v[1] = f.y;
 }
 
+// Two consecutive elements through a generic pointer (global or shared memory).
+__device__ __forceinline__ void load2_generic(const float* p, float (&v)[2]) {
+  const float2 t = *reinterpret_cast<const float2*>(p);
+  v[0] = t.x; v[1] = t.y;
+}
+__device__ __forceinline__ void load2_generic(const __nv_bfloat16* p, float (&v)[2]) {
+  const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+  v[0] = f.x; v[1] = f.y;
+}
+
 // Order-preserving map of a float to uint32 (larger float -> larger uint);
 // -0.0 is folded onto +0.0 so the two never order differently.
 __device__ __forceinline__ uint32_t orderable(float f) {

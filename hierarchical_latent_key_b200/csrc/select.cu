@@ -8,14 +8,15 @@
 // attention works": hierarchical search with a fixed budget per level, then a
 // fixed number of original keys taken from the chosen clusters.
 //
-// One CTA (4 warps) per (query t, KV group g).  Scores are fp32 inner products
-// of the group's latent query with fp32 centroids (exact enough that ordering
+// One warp per (query t, KV group g).  Scores are fp32 inner products of the
+// group's latent query with fp32 centroids (exact enough that ordering
 // decisions only differ from an fp64 evaluation inside a ~1e-6 relative band).
 // Candidates are ranked by a packed 64-bit key (orderable score, ~node id) so a
-// descending sort gives (score desc, node id asc).  All threads score candidates
-// into shared memory, each warp sorts a slice of 128 in registers (bitonic
-// network, shuffles across lanes), and one warp sorts the concatenated per-warp
-// heads: four CTA barriers per level instead of one per sorting-network stage.
+// descending sort gives (score desc, node id asc).  A level's candidates (at
+// most beam * branching <= 512) are scored by lane groups that read whole
+// centroid rows with coalesced loads, then sorted in registers by a warp-wide
+// bitonic network (shuffles across lanes); the walk needs no CTA barrier, so
+// many walks are in flight per SM to hide memory latency.
 
 #include <climits>
 
@@ -24,7 +25,12 @@
 
 namespace lsa {
 
-constexpr int kSelThreads = 128;   // 4 warps x 128 candidates >= beam * branching (32 * 16)
+constexpr int kSelWarps = 8;       // (query, group) units per CTA, one warp each
+constexpr int kSelMaxE = 16;       // sort width per lane: beam * branching <= 32 * 16
+constexpr int kWideWarps = 16;     // warps of the small-batch kernel: 32 * 16 candidate slots
+// Below this many (query, group) units the warp-per-unit kernel cannot fill the
+// 148 SMs (8 units per CTA), and one CTA per unit is used instead.
+constexpr int64_t kWideUnits = 148 * 8;
 
 // Bitonic sort (descending) of 32*E keys held in registers, E per lane; element
 // index i = lane * E + e.  Pairs closer than E sit in one lane; farther pairs are
@@ -84,158 +90,342 @@ __device__ __forceinline__ int emit_kept(const unsigned long long (&v)[E], int B
   return cnt;
 }
 
+// Shared-memory slot of sorted-list element i (lane i / E, register i % E): the
+// register index is XORed with the lane so that the E-strided reads of one
+// register index by the 32 lanes spread over all banks.
 template <int E>
-__device__ __forceinline__ int merge_sorted(const unsigned long long* src, int m, int B, int32_t* kept) {
-  const int lane = threadIdx.x & 31;
+__device__ __forceinline__ int key_slot(int i) {
+  const int ln = i / E, e = i % E;
+  return ln * E + (e ^ (ln % E));
+}
+
+// Centroid rows are scored by groups of LPR lanes; each lane holds F float4
+// pieces of the latent query, so one warp-wide load covers 32 / LPR whole rows.
+template <int R>
+struct RowSplit {
+  static constexpr int LPR = R >= 32 ? 8 : 4;
+  static constexpr int F = R / (4 * LPR);
+  static constexpr int RPI = 32 / LPR;
+};
+
+// One level of the walk: score the ncand children of the kept parents (all nodes
+// on level 0), write their keys to s_key, sort them in registers (E per lane)
+// and keep the first beam[l].  Returns the number of real candidates kept.
+template <int R, int E>
+__device__ __forceinline__ int level_pass(const SelectArgs& a, int l, int ncand, const float* cent,
+                                          const int32_t* mpos, bool all_eligible, int64_t qpos,
+                                          const float4 (&lat)[RowSplit<R>::F], const int32_t* kept, int b,
+                                          unsigned long long* s_key, int32_t* next, bool& bad) {
+  using RS = RowSplit<R>;
+  constexpr int U = 4;   // rows in flight per lane group
+  const int lane = threadIdx.x & 31, sub = lane % RS::LPR, grp = lane / RS::LPR;
+  for (int c0 = 0; c0 < ncand; c0 += RS::RPI * U) {
+    float4 x[U][RS::F];
+    bool ok[U];
+    int64_t id[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int c = c0 + u * RS::RPI + grp;
+      ok[u] = c < ncand;
+      id[u] = 0;
+      if (ok[u]) {
+        id[u] = l == 0 ? c : (int64_t)kept[c / b] * b + (c % b);
+        ok[u] = all_eligible || (int64_t)__ldg(&mpos[id[u]]) <= qpos;
+      }
+      const float4* cr = reinterpret_cast<const float4*>(cent + id[u] * R);
+#pragma unroll
+      for (int f = 0; f < RS::F; ++f) x[u][f] = ok[u] ? __ldg(&cr[f * RS::LPR + sub]) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      float sc = 0.f;
+#pragma unroll
+      for (int f = 0; f < RS::F; ++f) {
+        sc = fmaf(lat[f].x, x[u][f].x, sc);
+        sc = fmaf(lat[f].y, x[u][f].y, sc);
+        sc = fmaf(lat[f].z, x[u][f].z, sc);
+        sc = fmaf(lat[f].w, x[u][f].w, sc);
+      }
+#pragma unroll
+      for (int o = 1; o < RS::LPR; o <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+      const int c = c0 + u * RS::RPI + grp;
+      if (sub == 0 && c < ncand) {
+        unsigned long long key = 0ull;
+        if (ok[u]) {
+          if (isnan(sc)) bad = true;
+          else key = ((unsigned long long)orderable(sc) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)id[u]);
+        }
+        s_key[key_slot<E>(c)] = key;
+      }
+    }
+  }
+  __syncwarp();
   unsigned long long v[E];
 #pragma unroll
   for (int e = 0; e < E; ++e) {
     const int i = lane * E + e;
-    v[e] = i < m ? src[i] : 0ull;
+    v[e] = i < ncand ? s_key[key_slot<E>(i)] : 0ull;
   }
   warp_sort_desc<E>(v);
-  return emit_kept<E>(v, B, kept);
+  return emit_kept<E>(v, a.beam[l], next);
 }
 
+// Latent query of (t, g), computed by one warp: the group query (mean of the G
+// query heads) times W[g] (Wg: global or shared memory).  A lane owns columns (2 kp, 2 kp + 1) over the rows
+// j = js, js + JS, ...; the JS row slices are summed by shuffles.  Both select
+// kernels use this routine, so a query's latent (and its walk) does not depend
+// on the batch it is selected in.
 template <typename T, int R, int DK>
-__global__ void __launch_bounds__(kSelThreads, 4) k_select(SelectArgs a) {
-  __shared__ float s_q[DK];
-  __shared__ float s_part[kSelThreads];
-  __shared__ __align__(16) T s_w[DK * R];
-  __shared__ __align__(16) float s_lat[R];
-  __shared__ unsigned long long s_cand[(kSelThreads / 32) * 128];
-  __shared__ unsigned long long s_merge[(kSelThreads / 32) * LSA_MAX_BEAM];
-  __shared__ int32_t s_kept[LSA_MAX_BEAM];
-  __shared__ int32_t s_next[LSA_MAX_BEAM];
-  __shared__ int s_nkept;
-  const int64_t t = blockIdx.x;
-  const int g = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__device__ __forceinline__ void latent_query(const SelectArgs& a, int64_t t, int g, const T* Wg, float* s_q,
+                                             float* s_lat) {
+  const int lane = threadIdx.x & 31;
   const T* Q = static_cast<const T*>(a.Q);
-
-  // group query: mean of the G query heads of the group
-  for (int j = tid; j < DK; j += kSelThreads) {
-    float s = 0.f;
-    for (int i = 0; i < a.G; ++i) s += to_f32(Q[(t * a.Hq + (int64_t)g * a.G + i) * DK + j]);
-    s_q[j] = s / (float)a.G;
+  for (int j = lane; j < DK; j += 32) {
+    float sum = 0.f;
+    for (int i = 0; i < a.G; ++i) sum += to_f32(Q[(t * a.Hq + (int64_t)g * a.G + i) * DK + j]);
+    s_q[j] = sum / (float)a.G;
   }
-  __syncthreads();
-  // latent query = group query . W[g]: W[g] is staged in shared memory with
-  // 16-byte loads (one memory round trip), then thread (k, part) sums a slice of d
-  {
-    constexpr int PARTS = kSelThreads / R;
-    constexpr int SPAN = DK / PARTS;
-    constexpr int VEC = 16 / sizeof(T);
-    const T* W = static_cast<const T*>(a.W) + (int64_t)g * DK * R;
+  __syncwarp();
+  constexpr int JS = 64 / R;
+  const int kp = lane % (R / 2), js = lane / (R / 2);
+  const T* W = Wg + 2 * kp;
+  float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll 8
+  for (int j = js; j < DK; j += JS) {
+    float w[2];
+    load2_generic(W + (int64_t)j * R, w);
+    const float qj = s_q[j];
+    acc0 = fmaf(qj, w[0], acc0);
+    acc1 = fmaf(qj, w[1], acc1);
+  }
 #pragma unroll
-    for (int i = tid * VEC; i < DK * R; i += kSelThreads * VEC)
-      *reinterpret_cast<uint4*>(&s_w[i]) = __ldg(reinterpret_cast<const uint4*>(W + i));
-    __syncthreads();
-    const int k = tid % R, p = tid / R;
-    float acc = 0.f;
-#pragma unroll 16
-    for (int j = p * SPAN; j < (p + 1) * SPAN; ++j) acc = fmaf(s_q[j], to_f32(s_w[j * R + k]), acc);
-    s_part[tid] = acc;
-    __syncthreads();
-    if (tid < R) {
-      float v = 0.f;
-      for (int q = 0; q < PARTS; ++q) v += s_part[q * R + tid];
-      s_lat[tid] = v;
-      if (a.qlat_out) a.qlat_out[(t * a.Hkv + g) * R + tid] = v;
-    }
-    __syncthreads();
+  for (int o = R / 2; o < 32; o <<= 1) {
+    acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
+    acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
   }
+  if (js == 0) {
+    s_lat[2 * kp] = acc0;
+    s_lat[2 * kp + 1] = acc1;
+    if (a.qlat_out) {
+      a.qlat_out[(t * a.Hkv + g) * R + 2 * kp] = acc0;
+      a.qlat_out[(t * a.Hkv + g) * R + 2 * kp + 1] = acc1;
+    }
+  }
+  __syncwarp();
+}
+
+// One warp per (query t, KV group g), kSelWarps queries of one group per CTA.
+// The walk synchronises only its own warp.
+template <typename T, int R, int DK>
+__global__ void __launch_bounds__(kSelWarps * 32, 3) k_select(SelectArgs a) {
+  using RS = RowSplit<R>;
+  __shared__ unsigned long long s_key[kSelWarps][32 * kSelMaxE];
+  __shared__ float s_q[kSelWarps][DK];
+  __shared__ __align__(16) float s_lat[kSelWarps][R];
+  __shared__ int32_t s_kept[kSelWarps][2][LSA_MAX_BEAM];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = blockIdx.y;
+  const int64_t t = (int64_t)blockIdx.x * kSelWarps + warp;
+  if (t >= a.T) return;
+  latent_query<T, R, DK>(a, t, g, static_cast<const T*>(a.W) + (int64_t)g * DK * R, s_q[warp], s_lat[warp]);
+  float4 lat[RS::F];
+#pragma unroll
+  for (int f = 0; f < RS::F; ++f)
+    lat[f] = reinterpret_cast<const float4*>(s_lat[warp])[f * RS::LPR + lane % RS::LPR];
   const int64_t qpos = a.q_pos ? (int64_t)a.q_pos[t] : (int64_t)LLONG_MAX;
   // a query at or past the last indexed position sees every node (decode): no
   // per-node eligibility load is needed
   const bool all_eligible = qpos >= a.n_tree - 1;
+  unsigned long long* keys = s_key[warp];
   int ncand = (int)a.nodes[0];
   int n_kept = 0;
+  int cur = 0;
+  bool bad = false;
   for (int l = 0; l < a.levels; ++l) {
     const int b = a.branching[l];
     const float* cent = reinterpret_cast<const float*>(a.tree + a.off_c[l]) + (int64_t)g * a.nodes[l] * R;
     const int32_t* mpos = reinterpret_cast<const int32_t*>(a.tree + a.off_m[l]) + (int64_t)g * a.nodes[l];
-    // all threads score (one candidate each per pass) into shared memory; then each
-    // warp sorts a slice of 128 candidates (4 per lane) in registers
-    const int nw_act = (ncand + 127) / 128;
-    constexpr int KW = LSA_MAX_BEAM;                    // per-warp list kept for the merge
-    bool bad = false;
-    for (int i = tid; i < nw_act * 128; i += kSelThreads) {
-      unsigned long long key = 0ull;
-      if (i < ncand) {
-        const int64_t id = l == 0 ? i : (int64_t)s_kept[i / b] * b + (i % b);
-        if (all_eligible || (int64_t)__ldg(&mpos[id]) <= qpos) {
-          const float4* cr = reinterpret_cast<const float4*>(cent + id * R);
-          float sc = 0.f;
-#pragma unroll
-          for (int k = 0; k < R / 4; ++k) {
-            const float4 c = __ldg(&cr[k]);
-            sc = fmaf(s_lat[4 * k], c.x, sc);
-            sc = fmaf(s_lat[4 * k + 1], c.y, sc);
-            sc = fmaf(s_lat[4 * k + 2], c.z, sc);
-            sc = fmaf(s_lat[4 * k + 3], c.w, sc);
-          }
-          if (isnan(sc)) bad = true;
-          else key = ((unsigned long long)orderable(sc) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)id);
-        }
-      }
-      s_cand[i] = key;
+    const int32_t* kept = s_kept[warp][cur];
+    int32_t* next = s_kept[warp][cur ^ 1];
+    int valid;
+#define LSA_LEVEL(EE) level_pass<R, EE>(a, l, ncand, cent, mpos, all_eligible, qpos, lat, kept, b, keys, next, bad)
+    if (ncand <= 32) valid = LSA_LEVEL(1);
+    else if (ncand <= 64) valid = LSA_LEVEL(2);
+    else if (ncand <= 128) valid = LSA_LEVEL(4);
+    else if (ncand <= 256) valid = LSA_LEVEL(8);
+    else valid = LSA_LEVEL(16);
+#undef LSA_LEVEL
+    __syncwarp();
+    if (a.beam_out && lane < a.beam_max) {
+      const int32_t id = lane < valid ? next[lane] : -1;
+      a.beam_out[(((int64_t)l * a.Hkv + g) * a.T + t) * a.beam_max + lane] = id;
     }
-    __syncthreads();
-    if (warp < nw_act) {
-      unsigned long long v[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) v[e] = s_cand[warp * 128 + lane * 4 + e];
-      warp_sort_desc<4>(v);
-      if (nw_act == 1) {
-        const int cnt = emit_kept<4>(v, a.beam[l], s_next);
-        if (lane == 0) s_nkept = cnt;
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = lane * 4 + e;
-          if (i < KW) s_merge[warp * KW + i] = v[e];
-        }
-      }
-    }
-    if (bad) set_status(a.status, LSA_ERR_NONFINITE);
-    __syncthreads();
-    if (nw_act > 1 && warp == 0) {
-      const int m = nw_act * KW;
-      const int cnt = merge_sorted<4>(s_merge, m, a.beam[l], s_next);   // m <= 4 * 32
-      if (lane == 0) s_nkept = cnt;
-    }
-    __syncthreads();
-    const int valid = s_nkept;
-    if (tid < LSA_MAX_BEAM) {
-      const int32_t id = tid < valid ? s_next[tid] : -1;
-      s_kept[tid] = id;
-      if (a.beam_out && tid < a.beam_max)
-        a.beam_out[(((int64_t)l * a.Hkv + g) * a.T + t) * a.beam_max + tid] = id;
-    }
-    __syncthreads();
     n_kept = valid;
+    cur ^= 1;
     ncand = l + 1 < a.levels ? valid * a.branching[l + 1] : 0;
   }
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, LSA_ERR_NONFINITE);
+  const int32_t* kept = s_kept[warp][cur];
   const int leaf = a.leaf;
   const int B = a.beam[a.levels - 1];
-  if (a.leaves_out && tid < B) a.leaves_out[((int64_t)g * a.T + t) * B + tid] = tid < n_kept ? s_kept[tid] : -1;
+  if (a.leaves_out && lane < B) a.leaves_out[((int64_t)g * a.T + t) * B + lane] = lane < n_kept ? kept[lane] : -1;
   if (a.idx_out) {
     const int64_t K_sel = (int64_t)B * leaf;
     const int32_t* li = reinterpret_cast<const int32_t*>(a.tree + a.off_leaf) + (int64_t)g * a.n_tree;
     int32_t* out = a.idx_out + ((int64_t)g * a.T + t) * K_sel;
-    for (int64_t i = tid; i < K_sel; i += kSelThreads) {
+    for (int64_t i = lane; i < K_sel; i += 32) {
       const int k = (int)(i / leaf), q = (int)(i % leaf);
-      out[i] = k < n_kept ? __ldg(&li[(int64_t)s_kept[k] * leaf + q]) : -1;
+      out[i] = k < n_kept ? __ldg(&li[(int64_t)kept[k] * leaf + q]) : -1;
+    }
+  }
+}
+
+// Small batches (decode): one CTA of kWideWarps warps per (query t, KV group g),
+// so a level's candidates are scored in one or two memory round trips.  Each
+// warp sorts a chunk of 32 keys; chunk lists are then merged pairwise keeping
+// the first 32 (the elementwise max of one descending list and the other one
+// reversed holds the top 32 of both as a bitonic sequence, which five shuffle
+// steps sort).  Scores use the same lane-group sums as k_select.
+template <typename T, int R, int DK>
+__global__ void __launch_bounds__(kWideWarps * 32) k_select_wide(SelectArgs a) {
+  using RS = RowSplit<R>;
+  constexpr int NT = kWideWarps * 32;
+  __shared__ unsigned long long s_key[32 * kWideWarps];
+  __shared__ __align__(16) T s_w[DK * R];
+  __shared__ float s_q[DK];
+  __shared__ __align__(16) float s_lat[R];
+  __shared__ int32_t s_kept[2][LSA_MAX_BEAM];
+  __shared__ int s_valid;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = blockIdx.y;
+  const int64_t t = blockIdx.x;
+  {  // W[g] staged by the whole CTA in one memory round trip
+    constexpr int VEC = 16 / sizeof(T);
+    const T* W = static_cast<const T*>(a.W) + (int64_t)g * DK * R;
+    for (int i = tid * VEC; i < DK * R; i += NT * VEC)
+      *reinterpret_cast<uint4*>(&s_w[i]) = __ldg(reinterpret_cast<const uint4*>(W + i));
+  }
+  __syncthreads();
+  if (warp == 0) latent_query<T, R, DK>(a, t, g, s_w, s_q, s_lat);
+  __syncthreads();
+  float4 lat[RS::F];
+#pragma unroll
+  for (int f = 0; f < RS::F; ++f) lat[f] = reinterpret_cast<const float4*>(s_lat)[f * RS::LPR + lane % RS::LPR];
+  const int64_t qpos = a.q_pos ? (int64_t)a.q_pos[t] : (int64_t)LLONG_MAX;
+  const bool all_eligible = qpos >= a.n_tree - 1;
+  const int sub = lane % RS::LPR, gg = warp * RS::RPI + lane / RS::LPR;
+  constexpr int GROUPS = kWideWarps * RS::RPI;
+  int ncand = (int)a.nodes[0];
+  int n_kept = 0;
+  int cur = 0;
+  bool bad = false;
+  for (int l = 0; l < a.levels; ++l) {
+    const int b = a.branching[l];
+    const float* cent = reinterpret_cast<const float*>(a.tree + a.off_c[l]) + (int64_t)g * a.nodes[l] * R;
+    const int32_t* mpos = reinterpret_cast<const int32_t*>(a.tree + a.off_m[l]) + (int64_t)g * a.nodes[l];
+    const int32_t* kept = s_kept[cur];
+    constexpr int U = 32 * kWideWarps / GROUPS;   // every candidate slot in flight at once
+    for (int c0 = 0; c0 < ncand; c0 += GROUPS * U) {
+      float4 x[U][RS::F];
+      bool ok[U];
+      int64_t id[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int c = c0 + u * GROUPS + gg;
+        ok[u] = c < ncand;
+        id[u] = 0;
+        if (ok[u]) {
+          id[u] = l == 0 ? c : (int64_t)kept[c / b] * b + (c % b);
+          ok[u] = all_eligible || (int64_t)__ldg(&mpos[id[u]]) <= qpos;
+        }
+        const float4* cr = reinterpret_cast<const float4*>(cent + id[u] * R);
+#pragma unroll
+        for (int f = 0; f < RS::F; ++f)
+          x[u][f] = ok[u] ? __ldg(&cr[f * RS::LPR + sub]) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        float sc = 0.f;
+#pragma unroll
+        for (int f = 0; f < RS::F; ++f) {
+          sc = fmaf(lat[f].x, x[u][f].x, sc);
+          sc = fmaf(lat[f].y, x[u][f].y, sc);
+          sc = fmaf(lat[f].z, x[u][f].z, sc);
+          sc = fmaf(lat[f].w, x[u][f].w, sc);
+        }
+#pragma unroll
+        for (int o = 1; o < RS::LPR; o <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+        const int c = c0 + u * GROUPS + gg;
+        if (sub == 0 && c < ncand) {
+          unsigned long long key = 0ull;
+          if (ok[u]) {
+            if (isnan(sc)) bad = true;
+            else key = ((unsigned long long)orderable(sc) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)id[u]);
+          }
+          s_key[c] = key;
+        }
+      }
+    }
+    __syncthreads();
+    const int nchunks = (ncand + 31) / 32;
+    unsigned long long v[1];
+    v[0] = warp < nchunks && warp * 32 + lane < ncand ? s_key[warp * 32 + lane] : 0ull;
+    if (warp < nchunks) warp_sort_desc<1>(v);
+    // a warp's list replaces its own chunk, which only that warp has read
+    for (int step = 1; step < nchunks; step <<= 1) {
+      if (warp % (2 * step) == step && warp < nchunks) s_key[warp * 32 + lane] = v[0];
+      __syncthreads();
+      if (warp % (2 * step) == 0 && warp + step < nchunks) {
+        const unsigned long long o = s_key[(warp + step) * 32 + 31 - lane];
+        v[0] = v[0] > o ? v[0] : o;
+#pragma unroll
+        for (int j = 16; j; j >>= 1) {
+          const unsigned long long p = __shfl_xor_sync(0xffffffffu, v[0], j);
+          const bool lower = (lane & j) == 0;
+          v[0] = lower ? (v[0] > p ? v[0] : p) : (v[0] < p ? v[0] : p);
+        }
+      }
+      __syncthreads();
+    }
+    int32_t* next = s_kept[cur ^ 1];
+    if (warp == 0) {
+      const int valid = emit_kept<1>(v, a.beam[l], next);
+      if (lane == 0) s_valid = valid;
+    }
+    __syncthreads();
+    const int valid = s_valid;
+    if (a.beam_out && tid < a.beam_max) {
+      const int32_t id = tid < valid ? next[tid] : -1;
+      a.beam_out[(((int64_t)l * a.Hkv + g) * a.T + t) * a.beam_max + tid] = id;
+    }
+    n_kept = valid;
+    cur ^= 1;
+    ncand = l + 1 < a.levels ? valid * a.branching[l + 1] : 0;
+  }
+  if (__syncthreads_or(bad) && tid == 0) set_status(a.status, LSA_ERR_NONFINITE);
+  const int32_t* kept = s_kept[cur];
+  const int leaf = a.leaf;
+  const int B = a.beam[a.levels - 1];
+  if (a.leaves_out && tid < B) a.leaves_out[((int64_t)g * a.T + t) * B + tid] = tid < n_kept ? kept[tid] : -1;
+  if (a.idx_out) {
+    const int64_t K_sel = (int64_t)B * leaf;
+    const int32_t* li = reinterpret_cast<const int32_t*>(a.tree + a.off_leaf) + (int64_t)g * a.n_tree;
+    int32_t* out = a.idx_out + ((int64_t)g * a.T + t) * K_sel;
+    for (int64_t i = tid; i < K_sel; i += NT) {
+      const int k = (int)(i / leaf), q = (int)(i % leaf);
+      out[i] = k < n_kept ? __ldg(&li[(int64_t)kept[k] * leaf + q]) : -1;
     }
   }
 }
 
 template <typename T>
 static cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
-  dim3 grid((unsigned)a.T, (unsigned)a.Hkv);
+  const bool wide = a.T * a.Hkv < kWideUnits;
+  dim3 grid((unsigned)(wide ? a.T : ceil_div(a.T, kSelWarps)), (unsigned)a.Hkv);
 #define LSA_SEL(RR, DD)                                                     \
   if (a.r == RR && a.d == DD) {                                             \
-    k_select<T, RR, DD><<<grid, kSelThreads, 0, st>>>(a);                   \
+    if (wide) k_select_wide<T, RR, DD><<<grid, kWideWarps * 32, 0, st>>>(a); \
+    else k_select<T, RR, DD><<<grid, kSelWarps * 32, 0, st>>>(a);           \
     return cudaGetLastError();                                              \
   }
   LSA_SEL(16, 64) LSA_SEL(32, 64) LSA_SEL(64, 64) LSA_SEL(16, 128) LSA_SEL(32, 128) LSA_SEL(64, 128)

@@ -311,3 +311,35 @@ def test_tree_attention_backward(lsa, G):
     for a, b in ((dQ, dQ2), (dK, dK2), (dV, dV2)):
         ref = b.abs().max().item()
         assert (a - b).abs().max().item() <= 2e-2 * ref
+
+
+@pytest.mark.parametrize("name,T,Hkv,extra", [
+    ("tiny", 1536, 1, {}),
+    ("decode_128k", 640, 2, {}),
+    ("prefill_1m", 640, 2, dict(n=8 * 8 * 4 * 2 * 64, branching=(8, 8, 4, 2), beam=(4, 16, 16, 8), comps=256)),
+])
+def test_select_batch_kernels_agree(lsa, name, T, Hkv, extra):
+    """A large batch runs the warp-per-query walk, a small one the CTA-per-query walk; both
+    sum scores in the same order, so a query's selection must not depend on the batch it
+    came in.  The large batch is also checked stage-wise against the oracle."""
+    base = configs.get(name)
+    cfg = base.scaled(T=T, Hkv=Hkv, Hq=Hkv * (base.Hq // base.Hkv), **extra)
+    case = cfg.case("cpu")
+    g = _to(case)
+    tree = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    assert T * Hkv >= 148 * 8 and 100 * Hkv < 148 * 8
+    idx, qlat, beams = lsa.select(tree, g["Q"], g["W"], cfg.beam, g["q_pos"], qlat=True, beams=True)
+    lo, hi = T // 3, T // 3 + 100
+    qp = None if g["q_pos"] is None else g["q_pos"][lo:hi].contiguous()
+    idx_s, qlat_s = lsa.select(tree, g["Q"][lo:hi].contiguous(), g["W"], cfg.beam, qp, qlat=True)
+    torch.cuda.synchronize()
+    assert torch.equal(idx[:, lo:hi], idx_s)
+    assert torch.equal(qlat[lo:hi], qlat_s)
+    qpn = None if case.q_pos is None else case.q_pos.numpy()
+    for h in range(Hkv):
+        Z = orc.project(case.K[h, :cfg.n], case.W[h])
+        th = parity.export_tree(tree, h)
+        oq = orc.query_latent(case.Q[:, h * cfg.G:(h + 1) * cfg.G], case.W[h])
+        np.testing.assert_allclose(qlat[:, h].cpu().numpy(), oq, rtol=1e-4, atol=1e-5)
+        parity.check_select_stagewise(oq, th, cfg.branching, cfg.leaf, cfg.beam, qpn,
+                                      beams[:, h].cpu().numpy(), idx[h].cpu().numpy())
