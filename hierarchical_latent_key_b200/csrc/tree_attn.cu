@@ -138,7 +138,8 @@ struct TreeAttnArgs {
   int32_t* ent;                // [H][T * B] (query << 6 | rank), grouped by leaf
   float2* stats;               // [T][Hq][B] (max, sum) in base 2
   float* lse2;                 // [T][Hq]
-  float* oacc;                 // [T][Hq][d]
+  float* oacc;                 // [T][Hq][d] (red-add mode)
+  float* part;                 // [T][Hq][B][d] unnormalised leaf outputs (partial mode)
   __nv_bfloat16* O;
   float* LSE;
   int32_t* status;
@@ -518,6 +519,175 @@ __global__ void k_tl_finish(TreeAttnArgs a) {
   reinterpret_cast<uint2*>(a.O)[i] = w;
 }
 
+// ---- partial mode: one pass, per (row, leaf) partial outputs, then combine -----
+//
+// Each (row, leaf) pair writes its leaf max m (base 2), exp-sum l and the
+// unnormalised P.V with P = exp2(S - m); k_tl_combine merges a row's leaves
+// (weights 2^(m - M)).  No pass over the statistics first and no atomics, at
+// the cost of T * Hq * n_leaves * d * 4 bytes of partials.
+
+__global__ void __launch_bounds__(kTL) k_tl_part(TreeAttnArgs a) {
+  extern __shared__ char smem_raw[];
+  __shared__ int32_t s_pos[kLeafKeys];
+  __shared__ __align__(8) uint64_t s_mbar;
+  __shared__ uint32_t s_taddr;
+  const int64_t g = blockIdx.y, leaf = blockIdx.x;
+  const int32_t* offg = a.off + g * (a.NL + 1);
+  const int64_t e_lo = offg[leaf], n_ent = offg[leaf + 1] - e_lo;
+  if (n_ent == 0) return;
+  const int32_t* ent = a.ent + g * a.T * a.B + e_lo;
+  char* base = align1024(smem_raw);
+  LeafSmem s;
+  s.sA = smem_u32(base);                       // 32 KB: rows x d
+  s.sK = s.sA + kTL * 256;                     // 16 KB
+  s.sV = s.sK + kLeafKeys * 256;               // 16 KB
+  s.sP = s.sA;                                 // P (rows x 64 keys) overwrites the consumed Q tile
+  s.pos = s_pos;
+  s.mbar = smem_u32(&s_mbar);
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
+    asm volatile("fence.mbarrier_init.release.cluster;");
+  }
+  int64_t tq;
+  int rank, h;
+  row_of(a, ent, n_ent, 0, tq, rank, h);
+  if (threadIdx.x < kLeafKeys) s_pos[threadIdx.x] = a.leaf_index[g * a.n_tree + leaf * kLeafKeys + threadIdx.x];
+  __syncthreads();
+  copy_leaf(a, g, s, true);
+  alloc_tmem(&s_taddr, 128);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_taddr;
+  const int warp = threadIdx.x >> 5;
+  uint32_t phase = 0;
+  bool ok = true;
+  char* sP_gen = base;
+  for (int64_t e0 = 0; e0 < n_ent && ok; e0 += kTL / a.G) {
+    if (e0 > 0) row_of(a, ent, n_ent, e0, tq, rank, h);
+    copy_row(a, g, tq, h, s.sA);
+    cp_async_wait_all();
+    fence_async_smem();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      issue_qk(s, tmem, 0);
+      tc_commit(s.mbar);
+    }
+    ok = __syncthreads_and(mbar_wait(s.mbar, phase));
+    phase ^= 1;
+    tc_fence_after();
+    const int64_t prow = tq >= 0 ? (tq * a.Hq + g * a.G + h) * a.B + rank : -1;
+    if (ok) {
+      float sc[64];
+      read_scores(a, s, tmem, tq, sc);
+      float m = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) m = fmaxf(m, sc[i]);
+      // a row with no visible key (or no query) gets P = 0
+      const float mref = m == -INFINITY ? 0.f : m;
+      float l = 0.f;
+      const int r = threadIdx.x;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float p0 = exp2f(sc[c * 8 + 2 * q] - mref), p1 = exp2f(sc[c * 8 + 2 * q + 1] - mref);
+          l += p0 + p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          w[q] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        *reinterpret_cast<uint4*>(sP_gen + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (prow >= 0) a.stats[prow] = make_float2(m, l);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (ok && threadIdx.x == 0) {
+      tc_fence_after();
+      constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint64_t da = sdesc_sw128(s.sP + kk * 32, 16, 1024);
+        const uint64_t db = sdesc_sw128(s.sV + kk * 2048, kLeafKeys * 128, 1024);
+        tc_mma(tmem, da, db, idesc, kk > 0 ? 1u : 0u);
+      }
+      tc_commit(s.mbar);
+    }
+    if (ok) {
+      ok = __syncthreads_and(mbar_wait(s.mbar, phase));
+      phase ^= 1;
+    }
+    tc_fence_after();
+    if (ok) {
+      float* dst = prow >= 0 ? a.part + prow * kDim : nullptr;
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        float v[32];
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + part * 32, v);
+        if (dst) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + part * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+      }
+    } else {
+      set_status(a.status, LSA_ERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
+  free_tmem(tmem, 128);
+}
+
+// One warp per (query, head) row: O = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k
+// over the row's leaves, in rank order.
+__global__ void k_tl_combine(TreeAttnArgs a) {
+  const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // t * Hq + head
+  const int lane = threadIdx.x & 31;
+  if (row >= a.T * a.Hq) return;
+  const int64_t t = row / a.Hq, head = row % a.Hq, g = head / a.G;
+  bool valid = false;
+  float mk = -INFINITY, lk = 0.f;
+  if (lane < a.B && a.leaves[(g * a.T + t) * a.B + lane] >= 0) {
+    const float2 st = a.stats[row * a.B + lane];
+    valid = st.y > 0.f;
+    mk = st.x;
+    lk = st.y;
+  }
+  float M = valid ? mk : -INFINITY;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float L = 0.f;
+  if (vmask) {
+    const float wk = valid ? exp2f(mk - M) : 0.f;
+    const float* pr = a.part + row * a.B * kDim + lane * 4;
+    for (int k = 0; k < a.B; ++k) {
+      if (!((vmask >> k) & 1u)) continue;
+      const float w = __shfl_sync(0xffffffffu, wk, k), l = __shfl_sync(0xffffffffu, lk, k);
+      const float4 v = *reinterpret_cast<const float4*>(pr + (int64_t)k * kDim);
+      acc[0] = fmaf(w, v.x, acc[0]);
+      acc[1] = fmaf(w, v.y, acc[1]);
+      acc[2] = fmaf(w, v.z, acc[2]);
+      acc[3] = fmaf(w, v.w, acc[3]);
+      L = fmaf(w, l, L);
+    }
+  }
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
+  __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
+  uint2 w2;
+  w2.x = *reinterpret_cast<uint32_t*>(&lo);
+  w2.y = *reinterpret_cast<uint32_t*>(&hi);
+  *reinterpret_cast<uint2*>(a.O + row * kDim + lane * 4) = w2;
+  if (lane == 0) a.LSE[row] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+}
+
 // ---- backward, leaf by leaf -------------------------------------------------
 //
 // Same leaf lists as the forward.  Per leaf CTA and chunk of up to 128 rows:
@@ -775,11 +945,17 @@ constexpr size_t kBwdSmem = 1024 + 2 * kTL * 256 + 2 * kLeafKeys * 256 + 2 * kTL
 
 }  // namespace
 
+// Partial mode while its per-(row, leaf) outputs stay within this many bytes.
+constexpr size_t kPartialMaxBytes = size_t(4) << 30;
+
+static bool partial_mode(int64_t T, int64_t Hq, int B) { return (size_t)T * Hq * B * kDim * 4 <= kPartialMaxBytes; }
+
 size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   if (!fast) return al((size_t)H * T * B * leaf * 4);
-  return al(H * NL * 4) + al(H * (NL + 1) * 4) + al((size_t)H * T * B * 4) + al((size_t)T * Hq * B * 8) +
-         al((size_t)T * Hq * 4) + al((size_t)T * Hq * d * 4);
+  const size_t lists = al(H * NL * 4) + al(H * (NL + 1) * 4) + al((size_t)H * T * B * 4) + al((size_t)T * Hq * B * 8);
+  if (partial_mode(T, Hq, B)) return lists + al((size_t)T * Hq * B * d * 4);
+  return lists + al((size_t)T * Hq * 4) + al((size_t)T * Hq * d * 4);
 }
 
 size_t tree_attn_bwd_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast) {
@@ -826,8 +1002,14 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
   a.off = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * (c.NL + 1) * 4);
   a.ent = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * c.B * 4);
   a.stats = reinterpret_cast<float2*>(ws + o); o += al((size_t)c.T * c.Hq * c.B * 8);
-  a.lse2 = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);
-  a.oacc = reinterpret_cast<float*>(ws + o);
+  const bool partial = partial_mode(c.T, c.Hq, c.B);
+  a.lse2 = a.oacc = a.part = nullptr;
+  if (partial) {
+    a.part = reinterpret_cast<float*>(ws + o);
+  } else {
+    a.lse2 = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);
+    a.oacc = reinterpret_cast<float*>(ws + o);
+  }
   a.O = static_cast<__nv_bfloat16*>(c.O);
   a.LSE = c.LSE;
   a.status = c.status;
@@ -836,10 +1018,16 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
   a.scale_log2 = c.scale * 1.44269504088896340736f;
   const int64_t n_sel = (int64_t)c.H * c.T * c.B;
   if ((e = cudaMemsetAsync(a.cnt, 0, (size_t)c.H * c.NL * 4, st)) != cudaSuccess) return e;
-  if ((e = cudaMemsetAsync(a.oacc, 0, (size_t)c.T * c.Hq * kDim * 4, st)) != cudaSuccess) return e;
   k_tl_count<<<(unsigned)ceil_div(n_sel, 256), 256, 0, st>>>(a);
   k_tl_scan<<<(unsigned)c.H, 1024, 0, st>>>(a);
   k_tl_fill<<<(unsigned)ceil_div(n_sel, 256), 256, 0, st>>>(a);
+  if (partial) {
+    cudaFuncSetAttribute(k_tl_part, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOutSmem);
+    k_tl_part<<<dim3((unsigned)c.NL, (unsigned)c.H), kTL, kOutSmem, st>>>(a);
+    k_tl_combine<<<(unsigned)ceil_div(c.T * c.Hq * 32, 256), 256, 0, st>>>(a);
+    return cudaGetLastError();
+  }
+  if ((e = cudaMemsetAsync(a.oacc, 0, (size_t)c.T * c.Hq * kDim * 4, st)) != cudaSuccess) return e;
   cudaFuncSetAttribute(k_tl_stats, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStatsSmem);
   cudaFuncSetAttribute(k_tl_out, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOutSmem);
   dim3 grid((unsigned)c.NL, (unsigned)c.H);

@@ -194,9 +194,13 @@ int lsa_tree_attn_workspace_bytes(const lsa_tree_desc *tree, int32_t T, int32_t 
  * Computed leaf by leaf: every selected leaf's K/V rows are read once per pass
  * and shared by all (query, head) rows that chose the leaf, with the products on
  * the tensor cores (bf16, d = 128, leaf size 64; other shapes run the generic
- * kernels on the expanded lists).  Outputs as lsa_sparse_attn.  The summation
- * order over leaves is not fixed (fp32 atomic adds), so results may differ from
- * run to run in the last bits.  n_leaves in [1, 32]. */
+ * kernels on the expanded lists).  Outputs as lsa_sparse_attn.  While
+ * T * Hq * n_leaves * d * 4 bytes stay within 4 GiB, every (row, leaf) pair
+ * stores its leaf maximum, exp-sum and unnormalised output in the workspace and
+ * a row's leaves are merged in rank order (results are reproducible bit for
+ * bit); larger calls take a second pass over the leaves instead and accumulate
+ * the outputs with fp32 atomic adds, whose order is not fixed, so results may
+ * differ from run to run in the last bits.  n_leaves in [1, 32]. */
 int lsa_tree_attn(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, int32_t T,
                   int32_t Hq, const void *K, const void *V, int64_t n_cap, int32_t d,
                   int32_t dtype, const int32_t *leaves, int32_t n_leaves, const int32_t *q_pos,

@@ -235,6 +235,9 @@ def test_tree_attention_matches_oracle(lsa, G, n_q):
         assert mx <= 2e-2 and mean <= 2e-3, (h, mx, mean)
         assert np.abs(LSE[:, sl].cpu().numpy() - Lo).max() <= 1e-3
     assert (O.float() - O2.float()).abs().max().item() <= 2e-2
+    # partial outputs merged in rank order: a second call reproduces every bit
+    O3, L3 = lsa.tree_attn(tree, g["Q"], g["K"], g["V"], leaves, g["q_pos"], causal=True)
+    assert torch.equal(O, O3) and torch.equal(LSE, L3)
 
 
 def test_tree_attention_many_queries_per_leaf(lsa):
