@@ -18,6 +18,7 @@
 // Rows of one CTA chunk: up to 128 (query, head) pairs of queries that chose the
 // leaf.  Shapes served here: bf16, d = 128, leaf size 64, G in {1, 2, 4, 8};
 // other shapes expand the leaves into key lists and use the generic kernels.
+#include <climits>
 #include <cstring>
 
 #include "lsa_common.cuh"
@@ -140,6 +141,11 @@ struct TreeAttnArgs {
   float* lse2;                 // [T][Hq]
   float* oacc;                 // [T][Hq][d] (red-add mode)
   float* part;                 // [T][Hq][B][d] unnormalised leaf outputs (partial mode)
+  int32_t* entq;               // [H][T * B] query position of each entry (INT_MAX: not causal)
+  int32_t* coff;               // [H][NL] first chunk of each leaf within its head
+  int32_t* ctotal;             // [H] chunks per head
+  int4* cdesc;                 // chunk descriptors {head, leaf, first entry, entries}
+  int32_t epc;                 // entries per chunk (rows / G)
   __nv_bfloat16* O;
   float* LSE;
   int32_t* status;
@@ -205,6 +211,56 @@ __global__ void k_tl_fill(TreeAttnArgs a) {
   if (leaf < 0 || leaf >= a.NL) return;
   const int32_t pos = a.off[g * (a.NL + 1) + leaf] + atomicAdd(&a.cnt[g * a.NL + leaf], 1);
   a.ent[g * a.T * a.B + pos] = (int32_t)((t << 6) | k);
+  if (a.entq) a.entq[g * a.T * a.B + pos] = a.causal ? a.q_pos[t] : INT_MAX;
+}
+
+// Chunk lists for the pipelined pass: per head, the first chunk of each leaf
+// (ceil(entries / epc) chunks per leaf) and the head's total.
+__global__ void __launch_bounds__(1024) k_tl_cscan(TreeAttnArgs a) {
+  __shared__ int32_t s_warp[32];
+  const int64_t g = blockIdx.x;
+  const int32_t* o = a.off + g * (a.NL + 1);
+  int32_t* c = a.coff + g * a.NL;
+  const int64_t per = ceil_div(a.NL, 1024);
+  const int64_t lo = threadIdx.x * per, hi = min64(a.NL, lo + per);
+  int32_t s = 0;
+  for (int64_t i = lo; i < hi; ++i) s += (o[i + 1] - o[i] + a.epc - 1) / a.epc;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t inc = s;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    int32_t y = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += y;
+  }
+  if (lane == 31) s_warp[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = s_warp[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      int32_t y = __shfl_up_sync(0xffffffffu, w, d);
+      if (lane >= d) w += y;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  int32_t run = inc - s + (warp ? s_warp[warp - 1] : 0);
+  for (int64_t i = lo; i < hi; ++i) {
+    c[i] = run;
+    run += (o[i + 1] - o[i] + a.epc - 1) / a.epc;
+  }
+  if (threadIdx.x == 1023) a.ctotal[g] = run;
+}
+
+__global__ void k_tl_chunks(TreeAttnArgs a) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= (int64_t)a.H * a.NL) return;
+  const int64_t g = i / a.NL, leaf = i % a.NL;
+  int64_t base = a.coff[i];
+  for (int64_t h = 0; h < g; ++h) base += a.ctotal[h];
+  const int32_t e0 = a.off[g * (a.NL + 1) + leaf], n = a.off[g * (a.NL + 1) + leaf + 1] - e0;
+  for (int32_t c = 0; c * a.epc < n; ++c)
+    a.cdesc[base + c] = make_int4((int)g, (int)leaf, e0 + c * a.epc, min(a.epc, n - c * a.epc));
 }
 
 // ---- shared pieces of the two passes ----------------------------------------
@@ -264,19 +320,33 @@ __device__ __forceinline__ void issue_qk(const LeafSmem& s, uint32_t tmem, int c
   }
 }
 
+// Number of a leaf's keys visible at query position qp.  A leaf lists its keys
+// in ascending position order (the index build keeps position order inside
+// every node), so the visible keys are a prefix; a branch-free binary search
+// finds its length and the masks below are register compares.
+__device__ __forceinline__ int visible_prefix(const int32_t* pos, int64_t qp) {
+  if ((int64_t)pos[kLeafKeys - 1] <= qp) return kLeafKeys;
+  int c = 0;   // < 64 from here on: steps 32 + 16 + ... + 1 reach 63 at most
+#pragma unroll
+  for (int step = kLeafKeys / 2; step; step >>= 1)
+    if ((int64_t)pos[c + step - 1] <= qp) c += step;
+  return c;
+}
+
 // This thread's 64 scores (base-2 scaled, causally masked) from TMEM.
 __device__ __forceinline__ void read_scores(const TreeAttnArgs& a, const LeafSmem& s, uint32_t tmem, int64_t tq,
                                             float (&sc)[64]) {
   const int warp = threadIdx.x >> 5;
   float v[32];
   const int64_t qp = (a.causal && tq >= 0) ? (int64_t)a.q_pos[tq] : INT64_MAX;
+  const int nvis = visible_prefix(s.pos, qp);
 #pragma unroll
   for (int half = 0; half < 2; ++half) {
     tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + half * 32, v);
 #pragma unroll
     for (int i = 0; i < 32; ++i) {
       const int key = half * 32 + i;
-      sc[key] = (int64_t)s.pos[key] <= qp ? v[i] * a.scale_log2 : -INFINITY;
+      sc[key] = key < nvis ? v[i] * a.scale_log2 : -INFINITY;
     }
   }
 }
@@ -519,129 +589,12 @@ __global__ void k_tl_finish(TreeAttnArgs a) {
   reinterpret_cast<uint2*>(a.O)[i] = w;
 }
 
-// ---- partial mode: one pass, per (row, leaf) partial outputs, then combine -----
+// ---- partial mode: per (row, leaf) partial outputs, then combine ---------------
 //
 // Each (row, leaf) pair writes its leaf max m (base 2), exp-sum l and the
-// unnormalised P.V with P = exp2(S - m); k_tl_combine merges a row's leaves
-// (weights 2^(m - M)).  No pass over the statistics first and no atomics, at
-// the cost of T * Hq * n_leaves * d * 4 bytes of partials.
-
-__global__ void __launch_bounds__(kTL) k_tl_part(TreeAttnArgs a) {
-  extern __shared__ char smem_raw[];
-  __shared__ int32_t s_pos[kLeafKeys];
-  __shared__ __align__(8) uint64_t s_mbar;
-  __shared__ uint32_t s_taddr;
-  const int64_t g = blockIdx.y, leaf = blockIdx.x;
-  const int32_t* offg = a.off + g * (a.NL + 1);
-  const int64_t e_lo = offg[leaf], n_ent = offg[leaf + 1] - e_lo;
-  if (n_ent == 0) return;
-  const int32_t* ent = a.ent + g * a.T * a.B + e_lo;
-  char* base = align1024(smem_raw);
-  LeafSmem s;
-  s.sA = smem_u32(base);                       // 32 KB: rows x d
-  s.sK = s.sA + kTL * 256;                     // 16 KB
-  s.sV = s.sK + kLeafKeys * 256;               // 16 KB
-  s.sP = s.sA;                                 // P (rows x 64 keys) overwrites the consumed Q tile
-  s.pos = s_pos;
-  s.mbar = smem_u32(&s_mbar);
-  if (threadIdx.x == 0) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
-    asm volatile("fence.mbarrier_init.release.cluster;");
-  }
-  int64_t tq;
-  int rank, h;
-  row_of(a, ent, n_ent, 0, tq, rank, h);
-  if (threadIdx.x < kLeafKeys) s_pos[threadIdx.x] = a.leaf_index[g * a.n_tree + leaf * kLeafKeys + threadIdx.x];
-  __syncthreads();
-  copy_leaf(a, g, s, true);
-  alloc_tmem(&s_taddr, 128);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = s_taddr;
-  const int warp = threadIdx.x >> 5;
-  uint32_t phase = 0;
-  bool ok = true;
-  char* sP_gen = base;
-  for (int64_t e0 = 0; e0 < n_ent && ok; e0 += kTL / a.G) {
-    if (e0 > 0) row_of(a, ent, n_ent, e0, tq, rank, h);
-    copy_row(a, g, tq, h, s.sA);
-    cp_async_wait_all();
-    fence_async_smem();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      tc_fence_after();
-      issue_qk(s, tmem, 0);
-      tc_commit(s.mbar);
-    }
-    ok = __syncthreads_and(mbar_wait(s.mbar, phase));
-    phase ^= 1;
-    tc_fence_after();
-    const int64_t prow = tq >= 0 ? (tq * a.Hq + g * a.G + h) * a.B + rank : -1;
-    if (ok) {
-      float sc[64];
-      read_scores(a, s, tmem, tq, sc);
-      float m = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) m = fmaxf(m, sc[i]);
-      // a row with no visible key (or no query) gets P = 0
-      const float mref = m == -INFINITY ? 0.f : m;
-      float l = 0.f;
-      const int r = threadIdx.x;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float p0 = exp2f(sc[c * 8 + 2 * q] - mref), p1 = exp2f(sc[c * 8 + 2 * q + 1] - mref);
-          l += p0 + p1;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          w[q] = *reinterpret_cast<uint32_t*>(&b2);
-        }
-        *reinterpret_cast<uint4*>(sP_gen + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      if (prow >= 0) a.stats[prow] = make_float2(m, l);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (ok && threadIdx.x == 0) {
-      tc_fence_after();
-      constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk) {
-        const uint64_t da = sdesc_sw128(s.sP + kk * 32, 16, 1024);
-        const uint64_t db = sdesc_sw128(s.sV + kk * 2048, kLeafKeys * 128, 1024);
-        tc_mma(tmem, da, db, idesc, kk > 0 ? 1u : 0u);
-      }
-      tc_commit(s.mbar);
-    }
-    if (ok) {
-      ok = __syncthreads_and(mbar_wait(s.mbar, phase));
-      phase ^= 1;
-    }
-    tc_fence_after();
-    if (ok) {
-      float* dst = prow >= 0 ? a.part + prow * kDim : nullptr;
-#pragma unroll
-      for (int part = 0; part < 4; ++part) {
-        float v[32];
-        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + part * 32, v);
-        if (dst) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + part * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-        }
-      }
-    } else {
-      set_status(a.status, LSA_ERR_TIMEOUT);
-    }
-    tc_fence_before();
-    __syncthreads();
-  }
-  free_tmem(tmem, 128);
-}
+// unnormalised P.V with P = exp2(S - m) (k_tl_pipe below); k_tl_combine merges
+// a row's leaves (weights 2^(m - M)).  No pass over the statistics first and no
+// atomics, at the cost of T * Hq * n_leaves * d * 4 bytes of partials.
 
 // One warp per (query, head) row: O = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k
 // over the row's leaves, in rank order.
@@ -686,6 +639,335 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
   w2.y = *reinterpret_cast<uint32_t*>(&hi);
   *reinterpret_cast<uint2*>(a.O + row * kDim + lane * 4) = w2;
   if (lane == 0) a.LSE[row] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
+}
+
+// ---- partial mode, pipelined ------------------------------------------------
+//
+// Persistent CTAs (one per SM), each walking a contiguous range of chunks with
+// four warp roles joined by mbarriers:
+//   warps 8-11 (loaders): chunk metadata into shared memory and 16-byte
+//     cp.async copies of the chunk's Q rows and the leaf's K and V rows into one
+//     of kPipeStages stages (128B-swizzled tiles); the next chunk's metadata is
+//     fetched while the current one is copied;
+//   warp 12 (one lane, MMA): S = Q.K^T into one of kPipeBufs TMEM buffers, and
+//     once P is in shared memory, O = P.V over the same columns;
+//   warps 0-3 (P, one TMEM lane per row): P and the (m, l) statistics from S;
+//   warps 4-7 (epilogue, same lanes): O from TMEM to the partial outputs.
+// Every wait is bounded; on a timeout the CTA records LSA_ERR_TIMEOUT, stops
+// its roles, waits for its copies and MMAs in flight and frees TMEM.
+
+constexpr int kPipeStages = 3;
+constexpr int kPipeBufs = 4;                       // TMEM buffers of 128 columns
+constexpr int kPipeLoaders = 128;                  // loader threads (warps 8-11)
+constexpr int kPipeThreads = 13 * 32;
+constexpr uint32_t kStageBytes = 65536;            // Q/P 32 KB, K 16 KB, V 16 KB
+
+struct PipeMeta {
+  int32_t ent[kPipeStages][kTL];
+  int32_t qpos[kPipeStages][kTL];
+  int32_t pos[kPipeStages][kLeafKeys];
+  int32_t qrow[kPipeStages][kTL];                  // global Q row of each tile row (loaders only)
+  int32_t info[kPipeStages][2];                    // head, entries
+  int32_t prow[kPipeBufs][kTL];                    // partial row of each TMEM lane (-1: none)
+  float2 stat[kPipeBufs][kTL];                     // (m, l) of each TMEM lane
+  uint64_t full[kPipeStages], sempty[kPipeStages], pready[kPipeStages];
+  uint64_t sfull[kPipeBufs], ofull[kPipeBufs], tempty[kPipeBufs], mready[kPipeBufs];
+  uint64_t done;
+  uint32_t taddr;
+  int32_t abort;
+};
+constexpr size_t kPipeSmem = 1024 + kPipeStages * kStageBytes + sizeof(PipeMeta);
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Arrive on `bar` once this thread's cp.async copies issued so far have landed
+// (counts as one of the barrier's expected arrivals).
+__device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+
+// Barrier of the loader threads (named barrier 1) that also returns, in every
+// one of them, whether any of them passed `v`: their stop decisions agree, so
+// none waits at the barrier for a loader that has left.
+__device__ __forceinline__ bool loaders_any(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.or.pred q, 1, %2, p;\nselp.u32 %0, 1, 0, q;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)v), "n"(kPipeLoaders)
+      : "memory");
+  return r != 0;
+}
+
+// Metadata one loader thread needs for one chunk.
+struct LoadMeta {
+  int g, leaf, e_lo, ne;
+  int32_t pos;      // position of key (lt mod 64)
+  int32_t qent;     // entry of Q row lt (or -1)
+  int32_t ev, eq;   // entry lt and its query position (metadata)
+};
+
+__global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
+  extern __shared__ char smem_raw[];
+  char* base = align1024(smem_raw);
+  PipeMeta& M = *reinterpret_cast<PipeMeta*>(base + kPipeStages * kStageBytes);
+  const uint32_t sbase = smem_u32(base);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int64_t C = 0;
+  for (int h = 0; h < a.H; ++h) C += a.ctotal[h];
+  const int64_t k0 = C * blockIdx.x / gridDim.x, k1 = C * (blockIdx.x + 1) / gridDim.x;
+  const int N = (int)(k1 - k0);
+  if (N == 0) return;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPipeStages; ++s) {
+      mbar_init(smem_u32(&M.full[s]), 2 * kPipeLoaders);
+      mbar_init(smem_u32(&M.sempty[s]), 1);
+      mbar_init(smem_u32(&M.pready[s]), kTL);
+    }
+    for (int b = 0; b < kPipeBufs; ++b) {
+      mbar_init(smem_u32(&M.sfull[b]), 1);
+      mbar_init(smem_u32(&M.ofull[b]), 1);
+      mbar_init(smem_u32(&M.tempty[b]), kTL);
+      mbar_init(smem_u32(&M.mready[b]), kTL);
+    }
+    mbar_init(smem_u32(&M.done), 1);
+    M.abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;");
+  }
+  alloc_tmem(&M.taddr, 128 * kPipeBufs);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = M.taddr;
+  volatile int32_t* abort_flag = &M.abort;
+  // warp-uniform view of the abort flag (the warps' collectives must not diverge)
+  auto aborted = [&]() { return __any_sync(0xffffffffu, *abort_flag != 0); };
+  auto fail = [&]() {
+    *abort_flag = 1;
+    set_status(a.status, LSA_ERR_TIMEOUT);
+  };
+
+  if (warp >= 8 && warp < 12) {
+    // ---- loaders: lanes (lt & 15) x rows (lt >> 4) + 8 i, 16-byte chunks ----
+    const int lt = threadIdx.x - 256;
+    const int kr = lt & (kLeafKeys - 1);
+    // descriptors come 32 at a time (one per lane) and are broadcast by shuffles;
+    // a chunk's metadata is fetched two chunks before its copies are issued
+    int4 dcur = lane < N ? a.cdesc[k0 + lane] : make_int4(0, 0, 0, 0);
+    int4 dnxt = 32 + lane < N ? a.cdesc[k0 + 32 + lane] : make_int4(0, 0, 0, 0);
+    auto fetch = [&](int k, LoadMeta& L) {
+      const int4& dr = (k >> 5) == 0 ? dcur : dnxt;   // k lies in the current or the next block of 32
+      const int j = k & 31;
+      L.g = __shfl_sync(0xffffffffu, dr.x, j);
+      L.leaf = __shfl_sync(0xffffffffu, dr.y, j);
+      L.e_lo = __shfl_sync(0xffffffffu, dr.z, j);
+      L.ne = __shfl_sync(0xffffffffu, dr.w, j);
+      const int32_t* entg = a.ent + (int64_t)L.g * a.T * a.B + L.e_lo;
+      L.pos = a.leaf_index[(int64_t)L.g * a.n_tree + (int64_t)L.leaf * kLeafKeys + kr];
+      const int n_rows = L.ne * a.G;
+      L.qent = lt < n_rows ? entg[lt / a.G] : -1;
+      L.ev = lt < L.ne ? entg[lt] : -1;
+      L.eq = lt < L.ne ? a.entq[(int64_t)L.g * a.T * a.B + L.e_lo + lt] : 0;
+    };
+    LoadMeta cur, n1, n2;
+    fetch(0, cur);
+    if (N > 1) fetch(1, n1);
+    for (int k = 0; k < N; ++k) {
+      if ((k & 31) == 0 && k > 0) {   // entering block k / 32: shift the descriptor window
+        dcur = dnxt;
+        const int64_t nb = k + 32 + lane;
+        dnxt = nb < N ? a.cdesc[k0 + nb] : make_int4(0, 0, 0, 0);
+      }
+      // item k + 2 lies in block (k + 2) / 32, i.e. the current one or the next
+      if (k + 2 < N) {
+        const int kb = (k + 2) & ~31;
+        const int4& dr = kb == (k & ~31) ? dcur : dnxt;
+        const int j = (k + 2) & 31;
+        n2.g = __shfl_sync(0xffffffffu, dr.x, j);
+        n2.leaf = __shfl_sync(0xffffffffu, dr.y, j);
+        n2.e_lo = __shfl_sync(0xffffffffu, dr.z, j);
+        n2.ne = __shfl_sync(0xffffffffu, dr.w, j);
+        const int32_t* entg = a.ent + (int64_t)n2.g * a.T * a.B + n2.e_lo;
+        n2.pos = a.leaf_index[(int64_t)n2.g * a.n_tree + (int64_t)n2.leaf * kLeafKeys + kr];
+        const int n_rows = n2.ne * a.G;
+        n2.qent = lt < n_rows ? entg[lt / a.G] : -1;
+        n2.ev = lt < n2.ne ? entg[lt] : -1;
+        n2.eq = lt < n2.ne ? a.entq[(int64_t)n2.g * a.T * a.B + n2.e_lo + lt] : 0;
+      }
+      const int s = k % kPipeStages;
+      const bool ok = k < kPipeStages || mbar_wait(smem_u32(&M.sempty[s]), ((k / kPipeStages) - 1) & 1);
+      const uint32_t st = sbase + s * kStageBytes;
+      // row addresses through shared memory, so that 16 lanes copy one 256-B row
+      const int n_rows = cur.ne * a.G;
+      if (ok) {
+        if (lt < kLeafKeys) M.pos[s][lt] = cur.pos;
+        if (lt < n_rows) M.qrow[s][lt] = (cur.qent >> 6) * a.Hq + cur.g * a.G + lt % a.G;
+      }
+      if (loaders_any(!ok || *abort_flag != 0)) {   // also the barrier before the copies read them
+        if (!ok) fail();
+        break;
+      }
+      {
+        const int c = lt & 15, rg = lt >> 4;
+        const int64_t kv_base = (int64_t)cur.g * a.n_cap;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {   // K and V rows rg, rg + 8, ..., chunk c
+          const int kr2 = rg + 8 * i;
+          const int64_t row = kv_base + M.pos[s][kr2];
+          cp_async16(st + 32768u + sw128_off(kr2, c, kLeafKeys * 128), a.K + row * kDim + c * 8);
+          cp_async16(st + 49152u + sw128_off(kr2, c, kLeafKeys * 128), a.V + row * kDim + c * 8);
+        }
+        for (int r = rg; r < n_rows; r += 8)   // Q rows
+          cp_async16(st + sw128_off(r, c, kTL * 128), a.Q + (int64_t)M.qrow[s][r] * kDim + c * 8);
+      }
+      const uint32_t bar = smem_u32(&M.full[s]);
+      cp_async_arrive(bar);
+      if (lt < a.epc) {
+        M.ent[s][lt] = cur.ev;
+        M.qpos[s][lt] = cur.eq;
+      }
+      if (lt == 0) {
+        M.info[s][0] = cur.g;
+        M.info[s][1] = cur.ne;
+      }
+      mbar_arrive(bar);
+      cur = n1;
+      n1 = n2;
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");   // nothing in flight when the CTA exits
+  } else if (warp == 12) {
+    // ---- MMA issuer ----
+    if (lane == 0) {
+      constexpr uint32_t id_qk = idesc_bf16(128, 64, false, false);
+      constexpr uint32_t id_pv = idesc_bf16(128, 128, false, true);
+      auto qk = [&](int k) -> bool {
+        const int s = k % kPipeStages, b = k % kPipeBufs;
+        if (!mbar_wait(smem_u32(&M.full[s]), (k / kPipeStages) & 1)) return false;
+        if (k >= kPipeBufs && !mbar_wait(smem_u32(&M.tempty[b]), ((k / kPipeBufs) - 1) & 1)) return false;
+        fence_async_smem();    // the loaders' cp.async writes, seen through the barrier, before the MMA reads
+        tc_fence_after();
+        const uint32_t sA = sbase + s * kStageBytes, sK = sA + 32768;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t koff = (uint32_t)((kk & 3) * 32);
+          tc_mma(tmem + b * 128, sdesc_sw128(sA + (kk >> 2) * (kTL * 128) + koff, 16, 1024),
+                 sdesc_sw128(sK + (kk >> 2) * (kLeafKeys * 128) + koff, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&M.sfull[b]));
+        return true;
+      };
+      auto pv = [&](int k) -> bool {
+        const int s = k % kPipeStages, b = k % kPipeBufs;
+        if (!mbar_wait(smem_u32(&M.pready[s]), (k / kPipeStages) & 1)) return false;
+        tc_fence_after();
+        const uint32_t sP = sbase + s * kStageBytes, sV = sP + 49152;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma(tmem + b * 128, sdesc_sw128(sP + kk * 32, 16, 1024),
+                 sdesc_sw128(sV + kk * 2048, kLeafKeys * 128, 1024), id_pv, kk > 0 ? 1u : 0u);
+        tc_commit(smem_u32(&M.ofull[b]));
+        tc_commit(smem_u32(&M.sempty[s]));
+        return true;
+      };
+      bool ok = qk(0);
+      for (int k = 1; k < N && ok && !*abort_flag; ++k) ok = pv(k - 1) && qk(k);
+      if (ok && !*abort_flag) ok = pv(N - 1);
+      if (!ok) fail();
+      tc_commit(smem_u32(&M.done));    // every MMA issued above has completed
+      if (!mbar_wait(smem_u32(&M.done), 0)) fail();
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ---- P: row r = TMEM lane r ----
+    const int r = threadIdx.x;
+    const int e = r / a.G, hh = r % a.G;
+    bool ok = true;
+    for (int k = 0; k < N; ++k) {
+      if (aborted()) break;
+      const int s = k % kPipeStages, b = k % kPipeBufs;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&M.full[s]), (k / kPipeStages) & 1));
+      if (!ok) break;
+      const int g = M.info[s][0];
+      const int v = M.ent[s][e];
+      const int64_t tq = v >= 0 ? (v >> 6) : -1;
+      const int nvis = tq >= 0 ? visible_prefix(M.pos[s], (int64_t)M.qpos[s][e]) : 0;
+      const int prow = tq >= 0 ? (int)((tq * a.Hq + g * a.G + hh) * a.B + (v & 63)) : -1;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&M.sfull[b]), (k / kPipeBufs) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      float sc[64];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        float t32[32];
+        tmem_ld32(tmem + b * 128 + ((uint32_t)(warp * 32) << 16) + half * 32, t32);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sc[half * 32 + i] = half * 32 + i < nvis ? t32[i] * a.scale_log2 : -INFINITY;
+      }
+      float m = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) m = fmaxf(m, sc[i]);
+      const float mref = m == -INFINITY ? 0.f : m;
+      float l = 0.f;
+      char* sP = base + s * kStageBytes;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float p0 = exp2f(sc[c * 8 + 2 * q] - mref), p1 = exp2f(sc[c * 8 + 2 * q + 1] - mref);
+          l += p0 + p1;
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+          w[q] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        *reinterpret_cast<uint4*>(sP + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      M.prow[b][r] = prow;
+      M.stat[b][r] = make_float2(m, l);
+      mbar_arrive(smem_u32(&M.mready[b]));
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&M.pready[s]));
+    }
+    if (!ok && lane == 0) fail();
+  } else if (warp < 8) {
+    // ---- epilogue: row r = TMEM lane r ----
+    const int r = (warp & 3) * 32 + lane;
+    bool ok = true;
+    for (int k = 0; k < N; ++k) {
+      if (aborted()) break;
+      const int b = k % kPipeBufs;
+      ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&M.mready[b]), (k / kPipeBufs) & 1) &&
+                                       mbar_wait(smem_u32(&M.ofull[b]), (k / kPipeBufs) & 1));
+      if (!ok) break;
+      tc_fence_after();
+      const int prow = M.prow[b][r];
+      const float2 st = M.stat[b][r];
+      float* dst = prow >= 0 ? a.part + (int64_t)prow * kDim : nullptr;
+#pragma unroll
+      for (int part = 0; part < 4; ++part) {
+        float v[32];
+        tmem_ld32(tmem + b * 128 + ((uint32_t)((warp & 3) * 32) << 16) + part * 32, v);
+        if (dst) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            *reinterpret_cast<float4*>(dst + part * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+        }
+      }
+      if (prow >= 0) a.stats[prow] = st;
+      tc_fence_before();
+      mbar_arrive(smem_u32(&M.tempty[b]));
+    }
+    if (!ok && lane == 0) fail();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  free_tmem(tmem, 128 * kPipeBufs);
 }
 
 // ---- backward, leaf by leaf -------------------------------------------------
@@ -824,6 +1106,7 @@ __global__ void __launch_bounds__(kTL) k_tlb_leaf(TreeBwdArgs b) {
     }
     {
       const int64_t qpos = (a.causal && tq >= 0) ? (int64_t)a.q_pos[tq] : INT64_MAX;
+      const int nvis = row >= 0 ? visible_prefix(s_pos, qpos) : 0;
       const int r = threadIdx.x;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
@@ -839,7 +1122,7 @@ __global__ void __launch_bounds__(kTL) k_tlb_leaf(TreeBwdArgs b) {
 #pragma unroll
             for (int u = 0; u < 2; ++u) {
               const int i = c * 8 + 2 * q + u, key = half * 32 + i;
-              const bool vis = row >= 0 && (int64_t)s_pos[key] <= qpos;
+              const bool vis = key < nvis;
               const float p = vis ? exp2f(sv[i] * a.scale_log2 - lse) : 0.f;
               p2[u] = p;
               d2[u] = p * (dv[i] - dlt);
@@ -945,17 +1228,26 @@ constexpr size_t kBwdSmem = 1024 + 2 * kTL * 256 + 2 * kLeafKeys * 256 + 2 * kTL
 
 }  // namespace
 
-// Partial mode while its per-(row, leaf) outputs stay within this many bytes.
+// Partial mode while its per-(row, leaf) outputs stay within this many bytes
+// and every gathered row index fits the tensor maps' 32-bit coordinates.
 constexpr size_t kPartialMaxBytes = size_t(4) << 30;
 
-static bool partial_mode(int64_t T, int64_t Hq, int B) { return (size_t)T * Hq * B * kDim * 4 <= kPartialMaxBytes; }
+static bool partial_fits(int64_t T, int64_t Hq, int B) { return (size_t)T * Hq * B * kDim * 4 <= kPartialMaxBytes; }
+
+static int64_t max_chunks(int64_t H, int64_t NL, int64_t T, int B, int epc) {
+  return H * NL + ceil_div(H * T * B, (int64_t)epc);
+}
 
 size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   if (!fast) return al((size_t)H * T * B * leaf * 4);
   const size_t lists = al(H * NL * 4) + al(H * (NL + 1) * 4) + al((size_t)H * T * B * 4) + al((size_t)T * Hq * B * 8);
-  if (partial_mode(T, Hq, B)) return lists + al((size_t)T * Hq * B * d * 4);
-  return lists + al((size_t)T * Hq * 4) + al((size_t)T * Hq * d * 4);
+  const size_t red = lists + al((size_t)T * Hq * 4) + al((size_t)T * Hq * d * 4);
+  if (!partial_fits(T, Hq, B)) return red;
+  const int epc = kTL / (int)(Hq / H);
+  const size_t part = lists + al((size_t)T * Hq * B * d * 4) + al((size_t)H * T * B * 4) + al(H * NL * 4) +
+                      al(H * 4) + al((size_t)max_chunks(H, NL, T, B, epc) * 16);
+  return part > red ? part : red;
 }
 
 size_t tree_attn_bwd_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast) {
@@ -1002,11 +1294,20 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
   a.off = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * (c.NL + 1) * 4);
   a.ent = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * c.B * 4);
   a.stats = reinterpret_cast<float2*>(ws + o); o += al((size_t)c.T * c.Hq * c.B * 8);
-  const bool partial = partial_mode(c.T, c.Hq, c.B);
   a.lse2 = a.oacc = a.part = nullptr;
+  a.entq = a.coff = a.ctotal = nullptr;
+  a.cdesc = nullptr;
+  a.epc = kTL / G;
+  const bool partial = partial_fits(c.T, c.Hq, c.B);
+  const size_t o_lists = o;
   if (partial) {
-    a.part = reinterpret_cast<float*>(ws + o);
+    a.part = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * c.B * kDim * 4);
+    a.entq = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * c.B * 4);
+    a.coff = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.NL * 4);
+    a.ctotal = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * 4);
+    a.cdesc = reinterpret_cast<int4*>(ws + o);
   } else {
+    o = o_lists;
     a.lse2 = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);
     a.oacc = reinterpret_cast<float*>(ws + o);
   }
@@ -1022,8 +1323,13 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
   k_tl_scan<<<(unsigned)c.H, 1024, 0, st>>>(a);
   k_tl_fill<<<(unsigned)ceil_div(n_sel, 256), 256, 0, st>>>(a);
   if (partial) {
-    cudaFuncSetAttribute(k_tl_part, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kOutSmem);
-    k_tl_part<<<dim3((unsigned)c.NL, (unsigned)c.H), kTL, kOutSmem, st>>>(a);
+    int dev = 0, nsm = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    k_tl_cscan<<<(unsigned)c.H, 1024, 0, st>>>(a);
+    k_tl_chunks<<<(unsigned)ceil_div((int64_t)c.H * c.NL, 256), 256, 0, st>>>(a);
+    cudaFuncSetAttribute(k_tl_pipe, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPipeSmem);
+    k_tl_pipe<<<(unsigned)nsm, kPipeThreads, kPipeSmem, st>>>(a);
     k_tl_combine<<<(unsigned)ceil_div(c.T * c.Hq * 32, 256), 256, 0, st>>>(a);
     return cudaGetLastError();
   }
