@@ -635,7 +635,7 @@ def run_cuda(args, rank, world, local_rank):
             "breakdown_ms": {"select": statistics.mean(sel), "attention": statistics.mean(att),
                              "build_once": build_ms},
             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "roofline": {"kernel": "lsa_tree_attn (k_tl_stats + k_tl_out + list/finish kernels)", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
+            "roofline": {"kernel": "lsa_tree_attn (leaf lists + k_tl_pipe + k_tl_combine)", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
                          "peak_source": peaks["source"],
                          "algorithmic_bytes": alg_bytes, "distinct_kv_rows": rows,

@@ -140,7 +140,7 @@ struct TreeAttnArgs {
   float2* stats;               // [T][Hq][B] (max, sum) in base 2
   float* lse2;                 // [T][Hq]
   float* oacc;                 // [T][Hq][d] (red-add mode)
-  float* part;                 // [T][Hq][B][d] unnormalised leaf outputs (partial mode)
+  __nv_bfloat16* part;         // [T][Hq][B][d] leaf outputs over their own exp-sum (partial mode)
   int32_t* entq;               // [H][T * B] query position of each entry (INT_MAX: not causal)
   int32_t* coff;               // [H][NL] first chunk of each leaf within its head
   int32_t* ctotal;             // [H] chunks per head
@@ -592,12 +592,14 @@ __global__ void k_tl_finish(TreeAttnArgs a) {
 // ---- partial mode: per (row, leaf) partial outputs, then combine ---------------
 //
 // Each (row, leaf) pair writes its leaf max m (base 2), exp-sum l and the
-// unnormalised P.V with P = exp2(S - m) (k_tl_pipe below); k_tl_combine merges
-// a row's leaves (weights 2^(m - M)).  No pass over the statistics first and no
-// atomics, at the cost of T * Hq * n_leaves * d * 4 bytes of partials.
+// leaf output P.V / l with P = exp2(S - m), rounded to bf16 (a convex
+// combination of the leaf's V rows, so bf16 keeps it to 2^-9 of their scale);
+// k_tl_combine merges a row's leaves with weights 2^(m - M) l.  No pass over the
+// statistics first and no atomics, at the cost of T * Hq * n_leaves * d * 2
+// bytes of partials.
 
-// One warp per (query, head) row: O = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k
-// over the row's leaves, in rank order.
+// One warp per (query, head) row: O = sum_k w_k o_k / sum_k w_k with
+// w_k = 2^(m_k - M) l_k over the row's leaves, in rank order.
 __global__ void k_tl_combine(TreeAttnArgs a) {
   const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // t * Hq + head
   const int lane = threadIdx.x & 31;
@@ -618,17 +620,18 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   float L = 0.f;
   if (vmask) {
-    const float wk = valid ? exp2f(mk - M) : 0.f;
-    const float* pr = a.part + row * a.B * kDim + lane * 4;
+    const float wk = valid ? exp2f(mk - M) * lk : 0.f;
+    const __nv_bfloat16* pr = a.part + row * a.B * kDim + lane * 4;
     for (int k = 0; k < a.B; ++k) {
       if (!((vmask >> k) & 1u)) continue;
-      const float w = __shfl_sync(0xffffffffu, wk, k), l = __shfl_sync(0xffffffffu, lk, k);
-      const float4 v = *reinterpret_cast<const float4*>(pr + (int64_t)k * kDim);
-      acc[0] = fmaf(w, v.x, acc[0]);
-      acc[1] = fmaf(w, v.y, acc[1]);
-      acc[2] = fmaf(w, v.z, acc[2]);
-      acc[3] = fmaf(w, v.w, acc[3]);
-      L = fmaf(w, l, L);
+      const float w = __shfl_sync(0xffffffffu, wk, k);
+      float v[4];
+      load4(pr + (int64_t)k * kDim, v);
+      acc[0] = fmaf(w, v[0], acc[0]);
+      acc[1] = fmaf(w, v[1], acc[1]);
+      acc[2] = fmaf(w, v[2], acc[2]);
+      acc[3] = fmaf(w, v[3], acc[3]);
+      L += w;
     }
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -645,31 +648,36 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
 //
 // Persistent CTAs (one per SM), each walking a contiguous range of chunks with
 // four warp roles joined by mbarriers:
-//   warps 8-11 (loaders): chunk metadata into shared memory and 16-byte
+//   warps 2, 3, 6, 7 (loaders): chunk metadata into shared memory and 16-byte
 //     cp.async copies of the chunk's Q rows and the leaf's K and V rows into one
-//     of kPipeStages stages (128B-swizzled tiles); the next chunk's metadata is
-//     fetched while the current one is copied;
-//   warp 12 (one lane, MMA): S = Q.K^T into one of kPipeBufs TMEM buffers, and
+//     of kPipeStages stages (128B-swizzled tiles); a chunk's metadata is
+//     fetched two chunks ahead;
+//   warp 8 (one lane, MMA): S = Q.K^T into one of kPipeBufs TMEM buffers, and
 //     once P is in shared memory, O = P.V over the same columns;
-//   warps 0-3 (P, one TMEM lane per row): P and the (m, l) statistics from S;
-//   warps 4-7 (epilogue, same lanes): O from TMEM to the partial outputs.
+//   warps 0-1 (P, one TMEM lane per row): P and the (m, l) statistics from S;
+//   warps 4-5 (epilogue, same lanes): O from TMEM to the partial outputs.
 // Every wait is bounded; on a timeout the CTA records LSA_ERR_TIMEOUT, stops
 // its roles, waits for its copies and MMAs in flight and frees TMEM.
 
-constexpr int kPipeStages = 3;
+constexpr int kPipeStages = 4;
 constexpr int kPipeBufs = 4;                       // TMEM buffers of 128 columns
-constexpr int kPipeLoaders = 128;                  // loader threads (warps 8-11)
-constexpr int kPipeThreads = 13 * 32;
-constexpr uint32_t kStageBytes = 65536;            // Q/P 32 KB, K 16 KB, V 16 KB
+constexpr int kChunkRows = 64;                     // rows of a chunk (TMEM lanes 0-63)
+constexpr int kPipeLoaders = 128;                  // loader threads (warps 2, 3, 6, 7)
+constexpr int kPipeThreads = 9 * 32;
+// Stage: Q/P tile [0, 16 KB), K [16, 32 KB), V [32, 48 KB).  The M = 128 products
+// read 128 tile rows; rows 64-127 fall on the next 8 KB of the same stage and
+// belong to no chunk row (their results are never used).
+constexpr uint32_t kStageBytes = 49152;
+constexpr uint32_t kQHalf = kChunkRows * 128;     // bytes between the two 64-column halves of Q
 
 struct PipeMeta {
-  int32_t ent[kPipeStages][kTL];
-  int32_t qpos[kPipeStages][kTL];
+  int32_t ent[kPipeStages][kChunkRows];
+  int32_t qpos[kPipeStages][kChunkRows];
   int32_t pos[kPipeStages][kLeafKeys];
-  int32_t qrow[kPipeStages][kTL];                  // global Q row of each tile row (loaders only)
+  int32_t qrow[kPipeStages][kChunkRows];           // global Q row of each tile row (loaders only)
   int32_t info[kPipeStages][2];                    // head, entries
-  int32_t prow[kPipeBufs][kTL];                    // partial row of each TMEM lane (-1: none)
-  float2 stat[kPipeBufs][kTL];                     // (m, l) of each TMEM lane
+  int32_t prow[kPipeBufs][kChunkRows];             // partial row of each TMEM lane (-1: none)
+  float2 stat[kPipeBufs][kChunkRows];              // (m, l) of each TMEM lane
   uint64_t full[kPipeStages], sempty[kPipeStages], pready[kPipeStages];
   uint64_t sfull[kPipeBufs], ofull[kPipeBufs], tempty[kPipeBufs], mready[kPipeBufs];
   uint64_t done;
@@ -683,6 +691,16 @@ __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
 }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// Non-blocking: has the phase with this parity completed?
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return done != 0;
 }
 // Arrive on `bar` once this thread's cp.async copies issued so far have landed
 // (counts as one of the barrier's expected arrivals).
@@ -726,13 +744,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
     for (int s = 0; s < kPipeStages; ++s) {
       mbar_init(smem_u32(&M.full[s]), 2 * kPipeLoaders);
       mbar_init(smem_u32(&M.sempty[s]), 1);
-      mbar_init(smem_u32(&M.pready[s]), kTL);
+      mbar_init(smem_u32(&M.pready[s]), kChunkRows);
     }
     for (int b = 0; b < kPipeBufs; ++b) {
       mbar_init(smem_u32(&M.sfull[b]), 1);
       mbar_init(smem_u32(&M.ofull[b]), 1);
-      mbar_init(smem_u32(&M.tempty[b]), kTL);
-      mbar_init(smem_u32(&M.mready[b]), kTL);
+      mbar_init(smem_u32(&M.tempty[b]), kChunkRows);
+      mbar_init(smem_u32(&M.mready[b]), kChunkRows);
     }
     mbar_init(smem_u32(&M.done), 1);
     M.abort = 0;
@@ -751,21 +769,24 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
     set_status(a.status, LSA_ERR_TIMEOUT);
   };
 
-  if (warp >= 8 && warp < 12) {
+  if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
     // ---- loaders: lanes (lt & 15) x rows (lt >> 4) + 8 i, 16-byte chunks ----
-    const int lt = threadIdx.x - 256;
+    const int lt = ((warp & 1) | ((warp >> 1) & 2)) * 32 + lane;
     const int kr = lt & (kLeafKeys - 1);
     // descriptors come 32 at a time (one per lane) and are broadcast by shuffles;
     // a chunk's metadata is fetched two chunks before its copies are issued
     int4 dcur = lane < N ? a.cdesc[k0 + lane] : make_int4(0, 0, 0, 0);
     int4 dnxt = 32 + lane < N ? a.cdesc[k0 + 32 + lane] : make_int4(0, 0, 0, 0);
-    auto fetch = [&](int k, LoadMeta& L) {
-      const int4& dr = (k >> 5) == 0 ? dcur : dnxt;   // k lies in the current or the next block of 32
-      const int j = k & 31;
-      L.g = __shfl_sync(0xffffffffu, dr.x, j);
-      L.leaf = __shfl_sync(0xffffffffu, dr.y, j);
-      L.e_lo = __shfl_sync(0xffffffffu, dr.z, j);
-      L.ne = __shfl_sync(0xffffffffu, dr.w, j);
+    // descriptor of chunk kk seen from iteration k (kk lies in k's block of 32 or the next)
+    auto desc = [&](int kk, int k) -> int4 {
+      const int4& dr = (kk & ~31) == (k & ~31) ? dcur : dnxt;
+      const int j = kk & 31;
+      return make_int4(__shfl_sync(0xffffffffu, dr.x, j), __shfl_sync(0xffffffffu, dr.y, j),
+                       __shfl_sync(0xffffffffu, dr.z, j), __shfl_sync(0xffffffffu, dr.w, j));
+    };
+    auto fetch = [&](int kk, int k, LoadMeta& L) {
+      const int4 d = desc(kk, k);
+      L.g = d.x; L.leaf = d.y; L.e_lo = d.z; L.ne = d.w;
       const int32_t* entg = a.ent + (int64_t)L.g * a.T * a.B + L.e_lo;
       L.pos = a.leaf_index[(int64_t)L.g * a.n_tree + (int64_t)L.leaf * kLeafKeys + kr];
       const int n_rows = L.ne * a.G;
@@ -773,31 +794,38 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       L.ev = lt < L.ne ? entg[lt] : -1;
       L.eq = lt < L.ne ? a.entq[(int64_t)L.g * a.T * a.B + L.e_lo + lt] : 0;
     };
+    // L2 prefetch of the K/V rows kPrefetch chunks ahead (no shared memory needed);
+    // the row position is loaded one iteration before the prefetch is issued
+    constexpr int kPrefetch = 4;
+    int32_t pf_pos = 0, pf_g = 0;
+    auto pf_issue = [&]() {
+      const __nv_bfloat16* row = (lt < kLeafKeys ? a.K : a.V) + ((int64_t)pf_g * a.n_cap + pf_pos) * kDim;
+      asm volatile("prefetch.global.L2 [%0];\nprefetch.global.L2 [%1];" ::"l"(row), "l"(row + 64));
+    };
+    auto pf_load = [&](int kk, int k) {
+      const int4 d = desc(kk, k);
+      pf_g = d.x;
+      pf_pos = a.leaf_index[(int64_t)pf_g * a.n_tree + (int64_t)d.y * kLeafKeys + kr];
+    };
+    for (int kk = 2; kk < kPrefetch && kk < N; ++kk) {   // chunks 2 .. kPrefetch-1 right away
+      pf_load(kk, 0);
+      pf_issue();
+    }
+    if (kPrefetch < N) pf_load(kPrefetch, 0);
     LoadMeta cur, n1, n2;
-    fetch(0, cur);
-    if (N > 1) fetch(1, n1);
+    fetch(0, 0, cur);
+    if (N > 1) fetch(1, 0, n1);
     for (int k = 0; k < N; ++k) {
       if ((k & 31) == 0 && k > 0) {   // entering block k / 32: shift the descriptor window
         dcur = dnxt;
         const int64_t nb = k + 32 + lane;
         dnxt = nb < N ? a.cdesc[k0 + nb] : make_int4(0, 0, 0, 0);
       }
-      // item k + 2 lies in block (k + 2) / 32, i.e. the current one or the next
-      if (k + 2 < N) {
-        const int kb = (k + 2) & ~31;
-        const int4& dr = kb == (k & ~31) ? dcur : dnxt;
-        const int j = (k + 2) & 31;
-        n2.g = __shfl_sync(0xffffffffu, dr.x, j);
-        n2.leaf = __shfl_sync(0xffffffffu, dr.y, j);
-        n2.e_lo = __shfl_sync(0xffffffffu, dr.z, j);
-        n2.ne = __shfl_sync(0xffffffffu, dr.w, j);
-        const int32_t* entg = a.ent + (int64_t)n2.g * a.T * a.B + n2.e_lo;
-        n2.pos = a.leaf_index[(int64_t)n2.g * a.n_tree + (int64_t)n2.leaf * kLeafKeys + kr];
-        const int n_rows = n2.ne * a.G;
-        n2.qent = lt < n_rows ? entg[lt / a.G] : -1;
-        n2.ev = lt < n2.ne ? entg[lt] : -1;
-        n2.eq = lt < n2.ne ? a.entq[(int64_t)n2.g * a.T * a.B + n2.e_lo + lt] : 0;
+      if (k + kPrefetch < N) {
+        pf_issue();
+        if (k + kPrefetch + 1 < N) pf_load(k + kPrefetch + 1, k);
       }
+      if (k + 2 < N) fetch(k + 2, k, n2);
       const int s = k % kPipeStages;
       const bool ok = k < kPipeStages || mbar_wait(smem_u32(&M.sempty[s]), ((k / kPipeStages) - 1) & 1);
       const uint32_t st = sbase + s * kStageBytes;
@@ -811,19 +839,17 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
         if (!ok) fail();
         break;
       }
-      {
-        const int c = lt & 15, rg = lt >> 4;
-        const int64_t kv_base = (int64_t)cur.g * a.n_cap;
+      const int c = lt & 15, rg = lt >> 4;
+      const int64_t kv_base = (int64_t)cur.g * a.n_cap;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {   // K and V rows rg, rg + 8, ..., chunk c
-          const int kr2 = rg + 8 * i;
-          const int64_t row = kv_base + M.pos[s][kr2];
-          cp_async16(st + 32768u + sw128_off(kr2, c, kLeafKeys * 128), a.K + row * kDim + c * 8);
-          cp_async16(st + 49152u + sw128_off(kr2, c, kLeafKeys * 128), a.V + row * kDim + c * 8);
-        }
-        for (int r = rg; r < n_rows; r += 8)   // Q rows
-          cp_async16(st + sw128_off(r, c, kTL * 128), a.Q + (int64_t)M.qrow[s][r] * kDim + c * 8);
+      for (int i = 0; i < 8; ++i) {   // K and V rows rg, rg + 8, ..., chunk c
+        const int kr2 = rg + 8 * i;
+        const int64_t row = kv_base + M.pos[s][kr2];
+        cp_async16(st + 16384u + sw128_off(kr2, c, kLeafKeys * 128), a.K + row * kDim + c * 8);
+        cp_async16(st + 32768u + sw128_off(kr2, c, kLeafKeys * 128), a.V + row * kDim + c * 8);
       }
+      for (int r = rg; r < n_rows; r += 8)   // Q rows
+        cp_async16(st + sw128_off(r, c, kQHalf), a.Q + (int64_t)M.qrow[s][r] * kDim + c * 8);
       const uint32_t bar = smem_u32(&M.full[s]);
       cp_async_arrive(bar);
       if (lt < a.epc) {
@@ -839,49 +865,68 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       n1 = n2;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");   // nothing in flight when the CTA exits
-  } else if (warp == 12) {
+  } else if (warp == 8) {
     // ---- MMA issuer ----
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, 64, false, false);
       constexpr uint32_t id_pv = idesc_bf16(128, 128, false, true);
-      auto qk = [&](int k) -> bool {
+      auto qk = [&](int k) {
         const int s = k % kPipeStages, b = k % kPipeBufs;
-        if (!mbar_wait(smem_u32(&M.full[s]), (k / kPipeStages) & 1)) return false;
-        if (k >= kPipeBufs && !mbar_wait(smem_u32(&M.tempty[b]), ((k / kPipeBufs) - 1) & 1)) return false;
         fence_async_smem();    // the loaders' cp.async writes, seen through the barrier, before the MMA reads
         tc_fence_after();
-        const uint32_t sA = sbase + s * kStageBytes, sK = sA + 32768;
+        const uint32_t sA = sbase + s * kStageBytes, sK = sA + 16384;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (uint32_t)((kk & 3) * 32);
-          tc_mma(tmem + b * 128, sdesc_sw128(sA + (kk >> 2) * (kTL * 128) + koff, 16, 1024),
+          tc_mma(tmem + b * 128, sdesc_sw128(sA + (kk >> 2) * kQHalf + koff, 16, 1024),
                  sdesc_sw128(sK + (kk >> 2) * (kLeafKeys * 128) + koff, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
         }
         tc_commit(smem_u32(&M.sfull[b]));
-        return true;
       };
-      auto pv = [&](int k) -> bool {
+      auto pv = [&](int k) {
         const int s = k % kPipeStages, b = k % kPipeBufs;
-        if (!mbar_wait(smem_u32(&M.pready[s]), (k / kPipeStages) & 1)) return false;
         tc_fence_after();
-        const uint32_t sP = sbase + s * kStageBytes, sV = sP + 49152;
+        const uint32_t sP = sbase + s * kStageBytes, sV = sP + 32768;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           tc_mma(tmem + b * 128, sdesc_sw128(sP + kk * 32, 16, 1024),
                  sdesc_sw128(sV + kk * 2048, kLeafKeys * 128, 1024), id_pv, kk > 0 ? 1u : 0u);
         tc_commit(smem_u32(&M.ofull[b]));
         tc_commit(smem_u32(&M.sempty[s]));
-        return true;
       };
-      bool ok = qk(0);
-      for (int k = 1; k < N && ok && !*abort_flag; ++k) ok = pv(k - 1) && qk(k);
-      if (ok && !*abort_flag) ok = pv(N - 1);
+      // issue whichever product is ready: P.V of the oldest chunk whose P is in
+      // shared memory, else S of the next chunk whose stage has landed and whose
+      // TMEM buffer is free; give up after kWaitNs without progress
+      int nq = 0, np = 0;
+      bool ok = true;
+      uint64_t t_last = now_ns();
+      while (np < N) {
+        if (*abort_flag) {
+          ok = false;
+          break;
+        }
+        bool progressed = false;
+        if (np < nq && mbar_test(smem_u32(&M.pready[np % kPipeStages]), (np / kPipeStages) & 1)) {
+          pv(np++);
+          progressed = true;
+        } else if (nq < N && mbar_test(smem_u32(&M.full[nq % kPipeStages]), (nq / kPipeStages) & 1) &&
+                   (nq < kPipeBufs || mbar_test(smem_u32(&M.tempty[nq % kPipeBufs]), ((nq / kPipeBufs) - 1) & 1))) {
+          qk(nq++);
+          progressed = true;
+        }
+        if (progressed) {
+          t_last = now_ns();
+        } else if (now_ns() - t_last > kWaitNs) {
+          ok = false;
+          break;
+        }
+      }
       if (!ok) fail();
       tc_commit(smem_u32(&M.done));    // every MMA issued above has completed
       if (!mbar_wait(smem_u32(&M.done), 0)) fail();
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 2) {
     // ---- P: row r = TMEM lane r ----
     const int r = threadIdx.x;
     const int e = r / a.G, hh = r % a.G;
@@ -899,32 +944,43 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&M.sfull[b]), (k / kPipeBufs) & 1));
       if (!ok) break;
       tc_fence_after();
-      float sc[64];
+      float m = -INFINITY, l = 0.f;
+      if (__any_sync(0xffffffffu, tq >= 0)) {   // a warp without chunk rows leaves its P rows unused
+        float sc[64];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float t32[32];
-        tmem_ld32(tmem + b * 128 + ((uint32_t)(warp * 32) << 16) + half * 32, t32);
+        for (int half = 0; half < 2; ++half) {
+          float t32[32];
+          tmem_ld32(tmem + b * 128 + ((uint32_t)(warp * 32) << 16) + half * 32, t32);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sc[half * 32 + i] = half * 32 + i < nvis ? t32[i] * a.scale_log2 : -INFINITY;
-      }
-      float m = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) m = fmaxf(m, sc[i]);
-      const float mref = m == -INFINITY ? 0.f : m;
-      float l = 0.f;
-      char* sP = base + s * kStageBytes;
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float p0 = exp2f(sc[c * 8 + 2 * q] - mref), p1 = exp2f(sc[c * 8 + 2 * q + 1] - mref);
-          l += p0 + p1;
-          __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
-          w[q] = *reinterpret_cast<uint32_t*>(&b2);
+          for (int i = 0; i < 32; ++i) sc[half * 32 + i] = half * 32 + i < nvis ? t32[i] * a.scale_log2 : -INFINITY;
         }
-        *reinterpret_cast<uint4*>(sP + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+        float mx[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) mx[i] = fmaxf(fmaxf(sc[4 * i], sc[4 * i + 1]), fmaxf(sc[4 * i + 2], sc[4 * i + 3]));
+#pragma unroll
+        for (int w = 8; w; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) mx[i] = fmaxf(mx[i], mx[i + w]);
+        m = mx[0];
+        const float mref = m == -INFINITY ? 0.f : m;
+        float ls[8];
+        char* sP = base + s * kStageBytes;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t w[4];
+          float lc = 0.f;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const float p0 = exp2f(sc[c * 8 + 2 * q] - mref), p1 = exp2f(sc[c * 8 + 2 * q + 1] - mref);
+            lc += p0 + p1;
+            __nv_bfloat162 b2 = __floats2bfloat162_rn(p0, p1);
+            w[q] = *reinterpret_cast<uint32_t*>(&b2);
+          }
+          ls[c] = lc;
+          *reinterpret_cast<uint4*>(sP + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+              make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        l = ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
       }
       M.prow[b][r] = prow;
       M.stat[b][r] = make_float2(m, l);
@@ -934,7 +990,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       mbar_arrive(smem_u32(&M.pready[s]));
     }
     if (!ok && lane == 0) fail();
-  } else if (warp < 8) {
+  } else if (warp == 4 || warp == 5) {
     // ---- epilogue: row r = TMEM lane r ----
     const int r = (warp & 3) * 32 + lane;
     bool ok = true;
@@ -947,15 +1003,23 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       tc_fence_after();
       const int prow = M.prow[b][r];
       const float2 st = M.stat[b][r];
-      float* dst = prow >= 0 ? a.part + (int64_t)prow * kDim : nullptr;
+      __nv_bfloat16* dst = prow >= 0 ? a.part + (int64_t)prow * kDim : nullptr;
+      const float inv_l = st.y > 0.f ? 1.f / st.y : 0.f;
 #pragma unroll
       for (int part = 0; part < 4; ++part) {
         float v[32];
         tmem_ld32(tmem + b * 128 + ((uint32_t)((warp & 3) * 32) << 16) + part * 32, v);
         if (dst) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4*>(dst + part * 32 + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
+          for (int i = 0; i < 32; i += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * q] * inv_l, v[i + 2 * q + 1] * inv_l);
+              w[q] = *reinterpret_cast<uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(dst + part * 32 + i) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
         }
       }
       if (prow >= 0) a.stats[prow] = st;
@@ -1228,11 +1292,10 @@ constexpr size_t kBwdSmem = 1024 + 2 * kTL * 256 + 2 * kLeafKeys * 256 + 2 * kTL
 
 }  // namespace
 
-// Partial mode while its per-(row, leaf) outputs stay within this many bytes
-// and every gathered row index fits the tensor maps' 32-bit coordinates.
+// Partial mode while its per-(row, leaf) outputs stay within this many bytes.
 constexpr size_t kPartialMaxBytes = size_t(4) << 30;
 
-static bool partial_fits(int64_t T, int64_t Hq, int B) { return (size_t)T * Hq * B * kDim * 4 <= kPartialMaxBytes; }
+static bool partial_fits(int64_t T, int64_t Hq, int B) { return (size_t)T * Hq * B * kDim * 2 <= kPartialMaxBytes; }
 
 static int64_t max_chunks(int64_t H, int64_t NL, int64_t T, int B, int epc) {
   return H * NL + ceil_div(H * T * B, (int64_t)epc);
@@ -1244,8 +1307,8 @@ size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, 
   const size_t lists = al(H * NL * 4) + al(H * (NL + 1) * 4) + al((size_t)H * T * B * 4) + al((size_t)T * Hq * B * 8);
   const size_t red = lists + al((size_t)T * Hq * 4) + al((size_t)T * Hq * d * 4);
   if (!partial_fits(T, Hq, B)) return red;
-  const int epc = kTL / (int)(Hq / H);
-  const size_t part = lists + al((size_t)T * Hq * B * d * 4) + al((size_t)H * T * B * 4) + al(H * NL * 4) +
+  const int epc = kChunkRows / (int)(Hq / H);
+  const size_t part = lists + al((size_t)T * Hq * B * d * 2) + al((size_t)H * T * B * 4) + al(H * NL * 4) +
                       al(H * 4) + al((size_t)max_chunks(H, NL, T, B, epc) * 16);
   return part > red ? part : red;
 }
@@ -1294,14 +1357,15 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
   a.off = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * (c.NL + 1) * 4);
   a.ent = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * c.B * 4);
   a.stats = reinterpret_cast<float2*>(ws + o); o += al((size_t)c.T * c.Hq * c.B * 8);
-  a.lse2 = a.oacc = a.part = nullptr;
+  a.lse2 = a.oacc = nullptr;
+  a.part = nullptr;
   a.entq = a.coff = a.ctotal = nullptr;
   a.cdesc = nullptr;
-  a.epc = kTL / G;
+  a.epc = kChunkRows / G;
   const bool partial = partial_fits(c.T, c.Hq, c.B);
   const size_t o_lists = o;
   if (partial) {
-    a.part = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * c.B * kDim * 4);
+    a.part = reinterpret_cast<__nv_bfloat16*>(ws + o); o += al((size_t)c.T * c.Hq * c.B * kDim * 2);
     a.entq = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * c.B * 4);
     a.coff = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.NL * 4);
     a.ctotal = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * 4);
