@@ -103,9 +103,10 @@ __device__ __forceinline__ int key_slot(int i) {
 // pieces of the latent query, so one warp-wide load covers 32 / LPR whole rows.
 template <int R>
 struct RowSplit {
-  static constexpr int LPR = R >= 32 ? 8 : 4;
+  static constexpr int LPR = 4;
   static constexpr int F = R / (4 * LPR);
   static constexpr int RPI = 32 / LPR;
+  static constexpr int U = F >= 8 ? 1 : (8 / F > 4 ? 4 : 8 / F);   // rows in flight per lane group
 };
 
 // One level of the walk: score the ncand children of the kept parents (all nodes
@@ -117,7 +118,7 @@ __device__ __forceinline__ int level_pass(const SelectArgs& a, int l, int ncand,
                                           const float4 (&lat)[RowSplit<R>::F], const int32_t* kept, int b,
                                           unsigned long long* s_key, int32_t* next, bool& bad) {
   using RS = RowSplit<R>;
-  constexpr int U = 4;   // rows in flight per lane group
+  constexpr int U = RS::U;
   const int lane = threadIdx.x & 31, sub = lane % RS::LPR, grp = lane / RS::LPR;
   for (int c0 = 0; c0 < ncand; c0 += RS::RPI * U) {
     float4 x[U][RS::F];
@@ -166,8 +167,49 @@ __device__ __forceinline__ int level_pass(const SelectArgs& a, int l, int ncand,
     const int i = lane * E + e;
     v[e] = i < ncand ? s_key[key_slot<E>(i)] : 0ull;
   }
+  const int B = a.beam[l];
+  if constexpr (E >= 8) {
+    // Threshold first: the B-th largest of the lanes' two largest keys is a lower
+    // bound of the B-th largest key overall (those 64 are keys of the level), so
+    // every kept key is >= tau.  Keys are distinct, so sorting the keys >= tau
+    // gives exactly the first B of the full order; when more than 64 pass, the
+    // full sort runs instead.
+    unsigned long long smp[2] = {0ull, 0ull};
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const unsigned long long x = v[e];
+      const bool top = x > smp[0];
+      smp[1] = top ? smp[0] : (x > smp[1] ? x : smp[1]);
+      smp[0] = top ? x : smp[0];
+    }
+    warp_sort_desc<2>(smp);
+    const unsigned long long tau = __shfl_sync(0xffffffffu, ((B - 1) & 1) ? smp[1] : smp[0], (B - 1) >> 1);
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) c += (v[e] != 0ull && v[e] >= tau);
+    int inc = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, inc, 31);
+    if (total <= 64) {
+      __syncwarp();                       // every lane has read its keys: s_key is free
+      int o = inc - c;
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (v[e] != 0ull && v[e] >= tau) s_key[o++] = v[e];
+      __syncwarp();
+      unsigned long long w[2];
+      w[0] = 2 * lane < total ? s_key[2 * lane] : 0ull;
+      w[1] = 2 * lane + 1 < total ? s_key[2 * lane + 1] : 0ull;
+      warp_sort_desc<2>(w);
+      return emit_kept<2>(w, B, next);
+    }
+  }
   warp_sort_desc<E>(v);
-  return emit_kept<E>(v, a.beam[l], next);
+  return emit_kept<E>(v, B, next);
 }
 
 // Latent query of (t, g), computed by one warp: the group query (mean of the G
