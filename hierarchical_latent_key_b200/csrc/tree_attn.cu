@@ -92,16 +92,20 @@ __device__ __forceinline__ uint64_t now_ns() {
 }
 
 // Wait for phase `parity` of an mbarrier, giving up after kWaitNs.
+__device__ __forceinline__ bool mbar_try(uint32_t mbar, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(done)
+      : "r"(mbar), "r"(parity)
+      : "memory");
+  return done != 0;
+}
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity) {
+  if (mbar_try(mbar, parity)) return true;   // the common case reads no timer
   const uint64_t t0 = now_ns();
   while (true) {
-    uint32_t done;
-    asm volatile(
-        "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\nselp.u32 %0, 1, 0, p;\n}\n"
-        : "=r"(done)
-        : "r"(mbar), "r"(parity)
-        : "memory");
-    if (done) return true;
+    if (mbar_try(mbar, parity)) return true;
     if (now_ns() - t0 > kWaitNs) return false;
   }
 }
@@ -648,13 +652,14 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
 //
 // Persistent CTAs (one per SM), each walking a contiguous range of chunks with
 // four warp roles joined by mbarriers:
-//   warps 2, 3, 6, 7 (loaders): chunk metadata into shared memory and 16-byte
-//     cp.async copies of the chunk's Q rows and the leaf's K and V rows into one
-//     of kPipeStages stages (128B-swizzled tiles); a chunk's metadata is
-//     fetched two chunks ahead;
+//   warps 2-3 and 6-7 (two loader groups, alternate chunks): chunk metadata
+//     into shared memory and 16-byte cp.async copies of the chunk's Q rows and
+//     the leaf's K and V rows into one of kPipeStages stages (128B-swizzled
+//     tiles), after an L2 prefetch of the K/V rows two chunks earlier;
 //   warp 8 (one lane, MMA): S = Q.K^T into one of kPipeBufs TMEM buffers, and
 //     once P is in shared memory, O = P.V over the same columns;
-//   warps 0-1 (P, one TMEM lane per row): P and the (m, l) statistics from S;
+//   warps 0-1 and 12-13 (P, alternate chunks, one TMEM lane per row): P and
+//     the (m, l) statistics from S;
 //   warps 4-5 (epilogue, same lanes): O from TMEM to the partial outputs.
 // Every wait is bounded; on a timeout the CTA records LSA_ERR_TIMEOUT, stops
 // its roles, waits for its copies and MMAs in flight and frees TMEM.
@@ -662,8 +667,8 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
 constexpr int kPipeStages = 4;
 constexpr int kPipeBufs = 4;                       // TMEM buffers of 128 columns
 constexpr int kChunkRows = 64;                     // rows of a chunk (TMEM lanes 0-63)
-constexpr int kPipeLoaders = 128;                  // loader threads (warps 2, 3, 6, 7)
-constexpr int kPipeThreads = 9 * 32;
+constexpr int kPipeLoaders = 64;                   // threads of a loader group (warps 2-3, 6-7)
+constexpr int kPipeThreads = 14 * 32;
 // Stage: Q/P tile [0, 16 KB), K [16, 32 KB), V [32, 48 KB).  The M = 128 products
 // read 128 tile rows; rows 64-127 fall on the next 8 KB of the same stage and
 // belong to no chunk row (their results are never used).
@@ -675,6 +680,7 @@ struct PipeMeta {
   int32_t qpos[kPipeStages][kChunkRows];
   int32_t pos[kPipeStages][kLeafKeys];
   int32_t qrow[kPipeStages][kChunkRows];           // global Q row of each tile row (loaders only)
+  int32_t nvis[kPipeStages][kChunkRows];           // visible-prefix length of each entry
   int32_t info[kPipeStages][2];                    // head, entries
   int32_t prow[kPipeBufs][kChunkRows];             // partial row of each TMEM lane (-1: none)
   float2 stat[kPipeBufs][kChunkRows];              // (m, l) of each TMEM lane
@@ -708,15 +714,15 @@ __device__ __forceinline__ void cp_async_arrive(uint32_t bar) {
   asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
-// Barrier of the loader threads (named barrier 1) that also returns, in every
-// one of them, whether any of them passed `v`: their stop decisions agree, so
-// none waits at the barrier for a loader that has left.
-__device__ __forceinline__ bool loaders_any(bool v) {
+// Barrier of one loader group (named barrier 1 + group) that also returns, in
+// every one of its threads, whether any of them passed `v`: their stop decisions
+// agree, so none waits at the barrier for a loader that has left.
+__device__ __forceinline__ bool loaders_any(bool v, int group) {
   uint32_t r;
   asm volatile(
-      "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.or.pred q, 1, %2, p;\nselp.u32 %0, 1, 0, q;\n}"
+      "{\n.reg .pred p, q;\nsetp.ne.u32 p, %1, 0;\nbar.red.or.pred q, %2, %3, p;\nselp.u32 %0, 1, 0, q;\n}"
       : "=r"(r)
-      : "r"((uint32_t)v), "n"(kPipeLoaders)
+      : "r"((uint32_t)v), "r"(1 + group), "n"(kPipeLoaders)
       : "memory");
   return r != 0;
 }
@@ -770,93 +776,106 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
   };
 
   if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
-    // ---- loaders: lanes (lt & 15) x rows (lt >> 4) + 8 i, 16-byte chunks ----
+    // ---- loaders: two groups of 64 threads take alternate chunks (and stages);
+    // in a group, lanes (j & 15) x rows (j >> 4) + 4 i copy 16-byte pieces ----
     const int lt = ((warp & 1) | ((warp >> 1) & 2)) * 32 + lane;
-    const int kr = lt & (kLeafKeys - 1);
+    const int group = lt >> 6, j = lt & 63;
     // descriptors come 32 at a time (one per lane) and are broadcast by shuffles;
-    // a chunk's metadata is fetched two chunks before its copies are issued
+    // a chunk's metadata is fetched two group iterations before its copies
     int4 dcur = lane < N ? a.cdesc[k0 + lane] : make_int4(0, 0, 0, 0);
     int4 dnxt = 32 + lane < N ? a.cdesc[k0 + 32 + lane] : make_int4(0, 0, 0, 0);
-    // descriptor of chunk kk seen from iteration k (kk lies in k's block of 32 or the next)
-    auto desc = [&](int kk, int k) -> int4 {
-      const int4& dr = (kk & ~31) == (k & ~31) ? dcur : dnxt;
-      const int j = kk & 31;
-      return make_int4(__shfl_sync(0xffffffffu, dr.x, j), __shfl_sync(0xffffffffu, dr.y, j),
-                       __shfl_sync(0xffffffffu, dr.z, j), __shfl_sync(0xffffffffu, dr.w, j));
+    int blk = 0;
+    // descriptor of chunk kk (in block blk or the next)
+    auto desc = [&](int kk) -> int4 {
+      const int4& dr = (kk >> 5) == blk ? dcur : dnxt;
+      const int q = kk & 31;
+      return make_int4(__shfl_sync(0xffffffffu, dr.x, q), __shfl_sync(0xffffffffu, dr.y, q),
+                       __shfl_sync(0xffffffffu, dr.z, q), __shfl_sync(0xffffffffu, dr.w, q));
     };
-    auto fetch = [&](int kk, int k, LoadMeta& L) {
-      const int4 d = desc(kk, k);
+    auto fetch = [&](int kk, LoadMeta& L) {
+      const int4 d = desc(kk);
       L.g = d.x; L.leaf = d.y; L.e_lo = d.z; L.ne = d.w;
       const int32_t* entg = a.ent + (int64_t)L.g * a.T * a.B + L.e_lo;
-      L.pos = a.leaf_index[(int64_t)L.g * a.n_tree + (int64_t)L.leaf * kLeafKeys + kr];
+      L.pos = a.leaf_index[(int64_t)L.g * a.n_tree + (int64_t)L.leaf * kLeafKeys + j];
       const int n_rows = L.ne * a.G;
-      L.qent = lt < n_rows ? entg[lt / a.G] : -1;
-      L.ev = lt < L.ne ? entg[lt] : -1;
-      L.eq = lt < L.ne ? a.entq[(int64_t)L.g * a.T * a.B + L.e_lo + lt] : 0;
+      L.qent = j < n_rows ? entg[j / a.G] : -1;
+      L.ev = j < L.ne ? entg[j] : -1;
+      L.eq = j < L.ne ? a.entq[(int64_t)L.g * a.T * a.B + L.e_lo + j] : 0;
     };
-    // L2 prefetch of the K/V rows kPrefetch chunks ahead (no shared memory needed);
-    // the row position is loaded one iteration before the prefetch is issued
-    constexpr int kPrefetch = 4;
+    // L2 prefetch of the K/V rows two group iterations ahead (no shared memory
+    // needed); the row position is loaded one iteration before the prefetch
     int32_t pf_pos = 0, pf_g = 0;
     auto pf_issue = [&]() {
-      const __nv_bfloat16* row = (lt < kLeafKeys ? a.K : a.V) + ((int64_t)pf_g * a.n_cap + pf_pos) * kDim;
-      asm volatile("prefetch.global.L2 [%0];\nprefetch.global.L2 [%1];" ::"l"(row), "l"(row + 64));
+      const int64_t row = ((int64_t)pf_g * a.n_cap + pf_pos) * kDim;
+      asm volatile("prefetch.global.L2 [%0];\nprefetch.global.L2 [%1];\nprefetch.global.L2 [%2];\nprefetch.global.L2 [%3];"
+                   ::"l"(a.K + row), "l"(a.K + row + 64), "l"(a.V + row), "l"(a.V + row + 64));
     };
-    auto pf_load = [&](int kk, int k) {
-      const int4 d = desc(kk, k);
+    auto pf_load = [&](int kk) {
+      const int4 d = desc(kk);
       pf_g = d.x;
-      pf_pos = a.leaf_index[(int64_t)pf_g * a.n_tree + (int64_t)d.y * kLeafKeys + kr];
+      pf_pos = a.leaf_index[(int64_t)pf_g * a.n_tree + (int64_t)d.y * kLeafKeys + j];
     };
-    for (int kk = 2; kk < kPrefetch && kk < N; ++kk) {   // chunks 2 .. kPrefetch-1 right away
-      pf_load(kk, 0);
+    if (group + 2 < N) {   // the group's second chunk right away
+      pf_load(group + 2);
       pf_issue();
     }
-    if (kPrefetch < N) pf_load(kPrefetch, 0);
+    if (group + 4 < N) pf_load(group + 4);
     LoadMeta cur, n1, n2;
-    fetch(0, 0, cur);
-    if (N > 1) fetch(1, 0, n1);
-    for (int k = 0; k < N; ++k) {
-      if ((k & 31) == 0 && k > 0) {   // entering block k / 32: shift the descriptor window
+    if (group < N) fetch(group, cur);
+    if (group + 2 < N) fetch(group + 2, n1);
+    for (int k = group; k < N; k += 2) {
+      if ((k >> 5) != blk) {   // entering block k / 32: shift the descriptor window
+        blk = k >> 5;
         dcur = dnxt;
-        const int64_t nb = k + 32 + lane;
+        const int64_t nb = (int64_t)(blk + 1) * 32 + lane;
         dnxt = nb < N ? a.cdesc[k0 + nb] : make_int4(0, 0, 0, 0);
       }
-      if (k + kPrefetch < N) {
+      if (k + 4 < N) {
         pf_issue();
-        if (k + kPrefetch + 1 < N) pf_load(k + kPrefetch + 1, k);
+        if (k + 6 < N) pf_load(k + 6);
       }
-      if (k + 2 < N) fetch(k + 2, k, n2);
+      if (k + 4 < N) fetch(k + 4, n2);
       const int s = k % kPipeStages;
       const bool ok = k < kPipeStages || mbar_wait(smem_u32(&M.sempty[s]), ((k / kPipeStages) - 1) & 1);
       const uint32_t st = sbase + s * kStageBytes;
       // row addresses through shared memory, so that 16 lanes copy one 256-B row
       const int n_rows = cur.ne * a.G;
       if (ok) {
-        if (lt < kLeafKeys) M.pos[s][lt] = cur.pos;
-        if (lt < n_rows) M.qrow[s][lt] = (cur.qent >> 6) * a.Hq + cur.g * a.G + lt % a.G;
+        M.pos[s][j] = cur.pos;
+        if (j < n_rows) M.qrow[s][j] = (cur.qent >> 6) * a.Hq + cur.g * a.G + j % a.G;
       }
-      if (loaders_any(!ok || *abort_flag != 0)) {   // also the barrier before the copies read them
+      if (loaders_any(!ok || *abort_flag != 0, group)) {   // also the barrier before the copies read them
         if (!ok) fail();
         break;
       }
-      const int c = lt & 15, rg = lt >> 4;
+      const int c = j & 15, rg = j >> 4;
       const int64_t kv_base = (int64_t)cur.g * a.n_cap;
+      // all row addresses first: each copy's asm is a compiler memory barrier, so a
+      // shared-memory read between two copies would wait out its full latency
+      int32_t kpos[16], qr[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {   // K and V rows rg, rg + 8, ..., chunk c
-        const int kr2 = rg + 8 * i;
-        const int64_t row = kv_base + M.pos[s][kr2];
+      for (int i = 0; i < 16; ++i) {
+        kpos[i] = M.pos[s][rg + 4 * i];
+        qr[i] = rg + 4 * i < n_rows ? M.qrow[s][rg + 4 * i] : -1;
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {   // K and V rows rg, rg + 4, ..., chunk c
+        const int kr2 = rg + 4 * i;
+        const int64_t row = kv_base + kpos[i];
         cp_async16(st + 16384u + sw128_off(kr2, c, kLeafKeys * 128), a.K + row * kDim + c * 8);
         cp_async16(st + 32768u + sw128_off(kr2, c, kLeafKeys * 128), a.V + row * kDim + c * 8);
       }
-      for (int r = rg; r < n_rows; r += 8)   // Q rows
-        cp_async16(st + sw128_off(r, c, kQHalf), a.Q + (int64_t)M.qrow[s][r] * kDim + c * 8);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)   // Q rows rg, rg + 4, ... below n_rows
+        if (qr[i] >= 0) cp_async16(st + sw128_off(rg + 4 * i, c, kQHalf), a.Q + (int64_t)qr[i] * kDim + c * 8);
       const uint32_t bar = smem_u32(&M.full[s]);
       cp_async_arrive(bar);
-      if (lt < a.epc) {
-        M.ent[s][lt] = cur.ev;
-        M.qpos[s][lt] = cur.eq;
+      if (j < a.epc) {
+        M.ent[s][j] = cur.ev;
+        M.qpos[s][j] = cur.eq;
+        M.nvis[s][j] = cur.ev >= 0 ? visible_prefix(M.pos[s], (int64_t)cur.eq) : 0;
       }
-      if (lt == 0) {
+      if (j == 0) {
         M.info[s][0] = cur.g;
         M.info[s][1] = cur.ne;
       }
@@ -926,12 +945,14 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       if (!mbar_wait(smem_u32(&M.done), 0)) fail();
     }
     __syncwarp();
-  } else if (warp < 2) {
-    // ---- P: row r = TMEM lane r ----
-    const int r = threadIdx.x;
+  } else if (warp < 2 || warp == 12 || warp == 13) {
+    // ---- P: two warp pairs take alternate chunks; row r = TMEM lane r ----
+    const int r = (warp & 1) * 32 + lane;
+    const int pgrp = warp >= 12 ? 1 : 0;
     const int e = r / a.G, hh = r % a.G;
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     bool ok = true;
-    for (int k = 0; k < N; ++k) {
+    for (int k = pgrp; k < N; k += 2) {
       if (aborted()) break;
       const int s = k % kPipeStages, b = k % kPipeBufs;
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&M.full[s]), (k / kPipeStages) & 1));
@@ -939,7 +960,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       const int g = M.info[s][0];
       const int v = M.ent[s][e];
       const int64_t tq = v >= 0 ? (v >> 6) : -1;
-      const int nvis = tq >= 0 ? visible_prefix(M.pos[s], (int64_t)M.qpos[s][e]) : 0;
+      const int nvis = M.nvis[s][e];
       const int prow = tq >= 0 ? (int)((tq * a.Hq + g * a.G + hh) * a.B + (v & 63)) : -1;
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&M.sfull[b]), (k / kPipeBufs) & 1));
       if (!ok) break;
@@ -950,7 +971,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           float t32[32];
-          tmem_ld32(tmem + b * 128 + ((uint32_t)(warp * 32) << 16) + half * 32, t32);
+          tmem_ld32(tmem + b * 128 + lane_base + half * 32, t32);
 #pragma unroll
           for (int i = 0; i < 32; ++i) sc[half * 32 + i] = half * 32 + i < nvis ? t32[i] * a.scale_log2 : -INFINITY;
         }
