@@ -656,11 +656,12 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
 //     into shared memory and 16-byte cp.async copies of the chunk's Q rows and
 //     the leaf's K and V rows into one of kPipeStages stages (128B-swizzled
 //     tiles), after an L2 prefetch of the K/V rows two chunks earlier;
-//   warp 8 (one lane, MMA): S = Q.K^T into one of kPipeBufs TMEM buffers, and
+//   warp 11 (one lane, MMA): S = Q.K^T into one of kPipeBufs TMEM buffers, and
 //     once P is in shared memory, O = P.V over the same columns;
 //   warps 0-1 and 12-13 (P, alternate chunks, one TMEM lane per row): P and
 //     the (m, l) statistics from S;
-//   warps 4-5 (epilogue, same lanes): O from TMEM to the partial outputs.
+//   warps 4-5 and 8-9 (epilogue, alternate chunks, same lanes): O from TMEM to
+//     the partial outputs.
 // Every wait is bounded; on a timeout the CTA records LSA_ERR_TIMEOUT, stops
 // its roles, waits for its copies and MMAs in flight and frees TMEM.
 
@@ -884,7 +885,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       n1 = n2;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");   // nothing in flight when the CTA exits
-  } else if (warp == 8) {
+  } else if (warp == 11) {
     // ---- MMA issuer ----
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, 64, false, false);
@@ -916,9 +917,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       // issue whichever product is ready: P.V of the oldest chunk whose P is in
       // shared memory, else S of the next chunk whose stage has landed and whose
       // TMEM buffer is free; give up after kWaitNs without progress
-      int nq = 0, np = 0;
+      int nq = 0, np = 0, idle = 0;
       bool ok = true;
-      uint64_t t_last = now_ns();
+      uint64_t t_idle = 0;
       while (np < N) {
         if (*abort_flag) {
           ok = false;
@@ -934,10 +935,15 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
           progressed = true;
         }
         if (progressed) {
-          t_last = now_ns();
-        } else if (now_ns() - t_last > kWaitNs) {
-          ok = false;
-          break;
+          idle = 0;
+        } else if ((++idle & 63) == 0) {   // the timer is read once every 64 idle polls
+          const uint64_t t = now_ns();
+          if (idle == 64) {
+            t_idle = t;
+          } else if (t - t_idle > kWaitNs) {
+            ok = false;
+            break;
+          }
         }
       }
       if (!ok) fail();
@@ -1011,11 +1017,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       mbar_arrive(smem_u32(&M.pready[s]));
     }
     if (!ok && lane == 0) fail();
-  } else if (warp == 4 || warp == 5) {
-    // ---- epilogue: row r = TMEM lane r ----
+  } else if (warp == 4 || warp == 5 || warp == 8 || warp == 9) {
+    // ---- epilogue: two warp pairs take alternate chunks; row r = TMEM lane r ----
     const int r = (warp & 3) * 32 + lane;
+    const int egrp = warp >= 8 ? 1 : 0;
     bool ok = true;
-    for (int k = 0; k < N; ++k) {
+    for (int k = egrp; k < N; k += 2) {
       if (aborted()) break;
       const int b = k % kPipeBufs;
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&M.mready[b]), (k / kPipeBufs) & 1) &&
