@@ -609,6 +609,13 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
   const int lane = threadIdx.x & 31;
   if (row >= a.T * a.Hq) return;
   const int64_t t = row / a.Hq, head = row % a.Hq, g = head / a.G;
+  // all of the row's partials are requested at once, together with the statistics
+  // (ranks without a partial are read too, the workspace is readable, and skipped)
+  const __nv_bfloat16* pr = a.part + row * a.B * kDim + lane * 4;
+  uint2 raw[LSA_MAX_BEAM];
+#pragma unroll
+  for (int k = 0; k < LSA_MAX_BEAM; ++k)
+    raw[k] = k < a.B ? *reinterpret_cast<const uint2*>(pr + (int64_t)k * kDim) : make_uint2(0u, 0u);
   bool valid = false;
   float mk = -INFINITY, lk = 0.f;
   if (lane < a.B && a.leaves[(g * a.T + t) * a.B + lane] >= 0) {
@@ -621,22 +628,20 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   const unsigned vmask = __ballot_sync(0xffffffffu, valid);
+  const float wk = valid ? exp2f(mk - M) * lk : 0.f;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
   float L = 0.f;
-  if (vmask) {
-    const float wk = valid ? exp2f(mk - M) * lk : 0.f;
-    const __nv_bfloat16* pr = a.part + row * a.B * kDim + lane * 4;
-    for (int k = 0; k < a.B; ++k) {
-      if (!((vmask >> k) & 1u)) continue;
-      const float w = __shfl_sync(0xffffffffu, wk, k);
-      float v[4];
-      load4(pr + (int64_t)k * kDim, v);
-      acc[0] = fmaf(w, v[0], acc[0]);
-      acc[1] = fmaf(w, v[1], acc[1]);
-      acc[2] = fmaf(w, v[2], acc[2]);
-      acc[3] = fmaf(w, v[3], acc[3]);
-      L += w;
-    }
+#pragma unroll
+  for (int k = 0; k < LSA_MAX_BEAM; ++k) {   // rank order
+    if (!((vmask >> k) & 1u)) continue;
+    const float w = __shfl_sync(0xffffffffu, wk, k);
+    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[k].x));
+    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[k].y));
+    acc[0] = fmaf(w, lo.x, acc[0]);
+    acc[1] = fmaf(w, lo.y, acc[1]);
+    acc[2] = fmaf(w, hi.x, acc[2]);
+    acc[3] = fmaf(w, hi.y, acc[3]);
+    L += w;
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
   __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
