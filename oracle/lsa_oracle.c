@@ -428,9 +428,22 @@ int orc_select(const double *qlat, int64_t T, int32_t r, const int32_t *branchin
 /* LSE = log sum exp(logit).  No visible key: O = 0, LSE = -inf.              */
 /* Q, O: [T, G, d];  K, V: [n_cap, d];  idx: [T, K_sel];  LSE: [T, G].        */
 /* ------------------------------------------------------------------------- */
+static int orc_cmp_i64(const void *x, const void *y) {
+  const int64_t a = *(const int64_t *)x, b = *(const int64_t *)y;
+  return (a > b) - (a < b);
+}
+
+/* Keys query t attends to: its index list, the dense tail range and, when n_sink
+ * or window is positive, the first n_sink positions (sink tokens) and the window
+ * positions q_pos - window + 1 .. q_pos (kongchang.com, "How LSA Sidesteps
+ * Per-Key Scoring with Hierarchical Clustering": the keys taken from the chosen
+ * clusters are used together with a window of recent tokens and a few initial
+ * sink tokens).  With sink or window the key set is a set: it is sorted and a
+ * position listed twice counts once. */
 static int64_t orc_visible_keys(int64_t t, const int32_t *idx, int32_t K_sel,
                                 const int32_t *q_pos, int32_t causal, int64_t tail_begin,
-                                int64_t tail_end, int64_t n_cap, int64_t *out) {
+                                int64_t tail_end, int64_t n_cap, int32_t n_sink, int32_t window,
+                                int64_t *out) {
   int64_t cnt = 0;
   for (int32_t k = 0; k < K_sel; ++k) {
     int64_t j = idx[t * K_sel + k];
@@ -442,22 +455,34 @@ static int64_t orc_visible_keys(int64_t t, const int32_t *idx, int32_t K_sel,
     if (causal && j > q_pos[t]) continue;
     out[cnt++] = j;
   }
-  return cnt;
+  if (n_sink == 0 && window == 0) return cnt;
+  for (int64_t j = 0; j < n_sink && j < n_cap; ++j)
+    if (j <= q_pos[t]) out[cnt++] = j;
+  for (int64_t j = (int64_t)q_pos[t] - window + 1; j <= q_pos[t]; ++j)
+    if (j >= 0 && j < n_cap) out[cnt++] = j;
+  qsort(out, (size_t)cnt, sizeof(int64_t), orc_cmp_i64);
+  int64_t u = 0;
+  for (int64_t k = 0; k < cnt; ++k)
+    if (u == 0 || out[k] != out[u - 1]) out[u++] = out[k];
+  return u;
 }
 
-int orc_attn_fwd(const double *Q, int64_t T, int32_t G, int32_t d, const double *K,
-                 const double *V, int64_t n_cap, const int32_t *idx, int32_t K_sel,
-                 const int32_t *q_pos, int32_t causal, int64_t tail_begin,
-                 int64_t tail_end, double scale, double *O, double *LSE) {
+static int orc_attn_fwd_keys(const double *Q, int64_t T, int32_t G, int32_t d, const double *K,
+                             const double *V, int64_t n_cap, const int32_t *idx, int32_t K_sel,
+                             const int32_t *q_pos, int32_t causal, int64_t tail_begin,
+                             int64_t tail_end, int32_t n_sink, int32_t window, double scale,
+                             double *O, double *LSE) {
   if (!Q || !K || !V || !O || !LSE || (K_sel > 0 && !idx) || (causal && !q_pos))
     return ORC_ERR_ARG;
   if (tail_begin < 0 || tail_end < tail_begin || tail_end > n_cap) return ORC_ERR_SHAPE;
-  const int64_t max_keys = K_sel + (tail_end - tail_begin);
+  if (n_sink < 0 || window < 0 || ((n_sink > 0 || window > 0) && !causal)) return ORC_ERR_ARG;
+  const int64_t max_keys = K_sel + (tail_end - tail_begin) + n_sink + window;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t t = 0; t < T; ++t) {
     int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (max_keys + 1));
     double *logit = (double *)malloc(sizeof(double) * (max_keys + 1));
-    int64_t cnt = orc_visible_keys(t, idx, K_sel, q_pos, causal, tail_begin, tail_end, n_cap, keys);
+    int64_t cnt = orc_visible_keys(t, idx, K_sel, q_pos, causal, tail_begin, tail_end, n_cap, n_sink,
+                                   window, keys);
     for (int32_t h = 0; h < G; ++h) {
       const double *q = &Q[(t * G + h) * d];
       double *o = &O[(t * G + h) * d];
@@ -486,29 +511,48 @@ int orc_attn_fwd(const double *Q, int64_t T, int32_t G, int32_t d, const double 
   return ORC_OK;
 }
 
+int orc_attn_fwd(const double *Q, int64_t T, int32_t G, int32_t d, const double *K,
+                 const double *V, int64_t n_cap, const int32_t *idx, int32_t K_sel,
+                 const int32_t *q_pos, int32_t causal, int64_t tail_begin,
+                 int64_t tail_end, double scale, double *O, double *LSE) {
+  return orc_attn_fwd_keys(Q, T, G, d, K, V, n_cap, idx, K_sel, q_pos, causal, tail_begin, tail_end, 0, 0,
+                           scale, O, LSE);
+}
+
+/* The same with the sink and recent-window keys added (causal). */
+int orc_attn_fwd_sw(const double *Q, int64_t T, int32_t G, int32_t d, const double *K,
+                    const double *V, int64_t n_cap, const int32_t *idx, int32_t K_sel,
+                    const int32_t *q_pos, int64_t tail_begin, int64_t tail_end, int32_t n_sink,
+                    int32_t window, double scale, double *O, double *LSE) {
+  return orc_attn_fwd_keys(Q, T, G, d, K, V, n_cap, idx, K_sel, q_pos, 1, tail_begin, tail_end, n_sink,
+                           window, scale, O, LSE);
+}
+
 /* Gradient of the same sparse attention for a fixed key selection, from the
  * upstream gradient dO (standard softmax-attention calculus restricted to the
  * visible (query, key) pairs):  P = softmax(logit);  dV_j += P_j dO;
  * dP_j = <dO, v_j>;  dS_j = P_j (dP_j - sum_i P_i dP_i);  dQ = scale sum_j dS_j k_j;
  * dK_j += scale dS_j q.  dK and dV ([n_cap, d]) are overwritten and sum over
  * the G heads of the group and over every query that sees key j. */
-int orc_attn_bwd(const double *Q, int64_t T, int32_t G, int32_t d, const double *K,
-                 const double *V, int64_t n_cap, const int32_t *idx, int32_t K_sel,
-                 const int32_t *q_pos, int32_t causal, int64_t tail_begin,
-                 int64_t tail_end, double scale, const double *dO, double *dQ,
-                 double *dK, double *dV) {
+static int orc_attn_bwd_keys(const double *Q, int64_t T, int32_t G, int32_t d, const double *K,
+                             const double *V, int64_t n_cap, const int32_t *idx, int32_t K_sel,
+                             const int32_t *q_pos, int32_t causal, int64_t tail_begin,
+                             int64_t tail_end, int32_t n_sink, int32_t window, double scale,
+                             const double *dO, double *dQ, double *dK, double *dV) {
   if (!Q || !K || !V || !dO || !dQ || !dK || !dV || (K_sel > 0 && !idx) || (causal && !q_pos))
     return ORC_ERR_ARG;
   if (tail_begin < 0 || tail_end < tail_begin || tail_end > n_cap) return ORC_ERR_SHAPE;
+  if (n_sink < 0 || window < 0 || ((n_sink > 0 || window > 0) && !causal)) return ORC_ERR_ARG;
   memset(dK, 0, sizeof(double) * (size_t)(n_cap * d));
   memset(dV, 0, sizeof(double) * (size_t)(n_cap * d));
-  const int64_t max_keys = K_sel + (tail_end - tail_begin);
+  const int64_t max_keys = K_sel + (tail_end - tail_begin) + n_sink + window;
 #pragma omp parallel for schedule(dynamic, 1)
   for (int64_t t = 0; t < T; ++t) {
     int64_t *keys = (int64_t *)malloc(sizeof(int64_t) * (max_keys + 1));
     double *p = (double *)malloc(sizeof(double) * (max_keys + 1));
     double *dp = (double *)malloc(sizeof(double) * (max_keys + 1));
-    int64_t cnt = orc_visible_keys(t, idx, K_sel, q_pos, causal, tail_begin, tail_end, n_cap, keys);
+    int64_t cnt = orc_visible_keys(t, idx, K_sel, q_pos, causal, tail_begin, tail_end, n_cap, n_sink,
+                                   window, keys);
     for (int32_t h = 0; h < G; ++h) {
       const double *q = &Q[(t * G + h) * d];
       const double *go = &dO[(t * G + h) * d];
@@ -553,4 +597,23 @@ int orc_attn_bwd(const double *Q, int64_t T, int32_t G, int32_t d, const double 
     free(dp);
   }
   return ORC_OK;
+}
+
+int orc_attn_bwd(const double *Q, int64_t T, int32_t G, int32_t d, const double *K,
+                 const double *V, int64_t n_cap, const int32_t *idx, int32_t K_sel,
+                 const int32_t *q_pos, int32_t causal, int64_t tail_begin,
+                 int64_t tail_end, double scale, const double *dO, double *dQ,
+                 double *dK, double *dV) {
+  return orc_attn_bwd_keys(Q, T, G, d, K, V, n_cap, idx, K_sel, q_pos, causal, tail_begin, tail_end, 0, 0,
+                           scale, dO, dQ, dK, dV);
+}
+
+/* Backward of orc_attn_fwd_sw. */
+int orc_attn_bwd_sw(const double *Q, int64_t T, int32_t G, int32_t d, const double *K,
+                    const double *V, int64_t n_cap, const int32_t *idx, int32_t K_sel,
+                    const int32_t *q_pos, int64_t tail_begin, int64_t tail_end, int32_t n_sink,
+                    int32_t window, double scale, const double *dO, double *dQ, double *dK,
+                    double *dV) {
+  return orc_attn_bwd_keys(Q, T, G, d, K, V, n_cap, idx, K_sel, q_pos, 1, tail_begin, tail_end, n_sink,
+                           window, scale, dO, dQ, dK, dV);
 }

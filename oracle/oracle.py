@@ -103,6 +103,10 @@ def _declare(lib):
                                         f64, P, P]),
         "orc_attn_bwd": (ctypes.c_int, [P, i64, i32, i32, P, P, i64, P, i32, P, i32, i64, i64,
                                         f64, P, P, P, P]),
+        "orc_attn_fwd_sw": (ctypes.c_int, [P, i64, i32, i32, P, P, i64, P, i32, P, i64, i64, i32, i32,
+                                           f64, P, P]),
+        "orc_attn_bwd_sw": (ctypes.c_int, [P, i64, i32, i32, P, P, i64, P, i32, P, i64, i64, i32, i32,
+                                           f64, P, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -269,8 +273,10 @@ def select(qlat, tree: Tree, beam, q_pos=None, trace: bool = False):
 
 # --- attention -------------------------------------------------------------------
 
-def attn_fwd(Qg, K, V, idx, q_pos=None, causal=False, tail=(0, 0), scale=None):
-    """Qg: [T, G, d]; K, V: [n_cap, d]; idx: [T, K_sel] or None -> (O [T,G,d], LSE [T,G])."""
+def attn_fwd(Qg, K, V, idx, q_pos=None, causal=False, tail=(0, 0), scale=None, sink=0, window=0):
+    """Qg: [T, G, d]; K, V: [n_cap, d]; idx: [T, K_sel] or None -> (O [T,G,d], LSE [T,G]).
+    sink / window > 0 (causal only): the first `sink` positions and the `window` positions up to
+    q_pos join every query's key set, each key counted once."""
     Qg, K, V = _f64(Qg), _f64(K), _f64(V)
     T, G, d = Qg.shape
     n_cap = K.shape[0]
@@ -283,14 +289,20 @@ def attn_fwd(Qg, K, V, idx, q_pos=None, causal=False, tail=(0, 0), scale=None):
     scale = 1.0 / np.sqrt(d) if scale is None else float(scale)
     O = np.empty((T, G, d), np.float64)
     LSE = np.empty((T, G), np.float64)
+    if sink or window:
+        assert causal, "sink and window keys need query positions (causal)"
+        _check(load().orc_attn_fwd_sw(_p(Qg), T, G, d, _p(K), _p(V), n_cap, _p(idx_a), K_sel, _p(qp),
+                                      int(tail[0]), int(tail[1]), int(sink), int(window), scale,
+                                      _p(O), _p(LSE)), "orc_attn_fwd_sw")
+        return O, LSE
     _check(load().orc_attn_fwd(_p(Qg), T, G, d, _p(K), _p(V), n_cap, _p(idx_a), K_sel, _p(qp),
                                int(bool(causal)), int(tail[0]), int(tail[1]), scale,
                                _p(O), _p(LSE)), "orc_attn_fwd")
     return O, LSE
 
 
-def attn_bwd(Qg, K, V, idx, dO, q_pos=None, causal=False, tail=(0, 0), scale=None):
-    """Returns (dQ [T,G,d], dK [n_cap,d], dV [n_cap,d])."""
+def attn_bwd(Qg, K, V, idx, dO, q_pos=None, causal=False, tail=(0, 0), scale=None, sink=0, window=0):
+    """Returns (dQ [T,G,d], dK [n_cap,d], dV [n_cap,d]); sink / window as in attn_fwd."""
     Qg, K, V, dO = _f64(Qg), _f64(K), _f64(V), _f64(dO)
     T, G, d = Qg.shape
     n_cap = K.shape[0]
@@ -304,6 +316,12 @@ def attn_bwd(Qg, K, V, idx, dO, q_pos=None, causal=False, tail=(0, 0), scale=Non
     dQ = np.empty((T, G, d), np.float64)
     dK = np.empty((n_cap, d), np.float64)
     dV = np.empty((n_cap, d), np.float64)
+    if sink or window:
+        assert causal, "sink and window keys need query positions (causal)"
+        _check(load().orc_attn_bwd_sw(_p(Qg), T, G, d, _p(K), _p(V), n_cap, _p(idx_a), K_sel, _p(qp),
+                                      int(tail[0]), int(tail[1]), int(sink), int(window), scale, _p(dO),
+                                      _p(dQ), _p(dK), _p(dV)), "orc_attn_bwd_sw")
+        return dQ, dK, dV
     _check(load().orc_attn_bwd(_p(Qg), T, G, d, _p(K), _p(V), n_cap, _p(idx_a), K_sel, _p(qp),
                                int(bool(causal)), int(tail[0]), int(tail[1]), scale, _p(dO),
                                _p(dQ), _p(dK), _p(dV)), "orc_attn_bwd")

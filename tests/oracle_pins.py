@@ -430,4 +430,65 @@ def pin_backward_finite_differences():
         assert abs(fd - grad[pick]) < 1e-6 * max(1.0, abs(fd)), (which, fd, grad[pick])
 
 
+
+def _sink_window_mask(idx, n, tail, q_pos, sink, window):
+    """Union of the index list, the tail, the first `sink` positions and the `window`
+    positions up to q_pos, then the causal cut (kongchang.com, "How LSA Sidesteps Per-Key
+    Scoring with Hierarchical Clustering": chosen keys plus recent and sink tokens)."""
+    m = _mask_from(idx, n, tail, q_pos, True)
+    for t in range(idx.shape[0]):
+        m[t, :sink] = True
+        m[t, max(0, int(q_pos[t]) - window + 1):int(q_pos[t]) + 1] = True
+        m[t, int(q_pos[t]) + 1:] = False
+    return m
+
+
+def pin_attention_sink_window():
+    rng, Qg, K, V, idx = _attn_case(4)
+    T = Qg.shape[0]
+    n, d = K.shape
+    scale = 1 / np.sqrt(d)
+    q_pos = rng.integers(n // 2, n, T).astype(np.int32)
+    q_pos[0] = 1                                   # a query before the end of the sink range
+    # a window reaching position 0 is full causal attention, whatever the index list says
+    O, _ = orc.attn_fwd(Qg, K, V, idx, q_pos=q_pos, causal=True, scale=scale, window=n)
+    full = _sdpa_dense(Qg, K, V, np.arange(n)[None, :] <= q_pos[:, None], scale)
+    np.testing.assert_allclose(O, full, rtol=1e-10, atol=1e-12)
+    # index list + tail + sink + window = SDPA over the union mask
+    sink, window = 3, 5
+    O, LSE = orc.attn_fwd(Qg, K, V, idx, q_pos=q_pos, causal=True, tail=(n - 8, n), scale=scale, sink=sink,
+                          window=window)
+    m = _sink_window_mask(idx, n, (n - 8, n), q_pos, sink, window)
+    np.testing.assert_allclose(O, _sdpa_dense(Qg, K, V, m, scale), rtol=1e-10, atol=1e-12)
+    s = scale * np.einsum("tgd,nd->tgn", Qg, K)
+    lse = np.log(np.where(m[:, None, :], np.exp(s), 0.0).sum(-1))
+    np.testing.assert_allclose(LSE, lse, rtol=1e-10)
+    # a key listed again in the index list (inside the window or the sink) counts once
+    extra = np.stack([np.r_[np.arange(q_pos[t] - 2, q_pos[t] + 1).clip(0), [0, 1]] for t in range(T)]).astype(np.int32)
+    dup = np.concatenate([idx, extra], 1)
+    a, la = orc.attn_fwd(Qg, K, V, idx, q_pos=q_pos, causal=True, scale=scale, sink=sink, window=window)
+    b, lb = orc.attn_fwd(Qg, K, V, dup, q_pos=q_pos, causal=True, scale=scale, sink=sink, window=window)
+    assert np.array_equal(a, b) and np.array_equal(la, lb)
+
+
+def pin_backward_sink_window_autograd():
+    rng, Qg, K, V, idx = _attn_case(5)
+    n, d = K.shape
+    q_pos = rng.integers(n // 2, n, Qg.shape[0]).astype(np.int32)
+    q_pos[1] = 2
+    dO = rng.standard_normal(Qg.shape)
+    scale, sink, window = 0.4, 2, 6
+    dQ, dK, dV = orc.attn_bwd(Qg, K, V, idx, dO, q_pos=q_pos, causal=True, tail=(n - 8, n), scale=scale,
+                              sink=sink, window=window)
+    mask = torch.from_numpy(_sink_window_mask(idx, n, (n - 8, n), q_pos, sink, window))
+    q = torch.from_numpy(Qg).requires_grad_()
+    k = torch.from_numpy(K).requires_grad_()
+    v = torch.from_numpy(V).requires_grad_()
+    sc = (scale * torch.einsum("tgd,nd->tgn", q, k)).masked_fill(~mask[:, None, :], float("-inf"))
+    o = torch.einsum("tgn,nd->tgd", torch.softmax(sc, -1), v)
+    o.backward(torch.from_numpy(dO))
+    np.testing.assert_allclose(dQ, q.grad.numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dK, k.grad.numpy(), rtol=1e-9, atol=1e-12)
+    np.testing.assert_allclose(dV, v.grad.numpy(), rtol=1e-9, atol=1e-12)
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

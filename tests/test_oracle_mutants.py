@@ -23,6 +23,7 @@ ORDER = [
     P.pin_select_beam_walk, P.pin_select_full_beam_equals_flat,
     P.pin_attention_equals_sdpa, P.pin_attention_special_cases,
     P.pin_backward_autograd, P.pin_backward_finite_differences,
+    P.pin_attention_sink_window, P.pin_backward_sink_window_autograd,
 ]
 assert sorted(f.__name__ for f in ORDER) == sorted(f.__name__ for f in P.ALL_PINS)
 
@@ -62,6 +63,10 @@ MUTANTS = [
     ("dK sign flipped", "gk[j] += scale * ds * q[j];", "gk[j] -= scale * ds * q[j];"),
     ("dV ignores probabilities", "gv[j] += p[k] * go[j];", "gv[j] += go[j];"),
     ("dQ unscaled", "gq[j] += scale * ds * kr[j];", "gq[j] += ds * kr[j];"),
+    ("window one key short", "for (int64_t j = (int64_t)q_pos[t] - window + 1; j <= q_pos[t]; ++j)",
+     "for (int64_t j = (int64_t)q_pos[t] - window + 2; j <= q_pos[t]; ++j)"),
+    ("sink ignores causality", "if (j <= q_pos[t]) out[cnt++] = j;", "out[cnt++] = j;"),
+    ("repeated key counted twice", "if (u == 0 || out[k] != out[u - 1]) out[u++] = out[k];", "out[u++] = out[k];"),
 ]
 
 
