@@ -439,6 +439,103 @@ int lsa_sparse_attn_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, con
   return ok();
 }
 
+static int sw_checks(int32_t n_sink, int32_t window, const int32_t* q_pos, int64_t n_cap) {
+  if (n_sink < 0 || window < 0 || n_sink > LSA_MAX_SINK_WINDOW || window > LSA_MAX_SINK_WINDOW)
+    return fail(LSA_ERR_SHAPE, "n_sink and window must lie in [0, %d]", LSA_MAX_SINK_WINDOW);
+  if (n_sink > n_cap) return fail(LSA_ERR_SHAPE, "n_sink (%d) > n_cap (%lld)", n_sink, (long long)n_cap);
+  if (!q_pos) return fail(LSA_ERR_INVALID_ARG, "q_pos is required with sink and window keys");
+  return LSA_OK;
+}
+
+int lsa_sparse_attn_sw_workspace_bytes(int32_t T, int32_t Hq, int32_t n_heads, int32_t d, int32_t K_sel,
+                                       int64_t tail_len, int32_t n_sink, int32_t window, size_t* bytes) {
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
+  if (n_sink < 0 || window < 0 || n_sink > LSA_MAX_SINK_WINDOW || window > LSA_MAX_SINK_WINDOW)
+    return fail(LSA_ERR_SHAPE, "n_sink and window must lie in [0, %d]", LSA_MAX_SINK_WINDOW);
+  const int32_t K2 = K_sel + n_sink + window;
+  size_t attn = 0;
+  int rc = lsa_attn_workspace_bytes(T, Hq, n_heads, d, K2, tail_len, &attn);
+  if (rc != LSA_OK) return rc;
+  *bytes = align256((size_t)n_heads * T * K2 * sizeof(int32_t)) + attn;
+  return ok();
+}
+
+int lsa_sparse_attn_sw(const void* Q, int32_t T, int32_t Hq, const void* K, const void* V, int32_t n_heads,
+                       int64_t n_cap, int32_t d, int32_t dtype, const int32_t* idx, int32_t K_sel,
+                       const int32_t* q_pos, int32_t n_sink, int32_t window, int64_t tail_begin, int64_t tail_end,
+                       float scale, void* O, float* LSE, void* workspace, size_t workspace_bytes, int32_t* status,
+                       void* stream) {
+  int rc = attn_common_checks(Q, T, Hq, K, V, n_heads, n_cap, d, dtype, idx, K_sel, q_pos, 1, tail_begin, tail_end);
+  if (rc != LSA_OK) return rc;
+  if ((rc = sw_checks(n_sink, window, q_pos, n_cap)) != LSA_OK) return rc;
+  if (!std::isfinite(scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite");
+  if (T == 0) return ok();
+  if (!O || !LSE) return fail(LSA_ERR_INVALID_ARG, "O and LSE must be non-NULL");
+  size_t need = 0;
+  if ((rc = lsa_sparse_attn_sw_workspace_bytes(T, Hq, n_heads, d, K_sel, tail_end - tail_begin, n_sink, window,
+                                               &need)) != LSA_OK)
+    return rc;
+  if (!workspace || workspace_bytes < need)
+    return fail(LSA_ERR_WORKSPACE, "attention with sink and window keys needs %zu workspace bytes (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  const int32_t K2 = K_sel + n_sink + window;
+  int32_t* idx2 = static_cast<int32_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = lsa::run_attn_extend(K_sel > 0 ? idx : nullptr, K_sel, T, n_heads, q_pos, n_sink, window,
+                                       tail_begin, tail_end, n_cap, idx2, st);
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_sw");
+  lsa::AttnArgs a;
+  fill_attn(a, Q, T, Hq, K, V, n_heads, n_cap, d, idx2, K2, q_pos, 1, tail_begin, tail_end, scale, status);
+  a.O = O;
+  a.LSE = LSE;
+  if (a.nsplit > 1)
+    a.part = reinterpret_cast<float*>(static_cast<char*>(workspace) + align256((size_t)n_heads * T * K2 * sizeof(int32_t)));
+  e = lsa::run_attn_fwd(a, dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_sw");
+  return ok();
+}
+
+int lsa_sparse_attn_sw_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, const void* V, int32_t n_heads,
+                           int64_t n_cap, int32_t d, int32_t dtype, const void* O, const float* LSE, const void* dO,
+                           const int32_t* idx, int32_t K_sel, const int32_t* q_pos, int32_t n_sink, int32_t window,
+                           int64_t tail_begin, int64_t tail_end, float scale, float* dQ, float* dK, float* dV,
+                           void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  int rc = attn_common_checks(Q, T, Hq, K, V, n_heads, n_cap, d, dtype, idx, K_sel, q_pos, 1, tail_begin, tail_end);
+  if (rc != LSA_OK) return rc;
+  if ((rc = sw_checks(n_sink, window, q_pos, n_cap)) != LSA_OK) return rc;
+  if (!std::isfinite(scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite");
+  if (!dK || !dV) return fail(LSA_ERR_INVALID_ARG, "dK and dV must be non-NULL");
+  const int32_t K2 = K_sel + n_sink + window;
+  const size_t need = align256((size_t)n_heads * T * K2 * sizeof(int32_t));
+  if (T > 0 && (!workspace || workspace_bytes < need))
+    return fail(LSA_ERR_WORKSPACE, "the backward with sink and window keys needs %zu workspace bytes (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t kv_bytes = (size_t)n_heads * n_cap * d * sizeof(float);
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(dK, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_sw_bwd");
+  if ((e = cudaMemsetAsync(dV, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_sw_bwd");
+  if (T == 0) return ok();
+  if (!O || !LSE || !dO || !dQ) return fail(LSA_ERR_INVALID_ARG, "O, LSE, dO and dQ must be non-NULL");
+  int32_t* idx2 = static_cast<int32_t*>(workspace);
+  e = lsa::run_attn_extend(K_sel > 0 ? idx : nullptr, K_sel, T, n_heads, q_pos, n_sink, window, tail_begin, tail_end,
+                           n_cap, idx2, st);
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_sw_bwd");
+  lsa::AttnArgs a;
+  fill_attn(a, Q, T, Hq, K, V, n_heads, n_cap, d, idx2, K2, q_pos, 1, tail_begin, tail_end, scale, status);
+  a.O = const_cast<void*>(O);
+  a.LSE = const_cast<float*>(LSE);
+  a.dO = dO;
+  a.dQ = dQ;
+  a.dK = dK;
+  a.dV = dV;
+  if (a.nsplit > 1 && (e = cudaMemsetAsync(dQ, 0, (size_t)T * Hq * d * sizeof(float), st)) != cudaSuccess)
+    return cuda_fail(e, "lsa_sparse_attn_sw_bwd");
+  e = lsa::run_attn_bwd(a, dtype, st);
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_sw_bwd");
+  return ok();
+}
+
 int lsa_kv_append(void* K, void* V, int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, int64_t pos,
                   const void* K_rows, const void* V_rows, void* stream) {
   if (!K || !V || !K_rows || !V_rows) return fail(LSA_ERR_INVALID_ARG, "K, V, K_rows and V_rows must be non-NULL");

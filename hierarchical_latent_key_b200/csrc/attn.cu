@@ -379,6 +379,48 @@ cudaError_t run_kv_append(void* K, void* V, int64_t n_heads, int64_t n_cap, int6
   return cudaGetLastError();
 }
 
+// Key lists with the sink and recent-window keys (kongchang.com, "How LSA
+// Sidesteps Per-Key Scoring with Hierarchical Clustering": the keys taken from the
+// chosen clusters are used together with a window of recent tokens and a few
+// initial sink tokens).  Row (g, t) of idx2 = the K_sel listed keys, then n_sink
+// sink slots, then `window` window slots; a position that the tail range attends
+// already, or that the sink or the window holds, is dropped from the earlier parts,
+// so every key of the union appears once (the sink wins over the window, the tail
+// over both).  Positions past q_pos are left to the attention's causal mask.
+__global__ void k_attn_extend(const int32_t* __restrict__ idx, int32_t K_sel, int64_t T, const int32_t* __restrict__ q_pos,
+                              int32_t n_sink, int32_t window, int64_t tail_begin, int64_t tail_end, int64_t n_cap,
+                              int32_t* __restrict__ idx2, int32_t K2) {
+  const int64_t g = blockIdx.y, t = blockIdx.x;
+  const int64_t q = q_pos[t];
+  const int64_t w_lo = q - window + 1;
+  auto in_tail = [&](int64_t j) { return j >= tail_begin && j < tail_end; };
+  const int32_t* src = idx + (g * T + t) * K_sel;
+  int32_t* dst = idx2 + (g * T + t) * K2;
+  for (int i = threadIdx.x; i < K2; i += blockDim.x) {
+    int64_t out = -1;
+    if (i < K_sel) {
+      const int64_t j = src[i];
+      if (j >= 0 && !(j < n_sink || (j >= w_lo && j <= q) || in_tail(j))) out = j;
+    } else if (i < K_sel + n_sink) {
+      const int64_t j = i - K_sel;
+      if (j <= q && j < n_cap && !in_tail(j)) out = j;
+    } else {
+      const int64_t j = w_lo + (i - K_sel - n_sink);
+      if (j >= n_sink && j >= 0 && j <= q && j < n_cap && !in_tail(j)) out = j;
+    }
+    dst[i] = (int32_t)out;
+  }
+}
+
+cudaError_t run_attn_extend(const int32_t* idx, int32_t K_sel, int64_t T, int32_t n_heads, const int32_t* q_pos,
+                            int32_t n_sink, int32_t window, int64_t tail_begin, int64_t tail_end, int64_t n_cap,
+                            int32_t* idx2, cudaStream_t st) {
+  if (T == 0) return cudaSuccess;
+  k_attn_extend<<<dim3((unsigned)T, (unsigned)n_heads), 256, 0, st>>>(idx, K_sel, T, q_pos, n_sink, window, tail_begin,
+                                                                      tail_end, n_cap, idx2, K_sel + n_sink + window);
+  return cudaGetLastError();
+}
+
 int attn_splits(int64_t T, int Hkv, int64_t keys) {
   const int64_t units = T * Hkv;
   const int64_t target = 4 * 148;

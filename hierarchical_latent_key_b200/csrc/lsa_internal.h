@@ -128,5 +128,9 @@ cudaError_t run_kv_append(void* K, void* V, int64_t n_heads, int64_t n_cap, int6
                           const void* Kr, const void* Vr, cudaStream_t st);
 cudaError_t run_attn_fwd(const AttnArgs& a, int dtype, cudaStream_t st);
 cudaError_t run_attn_bwd(const AttnArgs& a, int dtype, cudaStream_t st);
+// idx2 [n_heads][T][K_sel + n_sink + window]: the key lists with the sink and window keys
+cudaError_t run_attn_extend(const int32_t* idx, int32_t K_sel, int64_t T, int32_t n_heads, const int32_t* q_pos,
+                            int32_t n_sink, int32_t window, int64_t tail_begin, int64_t tail_end, int64_t n_cap,
+                            int32_t* idx2, cudaStream_t st);
 
 }  // namespace lsa

@@ -67,6 +67,12 @@ def _load():
                                                i64, i64, f32, P, P, P, P, P]),
         "lsa_sparse_attn_noalloc": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i64,
                                                    i64, f32, P, P, P, P]),
+        "lsa_sparse_attn_sw_workspace_bytes": (ctypes.c_int, [i32, i32, i32, i32, i32, i64, i32, i32,
+                                                              ctypes.POINTER(sz)]),
+        "lsa_sparse_attn_sw": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i32, i64, i64,
+                                              f32, P, P, P, sz, P, P]),
+        "lsa_sparse_attn_sw_bwd": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, P, P, P, i32, P, i32,
+                                                  i32, i64, i64, f32, P, P, P, P, sz, P, P]),
         "lsa_kv_append": (ctypes.c_int, [P, P, i32, i64, i32, i32, i64, P, P, P]),
         "lsa_tree_attn_bwd_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
         "lsa_tree_attn_bwd": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, P, P, P, i32, P, i32, f32,
@@ -212,6 +218,36 @@ def lsa_sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos, causal, tail_begin, tai
                                     _ptr(dV), _ptr(status), _stream(stream, Q)), "lsa_sparse_attn_bwd")
 
 
+def lsa_sparse_attn_sw_workspace_bytes(T, Hq, n_heads, d, K_sel, tail_len, n_sink, window) -> int:
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_sparse_attn_sw_workspace_bytes(T, Hq, n_heads, d, K_sel, int(tail_len), int(n_sink), int(window),
+                                                   ctypes.byref(n)), "lsa_sparse_attn_sw_workspace_bytes")
+    return int(n.value)
+
+
+def lsa_sparse_attn_sw(Q, K, V, idx, q_pos, n_sink, window, tail_begin, tail_end, scale, O, LSE, workspace,
+                       status=None, stream=None):
+    T, Hq, d = Q.shape
+    K_sel = 0 if idx is None else idx.shape[-1]
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _raise(_lib.lsa_sparse_attn_sw(_ptr(Q), T, Hq, _ptr(K), _ptr(V), K.shape[0], K.shape[1], d, _dtype(Q), _ptr(idx),
+                                   K_sel, _ptr(q_pos), int(n_sink), int(window), tail_begin, tail_end, float(scale),
+                                   _ptr(O), _ptr(LSE), _ptr(workspace), ws_n, _ptr(status), _stream(stream, Q)),
+           "lsa_sparse_attn_sw")
+
+
+def lsa_sparse_attn_sw_bwd(Q, K, V, O, LSE, dO, idx, q_pos, n_sink, window, tail_begin, tail_end, scale, dQ, dK, dV,
+                           workspace, status=None, stream=None):
+    T, Hq, d = Q.shape
+    K_sel = 0 if idx is None else idx.shape[-1]
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _raise(_lib.lsa_sparse_attn_sw_bwd(_ptr(Q), T, Hq, _ptr(K), _ptr(V), K.shape[0], K.shape[1], d, _dtype(Q),
+                                       _ptr(O), _ptr(LSE), _ptr(dO), _ptr(idx), K_sel, _ptr(q_pos), int(n_sink),
+                                       int(window), tail_begin, tail_end, float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
+                                       _ptr(workspace), ws_n, _ptr(status), _stream(stream, Q)),
+           "lsa_sparse_attn_sw_bwd")
+
+
 def lsa_kv_append(K, V, pos, K_rows, V_rows, stream=None):
     """K, V: [n_heads, n_cap, d] caches; K_rows, V_rows: [n_heads, d] rows written at `pos`."""
     _raise(_lib.lsa_kv_append(_ptr(K), _ptr(V), K.shape[0], K.shape[1], K.shape[2], _dtype(K), int(pos),
@@ -313,10 +349,23 @@ def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, leaves=F
 
 
 def sparse_attn(Q, K, V, idx, q_pos=None, causal=False, tail=(0, 0), scale=None, workspace=None, status=None,
-                check=True):
+                check=True, sink=0, window=0):
+    """Key-list attention; sink / window > 0 add the first `sink` positions and the `window` positions up to
+    q_pos to every query's keys (causal, lsa_sparse_attn_sw)."""
     T, Hq, d = Q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     K_sel = 0 if idx is None else idx.shape[-1]
+    if sink or window:
+        need = lsa_sparse_attn_sw_workspace_bytes(T, Hq, K.shape[0], d, K_sel, tail[1] - tail[0], sink, window)
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+        O = torch.empty_like(Q)
+        LSE = torch.empty(T, Hq, dtype=torch.float32, device=Q.device)
+        st = _new_status(Q.device) if status is None else status
+        lsa_sparse_attn_sw(Q, K, V, idx, q_pos, sink, window, tail[0], tail[1], scale, O, LSE, workspace, st)
+        if check:
+            check_status(st, "lsa_sparse_attn_sw")
+        return O, LSE
     need = lsa_attn_workspace_bytes(T, Hq, K.shape[0], d, K_sel, tail[1] - tail[0])
     if need and (workspace is None or workspace.numel() * workspace.element_size() < need):
         workspace = torch.empty(need, dtype=torch.uint8, device=Q.device)
@@ -381,13 +430,22 @@ def tree_attn_bwd(tree: Tree, Q, K, V, O, LSE, dO, leaves, q_pos=None, causal=Fa
 
 
 def sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos=None, causal=False, tail=(0, 0), scale=None, status=None,
-                    check=True):
+                    check=True, sink=0, window=0):
     T, Hq, d = Q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     dQ = torch.empty(T, Hq, d, dtype=torch.float32, device=Q.device)
     dK = torch.empty(K.shape, dtype=torch.float32, device=Q.device)
     dV = torch.empty(V.shape, dtype=torch.float32, device=Q.device)
     st = _new_status(Q.device) if status is None else status
+    if sink or window:
+        K_sel = 0 if idx is None else idx.shape[-1]
+        ws = torch.empty(max(K.shape[0] * T * (K_sel + sink + window) * 4 + 256, 1), dtype=torch.uint8,
+                         device=Q.device)
+        lsa_sparse_attn_sw_bwd(Q, K, V, O, LSE, dO, idx, q_pos, sink, window, tail[0], tail[1], scale, dQ, dK, dV, ws,
+                               st)
+        if check:
+            check_status(st, "lsa_sparse_attn_sw_bwd")
+        return dQ, dK, dV
     lsa_sparse_attn_bwd(Q, K, V, O, LSE, dO, idx, q_pos, causal, tail[0], tail[1], scale, dQ, dK, dV, st)
     if check:
         check_status(st, "lsa_sparse_attn_bwd")

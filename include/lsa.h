@@ -183,6 +183,43 @@ int lsa_sparse_attn(const void *Q, int32_t T, int32_t Hq, const void *K, const v
                     int64_t tail_end, float scale, void *O, float *LSE, void *workspace,
                     size_t workspace_bytes, int32_t *status, void *stream);
 
+/* Largest sink and window sizes lsa_sparse_attn_sw accepts. */
+#define LSA_MAX_SINK_WINDOW 65536
+
+/* Host only.  Workspace bytes lsa_sparse_attn_sw needs: the extended key lists
+ * ([n_heads][T][K_sel + n_sink + window] int32) and the split partials of the
+ * attention over them. */
+int lsa_sparse_attn_sw_workspace_bytes(int32_t T, int32_t Hq, int32_t n_heads, int32_t d, int32_t K_sel,
+                                       int64_t tail_len, int32_t n_sink, int32_t window, size_t *bytes);
+
+/* Sparse attention with sink and recent-window keys (kongchang.com, "How LSA
+ * Sidesteps Per-Key Scoring with Hierarchical Clustering": the keys taken from the
+ * chosen clusters are attended together with a window of recent tokens and a few
+ * initial sink tokens).  Arguments and outputs as lsa_sparse_attn with causal = 1
+ * (q_pos required), plus
+ *  n_sink : positions [0, n_sink) join every query's keys (where <= q_pos);
+ *  window : positions [q_pos[t] - window + 1, q_pos[t]] join query t's keys.
+ * Query t attends to the union of its index list, the tail range, the sink and
+ * its window, each key once: an index-list entry that also lies in the tail, the
+ * sink or the window is not counted twice.  n_sink, window in
+ * [0, LSA_MAX_SINK_WINDOW], n_sink <= n_cap.  Key lists are extended by a kernel
+ * into the workspace, then the key-list attention runs. */
+int lsa_sparse_attn_sw(const void *Q, int32_t T, int32_t Hq, const void *K, const void *V,
+                       int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, const int32_t *idx,
+                       int32_t K_sel, const int32_t *q_pos, int32_t n_sink, int32_t window,
+                       int64_t tail_begin, int64_t tail_end, float scale, void *O, float *LSE,
+                       void *workspace, size_t workspace_bytes, int32_t *status, void *stream);
+
+/* Backward of lsa_sparse_attn_sw (conventions of lsa_sparse_attn_bwd).  Needs
+ * workspace for the extended key lists: n_heads * T * (K_sel + n_sink + window)
+ * int32, rounded up to 256 bytes. */
+int lsa_sparse_attn_sw_bwd(const void *Q, int32_t T, int32_t Hq, const void *K, const void *V,
+                           int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, const void *O,
+                           const float *LSE, const void *dO, const int32_t *idx, int32_t K_sel,
+                           const int32_t *q_pos, int32_t n_sink, int32_t window, int64_t tail_begin,
+                           int64_t tail_end, float scale, float *dQ, float *dK, float *dV,
+                           void *workspace, size_t workspace_bytes, int32_t *status, void *stream);
+
 /* Host only.  Workspace bytes lsa_tree_attn needs. */
 int lsa_tree_attn_workspace_bytes(const lsa_tree_desc *tree, int32_t T, int32_t Hq, int32_t d,
                                   int32_t dtype, int32_t n_leaves, size_t *bytes);
