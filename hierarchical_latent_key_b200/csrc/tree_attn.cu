@@ -1326,7 +1326,7 @@ constexpr size_t kBwdSmem = 1024 + 2 * kTL * 256 + 2 * kLeafKeys * 256 + 2 * kTL
 }  // namespace
 
 // Partial mode while its per-(row, leaf) outputs stay within this many bytes.
-constexpr size_t kPartialMaxBytes = size_t(4) << 30;
+constexpr size_t kPartialMaxBytes = size_t(24) << 30;   // an eighth of a 180 GB part
 
 static bool partial_fits(int64_t T, int64_t Hq, int B) { return (size_t)T * Hq * B * kDim * 2 <= kPartialMaxBytes; }
 

@@ -232,7 +232,7 @@ int lsa_tree_attn_workspace_bytes(const lsa_tree_desc *tree, int32_t T, int32_t 
  * and shared by all (query, head) rows that chose the leaf, with the products on
  * the tensor cores (bf16, d = 128, leaf size 64; other shapes run the generic
  * kernels on the expanded lists).  Outputs as lsa_sparse_attn.  While
- * T * Hq * n_leaves * d * 4 bytes stay within 4 GiB, every (row, leaf) pair
+ * T * Hq * n_leaves * d * 2 bytes stay within 24 GiB, every (row, leaf) pair
  * stores its leaf maximum, exp-sum and unnormalised output in the workspace and
  * a row's leaves are merged in rank order (results are reproducible bit for
  * bit); larger calls take a second pass over the leaves instead and accumulate

@@ -197,3 +197,30 @@ def test_train_128k_full(lsa):
         for name, got, want in (("dK", dK[h, j].cpu().numpy(), oK[j]), ("dV", dV[h, j].cpu().numpy(), oV[j])):
             e = np.abs(got - want)
             assert e.max() <= 2e-2 * np.abs(want).max() + 1e-6, (name, j, e.max(), np.abs(want).max())
+
+
+def test_tree_attention_beyond_partial_budget(lsa):
+    """Above 24 GiB of per-(row, leaf) partials the tree attention takes its two-pass schedule
+    (statistics, then outputs with fp32 red-adds): 131072 causal queries x 32 heads x 32 leaves
+    (34 GB of partials).  Checked against the key-list attention on every row and against the
+    oracle on sampled rows."""
+    cfg = configs.get("train_128k").scaled(Hq=32)
+    assert cfg.T * cfg.Hq * cfg.beam[-1] * 128 * 2 > (24 << 30)
+    case = cfg.case(DEV)
+    tree = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select(tree, case.Q, case.W, cfg.beam, case.q_pos, leaves=True)
+    O, LSE = lsa.tree_attn(tree, case.Q, case.K, case.V, leaves, case.q_pos, causal=True)
+    O2, L2 = lsa.sparse_attn(case.Q, case.K, case.V, idx, case.q_pos, True)
+    torch.cuda.synchronize()
+    d = (O.float() - O2.float()).abs()
+    assert d.max().item() <= 2e-2 and d.mean().item() <= 2e-3
+    assert (LSE - L2).abs().max().item() <= 1e-3
+    rng = np.random.default_rng(5)
+    h = 2
+    sl = slice(h * cfg.G, (h + 1) * cfg.G)
+    rows = np.sort(rng.choice(cfg.T, 32, replace=False))
+    Oo, Lo = orc.attn_fwd(case.Q[rows][:, sl].double().cpu().numpy(), case.K[h].double().cpu().numpy(),
+                          case.V[h].double().cpu().numpy(), idx[h][rows].cpu().numpy(),
+                          q_pos=case.q_pos.cpu().numpy()[rows], causal=True)
+    mx, mean = parity.attn_errors(O[rows][:, sl].float().cpu(), Oo)
+    assert mx <= 2e-2 and mean <= 2e-3, (mx, mean)
