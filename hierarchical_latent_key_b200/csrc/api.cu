@@ -311,32 +311,46 @@ int lsa_sparse_attn(const void* Q, int32_t T, int32_t Hq, const void* K, const v
   return ok();
 }
 
-int lsa_tree_attn_workspace_bytes(const lsa_tree_desc* tree, int32_t T, int32_t Hq, int32_t d, int32_t dtype,
-                                  int32_t n_leaves, size_t* bytes) {
+static int tree_attn_ws(const lsa_tree_desc* tree, int32_t T, int32_t Hq, int32_t d, int32_t dtype,
+                        int32_t n_leaves, int32_t n_sink, int32_t window, size_t* bytes) {
   int rc = check_desc(tree);
   if (rc != LSA_OK) return rc;
   if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
   if (T < 0 || Hq < tree->n_heads || Hq % tree->n_heads || n_leaves < 1 || n_leaves > LSA_MAX_BEAM ||
       (d != 64 && d != 128))
     return fail(LSA_ERR_SHAPE, "bad sizes");
+  if (n_sink < 0 || window < 0 || n_sink > LSA_MAX_SINK_WINDOW || window > LSA_MAX_SINK_WINDOW)
+    return fail(LSA_ERR_SHAPE, "n_sink and window must lie in [0, %d]", LSA_MAX_SINK_WINDOW);
   if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   const int G = Hq / tree->n_heads;
   const bool fast = lsa::tree_attn_fast_path(dtype, d, G, tree->leaf_size);
   *bytes = lsa::tree_attn_workspace(tree->n_heads, tree->nodes[tree->levels - 1], T, Hq, d, n_leaves,
-                                    tree->leaf_size, fast);
+                                    tree->leaf_size, fast, n_sink, window);
   return ok();
 }
 
-int lsa_tree_attn(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
-                  const void* K, const void* V, int64_t n_cap, int32_t d, int32_t dtype, const int32_t* leaves,
-                  int32_t n_leaves, const int32_t* q_pos, int32_t causal, float scale, void* O, float* LSE,
-                  void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+int lsa_tree_attn_workspace_bytes(const lsa_tree_desc* tree, int32_t T, int32_t Hq, int32_t d, int32_t dtype,
+                                  int32_t n_leaves, size_t* bytes) {
+  return tree_attn_ws(tree, T, Hq, d, dtype, n_leaves, 0, 0, bytes);
+}
+
+int lsa_tree_attn_sw_workspace_bytes(const lsa_tree_desc* tree, int32_t T, int32_t Hq, int32_t d, int32_t dtype,
+                                     int32_t n_leaves, int32_t n_sink, int32_t window, size_t* bytes) {
+  return tree_attn_ws(tree, T, Hq, d, dtype, n_leaves, n_sink, window, bytes);
+}
+
+static int tree_attn_call(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
+                          const void* K, const void* V, int64_t n_cap, int32_t d, int32_t dtype,
+                          const int32_t* leaves, int32_t n_leaves, const int32_t* q_pos, int32_t causal,
+                          int32_t n_sink, int32_t window, float scale, void* O, float* LSE, void* workspace,
+                          size_t workspace_bytes, int32_t* status, void* stream, const char* name) {
   size_t need = 0;
-  int rc = lsa_tree_attn_workspace_bytes(tree, T, Hq, d, dtype, n_leaves, &need);
+  int rc = tree_attn_ws(tree, T, Hq, d, dtype, n_leaves, n_sink, window, &need);
   if (rc != LSA_OK) return rc;
   const int G = Hq / tree->n_heads;
   if (G != 1 && G != 2 && G != 4 && G != 8) return fail(LSA_ERR_SHAPE, "query heads per group must be 1, 2, 4 or 8");
   if (n_cap < tree->n_tree) return fail(LSA_ERR_SHAPE, "n_cap (%lld) < n_tree", (long long)n_cap);
+  if (n_sink > n_cap) return fail(LSA_ERR_SHAPE, "n_sink (%d) > n_cap (%lld)", n_sink, (long long)n_cap);
   if (!std::isfinite(scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite");
   if (T == 0) return ok();
   if (!tree_mem || !Q || !K || !V || !leaves || !O || !LSE)
@@ -352,10 +366,27 @@ int lsa_tree_attn(const lsa_tree_desc* tree, const void* tree_mem, const void* Q
   c.leaves = leaves; c.q_pos = q_pos; c.O = O; c.LSE = LSE; c.workspace = workspace; c.status = status;
   c.T = T; c.n_cap = n_cap; c.n_tree = tree->n_tree; c.NL = tree->nodes[tree->levels - 1];
   c.Hq = Hq; c.H = tree->n_heads; c.d = d; c.dtype = dtype; c.B = n_leaves; c.leaf = tree->leaf_size;
-  c.causal = causal ? 1 : 0; c.scale = scale;
+  c.causal = causal ? 1 : 0; c.scale = scale; c.n_sink = n_sink; c.window = window;
   cudaError_t e = lsa::run_tree_attn(c, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "lsa_tree_attn");
+  if (e != cudaSuccess) return cuda_fail(e, name);
   return ok();
+}
+
+int lsa_tree_attn(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
+                  const void* K, const void* V, int64_t n_cap, int32_t d, int32_t dtype, const int32_t* leaves,
+                  int32_t n_leaves, const int32_t* q_pos, int32_t causal, float scale, void* O, float* LSE,
+                  void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  return tree_attn_call(tree, tree_mem, Q, T, Hq, K, V, n_cap, d, dtype, leaves, n_leaves, q_pos, causal, 0, 0, scale,
+                        O, LSE, workspace, workspace_bytes, status, stream, "lsa_tree_attn");
+}
+
+int lsa_tree_attn_sw(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
+                     const void* K, const void* V, int64_t n_cap, int32_t d, int32_t dtype, const int32_t* leaves,
+                     int32_t n_leaves, const int32_t* q_pos, int32_t n_sink, int32_t window, float scale, void* O,
+                     float* LSE, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  if (!q_pos && T > 0) return fail(LSA_ERR_INVALID_ARG, "q_pos is required with sink and window keys");
+  return tree_attn_call(tree, tree_mem, Q, T, Hq, K, V, n_cap, d, dtype, leaves, n_leaves, q_pos, 1, n_sink, window,
+                        scale, O, LSE, workspace, workspace_bytes, status, stream, "lsa_tree_attn_sw");
 }
 
 int lsa_tree_attn_bwd_workspace_bytes(const lsa_tree_desc* tree, int32_t T, int32_t Hq, int32_t d, int32_t dtype,

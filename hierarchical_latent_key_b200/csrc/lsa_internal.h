@@ -114,9 +114,11 @@ struct TreeAttnCall {
   int32_t* status;
   int64_t T, n_cap, n_tree, NL;
   int32_t Hq, H, d, dtype, B, leaf, causal;
+  int32_t n_sink, window;     // sink and recent-window keys (0: none; causal calls only)
   float scale;
 };
-size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast);
+size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast,
+                           int n_sink = 0, int window = 0);
 bool tree_attn_fast_path(int dtype, int d, int G, int leaf);
 cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st);
 size_t tree_attn_bwd_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast);

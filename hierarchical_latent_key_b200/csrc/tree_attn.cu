@@ -150,6 +150,9 @@ struct TreeAttnArgs {
   int32_t* ctotal;             // [H] chunks per head
   int4* cdesc;                 // chunk descriptors {head, leaf, first entry, entries}
   int32_t epc;                 // entries per chunk (rows / G)
+  int32_t n_sink, window;      // leaf keys in [0, n_sink) or [q_pos - window + 1, q_pos] are left out
+  const __nv_bfloat16* Od;     // [T][Hq][d] attention over the sink and window keys (or null)
+  const float* LSEd;           // [T][Hq] its natural-log softmax denominator
   __nv_bfloat16* O;
   float* LSE;
   int32_t* status;
@@ -624,9 +627,12 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
     mk = st.x;
     lk = st.y;
   }
+  // the sink/window part (if any) is one more partial: base-2 max = its LSE / ln 2, l = 1
+  const float md = a.LSEd ? a.LSEd[row] * 1.44269504088896340736f : -INFINITY;
   float M = valid ? mk : -INFINITY;
 #pragma unroll
   for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  M = fmaxf(M, md);
   const unsigned vmask = __ballot_sync(0xffffffffu, valid);
   const float wk = valid ? exp2f(mk - M) * lk : 0.f;
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
@@ -641,6 +647,16 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
     acc[1] = fmaf(w, lo.y, acc[1]);
     acc[2] = fmaf(w, hi.x, acc[2]);
     acc[3] = fmaf(w, hi.y, acc[3]);
+    L += w;
+  }
+  if (md != -INFINITY) {   // after the leaves, in a fixed order
+    const float w = exp2f(md - M);
+    float v[4];
+    load4(a.Od + row * kDim + lane * 4, v);
+    acc[0] = fmaf(w, v[0], acc[0]);
+    acc[1] = fmaf(w, v[1], acc[1]);
+    acc[2] = fmaf(w, v[2], acc[2]);
+    acc[3] = fmaf(w, v[3], acc[3]);
     L += w;
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
@@ -686,7 +702,8 @@ struct PipeMeta {
   int32_t qpos[kPipeStages][kChunkRows];
   int32_t pos[kPipeStages][kLeafKeys];
   int32_t qrow[kPipeStages][kChunkRows];           // global Q row of each tile row (loaders only)
-  int32_t nvis[kPipeStages][kChunkRows];           // visible-prefix length of each entry
+  int32_t nvis[kPipeStages][kChunkRows];           // visible keys of each entry: [vlo, nvis)
+  int32_t vlo[kPipeStages][kChunkRows];
   int32_t info[kPipeStages][2];                    // head, entries
   int32_t prow[kPipeBufs][kChunkRows];             // partial row of each TMEM lane (-1: none)
   float2 stat[kPipeBufs][kChunkRows];              // (m, l) of each TMEM lane
@@ -879,7 +896,12 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       if (j < a.epc) {
         M.ent[s][j] = cur.ev;
         M.qpos[s][j] = cur.eq;
-        M.nvis[s][j] = cur.ev >= 0 ? visible_prefix(M.pos[s], (int64_t)cur.eq) : 0;
+        // visible: position <= q_pos, outside the sink [0, n_sink) and the window
+        // (q_pos - window, q_pos], whose keys the dense part attends instead
+        const int hi = cur.ev >= 0 ? visible_prefix(M.pos[s], (int64_t)cur.eq - a.window) : 0;
+        const int lo = cur.ev >= 0 && a.n_sink > 0 ? visible_prefix(M.pos[s], (int64_t)a.n_sink - 1) : 0;
+        M.nvis[s][j] = hi > lo ? hi : lo;
+        M.vlo[s][j] = lo;
       }
       if (j == 0) {
         M.info[s][0] = cur.g;
@@ -971,7 +993,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       const int g = M.info[s][0];
       const int v = M.ent[s][e];
       const int64_t tq = v >= 0 ? (v >> 6) : -1;
-      const int nvis = M.nvis[s][e];
+      const int nvis = M.nvis[s][e], vlo = M.vlo[s][e];
       const int prow = tq >= 0 ? (int)((tq * a.Hq + g * a.G + hh) * a.B + (v & 63)) : -1;
       ok = __all_sync(0xffffffffu, mbar_wait(smem_u32(&M.sfull[b]), (k / kPipeBufs) & 1));
       if (!ok) break;
@@ -984,7 +1006,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
           float t32[32];
           tmem_ld32(tmem + b * 128 + lane_base + half * 32, t32);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sc[half * 32 + i] = half * 32 + i < nvis ? t32[i] * a.scale_log2 : -INFINITY;
+          for (int i = 0; i < 32; ++i)
+            sc[half * 32 + i] = half * 32 + i < nvis && half * 32 + i >= vlo ? t32[i] * a.scale_log2 : -INFINITY;
         }
         float mx[16];
 #pragma unroll
@@ -1334,15 +1357,24 @@ static int64_t max_chunks(int64_t H, int64_t NL, int64_t T, int B, int epc) {
   return H * NL + ceil_div(H * T * B, (int64_t)epc);
 }
 
-size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast) {
+size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, int B, int leaf, bool fast,
+                           int n_sink, int window) {
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
-  if (!fast) return al((size_t)H * T * B * leaf * 4);
+  const bool sw = n_sink > 0 || window > 0;
+  const size_t expand = al((size_t)H * T * B * leaf * 4);
+  if (!fast || (sw && !partial_fits(T, Hq, B)))   // key lists (extended with the sink and window keys)
+    return expand + (sw ? al((size_t)H * T * ((size_t)B * leaf + n_sink + window) * 4) : 0);
   const size_t lists = al(H * NL * 4) + al(H * (NL + 1) * 4) + al((size_t)H * T * B * 4) + al((size_t)T * Hq * B * 8);
   const size_t red = lists + al((size_t)T * Hq * 4) + al((size_t)T * Hq * d * 4);
   if (!partial_fits(T, Hq, B)) return red;
   const int epc = kChunkRows / (int)(Hq / H);
-  const size_t part = lists + al((size_t)T * Hq * B * d * 2) + al((size_t)H * T * B * 4) + al(H * NL * 4) +
-                      al(H * 4) + al((size_t)max_chunks(H, NL, T, B, epc) * 16);
+  size_t part = lists + al((size_t)T * Hq * B * d * 2) + al((size_t)H * T * B * 4) + al(H * NL * 4) +
+                al(H * 4) + al((size_t)max_chunks(H, NL, T, B, epc) * 16);
+  if (sw) {   // dense part: its key lists, output, LSE and split partials
+    const int ns = attn_splits(T, (int)H, n_sink + window);
+    part += al((size_t)H * T * (n_sink + window) * 4) + al((size_t)T * Hq * d * 2) + al((size_t)T * Hq * 4) +
+            (ns > 1 ? al((size_t)T * Hq * ns * (d + 2) * 4) : 0);
+  }
   return part > red ? part : red;
 }
 
@@ -1363,20 +1395,34 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
   char* ws = static_cast<char*>(c.workspace);
   auto al = [](size_t x) { return (x + 255) & ~size_t(255); };
   cudaError_t e;
-  if (!fast) {
+  const bool sw = c.n_sink > 0 || c.window > 0;
+  // key-list attention over given lists (one CTA per (query, group): no split workspace)
+  auto keylist_attn = [&](const int32_t* idx, int32_t K_sel, void* O, float* LSE, float* part) {
+    AttnArgs a;
+    memset(&a, 0, sizeof(a));
+    a.Q = c.Q; a.K = c.K; a.V = c.V; a.idx = idx; a.q_pos = c.q_pos; a.O = O; a.LSE = LSE;
+    a.status = c.status; a.T = c.T; a.n_cap = c.n_cap; a.Hq = c.Hq; a.Hkv = c.H; a.G = G; a.d = c.d;
+    a.K_sel = K_sel; a.causal = c.causal;
+    a.nsplit = part ? attn_splits(c.T, c.H, K_sel) : 1;
+    int64_t kps = (K_sel + a.nsplit - 1) / a.nsplit;
+    kps = (kps + 15) / 16 * 16;
+    a.keys_per_split = (int32_t)(kps > 0 ? kps : 16);
+    a.part = part;
+    a.scale = c.scale; a.scale_log2 = c.scale * 1.44269504088896340736f;
+    return run_attn_fwd(a, c.dtype, st);
+  };
+  if (!fast || (sw && !partial_fits(c.T, c.Hq, c.B))) {
     int32_t* idx = reinterpret_cast<int32_t*>(ws);
     const int64_t total = (int64_t)c.H * c.T * c.B * c.leaf;
     k_tl_expand<<<(unsigned)ceil_div(total, 256), 256, 0, st>>>(c.leaves, c.leaf_index, c.H, c.T, c.B, c.leaf,
                                                                 c.n_tree, idx);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    AttnArgs a;
-    memset(&a, 0, sizeof(a));
-    a.Q = c.Q; a.K = c.K; a.V = c.V; a.idx = idx; a.q_pos = c.q_pos; a.O = c.O; a.LSE = c.LSE;
-    a.status = c.status; a.T = c.T; a.n_cap = c.n_cap; a.Hq = c.Hq; a.Hkv = c.H; a.G = G; a.d = c.d;
-    a.K_sel = c.B * c.leaf; a.causal = c.causal; a.nsplit = 1;
-    a.keys_per_split = (int32_t)((a.K_sel + 15) / 16 * 16);
-    a.scale = c.scale; a.scale_log2 = c.scale * 1.44269504088896340736f;
-    return run_attn_fwd(a, c.dtype, st);   // one CTA per (query, group): needs no split workspace
+    if (!sw) return keylist_attn(idx, c.B * c.leaf, c.O, c.LSE, nullptr);
+    int32_t* idx2 = reinterpret_cast<int32_t*>(ws + al((size_t)total * 4));
+    if ((e = run_attn_extend(idx, c.B * c.leaf, c.T, c.H, c.q_pos, c.n_sink, c.window, 0, 0, c.n_cap, idx2, st)) !=
+        cudaSuccess)
+      return e;
+    return keylist_attn(idx2, c.B * c.leaf + c.n_sink + c.window, c.O, c.LSE, nullptr);
   }
   TreeAttnArgs a;
   a.Q = static_cast<const __nv_bfloat16*>(c.Q);
@@ -1395,6 +1441,10 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
   a.entq = a.coff = a.ctotal = nullptr;
   a.cdesc = nullptr;
   a.epc = kChunkRows / G;
+  a.n_sink = c.n_sink;
+  a.window = c.window;
+  a.Od = nullptr;
+  a.LSEd = nullptr;
   const bool partial = partial_fits(c.T, c.Hq, c.B);
   const size_t o_lists = o;
   if (partial) {
@@ -1403,6 +1453,20 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
     a.coff = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.NL * 4);
     a.ctotal = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * 4);
     a.cdesc = reinterpret_cast<int4*>(ws + o);
+    o += al((size_t)max_chunks(c.H, c.NL, c.T, c.B, a.epc) * 16);
+    if (sw) {   // dense part: the sink and window keys through the key-list attention
+      const int32_t KD = c.n_sink + c.window;
+      int32_t* idxd = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * KD * 4);
+      __nv_bfloat16* Od = reinterpret_cast<__nv_bfloat16*>(ws + o); o += al((size_t)c.T * c.Hq * kDim * 2);
+      float* LSEd = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);
+      float* partd = attn_splits(c.T, c.H, KD) > 1 ? reinterpret_cast<float*>(ws + o) : nullptr;
+      if ((e = run_attn_extend(nullptr, 0, c.T, c.H, c.q_pos, c.n_sink, c.window, 0, 0, c.n_cap, idxd, st)) !=
+          cudaSuccess)
+        return e;
+      if ((e = keylist_attn(idxd, KD, Od, LSEd, partd)) != cudaSuccess) return e;
+      a.Od = Od;
+      a.LSEd = LSEd;
+    }
   } else {
     o = o_lists;
     a.lse2 = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);

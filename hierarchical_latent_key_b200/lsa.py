@@ -67,6 +67,10 @@ def _load():
                                                i64, i64, f32, P, P, P, P, P]),
         "lsa_sparse_attn_noalloc": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i64,
                                                    i64, f32, P, P, P, P]),
+        "lsa_tree_attn_sw_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, i32, i32,
+                                                            ctypes.POINTER(sz)]),
+        "lsa_tree_attn_sw": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, i32, P, i32, i32, f32, P, P,
+                                            P, sz, P, P]),
         "lsa_sparse_attn_sw_workspace_bytes": (ctypes.c_int, [i32, i32, i32, i32, i32, i64, i32, i32,
                                                               ctypes.POINTER(sz)]),
         "lsa_sparse_attn_sw": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i32, i64, i64,
@@ -378,10 +382,38 @@ def sparse_attn(Q, K, V, idx, q_pos=None, causal=False, tail=(0, 0), scale=None,
     return O, LSE
 
 
+def lsa_tree_attn_sw_workspace_bytes(desc, T, Hq, d, dtype, n_leaves, n_sink, window) -> int:
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_tree_attn_sw_workspace_bytes(ctypes.byref(desc), T, Hq, d, _DTYPE[dtype], n_leaves, int(n_sink),
+                                                 int(window), ctypes.byref(n)), "lsa_tree_attn_sw_workspace_bytes")
+    return int(n.value)
+
+
+def lsa_tree_attn_sw(desc, tree_mem, Q, K, V, leaves, q_pos, n_sink, window, scale, O, LSE, workspace, status=None,
+                     stream=None):
+    T, Hq, d = Q.shape
+    ws_n = workspace.numel() * workspace.element_size()
+    _raise(_lib.lsa_tree_attn_sw(ctypes.byref(desc), _ptr(tree_mem), _ptr(Q), T, Hq, _ptr(K), _ptr(V), K.shape[1], d,
+                                 _dtype(Q), _ptr(leaves), leaves.shape[-1], _ptr(q_pos), int(n_sink), int(window),
+                                 float(scale), _ptr(O), _ptr(LSE), _ptr(workspace), ws_n, _ptr(status),
+                                 _stream(stream, Q)), "lsa_tree_attn_sw")
+
+
 def tree_attn(tree: Tree, Q, K, V, leaves, q_pos=None, causal=False, scale=None, workspace=None, status=None,
-              check=True):
+              check=True, sink=0, window=0):
     T, Hq, d = Q.shape
     scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if sink or window:
+        need = lsa_tree_attn_sw_workspace_bytes(tree.desc, T, Hq, d, Q.dtype, leaves.shape[-1], sink, window)
+        if workspace is None or workspace.numel() * workspace.element_size() < need:
+            workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)
+        O = torch.empty_like(Q)
+        LSE = torch.empty(T, Hq, dtype=torch.float32, device=Q.device)
+        st = _new_status(Q.device) if status is None else status
+        lsa_tree_attn_sw(tree.desc, tree.mem, Q, K, V, leaves, q_pos, sink, window, scale, O, LSE, workspace, st)
+        if check:
+            check_status(st, "lsa_tree_attn_sw")
+        return O, LSE
     need = lsa_tree_attn_workspace_bytes(tree.desc, T, Hq, d, Q.dtype, leaves.shape[-1])
     if workspace is None or workspace.numel() * workspace.element_size() < need:
         workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=Q.device)

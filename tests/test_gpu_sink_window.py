@@ -118,3 +118,49 @@ def test_rejects_bad_sink_window(lsa):
     with pytest.raises(lsa.LsaError) as e:
         lsa.sparse_attn(Q, K, K, None, qp, True, sink=300, window=4)   # sink beyond n_cap
     assert e.value.code == lsa.LSA_ERR_SHAPE
+
+
+@pytest.mark.parametrize("G", [4, 1, 8])
+def test_tree_attention_sink_window(lsa, G):
+    """Leaf-by-leaf attention with sink and window keys (leaf keys inside them left out, the dense
+    part merged as one more partial) = the key-list attention over the same union = the oracle."""
+    cfg = configs.get("prefill_1m").scaled(n=8 * 8 * 4 * 2 * 64, branching=(8, 8, 4, 2), beam=(4, 16, 16, 8),
+                                           Hkv=2, Hq=2 * G, T=300, comps=256)
+    case = cfg.case("cpu", seed=21 + G)
+    g = {k: getattr(case, k).to(DEV) for k in ("Q", "K", "V", "W")}
+    qp = case.q_pos.to(DEV)
+    tree = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select(tree, g["Q"], g["W"], cfg.beam, qp, leaves=True)
+    for sink, window in ((8, 96), (0, 64), (32, 0)):
+        O, LSE = lsa.tree_attn(tree, g["Q"], g["K"], g["V"], leaves, qp, causal=True, sink=sink, window=window)
+        O2, L2 = lsa.sparse_attn(g["Q"], g["K"], g["V"], idx, qp, True, sink=sink, window=window)
+        torch.cuda.synchronize()
+        d = (O.float() - O2.float()).abs()
+        assert d.max().item() <= 2e-2 and d.mean().item() <= 2e-3, (G, sink, window, d.max().item())
+        assert (LSE - L2).abs().max().item() <= 1e-3
+        rows = np.arange(0, cfg.T, 37)
+        h = 1
+        sl = slice(h * G, (h + 1) * G)
+        Oo, Lo = orc.attn_fwd(case.Q[rows][:, sl], case.K[h], case.V[h], idx[h][rows].cpu(),
+                              q_pos=case.q_pos.numpy()[rows], causal=True, sink=sink, window=window)
+        err = np.abs(O[rows][:, sl].float().cpu().numpy() - Oo)
+        assert err.max() <= 2e-2 and err.mean() <= 2e-3, (G, sink, window, err.max(), err.mean())
+        assert np.abs(LSE[rows][:, sl].cpu().numpy() - Lo).max() <= 1e-3
+
+
+def test_tree_attention_sink_window_fallback(lsa):
+    """fp32, d = 64 (not the tensor-core path): expanded key lists with the sink and window."""
+    cfg = configs.get("tiny").scaled(T=64)
+    case = cfg.case("cpu")
+    n = cfg.n
+    case.q_pos = torch.arange(n - 64, n, dtype=torch.int32)
+    g = {k: getattr(case, k).to(DEV) for k in ("Q", "K", "V", "W")}
+    qp = case.q_pos.to(DEV)
+    tree = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select(tree, g["Q"], g["W"], cfg.beam, qp, leaves=True)
+    O, LSE = lsa.tree_attn(tree, g["Q"], g["K"], g["V"], leaves, qp, causal=True, sink=3, window=50)
+    torch.cuda.synchronize()
+    Oo, Lo = orc.attn_fwd(case.Q, case.K[0], case.V[0], idx[0].cpu(), q_pos=case.q_pos.numpy(), causal=True,
+                          sink=3, window=50)
+    assert np.abs(O.cpu().numpy() - Oo).max() <= 1e-4
+    assert np.abs(LSE.cpu().numpy() - Lo).max() <= 1e-4
