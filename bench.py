@@ -463,6 +463,45 @@ def time_steps(w, steps, warmup, flush, stream):
     return sel, att
 
 
+SINK, WINDOW = 16, 512   # sink tokens and recent window of the sink/window measurement
+
+
+def time_sink_window(w, steps, warmup, flush, stream, sink=SINK, window=WINDOW):
+    """The prefill step with sink and recent-window keys added to every query (lsa_tree_attn_sw)."""
+    lsa = w.lsa
+    T, Hq, d = w.Q.shape
+    need = lsa.lsa_tree_attn_sw_workspace_bytes(w.tree.desc, T, Hq, d, w.Q.dtype, w.cfg.beam[-1], sink, window)
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=w.Q.device)
+
+    def attend():
+        lsa.lsa_tree_attn_sw(w.tree.desc, w.tree.mem, w.Q, w.K, w.V, w.leaves, w.q_pos, sink, window, w.scale, w.O,
+                             w.LSE, ws, w.status)
+
+    for _ in range(warmup):
+        flush.zero_()
+        w.select()
+        attend()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        w.select()
+        ev[k][1].record(stream)
+        attend()
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    code = lsa.lsa_status_check(w.status)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code}: {lsa.lsa_strerror(code)}")
+    sel = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(steps))
+    att = statistics.mean(ev[k][1].elapsed_time(ev[k][2]) for k in range(steps))
+    return {"value": T / ((sel + att) / 1e3), "unit": "queries/s", "n_sink": sink, "window": window,
+            "breakdown_ms": {"select": sel, "attention": att},
+            "config": f"prefill step as above, every query also attends to positions [0, {sink}) and its last "
+                      f"{window} positions (each key once)"}
+
+
 def time_e2e(w, steps, flush, stream):
     """Same step through the public API with pinned host buffers: H2D of the chunk's
     queries, select + attention, D2H of the outputs, all inside the timed region."""
@@ -601,6 +640,10 @@ def run_cuda(args, rank, world, local_rank):
     peaks = measured_peaks()
     achieved = alg_bytes / att_s / 1e9
     launches = w.launches_per_step * args.steps
+    try:
+        sink_window = time_sink_window(w, args.steps, args.warmup, flush, stream)
+    except Exception as e:  # noqa: BLE001
+        sink_window = {"error": f"{type(e).__name__}: {e}"}
     decode = train = None
     del w
     torch.cuda.empty_cache()
@@ -643,6 +686,7 @@ def run_cuda(args, rank, world, local_rank):
             "gpu_launches": launches,
             "clocks": clocks,
             "cpu_baseline": cpu,
+            "prefill_1m_sink_window": sink_window,
             "decode_10m": decode,
             "train_128k": train,
         }
