@@ -502,6 +502,41 @@ def time_sink_window(w, steps, warmup, flush, stream, sink=SINK, window=WINDOW):
                       f"{window} positions (each key once)"}
 
 
+def time_flat(w, steps, warmup, flush, stream):
+    """The prefill step with flat search (every leaf centroid scored, lsa_select_flat) in place of
+    the beam walk, then the same tree attention."""
+    lsa = w.lsa
+
+    def select():
+        lsa.lsa_select_flat(w.tree.desc, w.tree.mem, w.Q, w.W, w.cfg.beam[-1], w.q_pos, None, w.leaves,
+                            status=w.status)
+
+    for _ in range(warmup):
+        flush.zero_()
+        select()
+        w.attend()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        select()
+        ev[k][1].record(stream)
+        w.attend()
+        ev[k][2].record(stream)
+    torch.cuda.synchronize()
+    code = lsa.lsa_status_check(w.status)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code}: {lsa.lsa_strerror(code)}")
+    sel = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(steps))
+    att = statistics.mean(ev[k][1].elapsed_time(ev[k][2]) for k in range(steps))
+    T = w.Q.shape[0]
+    nl = w.cfg.nodes[-1]
+    return {"value": T / ((sel + att) / 1e3), "unit": "queries/s", "breakdown_ms": {"select": sel, "attention": att},
+            "config": f"prefill step as above with flat search: {nl} leaf centroids scored per query and group, "
+                      f"the best {w.cfg.beam[-1]} kept"}
+
+
 def time_e2e(w, steps, flush, stream):
     """Same step through the public API with pinned host buffers: H2D of the chunk's
     queries, select + attention, D2H of the outputs, all inside the timed region."""
@@ -644,6 +679,10 @@ def run_cuda(args, rank, world, local_rank):
         sink_window = time_sink_window(w, args.steps, args.warmup, flush, stream)
     except Exception as e:  # noqa: BLE001
         sink_window = {"error": f"{type(e).__name__}: {e}"}
+    try:
+        flat = time_flat(w, args.steps, args.warmup, flush, stream)
+    except Exception as e:  # noqa: BLE001
+        flat = {"error": f"{type(e).__name__}: {e}"}
     decode = train = None
     del w
     torch.cuda.empty_cache()
@@ -687,6 +726,7 @@ def run_cuda(args, rank, world, local_rank):
             "clocks": clocks,
             "cpu_baseline": cpu,
             "prefill_1m_sink_window": sink_window,
+            "prefill_1m_flat": flat,
             "decode_10m": decode,
             "train_128k": train,
         }

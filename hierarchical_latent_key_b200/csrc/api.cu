@@ -260,6 +260,42 @@ static int attn_common_checks(const void* Q, int32_t T, int32_t Hq, const void* 
   return LSA_OK;
 }
 
+int lsa_select_flat(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
+                    int32_t d, int32_t dtype, const void* W, int32_t n_leaves, const int32_t* q_pos,
+                    int32_t* idx_out, int32_t* leaves_out, float* qlat_out, int32_t* status, void* stream) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (T < 0) return fail(LSA_ERR_SHAPE, "T must be >= 0");
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  if (Hq < tree->n_heads || Hq % tree->n_heads) return fail(LSA_ERR_SHAPE, "Hq (%d) must be a multiple of n_heads (%d)", Hq, tree->n_heads);
+  if (Hq / tree->n_heads > 64) return fail(LSA_ERR_SHAPE, "more than 64 query heads per group");
+  const int L = tree->levels - 1;
+  if (n_leaves < 1 || n_leaves > LSA_MAX_BEAM || n_leaves > tree->nodes[L])
+    return fail(LSA_ERR_SHAPE, "n_leaves = %d must be in [1, min(%d, %lld)]", n_leaves, LSA_MAX_BEAM,
+                (long long)tree->nodes[L]);
+  if (T == 0) return ok();
+  if (!tree_mem || !Q || !W) return fail(LSA_ERR_INVALID_ARG, "tree_mem, Q and W must be non-NULL");
+  if (!idx_out && !leaves_out) return fail(LSA_ERR_INVALID_ARG, "give idx_out, leaves_out or both");
+  lsa::SelectArgs a;
+  memset(&a, 0, sizeof(a));
+  for (int l = 0; l < tree->levels; ++l) {
+    a.branching[l] = tree->branching[l];
+    a.nodes[l] = tree->nodes[l];
+    a.off_c[l] = tree->off_centroids[l];
+    a.off_m[l] = tree->off_min_pos[l];
+  }
+  a.beam[L] = n_leaves;
+  a.Q = Q; a.W = W; a.tree = static_cast<const char*>(tree_mem); a.q_pos = q_pos; a.idx_out = idx_out;
+  a.leaves_out = leaves_out; a.qlat_out = qlat_out; a.status = status;
+  a.T = T; a.Hq = Hq; a.Hkv = tree->n_heads; a.G = Hq / tree->n_heads; a.d = d; a.r = tree->r;
+  a.levels = tree->levels; a.leaf = tree->leaf_size; a.beam_max = n_leaves; a.n_tree = tree->n_tree;
+  a.off_leaf = tree->off_leaf_index;
+  cudaError_t e = lsa::run_select_flat(a, dtype, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_select_flat");
+  return ok();
+}
+
 int lsa_attn_workspace_bytes(int32_t T, int32_t Hq, int32_t n_heads, int32_t d, int32_t K_sel, int64_t tail_len,
                              size_t* bytes) {
   if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");

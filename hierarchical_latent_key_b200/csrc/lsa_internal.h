@@ -81,6 +81,8 @@ struct SelectArgs {
   uint64_t off_leaf;
 };
 cudaError_t run_select(const SelectArgs& a, int dtype, cudaStream_t st);
+// flat search: every leaf of the last level scored, the best beam[levels - 1] kept
+cudaError_t run_select_flat(const SelectArgs& a, int dtype, cudaStream_t st);
 
 struct AttnArgs {
   const void* Q;

@@ -475,6 +475,209 @@ static cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   return cudaErrorInvalidValue;
 }
 
+// ---- flat search: every leaf centroid scored ----------------------------------
+//
+// bdtechtalks.com, "Latent sparse attention", section "How latent sparse attention
+// works" (first strategy): the query is compared against all cluster centroids.
+// A CTA takes kFlatQ queries of one KV group and streams the group's leaf
+// centroids through shared memory in tiles of kFlatTile leaves; a thread scores
+// 4 queries x 8 leaves (sequential fp32 FMAs over the r dimensions).  Keys above a
+// query's running threshold (its B-th best key so far) go to a shared buffer;
+// when a buffer holds more than kFlatKeep keys a warp sorts it, keeps the best B
+// and raises the threshold.  Keys as in the beam walk: (orderable score, ~leaf id),
+// so the order is (score desc, leaf id asc).
+constexpr int kFlatQ = 32;              // queries per CTA (4 per warp)
+constexpr int kFlatTile = 256;          // leaves per tile (8 per lane)
+constexpr int kFlatKeep = 64;           // buffer size that triggers a reduction
+constexpr int kFlatCap = kFlatKeep + kFlatTile;
+
+template <int R>
+struct FlatSmem {
+  float cent[kFlatTile][R + 4];          // padded rows: a quarter-warp's float4 reads hit distinct banks
+  int32_t mpos[kFlatTile];
+  unsigned long long buf[kFlatQ][kFlatCap];
+  unsigned long long tau[kFlatQ];
+  int32_t cnt[kFlatQ];
+  __align__(16) float lat[kFlatQ][R];
+  float q[kSelWarps][128];
+  int32_t qpos[kFlatQ];
+  int32_t kept[kFlatQ][LSA_MAX_BEAM];
+  int32_t nkept[kFlatQ];
+};
+
+// Warp: the best B keys of query q's buffer into its first slots; returns how many.
+template <int R>
+__device__ __forceinline__ void flat_reduce(FlatSmem<R>& S, int q, int B) {
+  const int lane = threadIdx.x & 31;
+  const int n = S.cnt[q];
+  unsigned long long v[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int i = lane * 16 + e;
+    v[e] = i < n ? S.buf[q][i] : 0ull;
+  }
+  warp_sort_desc<16>(v);
+  __syncwarp();
+  int valid = 0;
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const int i = lane * 16 + e;
+    if (i < B) {
+      S.buf[q][i] = v[e];
+      valid += v[e] != 0ull;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) valid += __shfl_xor_sync(0xffffffffu, valid, o);
+  const unsigned long long last = __shfl_sync(0xffffffffu, v[(B - 1) & 15], (B - 1) >> 4);
+  __syncwarp();
+  if (lane == 0) {
+    S.cnt[q] = valid;
+    S.tau[q] = valid >= B ? last : 0ull;
+  }
+  __syncwarp();
+}
+
+template <typename T, int R, int DK>
+__global__ void __launch_bounds__(kSelWarps * 32, 1) k_select_flat(SelectArgs a) {
+  extern __shared__ __align__(16) char flat_raw[];
+  FlatSmem<R>& S = *reinterpret_cast<FlatSmem<R>*>(flat_raw);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
+  const int g = blockIdx.y;
+  const int64_t t0 = (int64_t)blockIdx.x * kFlatQ;
+  const int L = a.levels - 1, B = a.beam[L];
+  const int64_t NL = a.nodes[L];
+  const float* cent = reinterpret_cast<const float*>(a.tree + a.off_c[L]) + (int64_t)g * NL * R;
+  const int32_t* mpos = reinterpret_cast<const int32_t*>(a.tree + a.off_m[L]) + (int64_t)g * NL;
+  const T* Wg = static_cast<const T*>(a.W) + (int64_t)g * DK * R;
+  for (int qq = warp * 4; qq < warp * 4 + 4; ++qq) {   // latents of this warp's 4 queries
+    const int64_t t = t0 + qq;
+    if (t < a.T) {
+      latent_query<T, R, DK>(a, t, g, Wg, S.q[warp], S.lat[qq]);
+    } else {
+      for (int k = lane; k < R; k += 32) S.lat[qq][k] = 0.f;
+    }
+    if (lane == 0) {
+      S.cnt[qq] = 0;
+      S.tau[qq] = 0ull;
+      S.qpos[qq] = t < a.T ? (a.q_pos ? a.q_pos[t] : INT32_MAX) : -1;
+    }
+  }
+  __syncthreads();
+  bool bad = false;
+  for (int64_t L0 = 0; L0 < NL; L0 += kFlatTile) {
+    const int nt = (int)min64(kFlatTile, NL - L0);
+    {  // all of a thread's loads in flight before its stores
+      constexpr int PER = kFlatTile * (R / 4) / (kSelWarps * 32);
+      float4 x[PER];
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int i = tid + j * kSelWarps * 32, l = i / (R / 4), kc = i % (R / 4);
+        x[j] = l < nt ? __ldg(reinterpret_cast<const float4*>(cent + (L0 + l) * R) + kc) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int j = 0; j < PER; ++j) {
+        const int i = tid + j * kSelWarps * 32, l = i / (R / 4), kc = i % (R / 4);
+        *reinterpret_cast<float4*>(&S.cent[l][kc * 4]) = x[j];
+      }
+    }
+    for (int l = tid; l < kFlatTile; l += kSelWarps * 32) S.mpos[l] = l < nt ? __ldg(&mpos[L0 + l]) : INT32_MAX;
+    __syncthreads();
+    float acc[4][8];
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[qq][i] = 0.f;
+#pragma unroll 2
+    for (int k = 0; k < R; k += 4) {
+      float4 lq[4], cl[8];
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq) lq[qq] = *reinterpret_cast<const float4*>(&S.lat[warp * 4 + qq][k]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) cl[i] = *reinterpret_cast<const float4*>(&S.cent[lane + 32 * i][k]);
+#pragma unroll
+      for (int qq = 0; qq < 4; ++qq)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          acc[qq][i] = fmaf(lq[qq].x, cl[i].x, acc[qq][i]);
+          acc[qq][i] = fmaf(lq[qq].y, cl[i].y, acc[qq][i]);
+          acc[qq][i] = fmaf(lq[qq].z, cl[i].z, acc[qq][i]);
+          acc[qq][i] = fmaf(lq[qq].w, cl[i].w, acc[qq][i]);
+        }
+    }
+#pragma unroll
+    for (int qq = 0; qq < 4; ++qq) {
+      const int q = warp * 4 + qq;
+      const int64_t qp = S.qpos[q];
+      if (qp < 0) continue;
+      const unsigned long long tau = S.tau[q];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int l = lane + 32 * i;
+        if (l >= nt || (int64_t)S.mpos[l] > qp) continue;
+        const float sc = acc[qq][i];
+        if (isnan(sc)) {
+          bad = true;
+          continue;
+        }
+        const unsigned long long key =
+            ((unsigned long long)orderable(sc) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)(L0 + l));
+        if (key > tau) S.buf[q][atomicAdd(&S.cnt[q], 1)] = key;
+      }
+    }
+    __syncthreads();
+    const bool last = L0 + kFlatTile >= NL;
+    for (int qq = warp * 4; qq < warp * 4 + 4; ++qq)
+      if (S.qpos[qq] >= 0 && (S.cnt[qq] > kFlatKeep || (last && S.cnt[qq] > 0))) flat_reduce<R>(S, qq, B);
+    __syncthreads();
+  }
+  if (__syncthreads_or(bad) && tid == 0) set_status(a.status, LSA_ERR_NONFINITE);
+  // outputs: kept leaves in order, then their keys
+  for (int qq = warp * 4; qq < warp * 4 + 4; ++qq) {
+    const int64_t t = t0 + qq;
+    if (t >= a.T) continue;
+    const int n = S.cnt[qq];
+    for (int i = lane; i < B; i += 32) {
+      const int32_t leaf = i < n ? key_id(S.buf[qq][i]) : -1;
+      S.kept[qq][i] = leaf;
+      if (a.leaves_out) a.leaves_out[((int64_t)g * a.T + t) * B + i] = leaf;
+    }
+    __syncwarp();
+    if (a.idx_out) {
+      const int leaf = a.leaf;
+      const int64_t K_sel = (int64_t)B * leaf;
+      const int32_t* li = reinterpret_cast<const int32_t*>(a.tree + a.off_leaf) + (int64_t)g * a.n_tree;
+      int32_t* out = a.idx_out + ((int64_t)g * a.T + t) * K_sel;
+      for (int64_t i = lane; i < K_sel; i += 32) {
+        const int k = (int)(i / leaf), q = (int)(i % leaf);
+        out[i] = k < n ? __ldg(&li[(int64_t)S.kept[qq][k] * leaf + q]) : -1;
+      }
+    }
+  }
+}
+
+template <typename T>
+static cudaError_t launch_flat(const SelectArgs& a, cudaStream_t st) {
+  dim3 grid((unsigned)ceil_div(a.T, kFlatQ), (unsigned)a.Hkv);
+#define LSA_FLAT(RR, DD)                                                                              \
+  if (a.r == RR && a.d == DD) {                                                                       \
+    const size_t smem = sizeof(FlatSmem<RR>);                                                         \
+    cudaError_t e = cudaFuncSetAttribute(k_select_flat<T, RR, DD>,                                    \
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);     \
+    if (e != cudaSuccess) return e;                                                                   \
+    k_select_flat<T, RR, DD><<<grid, kSelWarps * 32, smem, st>>>(a);                                  \
+    return cudaGetLastError();                                                                        \
+  }
+  LSA_FLAT(16, 64) LSA_FLAT(32, 64) LSA_FLAT(64, 64) LSA_FLAT(16, 128) LSA_FLAT(32, 128) LSA_FLAT(64, 128)
+#undef LSA_FLAT
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t run_select_flat(const SelectArgs& a, int dtype, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  return dtype == LSA_BF16 ? launch_flat<__nv_bfloat16>(a, st) : launch_flat<float>(a, st);
+}
+
 cudaError_t run_select(const SelectArgs& a, int dtype, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
   return dtype == LSA_BF16 ? launch_select<__nv_bfloat16>(a, st) : launch_select<float>(a, st);

@@ -67,6 +67,7 @@ def _load():
                                                i64, i64, f32, P, P, P, P, P]),
         "lsa_sparse_attn_noalloc": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, i32, P, i32, i64,
                                                    i64, f32, P, P, P, P]),
+        "lsa_select_flat": (ctypes.c_int, [D, P, P, i32, i32, i32, i32, P, i32, P, P, P, P, P, P]),
         "lsa_tree_attn_sw_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, i32, i32,
                                                             ctypes.POINTER(sz)]),
         "lsa_tree_attn_sw": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, i32, P, i32, i32, f32, P, P,
@@ -349,6 +350,33 @@ def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, leaves=F
         out.append(ql)
     if beams:
         out.append(bo)
+    return out[0] if len(out) == 1 else tuple(out)
+
+
+def lsa_select_flat(desc, tree_mem, Q, W, n_leaves, q_pos, idx_out, leaves_out=None, qlat_out=None, status=None,
+                    stream=None):
+    T, Hq, d = Q.shape
+    _raise(_lib.lsa_select_flat(ctypes.byref(desc), _ptr(tree_mem), _ptr(Q), T, Hq, d, _dtype(Q), _ptr(W),
+                                int(n_leaves), _ptr(q_pos), _ptr(idx_out), _ptr(leaves_out), _ptr(qlat_out),
+                                _ptr(status), _stream(stream, Q)), "lsa_select_flat")
+
+
+def select_flat(tree: Tree, Q, W, n_leaves, q_pos=None, qlat=False, leaves=False, status=None, check=True):
+    """Flat search over every leaf; returns idx (and, when asked, leaves, query latents)."""
+    T = Q.shape[0]
+    d = tree.desc
+    idx = torch.empty(d.n_heads, T, n_leaves * d.leaf_size, dtype=torch.int32, device=Q.device)
+    lv = torch.empty(d.n_heads, T, n_leaves, dtype=torch.int32, device=Q.device) if leaves else None
+    ql = torch.empty(T, d.n_heads, d.r, dtype=torch.float32, device=Q.device) if qlat else None
+    st = _new_status(Q.device) if status is None else status
+    lsa_select_flat(d, tree.mem, Q, W, n_leaves, q_pos, idx, lv, ql, st)
+    if check:
+        check_status(st, "lsa_select_flat")
+    out = [idx]
+    if leaves:
+        out.append(lv)
+    if qlat:
+        out.append(ql)
     return out[0] if len(out) == 1 else tuple(out)
 
 

@@ -161,6 +161,21 @@ int lsa_select(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, i
                const int32_t *q_pos, int32_t *idx_out, int32_t *leaves_out, float *qlat_out,
                int32_t *beam_out, int32_t *status, void *stream);
 
+/* Flat search (bdtechtalks.com, "Latent sparse attention", section "How latent
+ * sparse attention works": the first of the two search strategies compares the
+ * query with all cluster centroids).  Arguments and outputs as lsa_select with a
+ * single budget: per (group g, query t) every leaf of the last level is scored,
+ * score = <q, leaf centroid> (fp32), a leaf is a candidate only if its min_pos <=
+ * q_pos[t] (when q_pos is given), and the n_leaves best by (score desc, leaf id asc)
+ * are kept, in that order.  idx_out [n_heads][T][n_leaves * leaf_size] and
+ * leaves_out [n_heads][T][n_leaves] as in lsa_select; qlat_out optional.
+ * n_leaves in [1, min(32, number of leaves)].  Quadratic in the context: every
+ * query reads every leaf centroid of its group. */
+int lsa_select_flat(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, int32_t T,
+                    int32_t Hq, int32_t d, int32_t dtype, const void *W, int32_t n_leaves,
+                    const int32_t *q_pos, int32_t *idx_out, int32_t *leaves_out, float *qlat_out,
+                    int32_t *status, void *stream);
+
 /* Host only.  Workspace bytes lsa_sparse_attn needs for these sizes (0 when the
  * call runs without key splitting). */
 int lsa_attn_workspace_bytes(int32_t T, int32_t Hq, int32_t n_heads, int32_t d, int32_t K_sel,

@@ -273,6 +273,16 @@ def select(qlat, tree: Tree, beam, q_pos=None, trace: bool = False):
 
 # --- attention -------------------------------------------------------------------
 
+def select_flat(qlat, tree: Tree, n_leaves, q_pos=None):
+    """Flat search (bdtechtalks.com, "Latent sparse attention", "How latent sparse attention
+    works": the query is compared with every cluster centroid): the beam walk with every node
+    kept above the leaf level scores every (eligible) leaf and keeps the n_leaves best.
+    Returns (idx [T, n_leaves * leaf], kept leaf ids [T, n_leaves], -1 padded)."""
+    full = [int(tree.nodes[l]) for l in range(len(tree.nodes) - 1)]
+    idx, beams, _ = select(qlat, tree, full + [int(n_leaves)], q_pos=q_pos, trace=True)
+    return idx, beams[-1][:, :int(n_leaves)]
+
+
 def attn_fwd(Qg, K, V, idx, q_pos=None, causal=False, tail=(0, 0), scale=None, sink=0, window=0):
     """Qg: [T, G, d]; K, V: [n_cap, d]; idx: [T, K_sel] or None -> (O [T,G,d], LSE [T,G]).
     sink / window > 0 (causal only): the first `sink` positions and the `window` positions up to

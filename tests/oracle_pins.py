@@ -278,6 +278,15 @@ def pin_select_full_beam_equals_flat():
     q_pos = rng.integers(0, Z.shape[0], 20)
     idx, bt, _ = orc.select(qlat, tree, full + [7], q_pos=q_pos, trace=True)
     np.testing.assert_array_equal(idx, _flat_topB(qlat, tree, 7, q_pos))
+    # the flat-search entry is that walk: same keys, and leaves in (score desc, id asc) order
+    idx_f, lv = orc.select_flat(qlat, tree, 7, q_pos=q_pos)
+    np.testing.assert_array_equal(idx_f, _flat_topB(qlat, tree, 7, q_pos))
+    li = tree.leaf_index.reshape(-1, tree.leaf_size)
+    for t in range(qlat.shape[0]):
+        got = lv[t][lv[t] >= 0]
+        np.testing.assert_array_equal(li[got].reshape(-1), idx_f[t][:len(got) * tree.leaf_size])
+        s = tree.centroids[-1][got] @ qlat[t]
+        assert np.all(np.diff(s) <= 0)
 
 
 def pin_select_beam_walk():

@@ -224,3 +224,21 @@ def test_tree_attention_beyond_partial_budget(lsa):
                           q_pos=case.q_pos.cpu().numpy()[rows], causal=True)
     mx, mean = parity.attn_errors(O[rows][:, sl].float().cpu(), Oo)
     assert mx <= 2e-2 and mean <= 2e-3, (mx, mean)
+
+
+def test_flat_prefill_1m_sampled(lsa):
+    """Flat search over the 16384 leaves of each head at 1,048,576 keys, 4096 causal queries;
+    the oracle checks sampled queries of two heads."""
+    from tests.test_gpu_flat import _check_flat
+    cfg = configs.get("prefill_1m")
+    case = cfg.case(DEV)
+    tree = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    idx, leaves = lsa.select_flat(tree, case.Q, case.W, cfg.beam[-1], case.q_pos, leaves=True)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(11)
+    rows = np.sort(rng.choice(cfg.T, 48, replace=False))
+    qp = case.q_pos.cpu().numpy()
+    for h in (0, 5):
+        th = parity.export_tree(tree, h)
+        oq = orc.query_latent(case.Q[:, h * cfg.G:(h + 1) * cfg.G].double().cpu().numpy(), case.W[h].double().cpu().numpy())
+        _check_flat(oq, th, cfg.beam[-1], qp, leaves[h].cpu().numpy(), idx[h].cpu().numpy(), cfg.leaf, rows)
