@@ -488,7 +488,7 @@ static cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
 // so the order is (score desc, leaf id asc).
 constexpr int kFlatQ = 32;              // queries per CTA (4 per warp)
 constexpr int kFlatTile = 256;          // leaves per tile (8 per lane)
-constexpr int kFlatKeep = 64;           // buffer size that triggers a reduction
+constexpr int kFlatKeep = 160;          // buffer size that triggers a reduction
 constexpr int kFlatCap = kFlatKeep + kFlatTile;
 
 template <int R>
