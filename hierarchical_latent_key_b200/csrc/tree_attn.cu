@@ -669,6 +669,223 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
   if (lane == 0) a.LSE[row] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
 }
 
+// ---- dense part: the sink and window keys, tile by tile -----------------------
+//
+// A CTA holds kTL rows, (query, head) pairs of one KV group: 128 / G consecutive
+// queries with their G heads.  Each row attends densely to the sink [0, n_sink)
+// and the window (q_pos - window, q_pos], each key once and none past q_pos or
+// the cache.  The CTA walks the 64-position key blocks that any of its rows
+// needs, twice: first for every row's softmax max and sum, then for
+// P = 2^(s - lse) and O = P.V on the tensor cores (O already normalised).
+
+struct BandArgs {
+  const __nv_bfloat16 *Q, *K, *V;
+  const int32_t* q_pos;
+  __nv_bfloat16* Od;           // [T][Hq][d]
+  float* LSEd;                 // [T][Hq] natural log (-inf: no dense key)
+  int32_t* status;
+  int64_t T, n_cap;
+  int32_t Hq, H, G, n_sink, window;
+  float scale_log2;
+};
+constexpr size_t kBandSmem = 1024 + kTL * 256 + 3 * kLeafKeys * 256;   // Q 32 KB; K, V, P 16 KB each
+
+__global__ void __launch_bounds__(kTL) k_tl_band(BandArgs a) {
+  extern __shared__ char smem_raw[];
+  __shared__ __align__(8) uint64_t s_mbar;
+  __shared__ uint32_t s_taddr;
+  __shared__ int32_t s_red[kTL / 32];
+  char* base = align1024(smem_raw);
+  char* gK = base + kTL * 256;
+  char* gV = gK + kLeafKeys * 256;
+  char* gP = gV + kLeafKeys * 256;
+  LeafSmem s;
+  s.sA = smem_u32(base);
+  s.sK = smem_u32(gK);
+  s.sV = smem_u32(gV);
+  s.sP = smem_u32(gP);
+  s.mbar = smem_u32(&s_mbar);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t g = blockIdx.y;
+  const int64_t t = (int64_t)blockIdx.x * (kTL / a.G) + threadIdx.x / a.G;
+  const int hh = threadIdx.x % a.G;
+  const bool valid = t < a.T;
+  const int64_t q = valid ? (int64_t)a.q_pos[t] : -1;
+  // this row's dense keys: [0, s_hi) and [w_lo, w_hi]
+  const int64_t s_hi = valid ? min(min((int64_t)a.n_sink, a.n_cap), q + 1) : 0;
+  const int64_t w_lo = max(max(q - a.window + 1, (int64_t)a.n_sink), (int64_t)0);
+  const int64_t w_hi = valid && a.window > 0 ? min(q, a.n_cap - 1) : -1;
+  // first block at or after b that this row needs (INT_MAX: none)
+  auto next_block = [&](int b) -> int {
+    if ((int64_t)b * kLeafKeys < s_hi) return b;
+    if (w_lo <= w_hi && (int64_t)b <= (w_hi >> 6)) return (int)max((int64_t)b, w_lo >> 6);
+    return INT_MAX;
+  };
+  auto cta_min = [&](int v) -> int {
+    v = __reduce_min_sync(0xffffffffu, v);
+    if (lane == 0) s_red[warp] = v;
+    __syncthreads();
+    int r = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kTL / 32; ++w) r = min(r, s_red[w]);
+    __syncthreads();
+    return r;
+  };
+  if (threadIdx.x == 0) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(s.mbar));
+    asm volatile("fence.mbarrier_init.release.cluster;");
+  }
+  // positions past every row's query are never attended, and the cache rows there
+  // may hold anything: their V rows are zeros (0 x NaN would still be NaN)
+  const int64_t qmax = -(int64_t)cta_min(valid ? -(int)q : INT_MAX);
+  if (valid) {
+    const __nv_bfloat16* qr = a.Q + (t * a.Hq + g * a.G + hh) * kDim;
+#pragma unroll
+    for (int c = 0; c < 16; ++c) cp_async16(s.sA + sw128_off(threadIdx.x, c, kTL * 128), qr + c * 8);
+  }
+  auto load_block = [&](int b, bool with_v) {
+    const int r = threadIdx.x >> 1, c0 = (threadIdx.x & 1) * 8;
+    const int64_t j = (int64_t)b * kLeafKeys + r;
+    if (j <= qmax && j < a.n_cap) {
+      const __nv_bfloat16* kr = a.K + (g * a.n_cap + j) * kDim;
+      const __nv_bfloat16* vr = a.V + (g * a.n_cap + j) * kDim;
+#pragma unroll
+      for (int c = c0; c < c0 + 8; ++c) {
+        cp_async16(s.sK + sw128_off(r, c, kLeafKeys * 128), kr + c * 8);
+        if (with_v) cp_async16(s.sV + sw128_off(r, c, kLeafKeys * 128), vr + c * 8);
+      }
+    } else {
+#pragma unroll
+      for (int c = c0; c < c0 + 8; ++c) {
+        *reinterpret_cast<uint4*>(gK + sw128_off(r, c, kLeafKeys * 128)) = make_uint4(0u, 0u, 0u, 0u);
+        if (with_v) *reinterpret_cast<uint4*>(gV + sw128_off(r, c, kLeafKeys * 128)) = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    cp_async_wait_all();
+    fence_async_smem();
+  };
+  // this row's 64 scores of block b (base-2 scaled; -inf outside its dense keys)
+  auto scores = [&](int b, uint32_t tmem, float (&sc)[64]) {
+    const int64_t j0 = (int64_t)b * kLeafKeys;
+    const int64_t sh = s_hi - j0, wl = w_lo - j0, wh = w_hi - j0;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      float v[32];
+      tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + half * 32, v);
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const int k = half * 32 + i;
+        sc[k] = (k < sh || (k >= wl && k <= wh)) ? v[i] * a.scale_log2 : -INFINITY;
+      }
+    }
+  };
+  alloc_tmem(&s_taddr, 256);   // S in columns [0, 64), O in [64, 192)
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s_taddr;
+  uint32_t phase = 0;
+  bool ok = true;
+  // product on the tensor cores, then every thread waits for it
+  auto run_mma = [&](bool pv, bool accumulate) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      tc_fence_after();
+      if (!pv) {
+        issue_qk(s, tmem, 0);
+      } else {
+        constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          tc_mma(tmem + 64, sdesc_sw128(s.sP + kk * 32, 16, 1024),
+                 sdesc_sw128(s.sV + kk * 2048, kLeafKeys * 128, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
+      }
+      tc_commit(s.mbar);
+    }
+    ok = __syncthreads_and(mbar_wait(s.mbar, phase));
+    phase ^= 1;
+    tc_fence_after();
+  };
+  // sweep 1: max and sum of every row
+  float m = -INFINITY, l = 0.f;
+  for (int b = cta_min(next_block(0)); b != INT_MAX && ok; b = cta_min(next_block(b + 1))) {
+    load_block(b, false);
+    run_mma(false, false);
+    if (!ok) break;
+    float sc[64];
+    scores(b, tmem, sc);
+    float bm = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 64; ++i) bm = fmaxf(bm, sc[i]);
+    const float mn = fmaxf(m, bm);
+    if (mn != -INFINITY) {
+      float sum = 0.f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) sum += exp2f(sc[i] - mn);
+      l = (m == -INFINITY ? 0.f : l * exp2f(m - mn)) + sum;
+      m = mn;
+    }
+    tc_fence_before();
+  }
+  const float lse2 = l > 0.f ? m + log2f(l) : INFINITY;   // +inf: P = 0
+  // sweep 2: O = sum over blocks of 2^(s - lse) . V
+  bool any = false;
+  for (int b = cta_min(next_block(0)); b != INT_MAX && ok; b = cta_min(next_block(b + 1))) {
+    load_block(b, true);
+    run_mma(false, false);
+    if (!ok) break;
+    float sc[64];
+    scores(b, tmem, sc);
+    const int r = threadIdx.x;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        __nv_bfloat162 b2 = __floats2bfloat162_rn(exp2f(sc[c * 8 + 2 * i] - lse2), exp2f(sc[c * 8 + 2 * i + 1] - lse2));
+        w[i] = *reinterpret_cast<uint32_t*>(&b2);
+      }
+      *reinterpret_cast<uint4*>(gP + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    run_mma(true, any);
+    any = true;
+    tc_fence_before();
+  }
+  if (!ok) set_status(a.status, LSA_ERR_TIMEOUT);
+  if (ok) {   // CTA-uniform: the TMEM loads are warp-collective, the stores per row
+    const int64_t row = t * a.Hq + g * a.G + hh;
+    __nv_bfloat16* dst = valid ? a.Od + row * kDim : nullptr;
+#pragma unroll
+    for (int part = 0; part < 4; ++part) {
+      float v[32];
+      if (any) {
+        tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + 64 + part * 32, v);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 32; i += 8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(v[i + 2 * k], v[i + 2 * k + 1]);
+          w[k] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        if (dst) *reinterpret_cast<uint4*>(dst + part * 32 + i) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    if (valid) a.LSEd[row] = l > 0.f ? (m + log2f(l)) * 0.69314718055994530942f : -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  free_tmem(tmem, 256);
+}
+
 // ---- partial mode, pipelined ------------------------------------------------
 //
 // Persistent CTAs (one per SM), each walking a contiguous range of chunks with
@@ -1370,11 +1587,7 @@ size_t tree_attn_workspace(int64_t H, int64_t NL, int64_t T, int64_t Hq, int d, 
   const int epc = kChunkRows / (int)(Hq / H);
   size_t part = lists + al((size_t)T * Hq * B * d * 2) + al((size_t)H * T * B * 4) + al(H * NL * 4) +
                 al(H * 4) + al((size_t)max_chunks(H, NL, T, B, epc) * 16);
-  if (sw) {   // dense part: its key lists, output, LSE and split partials
-    const int ns = attn_splits(T, (int)H, n_sink + window);
-    part += al((size_t)H * T * (n_sink + window) * 4) + al((size_t)T * Hq * d * 2) + al((size_t)T * Hq * 4) +
-            (ns > 1 ? al((size_t)T * Hq * ns * (d + 2) * 4) : 0);
-  }
+  if (sw) part += al((size_t)T * Hq * d * 2) + al((size_t)T * Hq * 4);   // dense part: output and LSE
   return part > red ? part : red;
 }
 
@@ -1454,18 +1667,19 @@ cudaError_t run_tree_attn(const TreeAttnCall& c, cudaStream_t st) {
     a.ctotal = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * 4);
     a.cdesc = reinterpret_cast<int4*>(ws + o);
     o += al((size_t)max_chunks(c.H, c.NL, c.T, c.B, a.epc) * 16);
-    if (sw) {   // dense part: the sink and window keys through the key-list attention
-      const int32_t KD = c.n_sink + c.window;
-      int32_t* idxd = reinterpret_cast<int32_t*>(ws + o); o += al((size_t)c.H * c.T * KD * 4);
-      __nv_bfloat16* Od = reinterpret_cast<__nv_bfloat16*>(ws + o); o += al((size_t)c.T * c.Hq * kDim * 2);
-      float* LSEd = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);
-      float* partd = attn_splits(c.T, c.H, KD) > 1 ? reinterpret_cast<float*>(ws + o) : nullptr;
-      if ((e = run_attn_extend(nullptr, 0, c.T, c.H, c.q_pos, c.n_sink, c.window, 0, 0, c.n_cap, idxd, st)) !=
-          cudaSuccess)
-        return e;
-      if ((e = keylist_attn(idxd, KD, Od, LSEd, partd)) != cudaSuccess) return e;
-      a.Od = Od;
-      a.LSEd = LSEd;
+    if (sw) {   // dense part: the sink and window keys, 64-position blocks on the tensor cores
+      BandArgs d;
+      d.Q = a.Q; d.K = a.K; d.V = a.V; d.q_pos = c.q_pos;
+      d.Od = reinterpret_cast<__nv_bfloat16*>(ws + o); o += al((size_t)c.T * c.Hq * kDim * 2);
+      d.LSEd = reinterpret_cast<float*>(ws + o); o += al((size_t)c.T * c.Hq * 4);
+      d.status = c.status; d.T = c.T; d.n_cap = c.n_cap;
+      d.Hq = (int32_t)c.Hq; d.H = (int32_t)c.H; d.G = G; d.n_sink = c.n_sink; d.window = c.window;
+      d.scale_log2 = c.scale * 1.44269504088896340736f;
+      cudaFuncSetAttribute(k_tl_band, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBandSmem);
+      k_tl_band<<<dim3((unsigned)ceil_div(c.T, (int64_t)(kTL / G)), (unsigned)c.H), kTL, kBandSmem, st>>>(d);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+      a.Od = d.Od;
+      a.LSEd = d.LSEd;
     }
   } else {
     o = o_lists;
