@@ -317,6 +317,62 @@ int orc_build_tree(const double *Z, int64_t n, int32_t r, const int32_t *branchi
 }
 
 /* ------------------------------------------------------------------------- */
+/* Pooling of consecutive keys ([P4] "How latent sparse attention works": the  */
+/* keys are first pooled into smaller representations, then clustered).       */
+/* Reading (the pages give neither the pooling operator nor the block size):   */
+/* block j holds the p consecutive keys at positions [j*p, (j+1)*p) and is     */
+/* represented by the mean of their latent rows.                              */
+/* Zp: [n/p, r].                                                               */
+/* ------------------------------------------------------------------------- */
+int orc_pool_keys(const double *Z, int64_t n, int32_t r, int32_t p, double *Zp) {
+  if (!Z || !Zp || p < 1 || r < 1) return ORC_ERR_ARG;
+  if (n % p) return ORC_ERR_SHAPE;
+  for (int64_t j = 0; j < n / p; ++j)
+    for (int32_t c = 0; c < r; ++c) {
+      double s = 0.0;
+      for (int32_t i = 0; i < p; ++i) s += Z[(j * p + i) * r + c];
+      Zp[j * r + c] = s / p;
+    }
+  return ORC_OK;
+}
+
+/* Tree over pooled blocks: the build above runs on the n/p block rows (a      */
+/* block's position is its index j, which orders pairs and seeds the start),  */
+/* with leaf_size/p blocks per leaf.  The cluster then references the         */
+/* original keys of its blocks ([P4]: centroids stored with references to the */
+/* original keys): leaf_index lists, for each block j of a leaf in ascending  */
+/* order, the keys j*p .. j*p+p-1, and min_pos is in key positions.            */
+/* trace (optional): [levels, iters, n/p] node id of each block.               */
+int orc_build_tree_pooled(const double *Z, int64_t n, int32_t r, int32_t p, const int32_t *branching,
+                          int32_t levels, int32_t leaf_size, int32_t iters, uint64_t seed,
+                          double *centroids, int32_t *min_pos, int32_t *leaf_index, int32_t *trace) {
+  if (!Z || !branching || !centroids || !min_pos || !leaf_index || p < 1) return ORC_ERR_ARG;
+  if (n % p || leaf_size % p) return ORC_ERR_SHAPE;
+  if (levels < 1 || levels > ORC_MAX_LEVELS) return ORC_ERR_ARG;
+  const int64_t nb = n / p;
+  double *Zp = (double *)malloc(sizeof(double) * nb * r);
+  int32_t *blocks = (int32_t *)malloc(sizeof(int32_t) * nb);
+  if (!Zp || !blocks) { free(Zp); free(blocks); return ORC_ERR_ALLOC; }
+  int err = orc_pool_keys(Z, n, r, p, Zp);
+  if (err == ORC_OK)
+    err = orc_build_tree(Zp, nb, r, branching, levels, leaf_size / p, iters, seed, centroids, min_pos, blocks,
+                         trace);
+  if (err == ORC_OK) {
+    int64_t nodes = 0, level_nodes = 1;
+    for (int32_t l = 0; l < levels; ++l) {
+      level_nodes *= branching[l];
+      nodes += level_nodes;
+    }
+    for (int64_t k = 0; k < nodes; ++k) min_pos[k] *= p;
+    for (int64_t s = 0; s < nb; ++s)
+      for (int32_t i = 0; i < p; ++i) leaf_index[s * p + i] = blocks[s] * p + i;
+  }
+  free(Zp);
+  free(blocks);
+  return err;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Hierarchical search ([P1]: the query starts at the root, scores a few      */
 /* candidate clusters per level and descends into a few branches; [P4]:       */
 /* fixed search budget per level; a fixed number of original keys retrieved  */

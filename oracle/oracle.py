@@ -16,6 +16,9 @@ Parity status of each function (what pins it, in ``tests/test_oracle_pins.py``):
                             an independent deferred-acceptance implementation
   build_tree                centroid == mean of members, parent == mean of
                             children, exact leaf sizes, permutation, init rule
+  pool_keys,                pool 1 == build_tree; centroids == means of the listed
+  build_tree_pooled         keys' latents; leaves are whole aligned blocks; block
+                            tree == build_tree on latents pooled by numpy
   select                    full beam == brute-force flat top-B over all leaves,
                             scored-node count, causal eligibility brute force
   attn_fwd                  torch SDPA (CPU, float64) with a boolean mask, one
@@ -98,6 +101,8 @@ def _declare(lib):
         "orc_level_init": (ctypes.c_int, [P, P, i64, i32, i32, u64, i32, P]),
         "orc_means": (ctypes.c_int, [P, i64, i32, P, i32, P]),
         "orc_build_tree": (ctypes.c_int, [P, i64, i32, P, i32, i32, i32, u64, P, P, P, P]),
+        "orc_pool_keys": (ctypes.c_int, [P, i64, i32, i32, P]),
+        "orc_build_tree_pooled": (ctypes.c_int, [P, i64, i32, i32, P, i32, i32, i32, u64, P, P, P, P]),
         "orc_select": (ctypes.c_int, [P, i64, i32, P, i32, i32, P, P, P, P, P, P, P, P]),
         "orc_attn_fwd": (ctypes.c_int, [P, i64, i32, i32, P, P, i64, P, i32, P, i32, i64, i64,
                                         f64, P, P]),
@@ -249,6 +254,32 @@ def build_tree(Z, branching, leaf_size: int, iters: int, seed: int, trace: bool 
     tr = np.empty((L, iters, n), np.int32) if trace else None
     _check(load().orc_build_tree(_p(Z), n, r, _p(br), L, leaf_size, iters, seed,
                                  _p(cent), _p(mpos), _p(leaf), _p(tr)), "orc_build_tree")
+    return Tree(br, leaf_size, r, cent, mpos, leaf, tr)
+
+
+def pool_keys(Z, p: int) -> np.ndarray:
+    """Mean latent row of every block of p consecutive keys: [n, r] -> [n / p, r]."""
+    Z = _f64(Z)
+    n, r = Z.shape
+    out = np.empty((n // p, r), np.float64)
+    _check(load().orc_pool_keys(_p(Z), n, r, p, _p(out)), "orc_pool_keys")
+    return out
+
+
+def build_tree_pooled(Z, p: int, branching, leaf_size: int, iters: int, seed: int, trace: bool = False) -> Tree:
+    """Tree over blocks of p consecutive keys (leaf_size / p blocks per leaf); leaf_index and
+    min_pos in key positions, trace (if asked) by block."""
+    Z = _f64(Z)
+    n, r = Z.shape
+    br = np.ascontiguousarray(branching, np.int32)
+    L = len(br)
+    total_nodes = int(np.sum(np.cumprod(br.astype(np.int64))))
+    cent = np.empty(total_nodes * r, np.float64)
+    mpos = np.empty(total_nodes, np.int32)
+    leaf = np.empty(n, np.int32)
+    tr = np.empty((L, iters, n // p), np.int32) if trace else None
+    _check(load().orc_build_tree_pooled(_p(Z), n, r, p, _p(br), L, leaf_size, iters, seed,
+                                        _p(cent), _p(mpos), _p(leaf), _p(tr)), "orc_build_tree_pooled")
     return Tree(br, leaf_size, r, cent, mpos, leaf, tr)
 
 

@@ -500,4 +500,36 @@ def pin_backward_sink_window_autograd():
     np.testing.assert_allclose(dK, k.grad.numpy(), rtol=1e-9, atol=1e-12)
     np.testing.assert_allclose(dV, v.grad.numpy(), rtol=1e-9, atol=1e-12)
 
+def pin_tree_pooled():
+    """Pooling then clustering (bdtechtalks.com, "How latent sparse attention works"): pool 1 is
+    the plain build; with pool p the tree over blocks is the plain build over block means taken
+    by numpy; every stored centroid is the mean of the latent rows of the keys its node lists,
+    min_pos is a key position, and a leaf is a union of whole aligned blocks."""
+    rng = np.random.default_rng(5)
+    n, d, r, p, br, leaf = 1024, 32, 8, 4, (8, 8), 16
+    K = _mixture(rng, n, d, 16)
+    W = rng.standard_normal((d, r)) / np.sqrt(d)
+    Z = K @ W
+    Zo = orc.project(K, W)
+    t0 = orc.build_tree(Zo, br, leaf, 3, seed=2, trace=True)
+    t1 = orc.build_tree_pooled(Zo, 1, br, leaf, 3, seed=2, trace=True)
+    np.testing.assert_array_equal(t1.leaf_index, t0.leaf_index)
+    np.testing.assert_array_equal(t1.centroids_flat, t0.centroids_flat)
+    np.testing.assert_array_equal(t1.min_pos_flat, t0.min_pos_flat)
+    np.testing.assert_array_equal(t1.trace, t0.trace)
+    tp = orc.build_tree_pooled(Zo, p, br, leaf, 3, seed=2, trace=True)
+    li = tp.leaf_index.astype(np.int64)
+    np.testing.assert_array_equal(np.sort(li), np.arange(n))
+    blk = li.reshape(-1, p)
+    assert np.all(blk[:, 0] % p == 0) and np.all(blk == blk[:, :1] + np.arange(p))
+    assert np.all(np.diff(li.reshape(-1, leaf), axis=1) > 0)
+    tb = orc.build_tree(Z.reshape(n // p, p, r).mean(axis=1), br, leaf // p, 3, seed=2, trace=True)
+    np.testing.assert_array_equal(blk[:, 0] // p, tb.leaf_index)
+    np.testing.assert_array_equal(tp.trace, tb.trace)
+    for l in range(len(br)):
+        groups = li.reshape(tp.nodes[l], -1)
+        np.testing.assert_allclose(tp.centroids[l], Z[groups].mean(axis=1), rtol=1e-10, atol=1e-12)
+        np.testing.assert_array_equal(tp.min_pos[l], groups.min(axis=1))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -23,7 +23,7 @@ ORDER = [
     P.pin_select_beam_walk, P.pin_select_full_beam_equals_flat,
     P.pin_attention_equals_sdpa, P.pin_attention_special_cases,
     P.pin_backward_autograd, P.pin_backward_finite_differences,
-    P.pin_attention_sink_window, P.pin_backward_sink_window_autograd,
+    P.pin_attention_sink_window, P.pin_backward_sink_window_autograd, P.pin_tree_pooled,
 ]
 assert sorted(f.__name__ for f in ORDER) == sorted(f.__name__ for f in P.ALL_PINS)
 
@@ -67,6 +67,12 @@ MUTANTS = [
      "for (int64_t j = (int64_t)q_pos[t] - window + 2; j <= q_pos[t]; ++j)"),
     ("sink ignores causality", "if (j <= q_pos[t]) out[cnt++] = j;", "out[cnt++] = j;"),
     ("repeated key counted twice", "if (u == 0 || out[k] != out[u - 1]) out[u++] = out[k];", "out[u++] = out[k];"),
+    ("pool drops a key", "for (int32_t i = 0; i < p; ++i) s += Z[(j * p + i) * r + c];",
+     "for (int32_t i = 1; i < p; ++i) s += Z[(j * p + i) * r + c];"),
+    ("pool sums instead of averaging", "Zp[j * r + c] = s / p;", "Zp[j * r + c] = s;"),
+    ("pooled keys not expanded", "leaf_index[s * p + i] = blocks[s] * p + i;", "leaf_index[s * p + i] = blocks[s] + i;"),
+    ("pooled min_pos left in blocks", "for (int64_t k = 0; k < nodes; ++k) min_pos[k] *= p;",
+     "for (int64_t k = 0; k < nodes; ++k) min_pos[k] *= 1;"),
 ]
 
 
