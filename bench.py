@@ -464,6 +464,7 @@ def time_steps(w, steps, warmup, flush, stream):
 
 
 SINK, WINDOW = 16, 512   # sink tokens and recent window of the sink/window measurement
+POOL = 4                 # keys per block of the pooled index
 
 
 def time_sink_window(w, steps, warmup, flush, stream, sink=SINK, window=WINDOW):
@@ -535,6 +536,61 @@ def time_flat(w, steps, warmup, flush, stream):
     return {"value": T / ((sel + att) / 1e3), "unit": "queries/s", "breakdown_ms": {"select": sel, "attention": att},
             "config": f"prefill step as above with flat search: {nl} leaf centroids scored per query and group, "
                       f"the best {w.cfg.beam[-1]} kept"}
+
+
+def time_pooled(w, steps, warmup, flush, stream, pool=POOL):
+    """The index over blocks of `pool` consecutive keys (lsa_build_tree_pooled): its build beside
+    the plain build (CUDA events, same workspace, median of 3), then the prefill step (select +
+    tree attention) on the pooled index."""
+    lsa, cfg = w.lsa, w.cfg
+    d = w.K.shape[2]
+    ws = torch.empty(lsa.lsa_build_workspace_bytes(w.tree.desc, d), dtype=torch.uint8, device=w.K.device)
+
+    def build(p):
+        times, tree = [], None
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            tree = lsa.build_tree(w.K, w.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed, workspace=ws,
+                                  status=w.status, check=False, pool=p)
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        return tree, statistics.median(times)
+
+    _, keys_ms = build(1)
+    tree, pooled_ms = build(pool)
+    plain = w.tree
+    w.tree = tree
+    try:
+        for _ in range(warmup):
+            flush.zero_()
+            w.select()
+            w.attend()
+        torch.cuda.synchronize()
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        for k in range(steps):
+            flush.zero_()
+            ev[k][0].record(stream)
+            w.select()
+            ev[k][1].record(stream)
+            w.attend()
+            ev[k][2].record(stream)
+        torch.cuda.synchronize()
+    finally:
+        w.tree = plain
+    code = lsa.lsa_status_check(w.status)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code}: {lsa.lsa_strerror(code)}")
+    sel = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(steps))
+    att = statistics.mean(ev[k][1].elapsed_time(ev[k][2]) for k in range(steps))
+    T = w.Q.shape[0]
+    return {"value": T / ((sel + att) / 1e3), "unit": "queries/s", "pool": pool,
+            "build_ms": {"pooled": pooled_ms, "keys": keys_ms},
+            "breakdown_ms": {"select": sel, "attention": att},
+            "config": f"prefill step as above on an index whose k-means levels cluster blocks of {pool} "
+                      f"consecutive keys ({cfg.n // pool:,} blocks per head, {cfg.leaf // pool} per leaf); "
+                      f"build times over all {cfg.Hkv} heads with CUDA events"}
 
 
 def time_e2e(w, steps, flush, stream):
@@ -683,6 +739,10 @@ def run_cuda(args, rank, world, local_rank):
         flat = time_flat(w, args.steps, args.warmup, flush, stream)
     except Exception as e:  # noqa: BLE001
         flat = {"error": f"{type(e).__name__}: {e}"}
+    try:
+        pooled = time_pooled(w, args.steps, args.warmup, flush, stream)
+    except Exception as e:  # noqa: BLE001
+        pooled = {"error": f"{type(e).__name__}: {e}"}
     decode = train = None
     del w
     torch.cuda.empty_cache()
@@ -727,6 +787,7 @@ def run_cuda(args, rank, world, local_rank):
             "cpu_baseline": cpu,
             "prefill_1m_sink_window": sink_window,
             "prefill_1m_flat": flat,
+            "prefill_1m_pooled": pooled,
             "decode_10m": decode,
             "train_128k": train,
         }

@@ -177,8 +177,17 @@ int lsa_build_workspace_bytes(const lsa_tree_desc* tree, int32_t d, size_t* byte
 int lsa_build_tree(const lsa_tree_desc* tree, void* tree_mem, const void* K, int64_t n_cap, int32_t d,
                    int32_t dtype, const void* W, int32_t iters, uint64_t seed, void* workspace,
                    size_t workspace_bytes, int32_t* trace, int32_t* status, void* stream) {
+  return lsa_build_tree_pooled(tree, tree_mem, K, n_cap, d, dtype, W, 1, iters, seed, workspace, workspace_bytes,
+                               trace, status, stream);
+}
+
+int lsa_build_tree_pooled(const lsa_tree_desc* tree, void* tree_mem, const void* K, int64_t n_cap, int32_t d,
+                          int32_t dtype, const void* W, int32_t pool, int32_t iters, uint64_t seed, void* workspace,
+                          size_t workspace_bytes, int32_t* trace, int32_t* status, void* stream) {
   int rc = check_desc(tree);
   if (rc != LSA_OK) return rc;
+  if (pool < 1 || tree->leaf_size % pool != 0)
+    return fail(LSA_ERR_SHAPE, "pool (%d) must be >= 1 and divide leaf_size (%d)", pool, tree->leaf_size);
   if (!tree_mem || !K || !W) return fail(LSA_ERR_INVALID_ARG, "tree_mem, K and W must be non-NULL");
   if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
@@ -195,8 +204,9 @@ int lsa_build_tree(const lsa_tree_desc* tree, void* tree_mem, const void* K, int
   if (P.coop_blocks <= 0) return fail(LSA_ERR_CUDA, "cannot size the cooperative assignment grid");
   cudaError_t e = cudaMemsetAsync(tree_mem, 0, tree->bytes, static_cast<cudaStream_t>(stream));
   if (e == cudaSuccess)
-    e = lsa::run_build(P, *tree, tree_mem, K, n_cap, d, dtype, W, trace, status, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "lsa_build_tree");
+    e = lsa::run_build(P, *tree, tree_mem, K, n_cap, d, dtype, W, pool, trace, status,
+                       static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_build_tree_pooled");
   return ok();
 }
 

@@ -687,14 +687,49 @@ __global__ void k_level_gather(const int32_t* __restrict__ order, const float* _
   if (part == 0) pb[q] = pa[src];
 }
 
-// smallest position of each node = position of its first member (ascending)
+// smallest key position of each node = that of its first member (ascending);
+// a member is a key, or with pooling a block of `pool` keys starting at pa * pool
 __global__ void k_min_pos(const int32_t* __restrict__ order, const int32_t* __restrict__ pa, int64_t nnodes,
-                          int64_t cap, int32_t* __restrict__ min_pos) {
+                          int64_t cap, int32_t pool, int32_t* __restrict__ min_pos) {
   const int64_t node = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (node >= nnodes) return;
   int64_t src = order[node * cap];
   if ((uint64_t)src >= (uint64_t)(nnodes * cap)) src = 0;  // only after a failed assignment
-  min_pos[node] = pa[src];
+  min_pos[node] = pa[src] * pool;
+}
+
+// ---------------------------------------------------------------------------
+// pooling (bdtechtalks.com, "Latent sparse attention", section "How latent
+// sparse attention works": consecutive keys pooled into smaller
+// representations before the clustering): block j of a head is the mean of the
+// latent rows of keys [j*pool, (j+1)*pool), summed in position order; its
+// position is j.
+// ---------------------------------------------------------------------------
+template <int R>
+__global__ void k_pool_keys(const float* __restrict__ Z, int64_t nblocks, int64_t per_head, int32_t pool,
+                            float* __restrict__ Zp, int32_t* __restrict__ pos) {
+  constexpr int V = R / 4;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // (head * nblocks + block) * V + part
+  if (i >= nblocks * V) return;
+  const int64_t blk = i / V, part = i % V;
+  const float4* src = reinterpret_cast<const float4*>(Z) + blk * pool * V + part;
+  float4 acc = src[0];
+  for (int k = 1; k < pool; ++k) {
+    const float4 v = src[(int64_t)k * V];
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  const float inv = 1.f / (float)pool;
+  reinterpret_cast<float4*>(Zp)[i] = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+  if (part == 0) pos[blk] = (int32_t)(blk % per_head);
+}
+
+// leaf_index of a pooled tree: block slot s (ascending inside its leaf) lists
+// the keys b*pool .. b*pool + pool - 1 of its block b
+__global__ void k_expand_leaves(const int32_t* __restrict__ blocks, int64_t nslots, int32_t pool,
+                                int32_t* __restrict__ leaf_index) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= nslots * pool) return;
+  leaf_index[i] = blocks[i / pool] * pool + (int32_t)(i % pool);
 }
 
 // ---------------------------------------------------------------------------
@@ -702,7 +737,7 @@ __global__ void k_min_pos(const int32_t* __restrict__ order, const int32_t* __re
 // ---------------------------------------------------------------------------
 template <int R>
 static cudaError_t build_levels(const BuildPlan& P, const lsa_tree_desc& t, char* tree_mem, int32_t* trace,
-                                int32_t* status, cudaStream_t st) {
+                                int32_t* status, int32_t pool, cudaStream_t st) {
   const int64_t H = t.n_heads, n = t.n_tree, nslots = H * n;
   float* Za = P.Za;
   float* Zb = P.Zb;
@@ -722,8 +757,12 @@ static cudaError_t build_levels(const BuildPlan& P, const lsa_tree_desc& t, char
     const int64_t cpn = ceil_div(cap, kMeanChunk);
     for (int it = 0; it < P.iters; ++it) {
       {
+        // centroids of every segment a CTA's 256 slots touch: (256 / m + 1) * b rows,
+        // at most (256 + b) * R floats (about 70 KB) when a segment holds b members
         const int64_t rows = (ceil_div(256, m) + 1) * b;
         const size_t smem = (size_t)rows * R * sizeof(float);
+        if (smem > 48 * 1024)
+          cudaFuncSetAttribute(k_dist_pref<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_dist_pref<R><<<(unsigned)ceil_div(nslots, 256), 256, smem, st>>>(Za, P.mu, nslots, m, b, P.D, P.pref,
                                                                           P.choice, P.ptr, P.dbits, status);
       }
@@ -770,7 +809,7 @@ static cudaError_t build_levels(const BuildPlan& P, const lsa_tree_desc& t, char
     if ((e = cudaMemcpyAsync(cent, P.mu, (size_t)nnodes * R * sizeof(float), cudaMemcpyDeviceToDevice, st)) !=
         cudaSuccess)
       return e;
-    k_min_pos<<<(unsigned)ceil_div(nnodes, 256), 256, 0, st>>>(P.order, pa, nnodes, cap, mpos);
+    k_min_pos<<<(unsigned)ceil_div(nnodes, 256), 256, 0, st>>>(P.order, pa, nnodes, cap, pool, mpos);
     k_level_gather<R><<<(unsigned)ceil_div(nslots * (R / 4), 256), 256, 0, st>>>(P.order, Za, pa, nslots, Zb, pb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     float* tz = Za; Za = Zb; Zb = tz;
@@ -778,7 +817,9 @@ static cudaError_t build_levels(const BuildPlan& P, const lsa_tree_desc& t, char
     S *= b;
   }
   int32_t* leaf = reinterpret_cast<int32_t*>(tree_mem + t.off_leaf_index);
-  return cudaMemcpyAsync(leaf, pa, (size_t)nslots * sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+  if (pool == 1) return cudaMemcpyAsync(leaf, pa, (size_t)nslots * sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+  k_expand_leaves<<<(unsigned)ceil_div(nslots * pool, 256), 256, 0, st>>>(pa, nslots, pool, leaf);
+  return cudaGetLastError();
 }
 
 template <typename T>
@@ -801,15 +842,34 @@ static cudaError_t project(const BuildPlan& P, const lsa_tree_desc& t, const voi
 }
 
 cudaError_t run_build(const BuildPlan& P, const lsa_tree_desc& t, void* tree_mem, const void* K, int64_t n_cap,
-                      int d, int dtype, const void* W, int32_t* trace, int32_t* status, cudaStream_t st) {
+                      int d, int dtype, const void* W, int32_t pool, int32_t* trace, int32_t* status,
+                      cudaStream_t st) {
   cudaError_t e = dtype == LSA_BF16 ? project<__nv_bfloat16>(P, t, K, n_cap, d, W, st)
                                     : project<float>(P, t, K, n_cap, d, W, st);
   if (e != cudaSuccess) return e;
   char* tm = static_cast<char*>(tree_mem);
+  // with pooling the levels cluster the blocks: same nodes and tree buffer,
+  // n_tree / pool members with leaf_size / pool per leaf
+  BuildPlan Q = P;
+  lsa_tree_desc tb = t;
+  if (pool > 1) {
+    const int64_t per_head = t.n_tree / pool, nblocks = t.n_heads * per_head;
+    const unsigned grid = (unsigned)ceil_div(nblocks * (t.r / 4), 256);
+    switch (t.r) {
+      case 16: k_pool_keys<16><<<grid, 256, 0, st>>>(P.Za, nblocks, per_head, pool, P.Zb, P.pb); break;
+      case 32: k_pool_keys<32><<<grid, 256, 0, st>>>(P.Za, nblocks, per_head, pool, P.Zb, P.pb); break;
+      default: k_pool_keys<64><<<grid, 256, 0, st>>>(P.Za, nblocks, per_head, pool, P.Zb, P.pb); break;
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    Q.Za = P.Zb; Q.Zb = P.Za;
+    Q.pa = P.pb; Q.pb = P.pa;
+    tb.n_tree = t.n_tree / pool;
+    tb.leaf_size = t.leaf_size / pool;
+  }
   switch (t.r) {
-    case 16: return build_levels<16>(P, t, tm, trace, status, st);
-    case 32: return build_levels<32>(P, t, tm, trace, status, st);
-    default: return build_levels<64>(P, t, tm, trace, status, st);
+    case 16: return build_levels<16>(Q, tb, tm, trace, status, pool, st);
+    case 32: return build_levels<32>(Q, tb, tm, trace, status, pool, st);
+    default: return build_levels<64>(Q, tb, tm, trace, status, pool, st);
   }
 }
 

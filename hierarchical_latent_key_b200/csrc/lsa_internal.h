@@ -57,7 +57,8 @@ struct BuildPlan {
 size_t build_workspace_layout(const lsa_tree_desc& t, char* base, BuildPlan* plan);
 
 cudaError_t run_build(const BuildPlan& P, const lsa_tree_desc& t, void* tree_mem, const void* K, int64_t n_cap,
-                      int d, int dtype, const void* W, int32_t* trace, int32_t* status, cudaStream_t st);
+                      int d, int dtype, const void* W, int32_t pool, int32_t* trace, int32_t* status,
+                      cudaStream_t st);
 int da_grid_blocks();
 
 struct SelectArgs {

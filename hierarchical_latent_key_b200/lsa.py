@@ -56,6 +56,7 @@ def _load():
         "lsa_tree_describe": (ctypes.c_int, [i32, i32, P, i32, i32, D]),
         "lsa_build_workspace_bytes": (ctypes.c_int, [D, i32, ctypes.POINTER(sz)]),
         "lsa_build_tree": (ctypes.c_int, [D, P, P, i64, i32, i32, P, i32, u64, P, sz, P, P, P]),
+        "lsa_build_tree_pooled": (ctypes.c_int, [D, P, P, i64, i32, i32, P, i32, i32, u64, P, sz, P, P, P]),
         "lsa_select": (ctypes.c_int, [D, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]),
         "lsa_tree_attn_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
         "lsa_tree_attn": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, i32, P, i32, f32, P, P, P, sz,
@@ -154,6 +155,14 @@ def lsa_build_tree(desc, tree_mem, K, W, iters, seed, workspace, trace=None, sta
     _raise(_lib.lsa_build_tree(ctypes.byref(desc), _ptr(tree_mem), _ptr(K), K.shape[1], K.shape[2], _dtype(K),
                                _ptr(W), iters, seed & ((1 << 64) - 1), _ptr(workspace), workspace.numel(),
                                _ptr(trace), _ptr(status), _stream(stream, K)), "lsa_build_tree")
+
+
+def lsa_build_tree_pooled(desc, tree_mem, K, W, pool, iters, seed, workspace, trace=None, status=None, stream=None):
+    """lsa_build_tree over blocks of `pool` consecutive keys (trace by block)."""
+    _raise(_lib.lsa_build_tree_pooled(ctypes.byref(desc), _ptr(tree_mem), _ptr(K), K.shape[1], K.shape[2],
+                                      _dtype(K), _ptr(W), pool, iters, seed & ((1 << 64) - 1), _ptr(workspace),
+                                      workspace.numel(), _ptr(trace), _ptr(status), _stream(stream, K)),
+           "lsa_build_tree_pooled")
 
 
 def lsa_select(desc, tree_mem, Q, W, beam, q_pos, idx_out, leaves_out=None, qlat_out=None, beam_out=None,
@@ -313,17 +322,23 @@ class Tree:
         return self.mem[off:off + 4 * n].view(torch.int32).view(d.n_heads, d.n_tree)
 
 
-def build_tree(K, W, branching, leaf_size, iters, seed, trace=False, workspace=None, status=None, check=True):
-    """Build the index over positions [0, leaf_size * prod(branching)) of K."""
+def build_tree(K, W, branching, leaf_size, iters, seed, trace=False, workspace=None, status=None, check=True,
+               pool=1):
+    """Build the index over positions [0, leaf_size * prod(branching)) of K; pool > 1 clusters
+    blocks of `pool` consecutive keys (the trace is then by block)."""
     Hkv, n_cap, d = K.shape
     desc = lsa_tree_describe(Hkv, W.shape[2], branching, leaf_size)
     mem = torch.empty(desc.bytes, dtype=torch.uint8, device=K.device)
     need = lsa_build_workspace_bytes(desc, d)
     if workspace is None or workspace.numel() < need:
         workspace = torch.empty(need, dtype=torch.uint8, device=K.device)
-    tr = torch.empty(len(branching), iters, Hkv, desc.n_tree, dtype=torch.int32, device=K.device) if trace else None
+    tr = (torch.empty(len(branching), iters, Hkv, desc.n_tree // pool, dtype=torch.int32, device=K.device)
+          if trace else None)
     st = _new_status(K.device) if status is None else status
-    lsa_build_tree(desc, mem, K, W, iters, seed, workspace, tr, st)
+    if pool == 1:
+        lsa_build_tree(desc, mem, K, W, iters, seed, workspace, tr, st)
+    else:
+        lsa_build_tree_pooled(desc, mem, K, W, pool, iters, seed, workspace, tr, st)
     if check:
         check_status(st, "lsa_build_tree")
     tree = Tree(desc, mem)

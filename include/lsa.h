@@ -132,6 +132,29 @@ int lsa_build_tree(const lsa_tree_desc *tree, void *tree_mem, const void *K, int
                    void *workspace, size_t workspace_bytes, int32_t *trace, int32_t *status,
                    void *stream);
 
+/* lsa_build_tree over pooled keys (bdtechtalks.com, "Latent sparse attention",
+ * section "How latent sparse attention works": consecutive keys are pooled into
+ * smaller representations, then clustered; each cluster keeps references to the
+ * original keys).
+ *  pool : keys per block, >= 1 and dividing tree->leaf_size.  Block j of a head
+ *         holds keys [j*pool, (j+1)*pool) and is represented by the mean of their
+ *         latent rows (fp32, summed in position order).  The k-means levels of
+ *         lsa_build_tree run on the n_tree/pool blocks (a block's position is j)
+ *         with leaf_size/pool blocks per leaf.
+ * Output layout is that of lsa_build_tree: leaf_index lists, for the blocks of a
+ * leaf in ascending order, their keys j*pool .. j*pool + pool - 1 (so every leaf
+ * still holds leaf_size keys in ascending position), min_pos is a key position,
+ * and every centroid is the mean of the latent rows of the keys under the node.
+ *  trace : optional int32 [levels][iters][n_heads][n_tree/pool], node id of every
+ *          block (indexed by block) after each round.
+ * pool = 1 is lsa_build_tree.  Workspace: lsa_build_workspace_bytes of the same
+ * tree.  Other arguments, limits and errors as lsa_build_tree; LSA_ERR_SHAPE if
+ * pool does not divide leaf_size. */
+int lsa_build_tree_pooled(const lsa_tree_desc *tree, void *tree_mem, const void *K, int64_t n_cap,
+                          int32_t d, int32_t dtype, const void *W, int32_t pool, int32_t iters,
+                          uint64_t seed, void *workspace, size_t workspace_bytes, int32_t *trace,
+                          int32_t *status, void *stream);
+
 /* Hierarchical search (kongchang.com, "How LSA Sidesteps ..."; bdtechtalks.com,
  * "How latent sparse attention works": fixed budget per level, a fixed number
  * of original keys from the chosen clusters).

@@ -99,6 +99,10 @@ def test_calls_validate_before_launch(lsa):
     rc = L.lsa_select(ctypes.byref(d2), None, None, 4, 3, 64, 0, None, ctypes.cast(bm, ctypes.c_void_p),
                       None, None, None, None, None, None, None)
     assert rc == lsa.LSA_ERR_SHAPE
+    for pool in (0, 3, 32):   # pool must be >= 1 and divide leaf_size (16)
+        rc = L.lsa_build_tree_pooled(ctypes.byref(d), None, None, 4096, 64, 1, None, pool, 1, 0, None, 0, None,
+                                     None, None)
+        assert rc == lsa.LSA_ERR_SHAPE and b"pool" in L.lsa_last_error()
     bad = lsa.lsa_tree_desc.from_buffer_copy(d)
     bad.off_leaf_index += 256
     n = ctypes.c_size_t()
