@@ -373,6 +373,70 @@ int orc_build_tree_pooled(const double *Z, int64_t n, int32_t r, int32_t p, cons
 }
 
 /* ------------------------------------------------------------------------- */
+/* Tree update on append ([P1]: the tree can be precomputed and then updated). */
+/* Reading (the pages give no update rule; every node of a level has the same */
+/* fan-out, so only the top level can grow): once U = leaf_size * b_1 * ...  */
+/* * b_{L-1} keys have been appended after the n_old indexed ones, they get a  */
+/* subtree of their own -- the build above run on those U keys alone with     */
+/* branching b_1..b_{L-1} (positions counted from the block's first key, the  */
+/* same seed) -- attached as top-level node b_0.  Its root centroid is the    */
+/* mean of the U keys' latent rows.  Every old node keeps its id and values;  */
+/* the subtree's nodes follow the old ones on each level, and its min_pos and */
+/* leaf_index are shifted by n_old.  One head; levels >= 2.                    */
+/* Outputs use the grown tree's layout (b_0 + 1 top nodes); trace (optional): */
+/* [levels-1, iters, U] of the subtree's build.                                */
+/* ------------------------------------------------------------------------- */
+int orc_tree_append(const double *old_cent, const int32_t *old_min_pos, const int32_t *old_leaf, int64_t n_old,
+                    const double *Znew, int64_t U, int32_t r, const int32_t *branching, int32_t levels,
+                    int32_t leaf_size, int32_t iters, uint64_t seed, double *cent, int32_t *min_pos,
+                    int32_t *leaf_index, int32_t *trace) {
+  if (!old_cent || !old_min_pos || !old_leaf || !Znew || !branching || !cent || !min_pos || !leaf_index)
+    return ORC_ERR_ARG;
+  if (levels < 2 || levels > ORC_MAX_LEVELS) return ORC_ERR_ARG;
+  int64_t sub_nodes_total = 0, level_nodes = 1;
+  for (int32_t l = 1; l < levels; ++l) {
+    level_nodes *= branching[l];
+    sub_nodes_total += level_nodes;
+  }
+  if (level_nodes * leaf_size != U) return ORC_ERR_SHAPE;
+  double *sc = (double *)malloc(sizeof(double) * sub_nodes_total * r);
+  int32_t *sm = (int32_t *)malloc(sizeof(int32_t) * sub_nodes_total);
+  int32_t *sl = (int32_t *)malloc(sizeof(int32_t) * U);
+  if (!sc || !sm || !sl) { free(sc); free(sm); free(sl); return ORC_ERR_ALLOC; }
+  int err = orc_build_tree(Znew, U, r, branching + 1, levels - 1, leaf_size, iters, seed, sc, sm, sl, trace);
+  if (err == ORC_OK) {
+    int64_t old_off = 0, new_off = 0, sub_off = 0;   /* node offsets of the level in each array */
+    int64_t old_nodes = branching[0], sub_nodes = 1;
+    for (int32_t l = 0; l < levels; ++l) {
+      if (l > 0) {
+        old_nodes *= branching[l];
+        sub_nodes *= branching[l];
+      }
+      memcpy(&cent[new_off * r], &old_cent[old_off * r], sizeof(double) * old_nodes * r);
+      memcpy(&min_pos[new_off], &old_min_pos[old_off], sizeof(int32_t) * old_nodes);
+      if (l == 0) {   /* the new top node: mean of every appended key */
+        for (int32_t c = 0; c < r; ++c) {
+          double s = 0.0;
+          for (int64_t i = 0; i < U; ++i) s += Znew[i * r + c];
+          cent[(new_off + old_nodes) * r + c] = s / (double)U;
+        }
+        min_pos[new_off + old_nodes] = (int32_t)n_old;
+      } else {
+        memcpy(&cent[(new_off + old_nodes) * r], &sc[sub_off * r], sizeof(double) * sub_nodes * r);
+        for (int64_t k = 0; k < sub_nodes; ++k) min_pos[new_off + old_nodes + k] = sm[sub_off + k] + (int32_t)n_old;
+        sub_off += sub_nodes;
+      }
+      old_off += old_nodes;
+      new_off += old_nodes + sub_nodes;
+    }
+    memcpy(leaf_index, old_leaf, sizeof(int32_t) * n_old);
+    for (int64_t i = 0; i < U; ++i) leaf_index[n_old + i] = sl[i] + (int32_t)n_old;
+  }
+  free(sc); free(sm); free(sl);
+  return err;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Hierarchical search ([P1]: the query starts at the root, scores a few      */
 /* candidate clusters per level and descends into a few branches; [P4]:       */
 /* fixed search budget per level; a fixed number of original keys retrieved  */

@@ -16,6 +16,9 @@ Parity status of each function (what pins it, in ``tests/test_oracle_pins.py``):
                             an independent deferred-acceptance implementation
   build_tree                centroid == mean of members, parent == mean of
                             children, exact leaf sizes, permutation, init rule
+  tree_append               old nodes unchanged; centroids == means of the keys
+                            listed under each node (new top node included); the
+                            full-beam walk == brute-force flat top-B
   pool_keys,                pool 1 == build_tree; centroids == means of the listed
   build_tree_pooled         keys' latents; leaves are whole aligned blocks; block
                             tree == build_tree on latents pooled by numpy
@@ -102,6 +105,7 @@ def _declare(lib):
         "orc_means": (ctypes.c_int, [P, i64, i32, P, i32, P]),
         "orc_build_tree": (ctypes.c_int, [P, i64, i32, P, i32, i32, i32, u64, P, P, P, P]),
         "orc_pool_keys": (ctypes.c_int, [P, i64, i32, i32, P]),
+        "orc_tree_append": (ctypes.c_int, [P, P, P, i64, P, i64, i32, P, i32, i32, i32, u64, P, P, P, P]),
         "orc_build_tree_pooled": (ctypes.c_int, [P, i64, i32, i32, P, i32, i32, i32, u64, P, P, P, P]),
         "orc_select": (ctypes.c_int, [P, i64, i32, P, i32, i32, P, P, P, P, P, P, P, P]),
         "orc_attn_fwd": (ctypes.c_int, [P, i64, i32, i32, P, P, i64, P, i32, P, i32, i64, i64,
@@ -281,6 +285,27 @@ def build_tree_pooled(Z, p: int, branching, leaf_size: int, iters: int, seed: in
     _check(load().orc_build_tree_pooled(_p(Z), n, r, p, _p(br), L, leaf_size, iters, seed,
                                         _p(cent), _p(mpos), _p(leaf), _p(tr)), "orc_build_tree_pooled")
     return Tree(br, leaf_size, r, cent, mpos, leaf, tr)
+
+
+def tree_append(tree: Tree, Znew, iters: int, seed: int, trace: bool = False) -> Tree:
+    """Attach a subtree over the U = leaf * b_1 * ... * b_{L-1} appended keys (latent rows Znew,
+    positions n_old ..) as top node b_0; returns the grown tree (trace: the subtree's build)."""
+    Znew = _f64(Znew)
+    U, r = Znew.shape
+    br = np.ascontiguousarray(tree.branching, np.int32)
+    L = len(br)
+    n_old = int(len(tree.leaf_index))
+    grown = br.copy()
+    grown[0] += 1
+    total_nodes = int(np.sum(np.cumprod(grown.astype(np.int64))))
+    cent = np.empty(total_nodes * r, np.float64)
+    mpos = np.empty(total_nodes, np.int32)
+    leaf = np.empty(n_old + U, np.int32)
+    tr = np.empty((L - 1, iters, U), np.int32) if trace else None
+    _check(load().orc_tree_append(_p(_f64(tree.centroids_flat)), _p(_i32(tree.min_pos_flat)),
+                                  _p(_i32(tree.leaf_index)), n_old, _p(Znew), U, r, _p(br), L, tree.leaf_size,
+                                  iters, seed, _p(cent), _p(mpos), _p(leaf), _p(tr)), "orc_tree_append")
+    return Tree(grown, tree.leaf_size, r, cent, mpos, leaf, tr)
 
 
 def select(qlat, tree: Tree, beam, q_pos=None, trace: bool = False):

@@ -532,4 +532,44 @@ def pin_tree_pooled():
         np.testing.assert_array_equal(tp.min_pos[l], groups.min(axis=1))
 
 
+def pin_tree_append():
+    """Update on append (kongchang.com, "How LSA Sidesteps Per-Key Scoring with Hierarchical
+    Clustering": the tree can be precomputed and updated): two subtrees attached in turn.  Old
+    nodes keep ids and values; every centroid of the grown tree (the new top nodes included) is
+    the mean of the latent rows of the keys listed under it; min_pos is their smallest position;
+    leaves stay ascending; the full-beam walk over the grown tree is brute-force flat top-B."""
+    rng = np.random.default_rng(9)
+    br, leaf, d, r = (4, 4, 2), 8, 16, 8
+    n_old, U = 4 * 4 * 2 * leaf, 4 * 2 * leaf
+    K = _mixture(rng, n_old + 2 * U, d, 12)
+    W = rng.standard_normal((d, r)) / np.sqrt(d)
+    Z = K @ W
+    Zo = orc.project(K, W)
+    tree = orc.build_tree(Zo[:n_old], br, leaf, 3, seed=4)
+    for step in range(2):
+        n = len(tree.leaf_index)
+        grown = orc.tree_append(tree, Zo[n:n + U], 3, seed=4)
+        assert grown.branching == (tree.branching[0] + 1,) + tree.branching[1:]
+        for l in range(len(br)):
+            k = tree.nodes[l]
+            np.testing.assert_array_equal(grown.centroids[l][:k], tree.centroids[l])
+            np.testing.assert_array_equal(grown.min_pos[l][:k], tree.min_pos[l])
+        np.testing.assert_array_equal(grown.leaf_index[:n], tree.leaf_index)
+        li = grown.leaf_index.astype(np.int64)
+        np.testing.assert_array_equal(np.sort(li), np.arange(n + U))
+        assert np.all(np.diff(li.reshape(-1, leaf), axis=1) > 0)
+        for l in range(len(br)):
+            groups = li.reshape(grown.nodes[l], -1)
+            np.testing.assert_allclose(grown.centroids[l], Z[groups].mean(axis=1), rtol=1e-10, atol=1e-12)
+            np.testing.assert_array_equal(grown.min_pos[l], groups.min(axis=1))
+        tree = grown
+    qlat = rng.standard_normal((12, d)) @ W
+    full = [tree.nodes[l] for l in range(len(tree.nodes) - 1)]
+    idx, _, _ = orc.select(qlat, tree, full + [5])
+    np.testing.assert_array_equal(idx, _flat_topB(qlat, tree, 5))
+    q_pos = rng.integers(0, n_old + 2 * U, 12)
+    idx, _, _ = orc.select(qlat, tree, full + [5], q_pos=q_pos)
+    np.testing.assert_array_equal(idx, _flat_topB(qlat, tree, 5, q_pos))
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

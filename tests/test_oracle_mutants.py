@@ -23,7 +23,7 @@ ORDER = [
     P.pin_select_beam_walk, P.pin_select_full_beam_equals_flat,
     P.pin_attention_equals_sdpa, P.pin_attention_special_cases,
     P.pin_backward_autograd, P.pin_backward_finite_differences,
-    P.pin_attention_sink_window, P.pin_backward_sink_window_autograd, P.pin_tree_pooled,
+    P.pin_attention_sink_window, P.pin_backward_sink_window_autograd, P.pin_tree_pooled, P.pin_tree_append,
 ]
 assert sorted(f.__name__ for f in ORDER) == sorted(f.__name__ for f in P.ALL_PINS)
 
@@ -73,6 +73,14 @@ MUTANTS = [
     ("pooled keys not expanded", "leaf_index[s * p + i] = blocks[s] * p + i;", "leaf_index[s * p + i] = blocks[s] + i;"),
     ("pooled min_pos left in blocks", "for (int64_t k = 0; k < nodes; ++k) min_pos[k] *= p;",
      "for (int64_t k = 0; k < nodes; ++k) min_pos[k] *= 1;"),
+    ("appended root not averaged", "cent[(new_off + old_nodes) * r + c] = s / (double)U;",
+     "cent[(new_off + old_nodes) * r + c] = s / (double)(U - 1);"),
+    ("appended min_pos not shifted", "min_pos[new_off + old_nodes + k] = sm[sub_off + k] + (int32_t)n_old;",
+     "min_pos[new_off + old_nodes + k] = sm[sub_off + k];"),
+    ("appended keys not shifted", "leaf_index[n_old + i] = sl[i] + (int32_t)n_old;", "leaf_index[n_old + i] = sl[i];"),
+    ("subtree centroids copied from the old nodes",
+     "memcpy(&cent[(new_off + old_nodes) * r], &sc[sub_off * r], sizeof(double) * sub_nodes * r);",
+     "memcpy(&cent[(new_off + old_nodes) * r], &cent[new_off * r], sizeof(double) * sub_nodes * r);"),
 ]
 
 
