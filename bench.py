@@ -394,6 +394,53 @@ def run_train(args, dev, rank, world, reduce_max, steps=3, warmup=2):
     return out
 
 
+def run_append(dev, seed):
+    """Update of the index on append (lsa_tree_append) at the decode_128k geometry: once a
+    top-level subtree's worth of keys (leaf * b_1 * b_2 = 8192) has been appended after the
+    131,072 indexed ones, a subtree is built over those keys alone and attached as one more top
+    node, instead of rebuilding the whole index.  CUDA events, median of 3, beside the build of
+    the 131,072-key index the decode started from; then one decode step's select over the grown
+    index."""
+    from hierarchical_latent_key_b200 import lsa
+    base = configs.get("decode_128k")
+    U = base.leaf * int(np.prod(base.branching[1:]))
+    cfg = base.scaled(T=U)
+    c = cfg.case(dev, seed)
+    K, W = c.K, c.W
+    stream = torch.cuda.current_stream(dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def timed(fn):
+        times, out = [], None
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            out = fn()
+            b.record(stream)
+            torch.cuda.synchronize()
+            times.append(a.elapsed_time(b))
+        return out, statistics.median(times)
+
+    desc = lsa.lsa_tree_describe(cfg.Hkv, cfg.r, cfg.branching, cfg.leaf)
+    bws = torch.empty(lsa.lsa_build_workspace_bytes(desc, cfg.d), dtype=torch.uint8, device=dev)
+    aws = torch.empty(lsa.lsa_tree_append_workspace_bytes(desc, cfg.d), dtype=torch.uint8, device=dev)
+    tree, build_ms = timed(lambda: lsa.build_tree(K, W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed, workspace=bws,
+                                                  status=status, check=False))
+    grown, append_ms = timed(lambda: lsa.tree_append(tree, K, W, cfg.iters, cfg.seed, workspace=aws, status=status,
+                                                     check=False))
+    q_pos = torch.full((1,), cfg.n + U - 1, dtype=torch.int32, device=dev)
+    (_, sel_ms) = timed(lambda: lsa.select(grown, c.Q[U - 1:U], W, cfg.beam, q_pos, status=status, check=False))
+    code = lsa.lsa_status_check(status)
+    if code != 0:
+        raise RuntimeError(f"kernel status {code}: {lsa.lsa_strerror(code)}")
+    return {"append_ms": append_ms, "build_ms": build_ms, "unit": "ms",
+            "keys_appended": U, "top_nodes": [int(tree.desc.nodes[0]), int(grown.desc.nodes[0])],
+            "select_after_ms": sel_ms,
+            "config": f"decode_128k geometry: tree {'/'.join(map(str, cfg.branching))} leaf {cfg.leaf} over "
+                      f"{cfg.n:,} keys x {cfg.Hkv} KV heads; {U:,} appended keys per head get their own subtree "
+                      f"({cfg.iters} k-means rounds per level); build_ms is the index of the {cfg.n:,} keys"}
+
+
 def run_decode(args, dev, rank, world, reduce_max):
     cfg = configs.get("decode_10m")
     steps, warmup = cfg.T, args.warmup
@@ -743,9 +790,15 @@ def run_cuda(args, rank, world, local_rank):
         pooled = time_pooled(w, args.steps, args.warmup, flush, stream)
     except Exception as e:  # noqa: BLE001
         pooled = {"error": f"{type(e).__name__}: {e}"}
-    decode = train = None
+    decode = train = append = None
     del w
     torch.cuda.empty_cache()
+    if not args.small:
+        try:
+            append = run_append(dev, rank_seed(5, rank))
+        except Exception as e:  # noqa: BLE001
+            append = {"error": f"{type(e).__name__}: {e}"}
+        torch.cuda.empty_cache()
     # secondary workloads: a failure is reported in the line instead of losing the headline
     if not args.no_decode and not args.small:
         try:
@@ -788,6 +841,7 @@ def run_cuda(args, rank, world, local_rank):
             "prefill_1m_sink_window": sink_window,
             "prefill_1m_flat": flat,
             "prefill_1m_pooled": pooled,
+            "tree_append_128k": append,
             "decode_10m": decode,
             "train_128k": train,
         }

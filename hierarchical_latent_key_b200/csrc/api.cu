@@ -139,8 +139,9 @@ int lsa_tree_describe(int32_t n_heads, int32_t r, const int32_t* branching, int3
   t.leaf_size = leaf_size;
   int64_t nodes = 1;
   for (int l = 0; l < levels; ++l) {
-    if (branching[l] < 2 || branching[l] > LSA_MAX_BRANCHING)
-      return fail(LSA_ERR_SHAPE, "branching[%d] must be in [2, 16] (got %d)", l, branching[l]);
+    const int bmax = l == 0 ? LSA_MAX_TOP_BRANCHING : LSA_MAX_BRANCHING;
+    if (branching[l] < 2 || branching[l] > bmax)
+      return fail(LSA_ERR_SHAPE, "branching[%d] must be in [2, %d] (got %d)", l, bmax, branching[l]);
     nodes *= branching[l];
     if (nodes * leaf_size > (int64_t(1) << 30)) return fail(LSA_ERR_SHAPE, "tree larger than 2^30 keys");
     t.branching[l] = branching[l];
@@ -188,6 +189,8 @@ int lsa_build_tree_pooled(const lsa_tree_desc* tree, void* tree_mem, const void*
   if (rc != LSA_OK) return rc;
   if (pool < 1 || tree->leaf_size % pool != 0)
     return fail(LSA_ERR_SHAPE, "pool (%d) must be >= 1 and divide leaf_size (%d)", pool, tree->leaf_size);
+  if (tree->branching[0] > LSA_MAX_BRANCHING)
+    return fail(LSA_ERR_SHAPE, "the k-means build splits at most 16 ways (branching[0] = %d)", tree->branching[0]);
   if (!tree_mem || !K || !W) return fail(LSA_ERR_INVALID_ARG, "tree_mem, K and W must be non-NULL");
   if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
@@ -207,6 +210,63 @@ int lsa_build_tree_pooled(const lsa_tree_desc* tree, void* tree_mem, const void*
     e = lsa::run_build(P, *tree, tree_mem, K, n_cap, d, dtype, W, pool, trace, status,
                        static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lsa_build_tree_pooled");
+  return ok();
+}
+
+static int append_subtree(const lsa_tree_desc* tree, lsa_tree_desc* sub) {
+  if (tree->levels < 2) return fail(LSA_ERR_SHAPE, "an update on append needs levels >= 2 (got %d)", tree->levels);
+  return lsa_tree_describe(tree->n_heads, tree->r, tree->branching + 1, tree->levels - 1, tree->leaf_size, sub);
+}
+
+int lsa_tree_append_workspace_bytes(const lsa_tree_desc* tree, int32_t d, size_t* bytes) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  lsa_tree_desc sub;
+  if ((rc = append_subtree(tree, &sub)) != LSA_OK) return rc;
+  *bytes = align256(sub.bytes) + lsa::build_workspace_layout(sub, nullptr, nullptr);
+  return ok();
+}
+
+int lsa_tree_append(const lsa_tree_desc* tree, const void* tree_mem, const lsa_tree_desc* grown, void* grown_mem,
+                    const void* K, int64_t n_cap, int32_t d, int32_t dtype, const void* W, int32_t iters,
+                    uint64_t seed, void* workspace, size_t workspace_bytes, int32_t* trace, int32_t* status,
+                    void* stream) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if ((rc = check_desc(grown)) != LSA_OK) return rc;
+  lsa_tree_desc sub;
+  if ((rc = append_subtree(tree, &sub)) != LSA_OK) return rc;
+  bool match = grown->n_heads == tree->n_heads && grown->r == tree->r && grown->levels == tree->levels &&
+               grown->leaf_size == tree->leaf_size && grown->branching[0] == tree->branching[0] + 1;
+  for (int l = 1; l < tree->levels; ++l) match = match && grown->branching[l] == tree->branching[l];
+  if (!match) return fail(LSA_ERR_SHAPE, "grown must describe the same tree with branching[0] + 1");
+  if (!tree_mem || !grown_mem || !K || !W) return fail(LSA_ERR_INVALID_ARG, "tree_mem, grown_mem, K and W must be non-NULL");
+  if (tree_mem == grown_mem) return fail(LSA_ERR_INVALID_ARG, "grown_mem must not be tree_mem");
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  if (n_cap < grown->n_tree)
+    return fail(LSA_ERR_SHAPE, "n_cap (%lld) < grown n_tree (%lld)", (long long)n_cap, (long long)grown->n_tree);
+  if (iters < 1 || iters > 1000) return fail(LSA_ERR_INVALID_ARG, "iters must be in [1, 1000] (got %d)", iters);
+  const size_t sub_bytes = align256(sub.bytes);
+  const size_t need = sub_bytes + lsa::build_workspace_layout(sub, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need)
+    return fail(LSA_ERR_WORKSPACE, "append needs %zu workspace bytes (got %zu)", need, workspace ? workspace_bytes : (size_t)0);
+  char* sub_mem = static_cast<char*>(workspace);
+  lsa::BuildPlan P;
+  lsa::build_workspace_layout(sub, sub_mem + sub_bytes, &P);
+  P.iters = iters;
+  P.seed = seed;
+  P.coop_blocks = lsa::da_grid_blocks();
+  if (P.coop_blocks <= 0) return fail(LSA_ERR_CUDA, "cannot size the cooperative assignment grid");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t esz = dtype == LSA_BF16 ? 2 : 4;
+  const char* Kb = static_cast<const char*>(K) + (size_t)tree->n_tree * d * esz;   // first appended key of head 0
+  cudaError_t e = cudaMemsetAsync(grown_mem, 0, grown->bytes, st);
+  if (e == cudaSuccess) e = lsa::run_build(P, sub, sub_mem, Kb, n_cap, d, dtype, W, 1, trace, status, st);
+  if (e == cudaSuccess) e = lsa::run_tree_attach(*tree, tree_mem, sub, sub_mem, *grown, grown_mem, st);
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_tree_append");
   return ok();
 }
 

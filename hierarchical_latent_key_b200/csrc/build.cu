@@ -873,6 +873,74 @@ cudaError_t run_build(const BuildPlan& P, const lsa_tree_desc& t, void* tree_mem
   }
 }
 
+// ---------------------------------------------------------------------------
+// update on append: one level of the grown tree -- the old nodes, then the
+// subtree's (its min_pos shifted by n_old); on the top level the subtree is one
+// node whose centroid is the mean of the subtree's top centroids (its children,
+// all of the same size) and whose min_pos is n_old
+// ---------------------------------------------------------------------------
+__global__ void k_attach_level(const float* __restrict__ oc, const int32_t* __restrict__ om, int64_t old_nodes,
+                               const float* __restrict__ sc, const int32_t* __restrict__ sm, int64_t sub_nodes,
+                               int root_children, int64_t H, int R, int32_t n_old, float* __restrict__ nc,
+                               int32_t* __restrict__ nm) {
+  const int64_t per = old_nodes + sub_nodes;
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;   // (head * per + node) * R + column
+  if (i >= H * per * R) return;
+  const int64_t h = i / (per * R), node = (i / R) % per;
+  const int c = (int)(i % R);
+  float v;
+  int32_t mp;
+  if (node < old_nodes) {
+    v = oc[(h * old_nodes + node) * R + c];
+    mp = om[h * old_nodes + node];
+  } else if (root_children > 0) {
+    float s = 0.f;
+    for (int j = 0; j < root_children; ++j) s += sc[(h * root_children + j) * R + c];
+    v = s / (float)root_children;
+    mp = n_old;
+  } else {
+    const int64_t k = node - old_nodes;
+    v = sc[(h * sub_nodes + k) * R + c];
+    mp = sm[h * sub_nodes + k] + n_old;
+  }
+  nc[i] = v;
+  if (c == 0) nm[h * per + node] = mp;
+}
+
+__global__ void k_attach_leaves(const int32_t* __restrict__ ol, const int32_t* __restrict__ sl, int64_t H,
+                                int64_t n_old, int64_t U, int32_t* __restrict__ nl) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= H * (n_old + U)) return;
+  const int64_t h = i / (n_old + U), k = i % (n_old + U);
+  nl[i] = k < n_old ? ol[h * n_old + k] : sl[h * U + (k - n_old)] + (int32_t)n_old;
+}
+
+cudaError_t run_tree_attach(const lsa_tree_desc& old_t, const void* old_mem, const lsa_tree_desc& sub,
+                            const void* sub_mem, const lsa_tree_desc& grown, void* grown_mem, cudaStream_t st) {
+  const char* om = static_cast<const char*>(old_mem);
+  const char* sb = static_cast<const char*>(sub_mem);
+  char* gm = static_cast<char*>(grown_mem);
+  const int64_t H = old_t.n_heads;
+  const int R = old_t.r;
+  for (int l = 0; l < old_t.levels; ++l) {
+    const int64_t on = old_t.nodes[l], sn = l == 0 ? 1 : sub.nodes[l - 1];
+    const int sl = l == 0 ? 0 : l - 1;   // subtree level feeding this one (its top for the new root)
+    const int64_t total = H * (on + sn) * R;
+    k_attach_level<<<(unsigned)ceil_div(total, 256), 256, 0, st>>>(
+        reinterpret_cast<const float*>(om + old_t.off_centroids[l]),
+        reinterpret_cast<const int32_t*>(om + old_t.off_min_pos[l]), on,
+        reinterpret_cast<const float*>(sb + sub.off_centroids[sl]),
+        reinterpret_cast<const int32_t*>(sb + sub.off_min_pos[sl]), sn, l == 0 ? (int)sub.nodes[0] : 0, H, R,
+        (int32_t)old_t.n_tree, reinterpret_cast<float*>(gm + grown.off_centroids[l]),
+        reinterpret_cast<int32_t*>(gm + grown.off_min_pos[l]));
+  }
+  const int64_t total = H * grown.n_tree;
+  k_attach_leaves<<<(unsigned)ceil_div(total, 256), 256, 0, st>>>(
+      reinterpret_cast<const int32_t*>(om + old_t.off_leaf_index), reinterpret_cast<const int32_t*>(sb + sub.off_leaf_index),
+      H, old_t.n_tree, sub.n_tree, reinterpret_cast<int32_t*>(gm + grown.off_leaf_index));
+  return cudaGetLastError();
+}
+
 int da_grid_blocks() {
   int dev = 0, sms = 0, per = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;

@@ -60,6 +60,10 @@ cudaError_t run_build(const BuildPlan& P, const lsa_tree_desc& t, void* tree_mem
                       int d, int dtype, const void* W, int32_t pool, int32_t* trace, int32_t* status,
                       cudaStream_t st);
 int da_grid_blocks();
+// The grown tree of an update on append: old levels as prefixes, the subtree's
+// nodes after them, the new top node = mean of the subtree's top centroids.
+cudaError_t run_tree_attach(const lsa_tree_desc& old_t, const void* old_mem, const lsa_tree_desc& sub,
+                            const void* sub_mem, const lsa_tree_desc& grown, void* grown_mem, cudaStream_t st);
 
 struct SelectArgs {
   const void* Q;

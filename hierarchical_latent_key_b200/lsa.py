@@ -57,6 +57,8 @@ def _load():
         "lsa_build_workspace_bytes": (ctypes.c_int, [D, i32, ctypes.POINTER(sz)]),
         "lsa_build_tree": (ctypes.c_int, [D, P, P, i64, i32, i32, P, i32, u64, P, sz, P, P, P]),
         "lsa_build_tree_pooled": (ctypes.c_int, [D, P, P, i64, i32, i32, P, i32, i32, u64, P, sz, P, P, P]),
+        "lsa_tree_append_workspace_bytes": (ctypes.c_int, [D, i32, ctypes.POINTER(ctypes.c_size_t)]),
+        "lsa_tree_append": (ctypes.c_int, [D, P, D, P, P, i64, i32, i32, P, i32, u64, P, sz, P, P, P]),
         "lsa_select": (ctypes.c_int, [D, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]),
         "lsa_tree_attn_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
         "lsa_tree_attn": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, i32, P, i32, f32, P, P, P, sz,
@@ -163,6 +165,22 @@ def lsa_build_tree_pooled(desc, tree_mem, K, W, pool, iters, seed, workspace, tr
                                       _dtype(K), _ptr(W), pool, iters, seed & ((1 << 64) - 1), _ptr(workspace),
                                       workspace.numel(), _ptr(trace), _ptr(status), _stream(stream, K)),
            "lsa_build_tree_pooled")
+
+
+def lsa_tree_append_workspace_bytes(desc, d):
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_tree_append_workspace_bytes(ctypes.byref(desc), d, ctypes.byref(n)),
+           "lsa_tree_append_workspace_bytes")
+    return int(n.value)
+
+
+def lsa_tree_append(desc, tree_mem, grown, grown_mem, K, W, iters, seed, workspace, trace=None, status=None,
+                    stream=None):
+    """Attach a subtree over keys [desc.n_tree, grown.n_tree) of K as top node desc.branching[0]."""
+    _raise(_lib.lsa_tree_append(ctypes.byref(desc), _ptr(tree_mem), ctypes.byref(grown), _ptr(grown_mem), _ptr(K),
+                                K.shape[1], K.shape[2], _dtype(K), _ptr(W), iters, seed & ((1 << 64) - 1),
+                                _ptr(workspace), workspace.numel(), _ptr(trace), _ptr(status), _stream(stream, K)),
+           "lsa_tree_append")
 
 
 def lsa_select(desc, tree_mem, Q, W, beam, q_pos, idx_out, leaves_out=None, qlat_out=None, beam_out=None,
@@ -343,6 +361,28 @@ def build_tree(K, W, branching, leaf_size, iters, seed, trace=False, workspace=N
         check_status(st, "lsa_build_tree")
     tree = Tree(desc, mem)
     return (tree, tr) if trace else tree
+
+
+def tree_append(tree: Tree, K, W, iters, seed, trace=False, workspace=None, status=None, check=True):
+    """The index grown by one top-level node over the next U = leaf * b_1 * ... keys of K
+    (positions tree.n_tree ..); returns the new Tree (and the subtree's build trace)."""
+    d0 = tree.desc
+    Hkv, n_cap, d = K.shape
+    levels = d0.levels
+    br = [d0.branching[l] for l in range(levels)]
+    grown = lsa_tree_describe(Hkv, d0.r, [br[0] + 1] + br[1:], d0.leaf_size)
+    mem = torch.empty(grown.bytes, dtype=torch.uint8, device=K.device)
+    need = lsa_tree_append_workspace_bytes(d0, d)
+    if workspace is None or workspace.numel() < need:
+        workspace = torch.empty(need, dtype=torch.uint8, device=K.device)
+    U = grown.n_tree - d0.n_tree
+    tr = torch.empty(levels - 1, iters, Hkv, U, dtype=torch.int32, device=K.device) if trace else None
+    st = _new_status(K.device) if status is None else status
+    lsa_tree_append(d0, tree.mem, grown, mem, K, W, iters, seed, workspace, tr, st)
+    if check:
+        check_status(st, "lsa_tree_append")
+    t = Tree(grown, mem)
+    return (t, tr) if trace else t
 
 
 def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, leaves=False, status=None, check=True):

@@ -47,7 +47,8 @@ extern "C" {
 
 #define LSA_VERSION 1
 #define LSA_MAX_LEVELS 8
-#define LSA_MAX_BRANCHING 16
+#define LSA_MAX_BRANCHING 16       /* children per node on a level the k-means build splits */
+#define LSA_MAX_TOP_BRANCHING 512  /* top-level nodes a tree can reach through lsa_tree_append */
 #define LSA_MAX_BEAM 32
 
 typedef enum lsa_status {
@@ -97,8 +98,9 @@ const char *lsa_strerror(int status);
 const char *lsa_last_error(void);
 
 /* Host only.  Fills *out for n_heads trees with latent dim r, `levels` levels of
- * fan-out branching[0..levels) (root to leaves, each in [2, 16]) and leaves of
- * leaf_size keys.  Limits: 1 <= levels <= 8, r in {16, 32, 64}, leaf_size in [8, 4096],
+ * fan-out branching[0..levels) (root to leaves; branching[0] in [2, 512], the others
+ * in [2, 16]; lsa_build_tree itself needs branching[0] <= 16 too, wider top levels
+ * come from lsa_tree_append) and leaves of leaf_size keys.  Limits: 1 <= levels <= 8, r in {16, 32, 64}, leaf_size in [8, 4096],
  * n_tree <= 2^30 and n_heads * n_tree < 2^31.
  * Returns LSA_ERR_SHAPE / LSA_ERR_INVALID_ARG on violations. */
 int lsa_tree_describe(int32_t n_heads, int32_t r, const int32_t *branching /* host */,
@@ -154,6 +156,35 @@ int lsa_build_tree_pooled(const lsa_tree_desc *tree, void *tree_mem, const void 
                           int32_t d, int32_t dtype, const void *W, int32_t pool, int32_t iters,
                           uint64_t seed, void *workspace, size_t workspace_bytes, int32_t *trace,
                           int32_t *status, void *stream);
+
+/* Host only.  Device workspace bytes lsa_tree_append needs for keys of width d
+ * (the subtree's buffer and its build workspace).  LSA_ERR_SHAPE if levels < 2. */
+int lsa_tree_append_workspace_bytes(const lsa_tree_desc *tree, int32_t d, size_t *bytes /* host */);
+
+/* Update of an index on append (kongchang.com, "How LSA Sidesteps Per-Key Scoring
+ * with Hierarchical Clustering": the tree can be precomputed and then updated).
+ * Every node of a level has the same fan-out, so only the top level can grow: once
+ * U = leaf_size * branching[1] * ... * branching[levels-1] keys have been appended
+ * after the tree->n_tree indexed ones, they get a subtree of their own, attached as
+ * top-level node branching[0].
+ *  tree, tree_mem   : the current index (read only; levels >= 2).
+ *  grown            : lsa_tree_describe of the same heads, r, levels and leaf_size with
+ *                     branching[0] + 1 (so grown->n_tree = tree->n_tree + U).
+ *  grown_mem        : grown->bytes of device memory (not tree_mem), written completely.
+ *  K, n_cap, d, dtype, W : as lsa_build_tree; keys [tree->n_tree, grown->n_tree) of
+ *                     every head are the appended block (n_cap >= grown->n_tree).
+ * The subtree is lsa_build_tree run on the U appended keys alone with branching
+ * branching[1..levels) (same iters and seed; positions, for the seeded start and the
+ * pair order, counted from the block's first key); its node ids follow the old ones
+ * on every level, its min_pos and leaf_index are shifted by tree->n_tree, and the new
+ * top node's centroid is the mean of its children's (= of the U keys' latent rows).
+ * Every old node keeps its id, centroid, min_pos and keys.
+ *  trace : optional int32 [levels-1][iters][n_heads][U] of the subtree's build.
+ * Errors as lsa_build_tree; LSA_ERR_SHAPE if grown does not match tree. */
+int lsa_tree_append(const lsa_tree_desc *tree, const void *tree_mem, const lsa_tree_desc *grown,
+                    void *grown_mem, const void *K, int64_t n_cap, int32_t d, int32_t dtype,
+                    const void *W, int32_t iters, uint64_t seed, void *workspace,
+                    size_t workspace_bytes, int32_t *trace, int32_t *status, void *stream);
 
 /* Hierarchical search (kongchang.com, "How LSA Sidesteps ..."; bdtechtalks.com,
  * "How latent sparse attention works": fixed budget per level, a fixed number

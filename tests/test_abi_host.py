@@ -44,7 +44,7 @@ def test_version_and_strerror(lsa):
 
 
 @pytest.mark.parametrize("kw,code", [
-    (dict(n_heads=0), 2), (dict(r=48), 2), (dict(branching=(16, 1)), 2), (dict(branching=(17,)), 2),
+    (dict(n_heads=0), 2), (dict(r=48), 2), (dict(branching=(16, 1)), 2), (dict(branching=(513,)), 2), (dict(branching=(16, 17)), 2),
     (dict(leaf_size=4), 2), (dict(branching=(16,) * 9), 2), (dict(branching=(16,) * 7, leaf_size=64), 2), (dict(n_heads=4, branching=(16,) * 6), 2),
 ])
 def test_describe_rejects(lsa, kw, code):
@@ -103,6 +103,34 @@ def test_calls_validate_before_launch(lsa):
         rc = L.lsa_build_tree_pooled(ctypes.byref(d), None, None, 4096, 64, 1, None, pool, 1, 0, None, 0, None,
                                      None, None)
         assert rc == lsa.LSA_ERR_SHAPE and b"pool" in L.lsa_last_error()
+    # the top level may grow to 512 through lsa_tree_append; the k-means build splits <= 16 ways
+    wide = lsa.lsa_tree_describe(1, 16, (17, 16), 16)
+    assert wide.nodes[0] == 17 and wide.n_tree == 17 * 16 * 16
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_tree_describe(1, 16, (513, 2), 16)
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_tree_describe(1, 16, (16, 17), 16)
+    rc = L.lsa_build_tree(ctypes.byref(wide), None, None, 1 << 20, 64, 1, None, 1, 0, None, 0, None, None, None)
+    assert rc == lsa.LSA_ERR_SHAPE and b"16 ways" in L.lsa_last_error()
+    # append: grown must be the same tree with branching[0] + 1, and levels >= 2
+    grown = lsa.lsa_tree_describe(1, 16, (17, 16), 16)
+    other = lsa.lsa_tree_describe(1, 16, (18, 16), 16)
+    base = lsa.lsa_tree_describe(1, 16, (16, 16), 16)
+    P16 = ctypes.c_void_p(16)
+    rc = L.lsa_tree_append(ctypes.byref(base), P16, ctypes.byref(other), P16, P16, 1 << 20, 64, 1, P16, 1, 0, None,
+                           0, None, None, None)
+    assert rc == lsa.LSA_ERR_SHAPE and b"branching[0] + 1" in L.lsa_last_error()
+    flat1 = lsa.lsa_tree_describe(1, 16, (16,), 16)
+    n = ctypes.c_size_t()
+    assert L.lsa_tree_append_workspace_bytes(ctypes.byref(flat1), 64, ctypes.byref(n)) == lsa.LSA_ERR_SHAPE
+    assert L.lsa_tree_append_workspace_bytes(ctypes.byref(base), 64, ctypes.byref(n)) == lsa.LSA_OK
+    P32 = ctypes.c_void_p(32)
+    rc = L.lsa_tree_append(ctypes.byref(base), P16, ctypes.byref(grown), P16, P16, 1 << 20, 64, 1, P16, 1, 0, P16,
+                           n.value, None, None, None)
+    assert rc == lsa.LSA_ERR_INVALID_ARG and b"not be tree_mem" in L.lsa_last_error()
+    rc = L.lsa_tree_append(ctypes.byref(base), P16, ctypes.byref(grown), P32, P16, 1 << 20, 64, 1, P16, 1, 0, P16,
+                           n.value - 1, None, None, None)
+    assert rc == lsa.LSA_ERR_WORKSPACE
     bad = lsa.lsa_tree_desc.from_buffer_copy(d)
     bad.off_leaf_index += 256
     n = ctypes.c_size_t()
