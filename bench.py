@@ -511,6 +511,11 @@ def time_steps(w, steps, warmup, flush, stream):
 
 
 SINK, WINDOW = 16, 512   # sink tokens and recent window of the sink/window measurement
+# DRAM bytes read + written by one lsa_tree_attn call of the prefill_1m step (its seven kernels:
+# leaf and chunk lists, k_tl_pipe, k_tl_combine), from one single-pass ncu capture of this
+# workload (dram__bytes_read.sum + dram__bytes_write.sum); to be taken again whenever one of
+# those kernels changes
+TREE_ATTN_TRAFFIC_BYTES = 7_223_064_320
 POOL = 4                 # keys per block of the pooled index
 
 
@@ -831,7 +836,8 @@ def run_cuda(args, rank, world, local_rank):
                              "build_once": build_ms},
             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "roofline": {"kernel": "lsa_tree_attn (leaf lists + k_tl_pipe + k_tl_combine)", "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                         "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                         "traffic": TREE_ATTN_TRAFFIC_BYTES if not args.small else None,
                          "peak_source": peaks["source"],
                          "algorithmic_bytes": alg_bytes, "distinct_kv_rows": rows,
                          "tensor_tflops": att_flops / att_s / 1e12},
