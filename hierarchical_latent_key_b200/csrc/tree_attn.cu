@@ -607,18 +607,31 @@ __global__ void k_tl_finish(TreeAttnArgs a) {
 
 // One warp per (query, head) row: O = sum_k w_k o_k / sum_k w_k with
 // w_k = 2^(m_k - M) l_k over the row's leaves, in rank order.
+// 16 bytes through the non-coherent path; volatile, so that every partial of a row
+// is requested before the first is used (the compiler would otherwise sink each
+// load to its use and keep only a few in flight)
+__device__ __forceinline__ uint4 ld_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+  return v;
+}
+
 __global__ void k_tl_combine(TreeAttnArgs a) {
   const int64_t row = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;   // t * Hq + head
   const int lane = threadIdx.x & 31;
   if (row >= a.T * a.Hq) return;
   const int64_t t = row / a.Hq, head = row % a.Hq, g = head / a.G;
-  // all of the row's partials are requested at once, together with the statistics
+  // half-warp h reads the partials of ranks h, h + 2, ...; lane (mod 16) owns dims
+  // [8 (lane mod 16), +8); all of them are requested at once, with the statistics
   // (ranks without a partial are read too, the workspace is readable, and skipped)
-  const __nv_bfloat16* pr = a.part + row * a.B * kDim + lane * 4;
-  uint2 raw[LSA_MAX_BEAM];
+  const int half = lane >> 4, sl = lane & 15;
+  const __nv_bfloat16* pr = a.part + row * a.B * kDim + sl * 8;
+  uint4 raw[LSA_MAX_BEAM / 2];
 #pragma unroll
-  for (int k = 0; k < LSA_MAX_BEAM; ++k)
-    raw[k] = k < a.B ? *reinterpret_cast<const uint2*>(pr + (int64_t)k * kDim) : make_uint2(0u, 0u);
+  for (int i = 0; i < LSA_MAX_BEAM / 2; ++i) {
+    const int k = 2 * i + half;
+    raw[i] = k < a.B ? ld_nc_v4(pr + (int64_t)k * kDim) : make_uint4(0u, 0u, 0u, 0u);
+  }
   bool valid = false;
   float mk = -INFINITY, lk = 0.f;
   if (lane < a.B && a.leaves[(g * a.T + t) * a.B + lane] >= 0) {
@@ -635,37 +648,53 @@ __global__ void k_tl_combine(TreeAttnArgs a) {
   M = fmaxf(M, md);
   const unsigned vmask = __ballot_sync(0xffffffffu, valid);
   const float wk = valid ? exp2f(mk - M) * lk : 0.f;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  float L = 0.f;
+  // L: butterfly sum (each step adds the same two values on both lanes: every lane
+  // ends with the same bits)
+  float L = wk;
 #pragma unroll
-  for (int k = 0; k < LSA_MAX_BEAM; ++k) {   // rank order
-    if (!((vmask >> k) & 1u)) continue;
-    const float w = __shfl_sync(0xffffffffu, wk, k);
-    const float2 lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[k].x));
-    const float2 hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&raw[k].y));
-    acc[0] = fmaf(w, lo.x, acc[0]);
-    acc[1] = fmaf(w, lo.y, acc[1]);
-    acc[2] = fmaf(w, hi.x, acc[2]);
-    acc[3] = fmaf(w, hi.y, acc[3]);
-    L += w;
+  for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+  for (int i = 0; i < LSA_MAX_BEAM / 2; ++i) {   // this half's ranks in order
+    const int k = 2 * i + half;
+    const float w = __shfl_sync(0xffffffffu, wk, k & 31);
+    if ((vmask >> k) & 1u) {
+      const uint32_t wd[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&wd[q]));
+        acc[2 * q] = fmaf(w, f.x, acc[2 * q]);
+        acc[2 * q + 1] = fmaf(w, f.y, acc[2 * q + 1]);
+      }
+    }
   }
+  // even ranks + odd ranks (the same sum on both halves)
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
   if (md != -INFINITY) {   // after the leaves, in a fixed order
     const float w = exp2f(md - M);
-    float v[4];
-    load4(a.Od + row * kDim + lane * 4, v);
-    acc[0] = fmaf(w, v[0], acc[0]);
-    acc[1] = fmaf(w, v[1], acc[1]);
-    acc[2] = fmaf(w, v[2], acc[2]);
-    acc[3] = fmaf(w, v[3], acc[3]);
+    float v0[4], v1[4];
+    load4(a.Od + row * kDim + sl * 8, v0);
+    load4(a.Od + row * kDim + sl * 8 + 4, v1);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      acc[e] = fmaf(w, v0[e], acc[e]);
+      acc[e + 4] = fmaf(w, v1[e], acc[e + 4]);
+    }
     L += w;
   }
   const float inv = L > 0.f ? 1.f / L : 0.f;
-  __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0] * inv, acc[1] * inv);
-  __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2] * inv, acc[3] * inv);
-  uint2 w2;
-  w2.x = *reinterpret_cast<uint32_t*>(&lo);
-  w2.y = *reinterpret_cast<uint32_t*>(&hi);
-  *reinterpret_cast<uint2*>(a.O + row * kDim + lane * 4) = w2;
+  if (half == 0) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * q] * inv, acc[2 * q + 1] * inv);
+      w4[q] = *reinterpret_cast<uint32_t*>(&b2);
+    }
+    *reinterpret_cast<uint4*>(a.O + row * kDim + sl * 8) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
   if (lane == 0) a.LSE[row] = L > 0.f ? (M + log2f(L)) * 0.69314718055994530942f : -INFINITY;
 }
 
