@@ -515,7 +515,7 @@ SINK, WINDOW = 16, 512   # sink tokens and recent window of the sink/window meas
 # leaf and chunk lists, k_tl_pipe, k_tl_combine), from one single-pass ncu capture of this
 # workload (dram__bytes_read.sum + dram__bytes_write.sum); to be taken again whenever one of
 # those kernels changes
-TREE_ATTN_TRAFFIC_BYTES = None
+TREE_ATTN_TRAFFIC_BYTES = 7_225_572_352
 POOL = 4                 # keys per block of the pooled index
 
 
