@@ -127,3 +127,45 @@ def test_append_top_level_past_32(lsa):
     idx_big = lsa.select(tree, g["Q"][big], g["W"], cfg.beam, qp)
     torch.cuda.synchronize()
     assert torch.equal(idx_big[:, cfg.T - 40:cfg.T], idx_small)
+
+
+def test_decode_loop_with_updates(lsa):
+    """Decode over a 4/8/4 index: each step's key joins the dense tail before the step attends;
+    when the tail holds U keys they are attached as a subtree (lsa_tree_append) and the tail
+    restarts after them.  Sampled steps around both updates: selection stage-wise against the
+    oracle on the grown index, attention over (selected keys + tail) against the oracle."""
+    U = 8 * 4 * 64
+    cfg = configs.get("decode_128k").scaled(n=4 * U, branching=(4, 8, 4), beam=(4, 16, 16), Hkv=2, Hq=8,
+                                            T=2 * U + 40, comps=128)
+    case = cfg.case("cpu", seed=47)
+    g = {k: getattr(case, k).to(DEV) for k in ("Q", "K", "V", "W")}
+    tree = lsa.build_tree(g["K"], g["W"], cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    tail_begin = cfg.n
+    sample = {0, 1, U - 2, U - 1, U, U + 1, 2 * U - 1, 2 * U, 2 * U + 39}
+    updates = 0
+    for s in range(cfg.T):
+        p = cfg.n + s                          # the step's key, appended before it attends
+        if p - tail_begin + 1 == U:            # the tail holds a full block: grow the index
+            assert int(tree.desc.n_tree) == tail_begin
+            tree = lsa.tree_append(tree, g["K"], g["W"], cfg.iters, cfg.seed)
+            tail_begin = p + 1
+            updates += 1
+        if s not in sample:
+            continue
+        qp = torch.tensor([p], dtype=torch.int32, device=DEV)
+        idx, qlat, beams = lsa.select(tree, g["Q"][s:s + 1], g["W"], cfg.beam, qp, qlat=True, beams=True)
+        tail = (tail_begin, p + 1)
+        O, LSE = lsa.sparse_attn(g["Q"][s:s + 1], g["K"], g["V"], idx, qp, True, tail)
+        torch.cuda.synchronize()
+        for h in range(cfg.Hkv):
+            _, th = _levels(tree, h)
+            Qg = case.Q[s:s + 1, h * cfg.G:(h + 1) * cfg.G]
+            oq = orc.query_latent(Qg, case.W[h])
+            parity.check_select_stagewise(oq, th, tree_branching(tree), cfg.leaf, cfg.beam, np.array([p]),
+                                          beams[:, h].cpu().numpy(), idx[h].cpu().numpy())
+            Oo, Lo = orc.attn_fwd(Qg, case.K[h], case.V[h], idx[h].cpu(), q_pos=np.array([p], np.int32),
+                                  causal=True, tail=tail)
+            err = np.abs(O[:, h * cfg.G:(h + 1) * cfg.G].float().cpu().numpy() - Oo)
+            assert err.max() <= 2e-2 and err.mean() <= 2e-3, (s, h, err.max(), err.mean())
+            assert np.abs(LSE[:, h * cfg.G:(h + 1) * cfg.G].cpu().numpy() - Lo).max() <= 1e-3
+    assert updates == 2 and int(tree.desc.nodes[0]) == 6
