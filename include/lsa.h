@@ -323,9 +323,10 @@ int lsa_tree_attn_sw_workspace_bytes(const lsa_tree_desc *tree, int32_t T, int32
  * [0, n_sink) and [q_pos[t] - window + 1, q_pos[t]], each key once.  On the leaf-by-
  * leaf path a leaf key inside the sink or the window is left out (a leaf lists its
  * keys in position order, so the kept keys are one index range) and the sink and
- * window keys are attended as one more partial through the key-list attention,
- * merged in the combine; other shapes run the key-list attention on the expanded
- * and extended lists.  n_sink, window in [0, LSA_MAX_SINK_WINDOW]. */
+ * window keys are attended as one more partial, tile by tile on the tensor cores
+ * (128 (query, head) rows of a KV group against the 64-position key blocks that any
+ * of them needs), merged in the combine; other shapes run the key-list attention on
+ * the expanded and extended lists.  n_sink, window in [0, LSA_MAX_SINK_WINDOW]. */
 int lsa_tree_attn_sw(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, int32_t T,
                      int32_t Hq, const void *K, const void *V, int64_t n_cap, int32_t d,
                      int32_t dtype, const int32_t *leaves, int32_t n_leaves, const int32_t *q_pos,
