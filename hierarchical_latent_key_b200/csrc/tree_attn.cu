@@ -717,7 +717,12 @@ struct BandArgs {
   int32_t Hq, H, G, n_sink, window;
   float scale_log2;
 };
-constexpr size_t kBandSmem = 1024 + kTL * 256 + 3 * kLeafKeys * 256;   // Q 32 KB; K, V, P 16 KB each
+constexpr size_t kBandSmem = 1024 + kTL * 256 + 4 * kLeafKeys * 256;   // Q 32 KB; two {K, V} buffers
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+// every committed group but the most recent one has landed (this thread's copies)
+__device__ __forceinline__ void cp_async_wait_prev() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_drain() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __global__ void __launch_bounds__(kTL) k_tl_band(BandArgs a) {
   extern __shared__ char smem_raw[];
@@ -725,14 +730,13 @@ __global__ void __launch_bounds__(kTL) k_tl_band(BandArgs a) {
   __shared__ uint32_t s_taddr;
   __shared__ int32_t s_red[kTL / 32];
   char* base = align1024(smem_raw);
-  char* gK = base + kTL * 256;
-  char* gV = gK + kLeafKeys * 256;
-  char* gP = gV + kLeafKeys * 256;
+  // two buffers of {K, V} (16 KB each): a block's copies land in one while the
+  // previous block is computed from the other; P overlays the K tile of its own
+  // block once S = Q.K^T has completed
+  auto gK = [&](int buf) { return base + kTL * 256 + buf * 2 * kLeafKeys * 256; };
+  auto gV = [&](int buf) { return gK(buf) + kLeafKeys * 256; };
   LeafSmem s;
   s.sA = smem_u32(base);
-  s.sK = smem_u32(gK);
-  s.sV = smem_u32(gV);
-  s.sP = smem_u32(gP);
   s.mbar = smem_u32(&s_mbar);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t g = blockIdx.y;
@@ -767,31 +771,31 @@ __global__ void __launch_bounds__(kTL) k_tl_band(BandArgs a) {
   // positions past every row's query are never attended, and the cache rows there
   // may hold anything: their V rows are zeros (0 x NaN would still be NaN)
   const int64_t qmax = -(int64_t)cta_min(valid ? -(int)q : INT_MAX);
-  if (valid) {
+  if (valid) {   // lands with the first block's group
     const __nv_bfloat16* qr = a.Q + (t * a.Hq + g * a.G + hh) * kDim;
 #pragma unroll
     for (int c = 0; c < 16; ++c) cp_async16(s.sA + sw128_off(threadIdx.x, c, kTL * 128), qr + c * 8);
   }
-  auto load_block = [&](int b, bool with_v) {
+  // copies of block b into buffer buf (issued, not waited for)
+  auto load_block = [&](int b, int buf, bool with_v) {
     const int r = threadIdx.x >> 1, c0 = (threadIdx.x & 1) * 8;
     const int64_t j = (int64_t)b * kLeafKeys + r;
+    const uint32_t sK = smem_u32(gK(buf)), sV = smem_u32(gV(buf));
     if (j <= qmax && j < a.n_cap) {
       const __nv_bfloat16* kr = a.K + (g * a.n_cap + j) * kDim;
       const __nv_bfloat16* vr = a.V + (g * a.n_cap + j) * kDim;
 #pragma unroll
       for (int c = c0; c < c0 + 8; ++c) {
-        cp_async16(s.sK + sw128_off(r, c, kLeafKeys * 128), kr + c * 8);
-        if (with_v) cp_async16(s.sV + sw128_off(r, c, kLeafKeys * 128), vr + c * 8);
+        cp_async16(sK + sw128_off(r, c, kLeafKeys * 128), kr + c * 8);
+        if (with_v) cp_async16(sV + sw128_off(r, c, kLeafKeys * 128), vr + c * 8);
       }
     } else {
 #pragma unroll
       for (int c = c0; c < c0 + 8; ++c) {
-        *reinterpret_cast<uint4*>(gK + sw128_off(r, c, kLeafKeys * 128)) = make_uint4(0u, 0u, 0u, 0u);
-        if (with_v) *reinterpret_cast<uint4*>(gV + sw128_off(r, c, kLeafKeys * 128)) = make_uint4(0u, 0u, 0u, 0u);
+        *reinterpret_cast<uint4*>(gK(buf) + sw128_off(r, c, kLeafKeys * 128)) = make_uint4(0u, 0u, 0u, 0u);
+        if (with_v) *reinterpret_cast<uint4*>(gV(buf) + sw128_off(r, c, kLeafKeys * 128)) = make_uint4(0u, 0u, 0u, 0u);
       }
     }
-    cp_async_wait_all();
-    fence_async_smem();
   };
   // this row's 64 scores of block b (base-2 scaled; -inf outside its dense keys)
   auto scores = [&](int b, uint32_t tmem, float (&sc)[64]) {
@@ -815,19 +819,22 @@ __global__ void __launch_bounds__(kTL) k_tl_band(BandArgs a) {
   const uint32_t tmem = s_taddr;
   uint32_t phase = 0;
   bool ok = true;
-  // product on the tensor cores, then every thread waits for it
-  auto run_mma = [&](bool pv, bool accumulate) {
+  // product on the tensor cores from buffer buf, then every thread waits for it
+  auto run_mma = [&](int buf, bool pv, bool accumulate) {
     __syncthreads();
     if (threadIdx.x == 0) {
       tc_fence_after();
       if (!pv) {
-        issue_qk(s, tmem, 0);
+        LeafSmem cs = s;
+        cs.sK = smem_u32(gK(buf));
+        issue_qk(cs, tmem, 0);
       } else {
         constexpr uint32_t idesc = idesc_bf16(128, 128, false, true);
+        const uint32_t sP = smem_u32(gK(buf)), sV = smem_u32(gV(buf));
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          tc_mma(tmem + 64, sdesc_sw128(s.sP + kk * 32, 16, 1024),
-                 sdesc_sw128(s.sV + kk * 2048, kLeafKeys * 128, 1024), idesc, (accumulate || kk > 0) ? 1u : 0u);
+          tc_mma(tmem + 64, sdesc_sw128(sP + kk * 32, 16, 1024), sdesc_sw128(sV + kk * 2048, kLeafKeys * 128, 1024),
+                 idesc, (accumulate || kk > 0) ? 1u : 0u);
       }
       tc_commit(s.mbar);
     }
@@ -837,51 +844,77 @@ __global__ void __launch_bounds__(kTL) k_tl_band(BandArgs a) {
   };
   // sweep 1: max and sum of every row
   float m = -INFINITY, l = 0.f;
-  for (int b = cta_min(next_block(0)); b != INT_MAX && ok; b = cta_min(next_block(b + 1))) {
-    load_block(b, false);
-    run_mma(false, false);
-    if (!ok) break;
-    float sc[64];
-    scores(b, tmem, sc);
-    float bm = -INFINITY;
+  {
+    int b = cta_min(next_block(0)), cur = 0;
+    if (b != INT_MAX) load_block(b, cur, false);
+    cp_async_commit();
+    while (b != INT_MAX && ok) {
+      const int nb = cta_min(next_block(b + 1));   // also: every thread is done with the other buffer
+      if (nb != INT_MAX) load_block(nb, cur ^ 1, false);
+      cp_async_commit();
+      cp_async_wait_prev();
+      fence_async_smem();
+      run_mma(cur, false, false);
+      if (!ok) break;
+      float sc[64];
+      scores(b, tmem, sc);
+      float bm = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 64; ++i) bm = fmaxf(bm, sc[i]);
-    const float mn = fmaxf(m, bm);
-    if (mn != -INFINITY) {
-      float sum = 0.f;
+      for (int i = 0; i < 64; ++i) bm = fmaxf(bm, sc[i]);
+      const float mn = fmaxf(m, bm);
+      if (mn != -INFINITY) {
+        float sum = 0.f;
 #pragma unroll
-      for (int i = 0; i < 64; ++i) sum += exp2f(sc[i] - mn);
-      l = (m == -INFINITY ? 0.f : l * exp2f(m - mn)) + sum;
-      m = mn;
+        for (int i = 0; i < 64; ++i) sum += exp2f(sc[i] - mn);
+        l = (m == -INFINITY ? 0.f : l * exp2f(m - mn)) + sum;
+        m = mn;
+      }
+      tc_fence_before();
+      b = nb;
+      cur ^= 1;
     }
-    tc_fence_before();
+    cp_async_drain();
   }
   const float lse2 = l > 0.f ? m + log2f(l) : INFINITY;   // +inf: P = 0
   // sweep 2: O = sum over blocks of 2^(s - lse) . V
   bool any = false;
-  for (int b = cta_min(next_block(0)); b != INT_MAX && ok; b = cta_min(next_block(b + 1))) {
-    load_block(b, true);
-    run_mma(false, false);
-    if (!ok) break;
-    float sc[64];
-    scores(b, tmem, sc);
-    const int r = threadIdx.x;
+  if (ok) {
+    __syncthreads();   // sweep 1's buffers are free
+    int b = cta_min(next_block(0)), cur = 0;
+    if (b != INT_MAX) load_block(b, cur, true);
+    cp_async_commit();
+    while (b != INT_MAX && ok) {
+      const int nb = cta_min(next_block(b + 1));
+      if (nb != INT_MAX) load_block(nb, cur ^ 1, true);
+      cp_async_commit();
+      cp_async_wait_prev();
+      fence_async_smem();
+      run_mma(cur, false, false);
+      if (!ok) break;
+      float sc[64];
+      scores(b, tmem, sc);
+      const int r = threadIdx.x;
+      char* gP = gK(cur);   // S = Q.K^T has completed: P takes the K tile's place
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      uint32_t w[4];
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(exp2f(sc[c * 8 + 2 * i] - lse2), exp2f(sc[c * 8 + 2 * i + 1] - lse2));
-        w[i] = *reinterpret_cast<uint32_t*>(&b2);
+        for (int i = 0; i < 4; ++i) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(exp2f(sc[c * 8 + 2 * i] - lse2), exp2f(sc[c * 8 + 2 * i + 1] - lse2));
+          w[i] = *reinterpret_cast<uint32_t*>(&b2);
+        }
+        *reinterpret_cast<uint4*>(gP + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
       }
-      *reinterpret_cast<uint4*>(gP + (r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4)) =
-          make_uint4(w[0], w[1], w[2], w[3]);
+      fence_async_smem();
+      tc_fence_before();
+      run_mma(cur, true, any);
+      any = true;
+      tc_fence_before();
+      b = nb;
+      cur ^= 1;
     }
-    fence_async_smem();
-    tc_fence_before();
-    run_mma(true, any);
-    any = true;
-    tc_fence_before();
+    cp_async_drain();
   }
   if (!ok) set_status(a.status, LSA_ERR_TIMEOUT);
   if (ok) {   // CTA-uniform: the TMEM loads are warp-collective, the stores per row
