@@ -826,12 +826,8 @@ def run_cuda(args, rank, world, local_rank):
             "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * t_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"{cfg.name}: {cfg.T} query tokens over {cfg.n:,} cached keys, "
-                                   f"{cfg.Hq}/{cfg.Hkv} heads, d={cfg.d}, r={cfg.r}, tree "
-                                   f"{'/'.join(map(str, cfg.branching))} leaf {cfg.leaf}, beam "
-                                   f"{'/'.join(map(str, cfg.beam))} ({cfg.K_sel} keys/query), causal",
-                       "global_batch": cfg.T * world, "seq_len": cfg.n, "parallelism": f"dp{world}",
-                       "l2": "flushed between timed steps (512 MiB write outside the events)"},
+            "config": dict(prefill_config(cfg, world),
+                           l2="flushed between timed steps (512 MiB write outside the events)"),
             "breakdown_ms": {"select": statistics.mean(sel), "attention": statistics.mean(att),
                              "build_once": build_ms},
             "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -857,6 +853,15 @@ def run_cuda(args, rank, world, local_rank):
 # ---------------------------------------------------------------------------
 # reference arm: the CPU oracle on this host
 # ---------------------------------------------------------------------------
+
+def prefill_config(cfg, world):
+    """The `config` object of the prefill line (both arms)."""
+    return {"workload": f"{cfg.name}: {cfg.T} query tokens over {cfg.n:,} cached keys, "
+                        f"{cfg.Hq}/{cfg.Hkv} heads, d={cfg.d}, r={cfg.r}, tree "
+                        f"{'/'.join(map(str, cfg.branching))} leaf {cfg.leaf}, beam "
+                        f"{'/'.join(map(str, cfg.beam))} ({cfg.K_sel} keys/query), causal",
+            "global_batch": cfg.T * world, "seq_len": cfg.n, "parallelism": f"dp{world}"}
+
 
 def run_reference(args):
     from oracle import oracle as orc
@@ -887,7 +892,7 @@ def run_reference(args):
     return {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": 1, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * statistics.mean(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": cfg.name, "global_batch": n_q, "seq_len": cfg.n, "parallelism": "none"},
+            "config": prefill_config(cfg, 1),
             "e2e": {"value": value, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "cpu_baseline": {"value": value, "unit": "queries/s", "cores": cores_used(), "kind": "oracle",
                              "sample": sample}}
