@@ -82,6 +82,21 @@ def test_workspace_queries(lsa):
     assert lsa.lsa_attn_workspace_bytes(1, 32, 8, 128, 2048, 64) > 0       # decode: split partials
 
 
+def test_workspace_of_the_next_rows(lsa):
+    """Sizes at the 1M prefill geometry: the sink/window pass adds only its per-(query, head)
+    output and LSE; the partials are T * Hq * n_leaves * d bf16; an update on append needs the
+    subtree's buffer and its build workspace."""
+    import torch
+    d = lsa.lsa_tree_describe(8, 64, (16, 16, 16, 4), 64)
+    T, Hq, B = 4096, 32, 32
+    base = lsa.lsa_tree_attn_workspace_bytes(d, T, Hq, 128, torch.bfloat16, B)
+    sw = lsa.lsa_tree_attn_sw_workspace_bytes(d, T, Hq, 128, torch.bfloat16, B, 16, 512)
+    assert base >= T * Hq * B * 128 * 2
+    assert sw - base == T * Hq * (128 * 2 + 4)
+    sub = lsa.lsa_tree_describe(8, 64, (16, 16, 4), 64)
+    assert lsa.lsa_tree_append_workspace_bytes(d, 128) >= sub.bytes + lsa.lsa_build_workspace_bytes(sub, 128)
+
+
 def test_calls_validate_before_launch(lsa):
     """Bad arguments come back as status codes; no device is needed to see them."""
     import torch
