@@ -606,7 +606,8 @@ __global__ void k_tl_finish(TreeAttnArgs a) {
 // bytes of partials.
 
 // One warp per (query, head) row: O = sum_k w_k o_k / sum_k w_k with
-// w_k = 2^(m_k - M) l_k over the row's leaves, in rank order.
+// w_k = 2^(m_k - M) l_k over the row's leaves, in a fixed order (even ranks and
+// odd ranks, each in rank order, then their sum).
 // 16 bytes through the non-coherent path; volatile, so that every partial of a row
 // is requested before the first is used (the compiler would otherwise sink each
 // load to its use and keep only a few in flight)

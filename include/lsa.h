@@ -303,7 +303,7 @@ int lsa_tree_attn_workspace_bytes(const lsa_tree_desc *tree, int32_t T, int32_t 
  * kernels on the expanded lists).  Outputs as lsa_sparse_attn.  While
  * T * Hq * n_leaves * d * 2 bytes stay within 24 GiB, every (row, leaf) pair
  * stores its leaf maximum, exp-sum and unnormalised output in the workspace and
- * a row's leaves are merged in rank order (results are reproducible bit for
+ * a row's leaves are merged in a fixed order (results are reproducible bit for
  * bit); larger calls take a second pass over the leaves instead and accumulate
  * the outputs with fp32 atomic adds, whose order is not fixed, so results may
  * differ from run to run in the last bits.  n_leaves in [1, 32]. */
