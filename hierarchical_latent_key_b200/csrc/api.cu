@@ -371,7 +371,7 @@ int lsa_attn_workspace_bytes(int32_t T, int32_t Hq, int32_t n_heads, int32_t d, 
   if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
   if (T < 0 || n_heads < 1 || Hq < 1 || K_sel < 0 || tail_len < 0 || (d != 64 && d != 128))
     return fail(LSA_ERR_SHAPE, "bad sizes");
-  const int ns = lsa::attn_splits(T, n_heads, K_sel + tail_len);
+  const int ns = T > 0 ? lsa::attn_splits(T, n_heads, K_sel + tail_len) : 1;
   *bytes = ns > 1 ? (size_t)T * Hq * ns * (d + 2) * sizeof(float) : 0;
   return ok();
 }

@@ -424,7 +424,7 @@ cudaError_t run_attn_extend(const int32_t* idx, int32_t K_sel, int64_t T, int32_
 int attn_splits(int64_t T, int Hkv, int64_t keys) {
   const int64_t units = T * Hkv;
   const int64_t target = 4 * 148;
-  if (units >= target || keys <= 64) return 1;
+  if (units <= 0 || units >= target || keys <= 64) return 1;
   int64_t s = (target + units - 1) / units;
   const int64_t max_s = (keys + 63) / 64;
   return (int)(s < max_s ? s : max_s);

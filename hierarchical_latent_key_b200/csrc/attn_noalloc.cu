@@ -46,6 +46,11 @@ extern "C" int lsa_sparse_attn_noalloc(const void* Q, int32_t T, int32_t Hq, con
                                        const int32_t* idx, int32_t K_sel, const int32_t* q_pos,
                                        int32_t causal, int64_t tail_begin, int64_t tail_end, float scale,
                                        void* O, float* LSE, int32_t* status, void* stream) {
+  // A call without queries launches nothing; lsa_sparse_attn validates the
+  // rest of its arguments and returns.
+  if (T == 0)
+    return lsa_sparse_attn(Q, T, Hq, K, V, n_heads, n_cap, d, dtype, idx, K_sel, q_pos, causal, tail_begin,
+                           tail_end, scale, O, LSE, nullptr, 0, status, stream);
   const int64_t tail_len = tail_end >= tail_begin ? tail_end - tail_begin : -1;
   size_t need = 0;
   int rc = lsa_attn_workspace_bytes(T, Hq, n_heads, d, K_sel, tail_len, &need);

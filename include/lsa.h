@@ -378,7 +378,10 @@ int lsa_sparse_attn_bwd(const void *Q, int32_t T, int32_t Hq, const void *K, con
  *    4.9 MB.  Calls that need no split use no scratch at all.
  *  - The first call on a device looks up that device's address of the array (once
  *    per device, with the device current); make that first call before any stream
- *    capture.
+ *    capture.  The address is kept for the life of the process: after
+ *    cudaDeviceReset (or anything else that destroys and recreates the device's
+ *    primary context) the kept address is stale, so do not call this entry point
+ *    on that device again in the same process.
  *  - All calls share the one array and it keeps the last call's contents; every
  *    call overwrites the partials it reads, so nothing needs clearing, but calls
  *    that overlap on the GPU (other streams, other host threads) race on it. */

@@ -165,3 +165,16 @@ def test_calls_validate_before_launch(lsa):
     assert call(args(d=96)) == lsa.LSA_ERR_SHAPE
     assert call(args(T=1, K_sel=2048)) == lsa.LSA_ERR_WORKSPACE
     assert call(args(T=0)) == lsa.LSA_OK
+
+
+def test_attn_no_queries(lsa):
+    """A call without queries needs no workspace and launches nothing, for every key count."""
+    L = lsa._lib
+    assert lsa.lsa_attn_workspace_bytes(0, 32, 8, 128, 2048, 0) == 0
+    assert lsa.lsa_attn_workspace_bytes(0, 32, 8, 128, 2048, 256) == 0
+    P = ctypes.c_void_p(16)
+    rc = L.lsa_sparse_attn_noalloc(P, 0, 32, P, P, 8, 1 << 20, 128, 1, P, 2048, None, 0, 0, 0, 0.1, P, P, None, None)
+    assert rc == lsa.LSA_OK
+    # the same call with an invalid argument is still rejected before anything else
+    rc = L.lsa_sparse_attn_noalloc(P, 0, 30, P, P, 8, 1 << 20, 128, 1, P, 2048, None, 0, 0, 0, 0.1, P, P, None, None)
+    assert rc == lsa.LSA_ERR_SHAPE
