@@ -379,8 +379,8 @@ cudaError_t run_kv_append(void* K, void* V, int64_t n_heads, int64_t n_cap, int6
   return cudaGetLastError();
 }
 
-// Key lists with the sink and recent-window keys (kongchang.com, "How LSA
-// Sidesteps Per-Key Scoring with Hierarchical Clustering": the keys taken from the
+// Key lists with the sink and recent-window keys (bdtechtalks.com, "Latent sparse
+// attention", section "How latent sparse attention works": the keys taken from the
 // chosen clusters are used together with a window of recent tokens and a few
 // initial sink tokens).  Row (g, t) of idx2 = the K_sel listed keys, then n_sink
 // sink slots, then `window` window slots; a position that the tail range attends

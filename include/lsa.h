@@ -261,10 +261,10 @@ int lsa_sparse_attn(const void *Q, int32_t T, int32_t Hq, const void *K, const v
 int lsa_sparse_attn_sw_workspace_bytes(int32_t T, int32_t Hq, int32_t n_heads, int32_t d, int32_t K_sel,
                                        int64_t tail_len, int32_t n_sink, int32_t window, size_t *bytes);
 
-/* Sparse attention with sink and recent-window keys (kongchang.com, "How LSA
- * Sidesteps Per-Key Scoring with Hierarchical Clustering": the keys taken from the
- * chosen clusters are attended together with a window of recent tokens and a few
- * initial sink tokens).  Arguments and outputs as lsa_sparse_attn with causal = 1
+/* Sparse attention with sink and recent-window keys (bdtechtalks.com, "Latent
+ * sparse attention", section "How latent sparse attention works": the keys taken
+ * from the chosen clusters are attended together with a window of recent tokens
+ * and a few initial sink tokens).  Arguments and outputs as lsa_sparse_attn with causal = 1
  * (q_pos required), plus
  *  n_sink : positions [0, n_sink) join every query's keys (where <= q_pos);
  *  window : positions [q_pos[t] - window + 1, q_pos[t]] join query t's keys.

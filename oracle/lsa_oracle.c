@@ -555,10 +555,10 @@ static int orc_cmp_i64(const void *x, const void *y) {
 
 /* Keys query t attends to: its index list, the dense tail range and, when n_sink
  * or window is positive, the first n_sink positions (sink tokens) and the window
- * positions q_pos - window + 1 .. q_pos (kongchang.com, "How LSA Sidesteps
- * Per-Key Scoring with Hierarchical Clustering": the keys taken from the chosen
- * clusters are used together with a window of recent tokens and a few initial
- * sink tokens).  With sink or window the key set is a set: it is sorted and a
+ * positions q_pos - window + 1 .. q_pos (bdtechtalks.com, "Latent sparse
+ * attention", section "How latent sparse attention works": the keys taken from
+ * the chosen clusters are used together with a window of recent tokens and a few
+ * initial sink tokens).  With sink or window the key set is a set: it is sorted and a
  * position listed twice counts once. */
 static int64_t orc_visible_keys(int64_t t, const int32_t *idx, int32_t K_sel,
                                 const int32_t *q_pos, int32_t causal, int64_t tail_begin,

@@ -442,8 +442,8 @@ def pin_backward_finite_differences():
 
 def _sink_window_mask(idx, n, tail, q_pos, sink, window):
     """Union of the index list, the tail, the first `sink` positions and the `window`
-    positions up to q_pos, then the causal cut (kongchang.com, "How LSA Sidesteps Per-Key
-    Scoring with Hierarchical Clustering": chosen keys plus recent and sink tokens)."""
+    positions up to q_pos, then the causal cut (bdtechtalks.com, "Latent sparse attention",
+    section "How latent sparse attention works": chosen keys plus recent and sink tokens)."""
     m = _mask_from(idx, n, tail, q_pos, True)
     for t in range(idx.shape[0]):
         m[t, :sink] = True
