@@ -235,6 +235,78 @@ def _deferred_acceptance_fast(D, pos, b):
             return ch
 
 
+def _numpy_build(Z, branching, leaf, iters, seed):
+    """The whole top-down build restated in numpy: per level, every parent's members (in
+    ascending position) start from the seeded picks, then `iters` rounds of (squared
+    distances, stable balanced assignment by the independent deferred-acceptance solver,
+    member means).  Returns (centroids per level, leaf_index, trace [L, iters, n])."""
+    n, r = Z.shape
+    L = len(branching)
+    members = [np.arange(n)]
+    trace = np.full((L, iters, n), -1, np.int64)
+    cents = []
+    for l, b in enumerate(branching):
+        nxt, cl = [], []
+        for s, pos in enumerate(members):
+            Zs = Z[pos]
+            h = np.array([orc.init_hash(seed, l, int(p)) for p in pos], dtype=np.uint64)
+            mu = Zs[np.argsort(h, kind="stable")[:b]]
+            for t in range(iters):
+                D = ((Zs[:, None, :] - mu[None]) ** 2).sum(-1)
+                a = _deferred_acceptance_fast(D, pos, b)
+                trace[l, t, pos] = s * b + a
+                mu = np.stack([Zs[a == c].mean(axis=0) for c in range(b)])
+            cl.append(mu)
+            nxt += [pos[a == c] for c in range(b)]
+        members = nxt
+        cents.append(np.concatenate(cl))
+    return cents, np.concatenate(members), trace
+
+
+def pin_tree_independent_rebuild():
+    """The oracle's composite build equals the numpy restatement of the same steps
+    (kongchang.com, "How LSA Sidesteps Per-Key Scoring with Hierarchical Clustering":
+    the tree is built like hierarchical k-means, root = all keys), on two trees: the
+    two-level tiny case and a three-level one, every round of every level compared."""
+    for kw in (dict(), dict(seed=5, branching=(4, 4, 4), leaf=16, iters=5)):
+        K, W, Z, tree = tiny_tree_case(**kw)
+        seed = kw.get("seed", 0)
+        iters = kw.get("iters", 4)
+        cents, li, tr = _numpy_build(Z, tree.branching, tree.leaf_size, iters, seed)
+        np.testing.assert_array_equal(tree.trace, tr)
+        np.testing.assert_array_equal(tree.leaf_index, li)
+        for l in range(len(tree.branching)):
+            np.testing.assert_allclose(tree.centroids[l], cents[l], rtol=1e-10, atol=1e-12)
+
+
+def pin_tree_rounds_from_trace():
+    """Every k-means round of every level follows from the round before it: round 0 of
+    level l from the seeded picks inside each level-(l-1) node, round t > 0 from the
+    numpy means of round t-1's partition; each assignment is the stable balanced one
+    (independent solver).  Also checks that exactly `iters` rounds ran per level."""
+    K, W, Z, tree = tiny_tree_case(seed=7, branching=(4, 4, 4), leaf=16, iters=6)
+    n, L, iters = Z.shape[0], len(tree.branching), tree.trace.shape[1]
+    assert iters == 6
+    parent = np.zeros(n, np.int64)
+    for l in range(L):
+        b = tree.branching[l]
+        for t in range(iters):
+            for s in np.unique(parent):
+                pos = np.nonzero(parent == s)[0]
+                Zs = Z[pos]
+                if t == 0:
+                    h = np.array([orc.init_hash(7, l, int(p)) for p in pos], dtype=np.uint64)
+                    mu = Zs[np.argsort(h, kind="stable")[:b]]
+                else:
+                    prev = tree.trace[l, t - 1, pos] - s * b
+                    assert prev.min() >= 0 and prev.max() < b
+                    mu = np.stack([Zs[prev == c].mean(axis=0) for c in range(b)])
+                D = ((Zs[:, None, :] - mu[None]) ** 2).sum(-1)
+                a = _deferred_acceptance_fast(D, pos, b)
+                np.testing.assert_array_equal(tree.trace[l, t, pos], s * b + a, err_msg=f"level {l} round {t}")
+        parent = tree.trace[l, iters - 1].astype(np.int64)
+
+
 def pin_tree_deterministic_and_seeded():
     _, _, Z, t1 = tiny_tree_case()
     t2 = orc.build_tree(Z, t1.branching, t1.leaf_size, 4, seed=0)

@@ -19,7 +19,8 @@ ORDER = [
     P.pin_splitmix64_published_vectors, P.pin_init_rule, P.pin_projection_matches_numpy,
     P.pin_distances_closed_form, P.pin_balanced_assign_bruteforce,
     P.pin_balanced_assign_vs_deferred_acceptance, P.pin_tree_invariants,
-    P.pin_tree_first_step_from_init, P.pin_tree_deterministic_and_seeded,
+    P.pin_tree_first_step_from_init, P.pin_tree_rounds_from_trace, P.pin_tree_independent_rebuild,
+    P.pin_tree_deterministic_and_seeded,
     P.pin_select_beam_walk, P.pin_select_full_beam_equals_flat,
     P.pin_attention_equals_sdpa, P.pin_attention_special_cases,
     P.pin_backward_autograd, P.pin_backward_finite_differences,
@@ -40,6 +41,14 @@ MUTANTS = [
      "if (x->pos > y->pos) return -1;\n  if (x->pos < y->pos) return 1;"),
     ("mean over wrong count", "mu[(int64_t)c * r + k] / (double)cnt[c]",
      "mu[(int64_t)c * r + k] / (double)(cnt[c] + 1)"),
+    ("init of every level uses level 0", "e = orc_level_init(Zs, pos, m, r, b, seed, l, mu);",
+     "e = orc_level_init(Zs, pos, m, r, b, seed, 0, mu);"),
+    ("means updated only after the last round", "        orc_means(Zs, m, r, a, b, mu);\n      }",
+     "        if (t == iters - 1) orc_means(Zs, m, r, a, b, mu);\n      }"),
+    ("only the first and last rounds run", "for (int32_t t = 0; t < iters && e == ORC_OK; ++t) {",
+     "for (int32_t t = 0; t < iters && e == ORC_OK; t = (t == 0 ? iters - 1 : t + 1)) {"),
+    ("one round short", "for (int32_t t = 0; t < iters && e == ORC_OK; ++t) {",
+     "for (int32_t t = 0; t < iters - 1 && e == ORC_OK; ++t) {"),
     ("children numbered transposed", "next[(s * b + j) * cap + fill[j]] = pos[i];",
      "next[(j * segs + s) * cap + fill[j]] = pos[i];"),
     ("min position as max", "if (pos[i] < min_pos[node_off + s * b + j])",
