@@ -33,13 +33,18 @@ def _eps_stable(D, a, Zs, mu, rel=STABLE_EPS_REL):
 
 
 def check_build_stagewise(Z, trace, branching, leaf, iters, seed, max_segments=None, rng=None, check=None):
-    """Z: [n, r] float64 latents of one head (oracle projection); trace: [L, iters, n]
-    GPU node ids by position; check(level, round, segment_size) -> bool selects which
-    rounds are recomputed (all by default).  Returns (rounds that differed, keys that
-    differed)."""
-    Z = np.asarray(Z, np.float64)
+    """Z: [n, r] float64 latents of one head (oracle projection), or a function that
+    returns the oracle latents of the given positions (for indexes too large to project
+    whole); trace: [L, iters, n] GPU node ids by position; check(level, round,
+    segment_size) -> bool selects which rounds are recomputed (all by default).  Returns
+    (rounds that differed, keys that differed)."""
     trace = np.asarray(trace)
-    n = Z.shape[0]
+    if callable(Z):
+        rows_of = Z
+    else:
+        Zfull = np.asarray(Z, np.float64)
+        rows_of = lambda pos: Zfull[pos]
+    n = trace.shape[-1]
     L = len(branching)
     parent = np.zeros(n, np.int64)
     rounds_diff = keys_diff = 0
@@ -55,8 +60,10 @@ def check_build_stagewise(Z, trace, branching, leaf, iters, seed, max_segments=N
         if max_segments is not None and S > max_segments:
             segs = sorted((rng or np.random.default_rng(0)).choice(S, max_segments, replace=False))
         for s in segs:
+            if check is not None and not any(check(l, t, m) for t in range(iters)):
+                continue
             pos = order[s]
-            Zs = Z[pos]
+            Zs = rows_of(pos)
             for t in range(iters):
                 if check is not None and not check(l, t, m):
                     continue
@@ -139,6 +146,40 @@ def check_select_stagewise(qlat, tree_h, branching, leaf, beam, q_pos, gpu_beam,
         expect[:len(keys)] = keys
         np.testing.assert_array_equal(gpu_idx[t], expect)
     return near
+
+
+GRAD_RMS_REL = 1e-2     # rms(error) <= 1e-2 * rms(reference), over the touched rows
+GRAD_ELEM_REL = 2 ** -5  # |error| <= 2^-5 |reference| + GRAD_ELEM_ABS * rms(reference), per element
+GRAD_ELEM_ABS = 4e-2
+
+
+def check_grad(name, got, want, zero_untouched=True, report=None):
+    """Gradient tolerance (the pages give none).  The kernels round P, dS and the stored
+    forward output O to bf16 (unit roundoff u = 2^-8) before their products, so a
+    gradient element carries a few u of relative error in each of its terms; summed over
+    hundreds of terms of either sign this stays near u of the gradient's own scale.  The
+    bound is taken over the rows a selection touches (with zero_untouched, for dK and dV,
+    rows no query sees must be exactly zero): rms(error) <= 1e-2 rms(ref), and per element
+    |error| <= 2^-5 |ref| + 4e-2 rms(ref)."""
+    got = np.asarray(got, np.float64).reshape(-1, np.shape(got)[-1])
+    want = np.asarray(want, np.float64).reshape(-1, np.shape(want)[-1])
+    touched = np.abs(want).max(axis=1) > 0
+    if zero_untouched:
+        assert np.all(got[~touched] == 0), (name, "nonzero gradient on an untouched row")
+    else:
+        touched[:] = True
+    g, w = got[touched], want[touched]
+    if w.size == 0:
+        return
+    err = np.abs(g - w)
+    rms = np.sqrt((w ** 2).mean())
+    rel_rms = np.sqrt((err ** 2).mean()) / rms
+    elem = (err - GRAD_ELEM_REL * np.abs(w)).max() / rms
+    if report is not None:
+        report[name] = (float(rel_rms), float(elem))
+    print(f"{name}: rms(err)/rms(ref) {rel_rms:.3g}, max(|err| - 2^-5|ref|)/rms(ref) {elem:.3g}")
+    assert rel_rms <= GRAD_RMS_REL, (name, rel_rms)
+    assert elem <= GRAD_ELEM_ABS, (name, elem)
 
 
 def attn_errors(O_gpu, O_ref):

@@ -130,34 +130,64 @@ def test_prefill_1m_full(lsa):
 
 
 def test_decode_10m_full(lsa):
-    """10,485,760 indexed keys, decode steps through select + key-list attention with tail."""
-    cfg = configs.get("decode_10m").scaled(T=8)
+    """10,485,760 indexed keys, all 128 decode steps (append, select, key-list attention with
+    the dense tail, one step at a time as bench.py runs them), every step checked on all 8
+    KV heads: the beam walk stage-wise (near-tie band), the key list exactly, attention on
+    the GPU's keys.  The build is checked stage-wise on sampled segments of one head (every
+    round of the three lowest levels) and by tree properties on every head."""
+    cfg = configs.get("decode_10m")
     case = cfg.case(DEV)
-    tree = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    n = cfg.n
+    Knew = case.K[:, n:].transpose(0, 1).contiguous()       # rows the steps append
+    Vnew = case.V[:, n:].transpose(0, 1).contiguous()
+    case.K[:, n:].zero_()
+    case.V[:, n:].zero_()
+    tree, trace = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed, trace=True)
+    torch.cuda.synchronize()
     rng = np.random.default_rng(2)
-    h = 6
-    _tree_props(tree, h, case.K, case.W[h].double().cpu().numpy(), cfg.n, cfg.leaf, rng, n_nodes=4)
-    # one decode step at a time, as bench.py runs them
-    th = parity.export_tree(tree, h)
-    W_h = case.W[h].double().cpu().numpy()
+    hb = 6
+    W_b = case.W[hb].double().cpu().numpy()
+    tr = trace[:, :, hb].cpu().numpy()
+    del trace
+    rd, kd = parity.check_build_stagewise(lambda pos: orc.project(_rows(case.K, hb, pos), W_b), tr, cfg.branching,
+                                          cfg.leaf, cfg.iters, cfg.seed, max_segments=4, rng=rng,
+                                          check=lambda l, t, m: m <= 81920)
+    del tr
+    print("decode_10m build rounds differing", rd, "keys", kd)
+    for h in range(cfg.Hkv):
+        _tree_props(tree, h, case.K, case.W[h].double().cpu().numpy(), n, cfg.leaf, rng, n_nodes=4)
+    # the decode loop on the GPU: one token per step, its key and value appended first
+    idx = torch.empty(cfg.Hkv, 1, cfg.K_sel, dtype=torch.int32, device=DEV)
+    st_idx, st_beams, st_O, st_LSE = [], [], [], []
     for s in range(cfg.T):
-        p = cfg.n + s
+        lsa.lsa_kv_append(case.K, case.V, n + s, Knew[s], Vnew[s])
         Qs = case.Q[s:s + 1]
         idx, beams = lsa.select(tree, Qs, case.W, cfg.beam, case.q_pos[s:s + 1], beams=True)
-        O, LSE = lsa.sparse_attn(Qs, case.K, case.V, idx, case.q_pos[s:s + 1], True, (cfg.n, p + 1))
-        Qg = Qs[:, h * cfg.G:(h + 1) * cfg.G].double().cpu().numpy()
-        oq = orc.query_latent(Qg, W_h)
-        parity.check_select_stagewise(oq, th, cfg.branching, cfg.leaf, cfg.beam, np.array([p]),
-                                      beams[:, h].cpu().numpy(), idx[h].cpu().numpy())
-        # every selected key and every tail key precedes the query: compact them (non-causal)
-        sel = idx[h, 0].cpu().numpy()
-        keys = np.concatenate([sel[sel >= 0], np.arange(cfg.n, p + 1)])
-        Kc, Vc = _rows(case.K, h, keys), _rows(case.V, h, keys)
-        n_sel = int((sel >= 0).sum())
-        Oo, Lo = orc.attn_fwd(Qg, Kc, Vc, np.arange(n_sel, dtype=np.int32)[None], tail=(n_sel, len(keys)))
-        mx, mean = parity.attn_errors(O[:, h * cfg.G:(h + 1) * cfg.G].float().cpu(), Oo)
-        assert mx <= 2e-2 and mean <= 2e-3, (s, mx, mean)
-        assert np.abs(LSE[:, h * cfg.G:(h + 1) * cfg.G].cpu().numpy() - Lo).max() <= 1e-3
+        O, LSE = lsa.sparse_attn(Qs, case.K, case.V, idx, case.q_pos[s:s + 1], True, (n, n + s + 1))
+        st_idx.append(idx.cpu()); st_beams.append(beams.cpu()); st_O.append(O.float().cpu()); st_LSE.append(LSE.cpu())
+    torch.cuda.synchronize()
+    near = 0
+    for h in range(cfg.Hkv):
+        th = parity.export_tree(tree, h)
+        W_h = case.W[h].double().cpu().numpy()
+        sl = slice(h * cfg.G, (h + 1) * cfg.G)
+        for s in range(cfg.T):
+            p = n + s
+            Qg = case.Q[s:s + 1, sl].double().cpu().numpy()
+            oq = orc.query_latent(Qg, W_h)
+            near += parity.check_select_stagewise(oq, th, cfg.branching, cfg.leaf, cfg.beam, np.array([p]),
+                                                  st_beams[s][:, h].numpy(), st_idx[s][h].numpy())
+            # every selected key and every tail key precedes the query: compact them (non-causal)
+            sel = st_idx[s][h, 0].numpy()
+            keys = np.concatenate([sel[sel >= 0], np.arange(n, p + 1)])
+            Kc, Vc = _rows(case.K, h, keys), _rows(case.V, h, keys)
+            n_sel = int((sel >= 0).sum())
+            Oo, Lo = orc.attn_fwd(Qg, Kc, Vc, np.arange(n_sel, dtype=np.int32)[None], tail=(n_sel, len(keys)))
+            mx, mean = parity.attn_errors(st_O[s][:, sl], Oo)
+            assert mx <= 2e-2 and mean <= 2e-3, (h, s, mx, mean)
+            assert np.abs(st_LSE[s][:, sl].numpy() - Lo).max() <= 1e-3
+    print("decode_10m near-ties", near, "of", cfg.T * cfg.Hkv * len(cfg.branching), "(query, head, level) beams")
+    assert near <= cfg.T * cfg.Hkv * len(cfg.branching) // 100
 
 
 def test_train_128k_full(lsa):
@@ -184,19 +214,22 @@ def test_train_128k_full(lsa):
     mx, mean = parity.attn_errors(O[rows][:, sl].float().cpu(), Oo)
     assert mx <= 2e-2 and mean <= 2e-3, (mx, mean)
     oQ, _, _ = orc.attn_bwd(Qh[rows], Kh, Vh, ih[rows], dOh[rows], q_pos=qp[rows], causal=True)
-    got = dQ[rows][:, sl].cpu().numpy()
-    err = np.abs(got - oQ)
-    assert err.max() <= 2e-2 * np.abs(oQ).max() and err.mean() <= 2e-3 * np.abs(oQ).mean()
-    # a few keys: every query that selected them contributes to dK, dV
-    keys = rng.choice(cfg.n // 2, 3, replace=False)
-    for j in keys:
-        users = np.nonzero((ih == j).any(axis=1) & (qp >= j))[0]
+    parity.check_grad("dQ", dQ[rows][:, sl].cpu().numpy(), oQ, zero_untouched=False)
+    # dK, dV of every key of 8 sampled leaves (512 keys): a leaf is selected whole, so the
+    # queries that listed its first key are every query that sees any of its keys
+    li = tree.leaf_index()[h].cpu().numpy().reshape(-1, cfg.leaf)
+    got_K, got_V, want_K, want_V = [], [], [], []
+    for leaf in rng.choice(li.shape[0], 8, replace=False):
+        keys = li[leaf]
+        users = np.nonzero((ih == keys[0]).any(axis=1))[0]
         if len(users) == 0:
             continue
         _, oK, oV = orc.attn_bwd(Qh[users], Kh, Vh, ih[users], dOh[users], q_pos=qp[users], causal=True)
-        for name, got, want in (("dK", dK[h, j].cpu().numpy(), oK[j]), ("dV", dV[h, j].cpu().numpy(), oV[j])):
-            e = np.abs(got - want)
-            assert e.max() <= 2e-2 * np.abs(want).max() + 1e-6, (name, j, e.max(), np.abs(want).max())
+        got_K.append(dK[h, keys].cpu().numpy()); want_K.append(oK[keys])
+        got_V.append(dV[h, keys].cpu().numpy()); want_V.append(oV[keys])
+    assert len(got_K) >= 4
+    parity.check_grad("dK", np.concatenate(got_K), np.concatenate(want_K))
+    parity.check_grad("dV", np.concatenate(got_V), np.concatenate(want_V))
 
 
 def test_tree_attention_beyond_partial_budget(lsa):

@@ -12,6 +12,7 @@ import torch
 
 from hierarchical_latent_key_b200 import configs
 from oracle import oracle as orc
+from tests import parity
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -102,10 +103,7 @@ def test_backward_with_sink_and_window(lsa):
         oQ, oK, oV = orc.attn_bwd(case.Q[:, sl], case.K[h], case.V[h], idx[h].cpu(), case.dO[:, sl],
                                   q_pos=case.q_pos.numpy(), causal=True, sink=sink, window=window)
         for name, got, want in (("dQ", dQ[:, sl], oQ), ("dK", dK[h], oK), ("dV", dV[h], oV)):
-            got = got.cpu().numpy()
-            err = np.abs(got - want)
-            assert err.max() <= 2e-2 * np.abs(want).max(), (name, err.max(), np.abs(want).max())
-            assert err.mean() <= 2e-3 * np.abs(want).mean(), (name, err.mean(), np.abs(want).mean())
+            parity.check_grad(name, got.cpu().numpy(), want, zero_untouched=name != "dQ")
 
 
 def test_rejects_bad_sink_window(lsa):
