@@ -645,6 +645,31 @@ def time_pooled(w, steps, warmup, flush, stream, pool=POOL):
                       f"build times over all {cfg.Hkv} heads with CUDA events"}
 
 
+def time_projection(w, steps, warmup, flush, stream):
+    """The latent projection Z = K . W of the index build (lsa_project_keys, tensor cores) over
+    all indexed keys of every KV head, L2 flushed between launches."""
+    lsa, cfg = w.lsa, w.cfg
+    Hkv, _, d = w.K.shape
+    Z = torch.empty(Hkv, cfg.n, cfg.r, dtype=torch.float32, device=w.K.device)
+    for _ in range(warmup):
+        lsa.lsa_project_keys(w.K, w.W, cfg.n, Z, w.status)
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+    for k in range(steps):
+        flush.zero_()
+        ev[k][0].record(stream)
+        lsa.lsa_project_keys(w.K, w.W, cfg.n, Z, w.status)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    ms = statistics.mean(ev[k][0].elapsed_time(ev[k][1]) for k in range(steps))
+    alg = Hkv * cfg.n * (d * w.K.element_size() + cfg.r * 4) + w.W.numel() * w.W.element_size()
+    peak = measured_peaks()["hbm_gbs"]
+    del Z
+    return {"kernel": "k_project_tc", "ms": ms, "keys": Hkv * cfg.n, "algorithmic_bytes": alg,
+            "achieved_gbs": alg / (ms / 1e3) / 1e9, "frac": alg / (ms / 1e3) / 1e9 / peak,
+            "tflops": 2.0 * Hkv * cfg.n * d * cfg.r / (ms / 1e3) / 1e12}
+
+
 def time_e2e(w, steps, flush, stream):
     """Same step through the public API with pinned host buffers: H2D of the chunk's
     queries, select + attention, D2H of the outputs, all inside the timed region."""
@@ -792,6 +817,10 @@ def run_cuda(args, rank, world, local_rank):
     except Exception as e:  # noqa: BLE001
         flat = {"error": f"{type(e).__name__}: {e}"}
     try:
+        projection = time_projection(w, args.steps, args.warmup, flush, stream)
+    except Exception as e:  # noqa: BLE001
+        projection = {"error": f"{type(e).__name__}: {e}"}
+    try:
         pooled = time_pooled(w, args.steps, args.warmup, flush, stream)
     except Exception as e:  # noqa: BLE001
         pooled = {"error": f"{type(e).__name__}: {e}"}
@@ -843,6 +872,7 @@ def run_cuda(args, rank, world, local_rank):
             "prefill_1m_sink_window": sink_window,
             "prefill_1m_flat": flat,
             "prefill_1m_pooled": pooled,
+            "projection_1m": projection,
             "tree_append_128k": append,
             "decode_10m": decode,
             "train_128k": train,

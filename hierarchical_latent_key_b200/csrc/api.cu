@@ -673,6 +673,19 @@ int lsa_sparse_attn_sw_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, 
   return ok();
 }
 
+int lsa_project_keys(const void* K, int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, const void* W,
+                     int32_t r, int64_t n, float* Z, int32_t* status, void* stream) {
+  if (!K || !W || !Z) return fail(LSA_ERR_INVALID_ARG, "K, W and Z must be non-NULL");
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (n_heads < 1 || (d != 64 && d != 128) || (r != 16 && r != 32 && r != 64))
+    return fail(LSA_ERR_SHAPE, "need n_heads >= 1, d in {64, 128} and r in {16, 32, 64}");
+  if (n < 0 || n > n_cap) return fail(LSA_ERR_SHAPE, "n %lld outside [0, n_cap]", (long long)n);
+  cudaError_t e = lsa::run_project(K, n_cap, W, n, n_heads, r, d, dtype, Z, nullptr, status,
+                                   static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_project_keys");
+  return ok();
+}
+
 int lsa_kv_append(void* K, void* V, int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, int64_t pos,
                   const void* K_rows, const void* V_rows, void* stream) {
   if (!K || !V || !K_rows || !V_rows) return fail(LSA_ERR_INVALID_ARG, "K, V, K_rows and V_rows must be non-NULL");

@@ -18,6 +18,7 @@
 // means over the partitioned order (fixed summation order, so deterministic).
 
 #include <cooperative_groups.h>
+#include <type_traits>
 
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
@@ -61,7 +62,7 @@ __global__ void __launch_bounds__(256) k_project_keys(const T* __restrict__ K, i
     float* zr = Z + ((int64_t)h * n + row) * R + q * CQ;
 #pragma unroll
     for (int c = 0; c < CQ; c += 4) *reinterpret_cast<float4*>(zr + c) = make_float4(acc[c], acc[c + 1], acc[c + 2], acc[c + 3]);
-    if (q == 0) pos[(int64_t)h * n + row] = (int32_t)row;
+    if (q == 0 && pos) pos[(int64_t)h * n + row] = (int32_t)row;
   }
 }
 
@@ -823,17 +824,22 @@ static cudaError_t build_levels(const BuildPlan& P, const lsa_tree_desc& t, char
 }
 
 template <typename T>
-static cudaError_t project(const BuildPlan& P, const lsa_tree_desc& t, const void* K, int64_t n_cap, int d,
-                           const void* W, cudaStream_t st) {
-  dim3 grid((unsigned)ceil_div(t.n_tree, 64), (unsigned)t.n_heads);
+static cudaError_t project(const void* K, int64_t n_cap, const void* W, int64_t n, int32_t n_heads, int r, int d,
+                           float* Z, int32_t* pos, int32_t* status, cudaStream_t st) {
+  // bf16 keys: tensor-core product (project.cu); fp32 keys keep fp32 FMAs, since a
+  // tf32 product would round the operands to 10 mantissa bits
+  if (project_tc_supported(std::is_same<T, float>::value ? LSA_F32 : LSA_BF16, r, d))
+    return run_project_tc(K, n_cap, W, n, n_heads, r, d, Z, pos, status, st);
+  if (n <= 0) return cudaSuccess;
+  dim3 grid((unsigned)ceil_div(n, 64), (unsigned)n_heads);
   const T* k = static_cast<const T*>(K);
   const T* w = static_cast<const T*>(W);
 #define LSA_PROJ(RR, DD)                                                                           \
-  if (t.r == RR && d == DD) {                                                                      \
+  if (r == RR && d == DD) {                                                                        \
     const size_t smem = (size_t)(DD * RR + 64 * (DD + 1)) * sizeof(float);                         \
     cudaFuncSetAttribute(k_project_keys<T, RR, DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
                          (int)smem);                                                               \
-    k_project_keys<T, RR, DD><<<grid, 256, smem, st>>>(k, n_cap, w, t.n_tree, P.Za, P.pa);        \
+    k_project_keys<T, RR, DD><<<grid, 256, smem, st>>>(k, n_cap, w, n, Z, pos);                   \
     return cudaGetLastError();                                                                     \
   }
   LSA_PROJ(16, 64) LSA_PROJ(32, 64) LSA_PROJ(64, 64) LSA_PROJ(16, 128) LSA_PROJ(32, 128) LSA_PROJ(64, 128)
@@ -841,11 +847,16 @@ static cudaError_t project(const BuildPlan& P, const lsa_tree_desc& t, const voi
   return cudaErrorInvalidValue;
 }
 
+cudaError_t run_project(const void* K, int64_t n_cap, const void* W, int64_t n, int32_t n_heads, int r, int d,
+                        int dtype, float* Z, int32_t* pos, int32_t* status, cudaStream_t st) {
+  return dtype == LSA_BF16 ? project<__nv_bfloat16>(K, n_cap, W, n, n_heads, r, d, Z, pos, status, st)
+                           : project<float>(K, n_cap, W, n, n_heads, r, d, Z, pos, status, st);
+}
+
 cudaError_t run_build(const BuildPlan& P, const lsa_tree_desc& t, void* tree_mem, const void* K, int64_t n_cap,
                       int d, int dtype, const void* W, int32_t pool, int32_t* trace, int32_t* status,
                       cudaStream_t st) {
-  cudaError_t e = dtype == LSA_BF16 ? project<__nv_bfloat16>(P, t, K, n_cap, d, W, st)
-                                    : project<float>(P, t, K, n_cap, d, W, st);
+  cudaError_t e = run_project(K, n_cap, W, t.n_tree, t.n_heads, t.r, d, dtype, P.Za, P.pa, status, st);
   if (e != cudaSuccess) return e;
   char* tm = static_cast<char*>(tree_mem);
   // with pooling the levels cluster the blocks: same nodes and tree buffer,

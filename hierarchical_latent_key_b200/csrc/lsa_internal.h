@@ -56,6 +56,15 @@ struct BuildPlan {
 // query and the carving of a caller buffer).
 size_t build_workspace_layout(const lsa_tree_desc& t, char* base, BuildPlan* plan);
 
+// Latent projection of keys on the tensor cores (bf16, r in {16, 32, 64}, d in {64, 128}):
+// Z[h][i] = K[h][i] . W[h] and pos[h][i] = i for i < n.
+// run_project picks the tensor-core kernel where supported, fp32 FMAs otherwise.
+bool project_tc_supported(int dtype, int r, int d);
+cudaError_t run_project(const void* K, int64_t n_cap, const void* W, int64_t n, int32_t n_heads, int r, int d,
+                        int dtype, float* Z, int32_t* pos, int32_t* status, cudaStream_t st);
+cudaError_t run_project_tc(const void* K, int64_t n_cap, const void* W, int64_t n, int32_t n_heads, int r, int d,
+                           float* Z, int32_t* pos, int32_t* status, cudaStream_t st);
+
 cudaError_t run_build(const BuildPlan& P, const lsa_tree_desc& t, void* tree_mem, const void* K, int64_t n_cap,
                       int d, int dtype, const void* W, int32_t pool, int32_t* trace, int32_t* status,
                       cudaStream_t st);

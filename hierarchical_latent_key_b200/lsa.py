@@ -82,6 +82,7 @@ def _load():
         "lsa_sparse_attn_sw_bwd": (ctypes.c_int, [P, i32, i32, P, P, i32, i64, i32, i32, P, P, P, P, i32, P, i32,
                                                   i32, i64, i64, f32, P, P, P, P, sz, P, P]),
         "lsa_kv_append": (ctypes.c_int, [P, P, i32, i64, i32, i32, i64, P, P, P]),
+        "lsa_project_keys": (ctypes.c_int, [P, i32, i64, i32, i32, P, i32, i64, P, P, P]),
         "lsa_tree_attn_bwd_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
         "lsa_tree_attn_bwd": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, P, P, P, i32, P, i32, f32,
                                              P, P, P, P, sz, P, P]),
@@ -278,6 +279,22 @@ def lsa_sparse_attn_sw_bwd(Q, K, V, O, LSE, dO, idx, q_pos, n_sink, window, tail
                                        int(window), tail_begin, tail_end, float(scale), _ptr(dQ), _ptr(dK), _ptr(dV),
                                        _ptr(workspace), ws_n, _ptr(status), _stream(stream, Q)),
            "lsa_sparse_attn_sw_bwd")
+
+
+def lsa_project_keys(K, W, n, Z, status=None, stream=None):
+    """K: [n_heads, n_cap, d]; W: [n_heads, d, r]; Z: [n_heads, n, r] fp32 (written)."""
+    _raise(_lib.lsa_project_keys(_ptr(K), K.shape[0], K.shape[1], K.shape[2], _dtype(K), _ptr(W), W.shape[2],
+                                 int(n), _ptr(Z), _ptr(status), _stream(stream, K)), "lsa_project_keys")
+
+
+def project_keys(K, W, n=None):
+    """Latents Z [n_heads, n, r] fp32 of the first n keys of K (all of them by default)."""
+    n = K.shape[1] if n is None else n
+    Z = torch.empty(K.shape[0], n, W.shape[2], dtype=torch.float32, device=K.device)
+    st = _new_status(K.device)
+    lsa_project_keys(K, W, n, Z, st)
+    check_status(st, "lsa_project_keys")
+    return Z
 
 
 def lsa_kv_append(K, V, pos, K_rows, V_rows, stream=None):

@@ -392,6 +392,20 @@ int lsa_sparse_attn_noalloc(const void *Q, int32_t T, int32_t Hq, const void *K,
                             int64_t tail_begin, int64_t tail_end, float scale, void *O, float *LSE,
                             int32_t *status, void *stream);
 
+/* Latent projection of the keys (kongchang.com, "Latent Sparse Attention Breaks
+ * Through the Million-Token Context Bottleneck", section "How LSA Sidesteps
+ * Per-Key Scoring with Hierarchical Clustering": keys are first mapped into a
+ * low-dimensional latent space).  The first step of lsa_build_tree, exposed on
+ * its own:  Z[h][i][c] = sum_j K[h][i][j] * W[h][j][c]  for i < n.
+ *  K : [n_heads][n_cap][d] (dtype), device;  W : [n_heads][d][r] (dtype), device;
+ *  Z : [n_heads][n][r] fp32, device, overwritten.
+ *  d in {64, 128}, r in {16, 32, 64}, 0 <= n <= n_cap.  bf16 inputs run on the
+ *  tensor cores (exact products, fp32 sums); fp32 inputs use fp32 FMAs.  An MMA
+ *  that does not complete within a second sets LSA_ERR_TIMEOUT in *status (may be
+ *  NULL).  Needs no workspace. */
+int lsa_project_keys(const void *K, int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype,
+                     const void *W, int32_t r, int64_t n, float *Z, int32_t *status, void *stream);
+
 /* Decode append (bdtechtalks.com, "How latent sparse attention works": the
  * recent tokens join the attended keys): write the new key row and value row of
  * every KV head at position `pos` of the caches K, V [n_heads][n_cap][d].

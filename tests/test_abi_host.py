@@ -178,3 +178,14 @@ def test_attn_no_queries(lsa):
     # the same call with an invalid argument is still rejected before anything else
     rc = L.lsa_sparse_attn_noalloc(P, 0, 30, P, P, 8, 1 << 20, 128, 1, P, 2048, None, 0, 0, 0, 0.1, P, P, None, None)
     assert rc == lsa.LSA_ERR_SHAPE
+
+
+def test_project_keys_rejects(lsa):
+    L = lsa._lib
+    P = ctypes.c_void_p(16)
+    assert L.lsa_project_keys(None, 2, 100, 128, 1, P, 64, 10, P, None, None) == lsa.LSA_ERR_INVALID_ARG
+    assert L.lsa_project_keys(P, 2, 100, 128, 9, P, 64, 10, P, None, None) == lsa.LSA_ERR_INVALID_ARG
+    assert L.lsa_project_keys(P, 2, 100, 96, 1, P, 64, 10, P, None, None) == lsa.LSA_ERR_SHAPE
+    assert L.lsa_project_keys(P, 2, 100, 128, 1, P, 48, 10, P, None, None) == lsa.LSA_ERR_SHAPE
+    assert L.lsa_project_keys(P, 2, 100, 128, 1, P, 64, 101, P, None, None) == lsa.LSA_ERR_SHAPE
+    assert L.lsa_project_keys(P, 0, 100, 128, 1, P, 64, 10, P, None, None) == lsa.LSA_ERR_SHAPE
