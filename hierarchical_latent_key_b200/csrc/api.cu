@@ -103,6 +103,30 @@ size_t build_workspace_layout(const lsa_tree_desc& t, char* base, BuildPlan* P) 
   return off;
 }
 
+size_t assign_workspace_layout(int64_t nseg, int64_t m, int b, char* base, BuildPlan* P) {
+  const int64_t nslots = nseg * m, nnodes = nseg * b;
+  const bool grid = m > kCtaMaxSeg;
+  uint64_t off = 0;
+  auto take = [&](uint64_t bytes) {
+    uint64_t at = off;
+    off = align256(off + (bytes ? bytes : 1));
+    return base ? base + at : nullptr;
+  };
+  char* p;
+  p = take(nslots * b * 4);                   if (P) P->D = reinterpret_cast<float*>(p);
+  p = take(nslots * 8);                       if (P) P->pref = reinterpret_cast<uint64_t*>(p);
+  p = take(nslots * 4);                       if (P) P->dbits = reinterpret_cast<uint32_t*>(p);
+  p = take(nslots);                           if (P) P->ptr = reinterpret_cast<uint8_t*>(p);
+  p = take(grid ? nnodes * 2048 * 4 : 0);     if (P) P->hist = reinterpret_cast<uint32_t*>(p);
+  p = take(grid ? nnodes * 8 : 0);            if (P) P->thr = reinterpret_cast<unsigned long long*>(p);
+  p = take(grid ? nnodes * 8 : 0);            if (P) P->prefix = reinterpret_cast<unsigned long long*>(p);
+  p = take(grid ? nnodes * 4 : 0);            if (P) P->need = reinterpret_cast<uint32_t*>(p);
+  p = take(grid ? nnodes * 4 : 0);            if (P) P->active = reinterpret_cast<int32_t*>(p);
+  p = take(24 * 4);                           if (P) P->flags = reinterpret_cast<int32_t*>(p);
+  p = take(sizeof(GridBarrier));              if (P) P->bar = reinterpret_cast<GridBarrier*>(p);
+  return off;
+}
+
 }  // namespace lsa
 
 extern "C" {
@@ -673,9 +697,50 @@ int lsa_sparse_attn_sw_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, 
   return ok();
 }
 
+static int assign_checks(int64_t nseg, int64_t m, int32_t b) {
+  if (nseg < 1 || m < 1) return fail(LSA_ERR_SHAPE, "need nseg >= 1 and m >= 1");
+  if (b < 2 || b > LSA_MAX_BRANCHING || m % b != 0)
+    return fail(LSA_ERR_SHAPE, "b must be in [2, 16] and divide m (b = %d, m = %lld)", b, (long long)m);
+  if (nseg * m >= (int64_t(1) << 31)) return fail(LSA_ERR_SHAPE, "nseg * m must stay below 2^31");
+  return LSA_OK;
+}
+
+int lsa_balanced_assign_workspace_bytes(int64_t nseg, int64_t m, int32_t b, size_t* bytes) {
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
+  int rc = assign_checks(nseg, m, b);
+  if (rc != LSA_OK) return rc;
+  *bytes = lsa::assign_workspace_layout(nseg, m, b, nullptr, nullptr);
+  return ok();
+}
+
+int lsa_balanced_assign(const float* Z, const float* mu, int64_t nseg, int64_t m, int32_t b, int32_t r,
+                        int32_t max_rounds, uint8_t* choice, void* workspace, size_t workspace_bytes,
+                        int32_t* status, void* stream) {
+  if (!Z || !mu || !choice) return fail(LSA_ERR_INVALID_ARG, "Z, mu and choice must be non-NULL");
+  int rc = assign_checks(nseg, m, b);
+  if (rc != LSA_OK) return rc;
+  if (r != 16 && r != 32 && r != 64) return fail(LSA_ERR_SHAPE, "r must be 16, 32 or 64 (got %d)", r);
+  if (max_rounds < 0) return fail(LSA_ERR_INVALID_ARG, "max_rounds must be >= 0 (0: the build's cap)");
+  const size_t need = lsa::assign_workspace_layout(nseg, m, b, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need)
+    return fail(LSA_ERR_WORKSPACE, "assignment needs %zu workspace bytes (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  lsa::BuildPlan P;
+  memset(&P, 0, sizeof(P));
+  lsa::assign_workspace_layout(nseg, m, b, static_cast<char*>(workspace), &P);
+  P.mu = const_cast<float*>(mu);
+  P.choice = choice;
+  P.coop_blocks = lsa::da_grid_blocks();
+  if (P.coop_blocks <= 0) return fail(LSA_ERR_CUDA, "cannot size the cooperative assignment grid");
+  cudaError_t e = lsa::run_assign(P, Z, nseg, m, b, r, max_rounds ? max_rounds : lsa::kMaxRounds, status,
+                                  static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_balanced_assign");
+  return ok();
+}
+
 int lsa_project_keys(const void* K, int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype, const void* W,
                      int32_t r, int64_t n, float* Z, int32_t* status, void* stream) {
-  if (!K || !W || !Z) return fail(LSA_ERR_INVALID_ARG, "K, W and Z must be non-NULL");
+  if (!K || !W || (!Z && n > 0)) return fail(LSA_ERR_INVALID_ARG, "K, W and Z must be non-NULL");
   if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
   if (n_heads < 1 || (d != 64 && d != 128) || (r != 16 && r != 32 && r != 64))
     return fail(LSA_ERR_SHAPE, "need n_heads >= 1, d in {64, 128} and r in {16, 32, 64}");

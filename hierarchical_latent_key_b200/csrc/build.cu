@@ -736,6 +736,48 @@ __global__ void k_expand_leaves(const int32_t* __restrict__ blocks, int64_t nslo
 // ---------------------------------------------------------------------------
 // host driver
 // ---------------------------------------------------------------------------
+// One balanced assignment of every segment: distances and preference lists
+// (k_dist_pref), then deferred acceptance, one CTA per segment up to kCtaMaxSeg
+// keys, else the cooperative grid kernel.  Writes P.choice [nslots].  A segment
+// still moving after max_rounds proposal rounds sets LSA_ERR_TIMEOUT.
+template <int R>
+static cudaError_t assign_round(const BuildPlan& P, const float* Za, int64_t nslots, int64_t m, int b,
+                                int max_rounds, int32_t* status, cudaStream_t st) {
+  const int64_t nseg = nslots / m, cap = m / b, nnodes = nseg * b;
+  cudaError_t e;
+  {
+    // centroids of every segment a CTA's 256 slots touch: (256 / m + 1) * b rows,
+    // at most (256 + b) * R floats (about 70 KB) when a segment holds b members
+    const int64_t rows = (ceil_div(256, m) + 1) * b;
+    const size_t smem = (size_t)rows * R * sizeof(float);
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(k_dist_pref<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    k_dist_pref<R><<<(unsigned)ceil_div(nslots, 256), 256, smem, st>>>(Za, P.mu, nslots, m, b, P.D, P.pref,
+                                                                      P.choice, P.ptr, P.dbits, status);
+  }
+  if (m <= kCtaMaxSeg) {
+    const int kpt = m <= 1024 ? 1 : m <= 2048 ? 2 : m <= 4096 ? 4 : 8;
+    const int nt = (int)((ceil_div(ceil_div(m, kpt), 32)) * 32);
+    switch (kpt) {
+      case 1: k_da_cta<1><<<(unsigned)nseg, nt, 0, st>>>(P.pref, P.D, P.choice, m, b, cap, max_rounds, status); break;
+      case 2: k_da_cta<2><<<(unsigned)nseg, nt, 0, st>>>(P.pref, P.D, P.choice, m, b, cap, max_rounds, status); break;
+      case 4: k_da_cta<4><<<(unsigned)nseg, nt, 0, st>>>(P.pref, P.D, P.choice, m, b, cap, max_rounds, status); break;
+      default: k_da_cta<8><<<(unsigned)nseg, nt, 0, st>>>(P.pref, P.D, P.choice, m, b, cap, max_rounds, status); break;
+    }
+    return cudaGetLastError();
+  }
+  DaGridArgs a;
+  a.pref = P.pref; a.D = P.D; a.choice = P.choice; a.ptr = P.ptr; a.dbits = P.dbits;
+  a.hist = P.hist; a.thr = P.thr; a.prefix = P.prefix; a.need = P.need; a.active = P.active;
+  a.flags = P.flags; a.bar = P.bar; a.nslots = nslots; a.m = m; a.cap = cap; a.nsegc = nnodes;
+  a.b = b; a.max_rounds = max_rounds; a.status = status;
+  if ((e = cudaMemsetAsync(P.hist, 0, (size_t)nnodes * 2048 * sizeof(uint32_t), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(P.flags, 0, 24 * sizeof(int32_t), st)) != cudaSuccess) return e;
+  if ((e = cudaMemsetAsync(P.bar, 0, sizeof(GridBarrier), st)) != cudaSuccess) return e;
+  void* args[] = {&a};
+  return cudaLaunchCooperativeKernel((const void*)k_da_grid, dim3(P.coop_blocks), dim3(512), args, 0, st);
+}
+
 template <int R>
 static cudaError_t build_levels(const BuildPlan& P, const lsa_tree_desc& t, char* tree_mem, int32_t* trace,
                                 int32_t* status, int32_t pool, cudaStream_t st) {
@@ -757,38 +799,7 @@ static cudaError_t build_levels(const BuildPlan& P, const lsa_tree_desc& t, char
     const int64_t nnodes = nseg * b;
     const int64_t cpn = ceil_div(cap, kMeanChunk);
     for (int it = 0; it < P.iters; ++it) {
-      {
-        // centroids of every segment a CTA's 256 slots touch: (256 / m + 1) * b rows,
-        // at most (256 + b) * R floats (about 70 KB) when a segment holds b members
-        const int64_t rows = (ceil_div(256, m) + 1) * b;
-        const size_t smem = (size_t)rows * R * sizeof(float);
-        if (smem > 48 * 1024)
-          cudaFuncSetAttribute(k_dist_pref<R>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        k_dist_pref<R><<<(unsigned)ceil_div(nslots, 256), 256, smem, st>>>(Za, P.mu, nslots, m, b, P.D, P.pref,
-                                                                          P.choice, P.ptr, P.dbits, status);
-      }
-      if (m <= kCtaMaxSeg) {
-        const int kpt = m <= 1024 ? 1 : m <= 2048 ? 2 : m <= 4096 ? 4 : 8;
-        const int nt = (int)((ceil_div(ceil_div(m, kpt), 32)) * 32);
-        switch (kpt) {
-          case 1: k_da_cta<1><<<(unsigned)nseg, nt, 0, st>>>(P.pref, P.D, P.choice, m, b, cap, kMaxRounds, status); break;
-          case 2: k_da_cta<2><<<(unsigned)nseg, nt, 0, st>>>(P.pref, P.D, P.choice, m, b, cap, kMaxRounds, status); break;
-          case 4: k_da_cta<4><<<(unsigned)nseg, nt, 0, st>>>(P.pref, P.D, P.choice, m, b, cap, kMaxRounds, status); break;
-          default: k_da_cta<8><<<(unsigned)nseg, nt, 0, st>>>(P.pref, P.D, P.choice, m, b, cap, kMaxRounds, status); break;
-        }
-      } else {
-        DaGridArgs a;
-        a.pref = P.pref; a.D = P.D; a.choice = P.choice; a.ptr = P.ptr; a.dbits = P.dbits;
-        a.hist = P.hist; a.thr = P.thr; a.prefix = P.prefix; a.need = P.need; a.active = P.active;
-        a.flags = P.flags; a.bar = P.bar; a.nslots = nslots; a.m = m; a.cap = cap; a.nsegc = nnodes;
-        a.b = b; a.max_rounds = kMaxRounds; a.status = status;
-        if ((e = cudaMemsetAsync(P.hist, 0, (size_t)nnodes * 2048 * sizeof(uint32_t), st)) != cudaSuccess) return e;
-        if ((e = cudaMemsetAsync(P.flags, 0, 24 * sizeof(int32_t), st)) != cudaSuccess) return e;
-        if ((e = cudaMemsetAsync(P.bar, 0, sizeof(GridBarrier), st)) != cudaSuccess) return e;
-        void* args[] = {&a};
-        e = cudaLaunchCooperativeKernel((const void*)k_da_grid, dim3(P.coop_blocks), dim3(512), args, 0, st);
-        if (e != cudaSuccess) return e;
-      }
+      if ((e = assign_round<R>(P, Za, nslots, m, b, kMaxRounds, status, st)) != cudaSuccess) return e;
       k_part_count<<<(unsigned)ntiles, kTile, 0, st>>>(P.choice, m, tps, b, P.tcnt);
       k_part_scan<<<(unsigned)nseg, 32, 0, st>>>(P.tcnt, tps, b, cap, P.toff);
       k_part_scatter<<<(unsigned)ntiles, kTile, 0, st>>>(P.choice, m, tps, b, cap, P.toff, P.order, status);
@@ -845,6 +856,16 @@ static cudaError_t project(const void* K, int64_t n_cap, const void* W, int64_t 
   LSA_PROJ(16, 64) LSA_PROJ(32, 64) LSA_PROJ(64, 64) LSA_PROJ(16, 128) LSA_PROJ(32, 128) LSA_PROJ(64, 128)
 #undef LSA_PROJ
   return cudaErrorInvalidValue;
+}
+
+cudaError_t run_assign(const BuildPlan& P, const float* Z, int64_t nseg, int64_t m, int b, int r, int max_rounds,
+                       int32_t* status, cudaStream_t st) {
+  const int64_t nslots = nseg * m;
+  switch (r) {
+    case 16: return assign_round<16>(P, Z, nslots, m, b, max_rounds, status, st);
+    case 32: return assign_round<32>(P, Z, nslots, m, b, max_rounds, status, st);
+    default: return assign_round<64>(P, Z, nslots, m, b, max_rounds, status, st);
+  }
 }
 
 cudaError_t run_project(const void* K, int64_t n_cap, const void* W, int64_t n, int32_t n_heads, int r, int d,

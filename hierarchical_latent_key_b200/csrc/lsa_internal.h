@@ -56,6 +56,14 @@ struct BuildPlan {
 // query and the carving of a caller buffer).
 size_t build_workspace_layout(const lsa_tree_desc& t, char* base, BuildPlan* plan);
 
+// One balanced assignment (distances, preference lists, deferred acceptance) of
+// nseg segments of m latent rows Z [nseg*m][r] to the b centroids of their segment
+// (P.mu [nseg*b][r]); the result goes to P.choice.  P needs D, pref, dbits, ptr and,
+// for m > kCtaMaxSeg, the grid fields.
+cudaError_t run_assign(const BuildPlan& P, const float* Z, int64_t nseg, int64_t m, int b, int r, int max_rounds,
+                       int32_t* status, cudaStream_t st);
+size_t assign_workspace_layout(int64_t nseg, int64_t m, int b, char* base, BuildPlan* P);
+
 // Latent projection of keys on the tensor cores (bf16, r in {16, 32, 64}, d in {64, 128}):
 // Z[h][i] = K[h][i] . W[h] and pos[h][i] = i for i < n.
 // run_project picks the tensor-core kernel where supported, fp32 FMAs otherwise.

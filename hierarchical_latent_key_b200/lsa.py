@@ -83,6 +83,8 @@ def _load():
                                                   i32, i64, i64, f32, P, P, P, P, sz, P, P]),
         "lsa_kv_append": (ctypes.c_int, [P, P, i32, i64, i32, i32, i64, P, P, P]),
         "lsa_project_keys": (ctypes.c_int, [P, i32, i64, i32, i32, P, i32, i64, P, P, P]),
+        "lsa_balanced_assign_workspace_bytes": (ctypes.c_int, [i64, i64, i32, ctypes.POINTER(sz)]),
+        "lsa_balanced_assign": (ctypes.c_int, [P, P, i64, i64, i32, i32, i32, P, P, sz, P, P]),
         "lsa_tree_attn_bwd_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
         "lsa_tree_attn_bwd": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, P, P, P, i32, P, i32, f32,
                                              P, P, P, P, sz, P, P]),
@@ -285,6 +287,31 @@ def lsa_project_keys(K, W, n, Z, status=None, stream=None):
     """K: [n_heads, n_cap, d]; W: [n_heads, d, r]; Z: [n_heads, n, r] fp32 (written)."""
     _raise(_lib.lsa_project_keys(_ptr(K), K.shape[0], K.shape[1], K.shape[2], _dtype(K), _ptr(W), W.shape[2],
                                  int(n), _ptr(Z), _ptr(status), _stream(stream, K)), "lsa_project_keys")
+
+
+def lsa_balanced_assign_workspace_bytes(nseg, m, b) -> int:
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_balanced_assign_workspace_bytes(int(nseg), int(m), int(b), ctypes.byref(n)),
+           "lsa_balanced_assign_workspace_bytes")
+    return n.value
+
+
+def lsa_balanced_assign(Z, mu, nseg, m, b, max_rounds, choice, workspace, status=None, stream=None):
+    """Z: [nseg*m, r] fp32; mu: [nseg*b, r] fp32; choice: [nseg*m] uint8 (written)."""
+    _raise(_lib.lsa_balanced_assign(_ptr(Z), _ptr(mu), int(nseg), int(m), int(b), Z.shape[1], int(max_rounds),
+                                    _ptr(choice), _ptr(workspace), workspace.numel(), _ptr(status),
+                                    _stream(stream, Z)), "lsa_balanced_assign")
+
+
+def balanced_assign(Z, mu, nseg, m, b, max_rounds=0, status=None, check=True):
+    """Centroid index (uint8) of every row of every segment; see lsa_balanced_assign."""
+    choice = torch.empty(nseg * m, dtype=torch.uint8, device=Z.device)
+    ws = torch.empty(lsa_balanced_assign_workspace_bytes(nseg, m, b), dtype=torch.uint8, device=Z.device)
+    st = _new_status(Z.device) if status is None else status
+    lsa_balanced_assign(Z, mu, nseg, m, b, max_rounds, choice, ws, st)
+    if check:
+        check_status(st, "lsa_balanced_assign")
+    return choice
 
 
 def project_keys(K, W, n=None):

@@ -392,13 +392,34 @@ int lsa_sparse_attn_noalloc(const void *Q, int32_t T, int32_t Hq, const void *K,
                             int64_t tail_begin, int64_t tail_end, float scale, void *O, float *LSE,
                             int32_t *status, void *stream);
 
+/* One balanced k-means assignment step of the build (kongchang.com, "How LSA
+ * Sidesteps Per-Key Scoring with Hierarchical Clustering": the tree is built like
+ * hierarchical k-means), exposed on its own.  Segment s holds the m latent rows
+ * Z[s*m .. s*m + m) (fp32, [nseg*m][r], device) and the b centroids
+ * mu[s*b .. s*b + b) ([nseg*b][r], device).  Each row goes to one of its segment's
+ * centroids, exactly m/b rows per centroid, by the unique stable assignment under
+ * the order (squared distance asc, row index in the segment asc, centroid asc).
+ * choice [nseg*m] uint8 (device) receives the centroid index of every row.
+ * Rows are identified by their index inside the segment.
+ *  b in [2, 16] dividing m; r in {16, 32, 64}; nseg * m < 2^31.
+ *  max_rounds: cap on the proposal rounds of the parallel deferred acceptance
+ *  (0 = the cap the build uses, 4096).  A segment whose assignment is still
+ *  changing when the cap is reached leaves choice balanced or not and sets
+ *  LSA_ERR_TIMEOUT in *status; the kernels return normally either way.  NaN
+ *  distances set LSA_ERR_NONFINITE.
+ *  workspace: lsa_balanced_assign_workspace_bytes(nseg, m, b) bytes (device). */
+int lsa_balanced_assign_workspace_bytes(int64_t nseg, int64_t m, int32_t b, size_t *bytes);
+int lsa_balanced_assign(const float *Z, const float *mu, int64_t nseg, int64_t m, int32_t b, int32_t r,
+                        int32_t max_rounds, uint8_t *choice, void *workspace, size_t workspace_bytes,
+                        int32_t *status, void *stream);
+
 /* Latent projection of the keys (kongchang.com, "Latent Sparse Attention Breaks
  * Through the Million-Token Context Bottleneck", section "How LSA Sidesteps
  * Per-Key Scoring with Hierarchical Clustering": keys are first mapped into a
  * low-dimensional latent space).  The first step of lsa_build_tree, exposed on
  * its own:  Z[h][i][c] = sum_j K[h][i][j] * W[h][j][c]  for i < n.
  *  K : [n_heads][n_cap][d] (dtype), device;  W : [n_heads][d][r] (dtype), device;
- *  Z : [n_heads][n][r] fp32, device, overwritten.
+ *  Z : [n_heads][n][r] fp32, device, overwritten (may be NULL when n = 0).
  *  d in {64, 128}, r in {16, 32, 64}, 0 <= n <= n_cap.  bf16 inputs run on the
  *  tensor cores (exact products, fp32 sums); fp32 inputs use fp32 FMAs.  An MMA
  *  that does not complete within a second sets LSA_ERR_TIMEOUT in *status (may be

@@ -189,3 +189,17 @@ def test_project_keys_rejects(lsa):
     assert L.lsa_project_keys(P, 2, 100, 128, 1, P, 48, 10, P, None, None) == lsa.LSA_ERR_SHAPE
     assert L.lsa_project_keys(P, 2, 100, 128, 1, P, 64, 101, P, None, None) == lsa.LSA_ERR_SHAPE
     assert L.lsa_project_keys(P, 0, 100, 128, 1, P, 64, 10, P, None, None) == lsa.LSA_ERR_SHAPE
+
+
+def test_balanced_assign_rejects(lsa):
+    L = lsa._lib
+    P = ctypes.c_void_p(16)
+    n = ctypes.c_size_t()
+    assert L.lsa_balanced_assign_workspace_bytes(4, 64, 4, ctypes.byref(n)) == lsa.LSA_OK and n.value > 0
+    assert L.lsa_balanced_assign_workspace_bytes(4, 66, 4, ctypes.byref(n)) == lsa.LSA_ERR_SHAPE
+    assert L.lsa_balanced_assign_workspace_bytes(4, 64, 17, ctypes.byref(n)) == lsa.LSA_ERR_SHAPE
+    assert L.lsa_balanced_assign_workspace_bytes(0, 64, 4, ctypes.byref(n)) == lsa.LSA_ERR_SHAPE
+    assert L.lsa_balanced_assign(P, P, 4, 64, 4, 48, 0, P, P, 1 << 20, None, None) == lsa.LSA_ERR_SHAPE
+    assert L.lsa_balanced_assign(P, P, 4, 64, 4, 64, -1, P, P, 1 << 20, None, None) == lsa.LSA_ERR_INVALID_ARG
+    assert L.lsa_balanced_assign(None, P, 4, 64, 4, 64, 0, P, P, 1 << 20, None, None) == lsa.LSA_ERR_INVALID_ARG
+    assert L.lsa_balanced_assign(P, P, 4, 64, 4, 64, 0, P, P, 16, None, None) == lsa.LSA_ERR_WORKSPACE
