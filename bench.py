@@ -178,7 +178,8 @@ class Prefill:
 class Decode:
     """Single-request decode: step s appends one key and one value row per KV head at
     position n + s, selects for the new token and attends to the selection plus the dense
-    tail of appended rows [n, n + s] (causal by position)."""
+    tail of appended rows [n, n + s] (causal by position), all in one lsa_decode_step call
+    (two kernel launches)."""
 
     def __init__(self, cfg, dev, seed, steps):
         from hierarchical_latent_key_b200 import lsa
@@ -188,34 +189,24 @@ class Decode:
         self.K, self.V, self.W, self.Q, self.q_pos = c.K, c.V, c.W, c.Q, c.q_pos
         del c
         n = cfg.n
-        self.Knew = self.K[:, n:].transpose(0, 1).contiguous()   # [steps, Hkv, d]: rows the steps append
-        self.Vnew = self.V[:, n:].transpose(0, 1).contiguous()
+        self.Knew = self.K[:, n:].transpose(0, 1).clone(memory_format=torch.contiguous_format)   # [steps, Hkv, d]: rows the steps append
+        self.Vnew = self.V[:, n:].transpose(0, 1).clone(memory_format=torch.contiguous_format)
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
         self.tree = lsa.build_tree(self.K, self.W, cfg.branching, cfg.leaf, cfg.iters, seed)
         torch.cuda.synchronize(dev)
         self.build_ms = 1e3 * (time.perf_counter() - t0)
         _, Hq, d = self.Q.shape
-        self.idx = torch.empty(cfg.Hkv, 1, cfg.K_sel, dtype=torch.int32, device=dev)
-        self.O = torch.empty(1, Hq, d, dtype=self.Q.dtype, device=dev)
-        self.LSE = torch.empty(1, Hq, dtype=torch.float32, device=dev)
-        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
-        need = lsa.lsa_attn_workspace_bytes(1, Hq, cfg.Hkv, d, cfg.K_sel, steps)
-        self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
-        self.scale = 1.0 / math.sqrt(d)
-        self.launches_per_step = 1 + 1 + 1 + (1 if need else 0)
+        self.dec = lsa.DecodeStep(self.tree, self.W, cfg.beam, self.K, Hq, steps)
+        self.O, self.LSE, self.status = self.dec.O, self.dec.LSE, self.dec.status
+        self.launches_per_step = 2      # select (with the append), attention (with the split merge)
 
-    def append(self, s):
-        self.lsa.lsa_kv_append(self.K, self.V, self.cfg.n + s, self.Knew[s], self.Vnew[s])
-
-    def step(self, s):
-        self.append(s)
-        self.select(s)
-        self.attend(s)
+    def step(self, s, Q=None):
+        n = self.cfg.n
+        self.dec.step(self.K, self.V, self.Q[s:s + 1] if Q is None else Q, self.Knew[s], self.Vnew[s], n + s, n)
 
     def capture(self, steps):
-        """One CUDA graph per decode step (append, select, attention): a step is then
-        one launch, so host launch latency does not separate its kernels."""
+        """One CUDA graph per decode step: a step is then one graph launch."""
         self.graphs = []
         for s in range(steps):
             g = torch.cuda.CUDAGraph()
@@ -224,31 +215,20 @@ class Decode:
             self.graphs.append(g)
         torch.cuda.synchronize()
 
-    def select(self, s, Q=None):
-        self.lsa.lsa_select(self.tree.desc, self.tree.mem, self.Q[s:s + 1] if Q is None else Q, self.W,
-                            self.cfg.beam, self.q_pos[s:s + 1], self.idx, status=self.status)
-
-    def attend(self, s, Q=None):
-        n = self.cfg.n
-        self.lsa.lsa_sparse_attn(self.Q[s:s + 1] if Q is None else Q, self.K, self.V, self.idx,
-                                 self.q_pos[s:s + 1], True, n, n + s + 1, self.scale, self.O, self.LSE, self.ws,
-                                 self.status)
-
     def bytes_per_step(self, s):
         """Algorithmic bytes of one step: gathered K/V rows of the selection and the tail,
-        centroid rows scored, projection, query/output, key lists."""
+        centroid rows scored, projection, query/output, leaf lists and the appended rows."""
         cfg, d = self.cfg, self.Q.shape[2]
         esz = self.Q.element_size()
         attn = cfg.Hkv * (cfg.K_sel + s + 1) * 2 * d * esz + 2 * cfg.Hq * d * esz + cfg.Hkv * cfg.K_sel * 4
         cand = cfg.nodes[0] + sum(cfg.beam[l - 1] * cfg.branching[l] for l in range(1, len(cfg.branching)))
         sel = (cfg.Hkv * cand * (cfg.r * 4 + 4) + cfg.Hkv * d * cfg.r * esz + cfg.Hq * d * esz
-               + 2 * cfg.Hkv * cfg.K_sel * 4)
+               + 2 * cfg.Hkv * d * esz)
         return attn, sel
 
 
 def time_decode(w, steps, warmup, flush, stream):
-    """Per step: one graph replay (append + select + attention), L2 flushed between
-    steps; a second pass with events between the kernels gives the breakdown."""
+    """Per step: one graph replay (append + select + attention), L2 flushed between steps."""
     for s in range(warmup):
         w.graphs[s].replay()
     torch.cuda.synchronize()
@@ -259,24 +239,7 @@ def time_decode(w, steps, warmup, flush, stream):
         w.graphs[warmup + k].replay()
         ev[k][1].record(stream)
     torch.cuda.synchronize()
-    total = [ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)]
-    # breakdown (eager launches, host gaps included): append / select / attention
-    parts = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(8)]
-    for k in range(8):
-        s = warmup + k
-        flush.zero_()
-        torch.cuda.synchronize()
-        parts[k][0].record(stream)
-        w.append(s)
-        parts[k][1].record(stream)
-        w.select(s)
-        parts[k][2].record(stream)
-        w.attend(s)
-        parts[k][3].record(stream)
-    torch.cuda.synchronize()
-    br = {name: statistics.median(parts[k][i].elapsed_time(parts[k][i + 1]) for k in range(8)) * 1e3
-          for i, name in enumerate(("append", "select", "attention"))}
-    return total, br
+    return [ev[k][0].elapsed_time(ev[k][1]) for k in range(steps)]
 
 
 def time_decode_e2e(w, steps, warmup, flush, stream):
@@ -389,6 +352,11 @@ def run_train(args, dev, rank, world, reduce_max, steps=3, warmup=2):
            "forward_tflops": flops_fwd / (br["forward"] / 1e3) / 1e12,
            "backward_tflops": 2.5 * flops_fwd / (br["backward"] / 1e3) / 1e12,
            "gpu_launches_per_step": None}
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            out["cpu_baseline"] = cpu_baseline_train(w)
+        except Exception as e:  # noqa: BLE001
+            out["cpu_baseline"] = {"error": f"{type(e).__name__}: {e}"}
     del w
     torch.cuda.empty_cache()
     return out
@@ -448,7 +416,7 @@ def run_decode(args, dev, rank, world, reduce_max):
     stream = torch.cuda.current_stream(dev)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     w.capture(warmup + steps)
-    total, br = time_decode(w, steps, warmup, flush, stream)
+    total = time_decode(w, steps, warmup, flush, stream)
     code = w.lsa.lsa_status_check(w.status)
     if code != 0:
         raise RuntimeError(f"kernel status {code}: {w.lsa.lsa_strerror(code)}")
@@ -459,7 +427,6 @@ def run_decode(args, dev, rank, world, reduce_max):
     peaks = measured_peaks()
     att_b = statistics.mean(w.bytes_per_step(warmup + k)[0] for k in range(steps))
     sel_b = w.bytes_per_step(0)[1]
-    a_s, s_s = br["attention"] / 1e6, br["select"] / 1e6
     step_s = total_s / steps
     out = {
         "value": value, "unit": "queries/s", "steps": steps, "ms_per_step": 1e3 * t_max / steps,
@@ -468,21 +435,22 @@ def run_decode(args, dev, rank, world, reduce_max):
                                f"{cfg.leaf}, beam {'/'.join(map(str, cfg.beam))} ({cfg.K_sel} keys) + dense tail "
                                f"of appended keys", "seq_len": cfg.n,
                    "l2": "flushed between timed steps (512 MiB write outside the events)"},
-        "breakdown_us": {"step_graph": 1e3 * statistics.mean(total), "eager_append": br["append"],
-                         "eager_select": br["select"], "eager_attention": br["attention"],
+        "breakdown_us": {"step_graph": 1e3 * statistics.mean(total), "step_graph_min": 1e3 * min(total),
                          "build_once_ms": w.build_ms},
         "e2e": {"value": e2e_value, "unit": "queries/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "roofline": {"bound": "hbm", "unit": "GB/s", "peak": peaks["hbm_gbs"], "peak_source": peaks["source"],
-                     "step": {"achieved": (att_b + sel_b) / step_s / 1e9,
-                              "frac": (att_b + sel_b) / step_s / 1e9 / peaks["hbm_gbs"],
-                              "algorithmic_bytes": att_b + sel_b},
-                     "k_attn_fwd": {"achieved": att_b / a_s / 1e9, "frac": att_b / a_s / 1e9 / peaks["hbm_gbs"],
-                                    "algorithmic_bytes": att_b},
-                     "k_select": {"achieved": sel_b / s_s / 1e9, "frac": sel_b / s_s / 1e9 / peaks["hbm_gbs"],
-                                  "algorithmic_bytes": sel_b}, "traffic": None},
+                     "achieved": (att_b + sel_b) / step_s / 1e9,
+                     "frac": (att_b + sel_b) / step_s / 1e9 / peaks["hbm_gbs"],
+                     "algorithmic_bytes": att_b + sel_b, "traffic": None,
+                     "kernels": "k_select_wide (append, 5-level walk) + k_dec_attn (gather, split merge)"},
         "gpu_launches": w.launches_per_step * steps,
-        "cuda_graph": "one graph per decode step (append, select, attention)",
+        "cuda_graph": "one graph per decode step (lsa_decode_step: select with the append, attention)",
     }
+    if rank == 0 and not args.no_cpu_baseline:
+        try:
+            out["cpu_baseline"] = cpu_baseline_decode(w)
+        except Exception as e:  # noqa: BLE001
+            out["cpu_baseline"] = {"error": f"{type(e).__name__}: {e}"}
     w.graphs = None
     del w
     torch.cuda.empty_cache()
@@ -718,9 +686,150 @@ def cpu_baseline_prefill(w, n_queries=4096):
     orc.attn_fwd(Qg, Kh, Vh, idx, q_pos=qp, causal=True)
     dt = time.perf_counter() - t0
     qps = n_queries / (dt * cfg.Hkv)
+    # single core: 64 of the queries in a one-thread child process (walk on the oracle, attention over
+    # each query's visible selected keys, gathered from the GPU's selection)
+    rows = np.arange(cfg.T - 64, cfg.T)
+    kc, vc = [], []
+    for t in rows:
+        lv = w.leaves[h][t]
+        kk = w.tree.leaf_index()[h].view(-1, cfg.leaf)[lv[lv >= 0].long()].reshape(-1)
+        kk = kk[kk <= w.q_pos[t]].long()
+        kc.append(w.K[h, kk].double().cpu().numpy())
+        vc.append(w.V[h, kk].double().cpu().numpy())
+    L = len(cfg.branching)
+    one = _single_core("prefill", dict(
+        branching=np.asarray(cfg.branching, np.int32), leaf=np.int64(cfg.leaf),
+        cents=[w.tree.centroids(l)[h].double().cpu().numpy() for l in range(L)],
+        mpos=[w.tree.min_pos(l)[h].cpu().numpy() for l in range(L)], leaf_index=w.tree.leaf_index()[h].cpu().numpy(),
+        W=Wh.double().numpy(), beam=np.asarray(cfg.beam), q_pos=w.q_pos[rows].cpu().numpy(),
+        Qg=w.Q[rows, h * cfg.G:(h + 1) * cfg.G].double().cpu().numpy(), Kc=kc, Vc=vc))
     return {"value": qps, "unit": "queries/s", "cores": cores_used(), "kind": "oracle",
+            "single_core_value": 64 / (one * cfg.Hkv),
             "sample": f"{n_queries} of {cfg.T} chunk queries on KV head 0 of {cfg.Hkv} (select + attention, "
-                      f"float64 C oracle, OpenMP), scaled x{cfg.Hkv} heads; index built on the GPU"}
+                      f"float64 C oracle, OpenMP), scaled x{cfg.Hkv} heads; index built on the GPU; "
+                      f"single_core_value: the last 64 queries with one OpenMP thread (walk on the oracle, attention "
+                      f"over each query's visible keys of the GPU's selection)"}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing on the host (the cpu_baseline entries)
+# ---------------------------------------------------------------------------
+
+def _oracle_sample(kind, arrays):
+    """Run one oracle sample in this process; returns seconds of oracle work."""
+    from oracle import oracle as orc
+    t0 = time.perf_counter()
+    if kind == "prefill":
+        tree = orc.Tree.from_levels(arrays["branching"], int(arrays["leaf"]), arrays["cents"], arrays["mpos"],
+                                    arrays["leaf_index"])
+        qlat = orc.query_latent(arrays["Qg"], arrays["W"])
+        orc.select(qlat, tree, arrays["beam"], q_pos=arrays["q_pos"])
+        for t in range(arrays["Qg"].shape[0]):
+            Kc, Vc = arrays["Kc"][t], arrays["Vc"][t]
+            orc.attn_fwd(arrays["Qg"][t:t + 1], Kc, Vc, np.zeros((1, 0), np.int32), tail=(0, Kc.shape[0]))
+    elif kind == "decode":
+        tree = orc.Tree.from_levels(arrays["branching"], int(arrays["leaf"]), arrays["cents"], arrays["mpos"],
+                                    arrays["leaf_index"])
+        for s in range(arrays["Qg"].shape[0]):
+            qlat = orc.query_latent(arrays["Qg"][s:s + 1], arrays["W"])
+            orc.select(qlat, tree, arrays["beam"])
+            Kc, Vc = arrays["Kc"][s], arrays["Vc"][s]
+            orc.attn_fwd(arrays["Qg"][s:s + 1], Kc, Vc, np.zeros((1, 0), np.int32), tail=(0, Kc.shape[0]))
+    elif kind == "train":
+        qp = arrays["q_pos"]
+        O, LSE = orc.attn_fwd(arrays["Qg"], arrays["K"], arrays["V"], arrays["idx"], q_pos=qp, causal=True)
+        orc.attn_bwd(arrays["Qg"], arrays["K"], arrays["V"], arrays["idx"], arrays["dO"], q_pos=qp, causal=True)
+    else:
+        raise ValueError(kind)
+    return time.perf_counter() - t0
+
+
+def _single_core(kind, arrays):
+    """The same oracle sample in a child process limited to one OpenMP thread."""
+    import subprocess
+    import tempfile
+    with tempfile.TemporaryDirectory() as d:
+        path = os.path.join(d, "sample.npz")
+        packed = {}
+        for k, v in arrays.items():
+            if isinstance(v, list):
+                obj = np.empty(len(v), dtype=object)
+                for i, x in enumerate(v):
+                    obj[i] = x
+                v = obj
+            packed[k] = v
+        np.savez(path, **packed)
+        code = ("import sys, json; sys.path.insert(0, %r); import numpy as np, bench; "
+                "z = np.load(%r, allow_pickle=True); a = {k: (list(z[k]) if z[k].dtype == object else z[k]) "
+                "for k in z.files}; print(json.dumps(bench._oracle_sample(%r, a)))") % (ROOT, path, kind)
+        env = dict(os.environ, OMP_NUM_THREADS="1", CUDA_VISIBLE_DEVICES="")
+        r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=900)
+        if r.returncode != 0:
+            raise RuntimeError(r.stderr[-500:])
+        return float(r.stdout.strip().splitlines()[-1])
+
+
+def cpu_baseline_decode(w, n_steps=8):
+    """The oracle per decode step on KV head 0 (of 8): group latent, the beam walk over the
+    index the GPU built (exported to float64), attention over the kept leaves' keys and the
+    tail (rows gathered on the device first); scaled x8 heads."""
+    cfg = w.cfg
+    h = 0
+    L = len(cfg.branching)
+    n = cfg.n
+    li = w.tree.leaf_index()[h]
+    qg, kcs, vcs = [], [], []
+    for s in range(n_steps):
+        keys = torch.cat([li.view(-1, cfg.leaf)[w.dec.leaves[h][w.dec.leaves[h] >= 0].long()].reshape(-1),
+                          torch.arange(n, n + s + 1, device=li.device, dtype=li.dtype)]).long()
+        kcs.append(w.K[h, keys].double().cpu().numpy())
+        vcs.append(w.V[h, keys].double().cpu().numpy())
+        qg.append(w.Q[s, h * cfg.G:(h + 1) * cfg.G].double().cpu().numpy())
+    arrays = dict(branching=np.asarray(cfg.branching, np.int32), leaf=np.int64(cfg.leaf),
+                  cents=[w.tree.centroids(l)[h].double().cpu().numpy() for l in range(L)],
+                  mpos=[w.tree.min_pos(l)[h].cpu().numpy() for l in range(L)],
+                  leaf_index=li.cpu().numpy(), W=w.W[h].double().cpu().numpy(), beam=np.asarray(cfg.beam),
+                  Qg=np.stack(qg), Kc=kcs, Vc=vcs)
+    dt = _oracle_sample("decode", arrays)
+    one = _single_core("decode", arrays)
+    return {"value": n_steps / (dt * cfg.Hkv), "unit": "queries/s", "cores": cores_used(), "kind": "oracle",
+            "single_core_value": n_steps / (one * cfg.Hkv),
+            "sample": f"{n_steps} decode steps on KV head 0 of {cfg.Hkv} (latent, beam walk over the GPU-built "
+                      f"index, attention over the kept leaves' keys + tail gathered on the device), float64 C "
+                      f"oracle, scaled x{cfg.Hkv} heads; single_core_value: the same with one OpenMP thread"}
+
+
+def cpu_baseline_train(w, n_queries=48):
+    """The oracle's forward + backward for a sample of queries on KV head 0 (of 4), over the
+    GPU's selection, extrapolated to the whole layer (all queries, all heads); the oracle's
+    own index build for one head is timed too and added once per head."""
+    from oracle import oracle as orc
+    cfg = w.cfg
+    h = 0
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.choice(cfg.T, n_queries, replace=False))
+    li = w.lsa.Tree(w.desc, w.tree_mem).leaf_index()[h].view(-1, cfg.leaf)
+    lv = w.leaves[h][torch.as_tensor(rows, device=w.leaves.device)].long()
+    idx = torch.where(lv[..., None] >= 0, li[lv.clamp(min=0)], -1).reshape(len(rows), -1).cpu().numpy()
+    arrays = dict(Qg=w.Q[rows][:, h * cfg.G:(h + 1) * cfg.G].double().cpu().numpy(),
+                  K=w.K[h].double().cpu().numpy(), V=w.V[h].double().cpu().numpy(), idx=idx,
+                  dO=w.dO[rows][:, h * cfg.G:(h + 1) * cfg.G].double().cpu().numpy(),
+                  q_pos=w.q_pos.cpu().numpy()[rows])
+    dt = _oracle_sample("train", arrays)
+    one = _single_core("train", dict(arrays, Qg=arrays["Qg"][:8], idx=idx[:8], dO=arrays["dO"][:8],
+                                     q_pos=arrays["q_pos"][:8]))
+    Z = orc.project(w.K[h, :cfg.n].cpu(), w.W[h].cpu())
+    t0 = time.perf_counter()
+    orc.build_tree(Z, cfg.branching, cfg.leaf, cfg.iters, cfg.seed)
+    build_s = time.perf_counter() - t0
+    per_q = dt / n_queries
+    total = cfg.Hkv * (build_s + per_q * cfg.T)
+    return {"value": cfg.T / total, "unit": "tokens/s", "cores": cores_used(), "kind": "oracle",
+            "extrapolated": True, "single_core_value": cfg.T / (cfg.Hkv * (one / 8) * cfg.T),
+            "sample": f"{n_queries} of {cfg.T} queries on KV head 0 of {cfg.Hkv}: forward + backward over the GPU's "
+                      f"selection ({per_q * 1e3:.1f} ms per query), plus the oracle's index build for one head "
+                      f"({build_s:.1f} s); extrapolated to all queries and heads; single_core_value: forward + "
+                      f"backward only (8 queries, one OpenMP thread), select and build excluded"}
 
 
 def bench_config(args):

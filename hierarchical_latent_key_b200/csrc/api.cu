@@ -294,6 +294,27 @@ int lsa_tree_append(const lsa_tree_desc* tree, const void* tree_mem, const lsa_t
   return ok();
 }
 
+// Beam checks shared by the select calls: fills a's per-level fields, returns
+// LSA_OK or the failure code (beam_max through *bmax).
+static int beam_checks(const lsa_tree_desc* tree, const int32_t* beam, lsa::SelectArgs& a, int* bmax) {
+  if (!beam) return fail(LSA_ERR_INVALID_ARG, "beam must be non-NULL");
+  int beam_max = 0;
+  for (int l = 0; l < tree->levels; ++l) {
+    const int64_t avail = l == 0 ? tree->nodes[0] : (int64_t)beam[l - 1] * tree->branching[l];
+    if (beam[l] < 1 || beam[l] > LSA_MAX_BEAM || beam[l] > avail ||
+        (l + 1 < tree->levels && (int64_t)beam[l] * tree->branching[l + 1] > 512))
+      return fail(LSA_ERR_SHAPE, "beam[%d] = %d must be in [1, min(64, %lld)]", l, beam[l], (long long)avail);
+    beam_max = beam[l] > beam_max ? beam[l] : beam_max;
+    a.beam[l] = beam[l];
+    a.branching[l] = tree->branching[l];
+    a.nodes[l] = tree->nodes[l];
+    a.off_c[l] = tree->off_centroids[l];
+    a.off_m[l] = tree->off_min_pos[l];
+  }
+  *bmax = beam_max;
+  return LSA_OK;
+}
+
 int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq, int32_t d,
                int32_t dtype, const void* W, const int32_t* beam, const int32_t* q_pos, int32_t* idx_out,
                int32_t* leaves_out, float* qlat_out, int32_t* beam_out, int32_t* status, void* stream) {
@@ -308,18 +329,7 @@ int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, i
   lsa::SelectArgs a;
   memset(&a, 0, sizeof(a));
   int beam_max = 0;
-  for (int l = 0; l < tree->levels; ++l) {
-    const int64_t avail = l == 0 ? tree->nodes[0] : (int64_t)beam[l - 1] * tree->branching[l];
-    if (beam[l] < 1 || beam[l] > LSA_MAX_BEAM || beam[l] > avail ||
-        (l + 1 < tree->levels && (int64_t)beam[l] * tree->branching[l + 1] > 512))
-      return fail(LSA_ERR_SHAPE, "beam[%d] = %d must be in [1, min(64, %lld)]", l, beam[l], (long long)avail);
-    beam_max = beam[l] > beam_max ? beam[l] : beam_max;
-    a.beam[l] = beam[l];
-    a.branching[l] = tree->branching[l];
-    a.nodes[l] = tree->nodes[l];
-    a.off_c[l] = tree->off_centroids[l];
-    a.off_m[l] = tree->off_min_pos[l];
-  }
+  if ((rc = beam_checks(tree, beam, a, &beam_max)) != LSA_OK) return rc;
   if (T == 0) return ok();
   if (!tree_mem || !Q || !W) return fail(LSA_ERR_INVALID_ARG, "tree_mem, Q and W must be non-NULL");
   if (!idx_out && !leaves_out) return fail(LSA_ERR_INVALID_ARG, "give idx_out, leaves_out or both");
@@ -694,6 +704,108 @@ int lsa_sparse_attn_sw_bwd(const void* Q, int32_t T, int32_t Hq, const void* K, 
     return cuda_fail(e, "lsa_sparse_attn_sw_bwd");
   e = lsa::run_attn_bwd(a, dtype, st);
   if (e != cudaSuccess) return cuda_fail(e, "lsa_sparse_attn_sw_bwd");
+  return ok();
+}
+
+static size_t decode_ws_layout(int64_t Hkv, int B, int G, int d, int nsplit, char* base, int32_t** leaves,
+                               int32_t** cnt, float** part) {
+  uint64_t off = 0;
+  auto take = [&](uint64_t bytes) {
+    uint64_t at = off;
+    off = align256(off + (bytes ? bytes : 1));
+    return base ? base + at : nullptr;
+  };
+  char* p = take((uint64_t)Hkv * B * 4);
+  if (leaves) *leaves = reinterpret_cast<int32_t*>(p);
+  p = take((uint64_t)Hkv * 4);
+  if (cnt) *cnt = reinterpret_cast<int32_t*>(p);
+  p = take((uint64_t)Hkv * nsplit * G * (d + 2) * 4);
+  if (part) *part = reinterpret_cast<float*>(p);
+  return off;
+}
+
+int lsa_decode_step_workspace_bytes(const lsa_tree_desc* tree, int32_t Hq, int32_t d, const int32_t* beam,
+                                    int64_t tail_len_max, size_t* bytes) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes is NULL");
+  lsa::SelectArgs a;
+  memset(&a, 0, sizeof(a));
+  int bmax = 0;
+  if ((rc = beam_checks(tree, beam, a, &bmax)) != LSA_OK) return rc;
+  if (Hq < tree->n_heads || Hq % tree->n_heads) return fail(LSA_ERR_SHAPE, "Hq must be a multiple of n_heads");
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  if (tail_len_max < 0) return fail(LSA_ERR_SHAPE, "tail_len_max must be >= 0");
+  const int B = beam[tree->levels - 1];
+  const int nsplit = lsa::dec_splits(B, tree->leaf_size, tail_len_max);
+  *bytes = decode_ws_layout(tree->n_heads, B, Hq / tree->n_heads, d, nsplit, nullptr, nullptr, nullptr, nullptr);
+  return ok();
+}
+
+int lsa_decode_step(const lsa_tree_desc* tree, const void* tree_mem, const void* W, const int32_t* beam, void* K,
+                    void* V, int64_t n_cap, int32_t d, int32_t dtype, const void* Q, int32_t Hq, const void* K_row,
+                    const void* V_row, int64_t pos, int64_t tail_begin, float scale, void* O, float* LSE,
+                    int32_t* leaves_out, void* workspace, size_t workspace_bytes, int32_t* status, void* stream) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  lsa::SelectArgs a;
+  memset(&a, 0, sizeof(a));
+  int bmax = 0;
+  if ((rc = beam_checks(tree, beam, a, &bmax)) != LSA_OK) return rc;
+  if (!valid_dtype(dtype)) return fail(LSA_ERR_INVALID_ARG, "unknown dtype %d", dtype);
+  if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
+  const int32_t H = tree->n_heads;
+  if (Hq < H || Hq % H) return fail(LSA_ERR_SHAPE, "Hq (%d) must be a multiple of n_heads (%d)", Hq, H);
+  const int G = Hq / H;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return fail(LSA_ERR_SHAPE, "query heads per group must be 1, 2, 4 or 8");
+  if (!tree_mem || !W || !K || !V || !Q || !O || !LSE)
+    return fail(LSA_ERR_INVALID_ARG, "tree_mem, W, K, V, Q, O and LSE must be non-NULL");
+  if ((K_row == nullptr) != (V_row == nullptr)) return fail(LSA_ERR_INVALID_ARG, "give both K_row and V_row or neither");
+  if (n_cap < tree->n_tree) return fail(LSA_ERR_SHAPE, "n_cap is smaller than the indexed keys");
+  if (pos < tree->n_tree - 1 || pos >= n_cap)
+    return fail(LSA_ERR_SHAPE, "pos %lld must lie in [n_tree - 1, n_cap) (n_tree %lld)", (long long)pos,
+                (long long)tree->n_tree);
+  if (tail_begin < tree->n_tree || tail_begin > pos + 1)
+    return fail(LSA_ERR_SHAPE, "tail_begin %lld must lie in [n_tree, pos + 1]", (long long)tail_begin);
+  if (!std::isfinite(scale)) return fail(LSA_ERR_INVALID_ARG, "scale must be finite");
+  const int B = beam[tree->levels - 1];
+  const int64_t tail_len = pos + 1 - tail_begin;
+  const int nsplit = lsa::dec_splits(B, tree->leaf_size, tail_len);
+  const size_t need = decode_ws_layout(H, B, G, d, nsplit, nullptr, nullptr, nullptr, nullptr);
+  if (!workspace || workspace_bytes < need)
+    return fail(LSA_ERR_WORKSPACE, "decode step needs %zu workspace bytes (got %zu)", need,
+                workspace ? workspace_bytes : (size_t)0);
+  int32_t *leaves = nullptr, *cnt = nullptr;
+  float* part = nullptr;
+  decode_ws_layout(H, B, G, d, nsplit, static_cast<char*>(workspace), &leaves, &cnt, &part);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // select (one CTA per KV group) with the append and the counter reset folded in
+  a.Q = Q; a.W = W; a.tree = static_cast<const char*>(tree_mem); a.q_pos = nullptr; a.idx_out = nullptr;
+  a.leaves_out = leaves; a.status = status;
+  a.T = 1; a.Hq = Hq; a.Hkv = H; a.G = G; a.d = d; a.r = tree->r;
+  a.levels = tree->levels; a.leaf = tree->leaf_size; a.beam_max = bmax; a.n_tree = tree->n_tree;
+  a.off_leaf = tree->off_leaf_index;
+  const int row_bytes = d * (dtype == LSA_BF16 ? 2 : 4);
+  if (K_row) {
+    a.app_K = K; a.app_V = V; a.app_Kr = K_row; a.app_Vr = V_row; a.app_pos = pos; a.app_ncap = n_cap;
+    a.app_row_bytes = row_bytes;
+  }
+  a.zero_cnt = cnt;
+  cudaError_t e = lsa::run_select(a, dtype, st);
+  if (e == cudaSuccess) {
+    lsa::DecAttnArgs b;
+    memset(&b, 0, sizeof(b));
+    b.Q = Q; b.K = K; b.V = V; b.leaves = leaves;
+    b.leaf_index = reinterpret_cast<const int32_t*>(static_cast<const char*>(tree_mem) + tree->off_leaf_index);
+    b.O = O; b.LSE = LSE; b.part = part; b.cnt = cnt;
+    b.n_cap = n_cap; b.n_tree = tree->n_tree; b.tail_begin = tail_begin; b.tail_end = pos + 1;
+    b.Hq = Hq; b.Hkv = H; b.B = B; b.leaf = tree->leaf_size; b.spl = (tree->leaf_size + 63) / 64;
+    b.nsplit = nsplit; b.scale_log2 = scale * 1.44269504088896340736f;
+    e = lsa::run_dec_attn(b, dtype, d, G, st);
+  }
+  if (e == cudaSuccess && leaves_out)
+    e = cudaMemcpyAsync(leaves_out, leaves, (size_t)H * B * sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_decode_step");
   return ok();
 }
 

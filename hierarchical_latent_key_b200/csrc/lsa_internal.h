@@ -101,8 +101,37 @@ struct SelectArgs {
   uint64_t off_c[LSA_MAX_LEVELS];
   uint64_t off_m[LSA_MAX_LEVELS];
   uint64_t off_leaf;
+  // decode step only (the small-batch kernel): append one K/V row per KV head at
+  // app_pos before selecting, and zero the attention's arrival counters
+  void* app_K;
+  void* app_V;
+  const void* app_Kr;
+  const void* app_Vr;
+  int64_t app_pos, app_ncap;
+  int32_t app_row_bytes;
+  int32_t* zero_cnt;
 };
 cudaError_t run_select(const SelectArgs& a, int dtype, cudaStream_t st);
+
+// Decode attention (decode.cu): one query token, keys = the kept leaves of every
+// KV group (leaf_index slices) + the tail [tail_begin, tail_end), split into
+// chunks of 64 keys over CTAs; the last CTA of a group merges the partials.
+struct DecAttnArgs {
+  const void* Q;              // [Hq][d]
+  const void* K;
+  const void* V;              // [Hkv][n_cap][d]
+  const int32_t* leaves;      // [Hkv][B]
+  const int32_t* leaf_index;  // [Hkv][n_tree]
+  void* O;                    // [Hq][d]
+  float* LSE;                 // [Hq]
+  float* part;                // [Hkv][nsplit][G][d + 2]
+  int32_t* cnt;               // [Hkv], zero on entry, re-zeroed by the last CTA
+  int64_t n_cap, n_tree, tail_begin, tail_end;
+  int32_t Hq, Hkv, B, leaf, spl, nsplit;
+  float scale_log2;
+};
+int dec_splits(int B, int leaf, int64_t tail_len);
+cudaError_t run_dec_attn(const DecAttnArgs& a, int dtype, int d, int G, cudaStream_t st);
 // flat search: every leaf of the last level scored, the best beam[levels - 1] kept
 cudaError_t run_select_flat(const SelectArgs& a, int dtype, cudaStream_t st);
 

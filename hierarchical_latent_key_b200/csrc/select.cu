@@ -322,6 +322,10 @@ __global__ void __launch_bounds__(kSelWarps * 32, 3) k_select(SelectArgs a) {
   }
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // Small batches (decode): one CTA of kWideWarps warps per (query t, KV group g),
 // so a level's candidates are scored in one or two memory round trips.  Each
 // warp sorts a chunk of 32 keys; chunk lists are then merged pairwise keeping
@@ -341,9 +345,25 @@ __global__ void __launch_bounds__(kWideWarps * 32) k_select_wide(SelectArgs a) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = blockIdx.y;
   const int64_t t = blockIdx.x;
-  {  // W[g] staged by the whole CTA in one memory round trip
+  if (t == 0) {   // decode step: this head's new key and value rows, the attention's counter
+    const int chunks = a.app_row_bytes / 16;
+    if (a.app_K && tid < 2 * chunks) {
+      const bool isv = tid >= chunks;
+      const int c = isv ? tid - chunks : tid;
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const char*>(isv ? a.app_Vr : a.app_Kr) +
+                                                        (int64_t)g * a.app_row_bytes) + c;
+      uint4* dst = reinterpret_cast<uint4*>(static_cast<char*>(isv ? a.app_V : a.app_K) +
+                                            ((int64_t)g * a.app_ncap + a.app_pos) * a.app_row_bytes) + c;
+      *dst = __ldg(src);
+    }
+    if (a.zero_cnt && tid == 0) a.zero_cnt[g] = 0;
+  }
+  {  // W[g] staged by the whole CTA in one memory round trip; the top level's rows requested meanwhile
     constexpr int VEC = 16 / sizeof(T);
     const T* W = static_cast<const T*>(a.W) + (int64_t)g * DK * R;
+    const char* top = a.tree + a.off_c[0] + (int64_t)g * a.nodes[0] * R * sizeof(float);
+    const int top_lines = (int)((a.nodes[0] * R * (int64_t)sizeof(float) + 127) / 128);
+    for (int x = tid; x < top_lines; x += NT) prefetch_l2(top + (int64_t)x * 128);
     for (int i = tid * VEC; i < DK * R; i += NT * VEC)
       *reinterpret_cast<uint4*>(&s_w[i]) = __ldg(reinterpret_cast<const uint4*>(W + i));
   }
@@ -406,6 +426,27 @@ __global__ void __launch_bounds__(kWideWarps * 32) k_select_wide(SelectArgs a) {
           }
           s_key[c] = key;
         }
+      }
+    }
+    // the next level's candidates are children of this level's kept nodes: bring the
+    // children of every candidate into L2 while the keys are sorted (a decode walk is a
+    // chain of dependent reads; this turns the next level's DRAM round trip into an L2 hit)
+    if (l + 1 < a.levels) {
+      const int b1 = a.branching[l + 1];
+      const char* nxt = a.tree + a.off_c[l + 1] + (int64_t)g * a.nodes[l + 1] * R * sizeof(float);
+      const int lines = (b1 * R * (int)sizeof(float) + 127) / 128;   // one candidate's children, 128-B lines
+      for (int x = tid; x < ncand * lines; x += NT) {
+        const int c = x / lines, ln = x % lines;
+        const int64_t id = l == 0 ? c : (int64_t)kept[c / b] * b + (c % b);
+        prefetch_l2(nxt + (id * b1 * R * (int64_t)sizeof(float)) + ln * 128);
+      }
+    } else if (a.leaves_out) {   // last level: the leaf_index slices the attention reads next
+      const char* li = reinterpret_cast<const char*>(a.tree + a.off_leaf) + (int64_t)g * a.n_tree * 4;
+      const int lines = (a.leaf * 4 + 127) / 128;
+      for (int x = tid; x < ncand * lines; x += NT) {
+        const int c = x / lines, ln = x % lines;
+        const int64_t id = l == 0 ? c : (int64_t)kept[c / b] * b + (c % b);
+        prefetch_l2(li + id * a.leaf * 4 + ln * 128);
       }
     }
     __syncthreads();

@@ -84,6 +84,11 @@ def _load():
         "lsa_kv_append": (ctypes.c_int, [P, P, i32, i64, i32, i32, i64, P, P, P]),
         "lsa_project_keys": (ctypes.c_int, [P, i32, i64, i32, i32, P, i32, i64, P, P, P]),
         "lsa_balanced_assign_workspace_bytes": (ctypes.c_int, [i64, i64, i32, ctypes.POINTER(sz)]),
+        "lsa_decode_step_workspace_bytes": (ctypes.c_int, [ctypes.POINTER(lsa_tree_desc), i32, i32,
+                                                           ctypes.POINTER(i32), i64, ctypes.POINTER(sz)]),
+        "lsa_decode_step": (ctypes.c_int, [ctypes.POINTER(lsa_tree_desc), P, P, ctypes.POINTER(i32), P, P, i64,
+                                           i32, i32, P, i32, P, P, i64, i64, ctypes.c_float, P, P, P, P, sz,
+                                           P, P]),
         "lsa_balanced_assign": (ctypes.c_int, [P, P, i64, i64, i32, i32, i32, P, P, sz, P, P]),
         "lsa_tree_attn_bwd_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
         "lsa_tree_attn_bwd": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, P, P, P, i32, P, i32, f32,
@@ -312,6 +317,46 @@ def balanced_assign(Z, mu, nseg, m, b, max_rounds=0, status=None, check=True):
     if check:
         check_status(st, "lsa_balanced_assign")
     return choice
+
+
+def lsa_decode_step_workspace_bytes(desc, Hq, d, beam, tail_len_max) -> int:
+    n = ctypes.c_size_t()
+    bm = (ctypes.c_int32 * len(beam))(*beam)
+    _raise(_lib.lsa_decode_step_workspace_bytes(ctypes.byref(desc), Hq, d, bm, int(tail_len_max), ctypes.byref(n)),
+           "lsa_decode_step_workspace_bytes")
+    return n.value
+
+
+def lsa_decode_step(desc, tree_mem, W, beam, K, V, Q, K_row, V_row, pos, tail_begin, scale, O, LSE, workspace,
+                    leaves_out=None, status=None, stream=None):
+    """K, V: [n_heads, n_cap, d] caches; Q: [1, Hq, d]; K_row, V_row: [n_heads, d] or None;
+    O: [1, Hq, d]; LSE: [1, Hq]; leaves_out: [n_heads, beam[-1]] int32 or None."""
+    bm = (ctypes.c_int32 * len(beam))(*beam)
+    _raise(_lib.lsa_decode_step(ctypes.byref(desc), _ptr(tree_mem), _ptr(W), bm, _ptr(K), _ptr(V), K.shape[1],
+                                K.shape[2], _dtype(K), _ptr(Q), Q.shape[1], _ptr(K_row), _ptr(V_row), int(pos),
+                                int(tail_begin), float(scale), _ptr(O), _ptr(LSE), _ptr(leaves_out),
+                                _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream, K)),
+           "lsa_decode_step")
+
+
+class DecodeStep:
+    """Buffers of a decode loop over one index: call step(...) once per token."""
+
+    def __init__(self, tree, W, beam, K, Hq, tail_len_max, scale=None):
+        d = K.shape[2]
+        self.tree, self.W, self.beam = tree, W, list(beam)
+        self.scale = 1.0 / math.sqrt(d) if scale is None else scale
+        need = lsa_decode_step_workspace_bytes(tree.desc, Hq, d, self.beam, tail_len_max)
+        self.ws = torch.empty(need, dtype=torch.uint8, device=K.device)
+        self.O = torch.empty(1, Hq, d, dtype=K.dtype, device=K.device)
+        self.LSE = torch.empty(1, Hq, dtype=torch.float32, device=K.device)
+        self.leaves = torch.empty(K.shape[0], self.beam[-1], dtype=torch.int32, device=K.device)
+        self.status = _new_status(K.device)
+
+    def step(self, K, V, Q, K_row, V_row, pos, tail_begin, stream=None):
+        lsa_decode_step(self.tree.desc, self.tree.mem, self.W, self.beam, K, V, Q, K_row, V_row, pos, tail_begin,
+                        self.scale, self.O, self.LSE, self.ws, self.leaves, self.status, stream)
+        return self.O, self.LSE
 
 
 def project_keys(K, W, n=None):

@@ -434,6 +434,32 @@ int lsa_project_keys(const void *K, int32_t n_heads, int64_t n_cap, int32_t d, i
 int lsa_kv_append(void *K, void *V, int32_t n_heads, int64_t n_cap, int32_t d, int32_t dtype,
                   int64_t pos, const void *K_rows, const void *V_rows, void *stream);
 
+/* One decode step of a single request (kongchang.com, "The Accuracy-Efficiency
+ * Dilemma of Sparse Attention": decode is memory-bound and latency-sensitive;
+ * bdtechtalks.com, "How latent sparse attention works": the query is compared
+ * with the centroids, a fixed number of keys is taken from the chosen clusters,
+ * and the recent tokens join them).  For the token at position `pos` it
+ *   1. appends K_row, V_row ([n_heads][d], device) at `pos` of the caches K, V
+ *      ([n_heads][n_cap][d]) when they are non-NULL (both or neither);
+ *   2. walks the index with the group query of Q ([1][Hq][d]), as lsa_select with
+ *      q_pos = pos (every indexed key precedes the token), keeping beam[levels-1]
+ *      leaves per KV group;
+ *   3. attends to the keys of the kept leaves and to the tail [tail_begin, pos]:
+ *      O [1][Hq][d] (dtype), LSE [Hq] fp32, as lsa_sparse_attn with causal = 1.
+ * Two kernel launches; no host synchronisation.  Requires n_tree - 1 <= pos <
+ * n_cap and n_tree <= tail_begin <= pos + 1.  leaves_out (optional, device,
+ * [n_heads][beam[levels-1]]) receives the kept leaf ids (-1 pads).
+ * workspace: lsa_decode_step_workspace_bytes(tree, Hq, d, beam, tail_len_max)
+ * bytes with tail_len_max >= pos + 1 - tail_begin; calls that share a workspace
+ * must not overlap on the GPU. */
+int lsa_decode_step_workspace_bytes(const lsa_tree_desc *tree, int32_t Hq, int32_t d, const int32_t *beam,
+                                    int64_t tail_len_max, size_t *bytes);
+int lsa_decode_step(const lsa_tree_desc *tree, const void *tree_mem, const void *W, const int32_t *beam,
+                    void *K, void *V, int64_t n_cap, int32_t d, int32_t dtype, const void *Q, int32_t Hq,
+                    const void *K_row, const void *V_row, int64_t pos, int64_t tail_begin, float scale,
+                    void *O, float *LSE, int32_t *leaves_out, void *workspace, size_t workspace_bytes,
+                    int32_t *status, void *stream);
+
 /* Zero the device status word on `stream`. */
 int lsa_status_clear(int32_t *status, void *stream);
 

@@ -203,3 +203,27 @@ def test_balanced_assign_rejects(lsa):
     assert L.lsa_balanced_assign(P, P, 4, 64, 4, 64, -1, P, P, 1 << 20, None, None) == lsa.LSA_ERR_INVALID_ARG
     assert L.lsa_balanced_assign(None, P, 4, 64, 4, 64, 0, P, P, 1 << 20, None, None) == lsa.LSA_ERR_INVALID_ARG
     assert L.lsa_balanced_assign(P, P, 4, 64, 4, 64, 0, P, P, 16, None, None) == lsa.LSA_ERR_WORKSPACE
+
+
+def test_decode_step_rejects(lsa):
+    L = lsa._lib
+    P = ctypes.c_void_p(16)
+    d = lsa.lsa_tree_describe(2, 64, (16, 16, 8), 64)
+    beam = (ctypes.c_int32 * 3)(8, 32, 32)
+    n = ctypes.c_size_t()
+    assert L.lsa_decode_step_workspace_bytes(ctypes.byref(d), 8, 128, beam, 256, ctypes.byref(n)) == lsa.LSA_OK
+    need = n.value
+    # 32 leaves + 4 tail splits of 64 keys, 2 heads x 4 query heads x 130 floats each
+    assert need >= 2 * 36 * 4 * 130 * 4
+
+    def call(pos, tail_begin, ws=need, Kr=P, Vr=P, Hq=8):
+        return L.lsa_decode_step(ctypes.byref(d), P, P, beam, P, P, d.n_tree + 256, 128, 1, P, Hq, Kr, Vr, pos,
+                                 tail_begin, 0.1, P, P, None, P, ws, None, None)
+    nt = d.n_tree
+    assert call(nt - 2, nt) == lsa.LSA_ERR_SHAPE            # token before the last indexed key
+    assert call(nt + 3, nt - 1) == lsa.LSA_ERR_SHAPE        # tail overlapping the index
+    assert call(nt + 3, nt + 5) == lsa.LSA_ERR_SHAPE        # tail past the token
+    assert call(nt + 256, nt) == lsa.LSA_ERR_SHAPE          # pos outside the cache
+    assert call(nt + 3, nt, Vr=None) == lsa.LSA_ERR_INVALID_ARG
+    assert call(nt + 3, nt, Hq=12) == lsa.LSA_ERR_SHAPE
+    assert call(nt + 3, nt, ws=16) == lsa.LSA_ERR_WORKSPACE

@@ -130,16 +130,16 @@ def test_prefill_1m_full(lsa):
 
 
 def test_decode_10m_full(lsa):
-    """10,485,760 indexed keys, all 128 decode steps (append, select, key-list attention with
-    the dense tail, one step at a time as bench.py runs them), every step checked on all 8
+    """10,485,760 indexed keys, all 128 decode steps (lsa_decode_step: append, select, attention
+    over the kept leaves and the dense tail, one step at a time as bench.py runs them), every step checked on all 8
     KV heads: the beam walk stage-wise (near-tie band), the key list exactly, attention on
     the GPU's keys.  The build is checked stage-wise on sampled segments of one head (every
     round of the three lowest levels) and by tree properties on every head."""
     cfg = configs.get("decode_10m")
     case = cfg.case(DEV)
     n = cfg.n
-    Knew = case.K[:, n:].transpose(0, 1).contiguous()       # rows the steps append
-    Vnew = case.V[:, n:].transpose(0, 1).contiguous()
+    Knew = case.K[:, n:].transpose(0, 1).clone(memory_format=torch.contiguous_format)       # rows the steps append
+    Vnew = case.V[:, n:].transpose(0, 1).clone(memory_format=torch.contiguous_format)
     case.K[:, n:].zero_()
     case.V[:, n:].zero_()
     tree, trace = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed, trace=True)
@@ -156,15 +156,17 @@ def test_decode_10m_full(lsa):
     print("decode_10m build rounds differing", rd, "keys", kd)
     for h in range(cfg.Hkv):
         _tree_props(tree, h, case.K, case.W[h].double().cpu().numpy(), n, cfg.leaf, rng, n_nodes=4)
-    # the decode loop on the GPU: one token per step, its key and value appended first
-    idx = torch.empty(cfg.Hkv, 1, cfg.K_sel, dtype=torch.int32, device=DEV)
+    # the decode loop on the GPU as bench.py runs it: one lsa_decode_step per token (append,
+    # select, attention); the select call alone gives the per-level beams for the stage-wise check
+    dec = lsa.DecodeStep(tree, case.W, cfg.beam, case.K, cfg.Hq, cfg.T)
     st_idx, st_beams, st_O, st_LSE = [], [], [], []
     for s in range(cfg.T):
-        lsa.lsa_kv_append(case.K, case.V, n + s, Knew[s], Vnew[s])
         Qs = case.Q[s:s + 1]
-        idx, beams = lsa.select(tree, Qs, case.W, cfg.beam, case.q_pos[s:s + 1], beams=True)
-        O, LSE = lsa.sparse_attn(Qs, case.K, case.V, idx, case.q_pos[s:s + 1], True, (n, n + s + 1))
+        O, LSE = dec.step(case.K, case.V, Qs, Knew[s], Vnew[s], n + s, n)
+        idx, leaves, beams = lsa.select(tree, Qs, case.W, cfg.beam, case.q_pos[s:s + 1], beams=True, leaves=True)
+        assert torch.equal(dec.leaves, leaves[:, 0]), s
         st_idx.append(idx.cpu()); st_beams.append(beams.cpu()); st_O.append(O.float().cpu()); st_LSE.append(LSE.cpu())
+    assert lsa.lsa_status_check(dec.status) == lsa.LSA_OK
     torch.cuda.synchronize()
     near = 0
     for h in range(cfg.Hkv):
