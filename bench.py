@@ -320,6 +320,9 @@ class Train:
 
 def run_train(args, dev, rank, world, reduce_max, steps=3, warmup=2):
     cfg = configs.get("train_128k")
+    if args.small:   # profiling case: the training geometry over 16,384 tokens
+        cfg = cfg.scaled(name="train_geometry_16k", n=16384, T=16384, branching=(16, 16), beam=(8, 32), comps=256)
+    # (--small: 16 x 16 leaves of 64 keys, beam 8/32 = 2048 keys per query, as the full tree's last level)
     w = Train(cfg, dev, rank_seed(cfg.seed, rank))
     stream = torch.cuda.current_stream(dev)
     ph = w.phases()
@@ -411,6 +414,8 @@ def run_append(dev, seed):
 
 def run_decode(args, dev, rank, world, reduce_max):
     cfg = configs.get("decode_10m")
+    if args.small:   # profiling case: the decode step over the 131,072-key index of decode_128k
+        cfg = configs.get("decode_128k").scaled(T=cfg.T, beam=(8, 32, 32))
     steps, warmup = cfg.T, args.warmup
     w = Decode(cfg, dev, rank_seed(cfg.seed, rank), warmup + steps)
     stream = torch.cuda.current_stream(dev)
@@ -1049,7 +1054,8 @@ def main(argv=None):
     ap.add_argument("--no-train", action="store_true", help="skip the training-shaped 128k layer step")
     ap.add_argument("--small", action="store_true",
                     help="profiling case: the prefill geometry (4096 queries x 2048 keys) over 131,072 cached "
-                         "keys, tree 8/8/8/4, so a kernel capture stays small")
+                         "keys, tree 8/8/8/4, so a kernel capture stays small; with --workload decode_10m the "
+                         "decode step over a 131,072-key index, with --workload train_128k a 16,384-token layer")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -719,7 +719,7 @@ static size_t decode_ws_layout(int64_t Hkv, int B, int G, int d, int nsplit, cha
   if (leaves) *leaves = reinterpret_cast<int32_t*>(p);
   p = take((uint64_t)Hkv * 4);
   if (cnt) *cnt = reinterpret_cast<int32_t*>(p);
-  p = take((uint64_t)Hkv * nsplit * G * (d + 2) * 4);
+  p = take((uint64_t)Hkv * nsplit * G * (d + 4) * 4);   // partial rows padded to 16 bytes
   if (part) *part = reinterpret_cast<float*>(p);
   return off;
 }
@@ -771,6 +771,9 @@ int lsa_decode_step(const lsa_tree_desc* tree, const void* tree_mem, const void*
   const int B = beam[tree->levels - 1];
   const int64_t tail_len = pos + 1 - tail_begin;
   const int nsplit = lsa::dec_splits(B, tree->leaf_size, tail_len);
+  if (nsplit > lsa::dec_max_splits(dtype, d, G))
+    return fail(LSA_ERR_SHAPE, "decode step: %d splits of 64 keys (kept leaves and tail) exceed the %d one call merges",
+                nsplit, lsa::dec_max_splits(dtype, d, G));
   const size_t need = decode_ws_layout(H, B, G, d, nsplit, nullptr, nullptr, nullptr, nullptr);
   if (!workspace || workspace_bytes < need)
     return fail(LSA_ERR_WORKSPACE, "decode step needs %zu workspace bytes (got %zu)", need,
@@ -778,6 +781,7 @@ int lsa_decode_step(const lsa_tree_desc* tree, const void* tree_mem, const void*
   int32_t *leaves = nullptr, *cnt = nullptr;
   float* part = nullptr;
   decode_ws_layout(H, B, G, d, nsplit, static_cast<char*>(workspace), &leaves, &cnt, &part);
+  if (leaves_out) leaves = leaves_out;   // the kept leaves go straight to the caller's buffer
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   // select (one CTA per KV group) with the append and the counter reset folded in
   a.Q = Q; a.W = W; a.tree = static_cast<const char*>(tree_mem); a.q_pos = nullptr; a.idx_out = nullptr;
@@ -803,8 +807,6 @@ int lsa_decode_step(const lsa_tree_desc* tree, const void* tree_mem, const void*
     b.nsplit = nsplit; b.scale_log2 = scale * 1.44269504088896340736f;
     e = lsa::run_dec_attn(b, dtype, d, G, st);
   }
-  if (e == cudaSuccess && leaves_out)
-    e = cudaMemcpyAsync(leaves_out, leaves, (size_t)H * B * sizeof(int32_t), cudaMemcpyDeviceToDevice, st);
   if (e != cudaSuccess) return cuda_fail(e, "lsa_decode_step");
   return ok();
 }

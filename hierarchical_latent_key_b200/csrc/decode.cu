@@ -57,22 +57,31 @@ __device__ __forceinline__ void unpack(const uint4& x, const __nv_bfloat16*, flo
 template <typename T, int DK, int G>
 __global__ void __launch_bounds__(kDT) k_dec_attn(DecAttnArgs a) {
   using S = DecSmem<T, DK>;
+  constexpr int kPS = DK + 4;   // floats per partial row: d outputs, max, sum, 2 pad (16-byte rows)
   constexpr int EPC = 16 / (int)sizeof(T);        // elements per 16-byte chunk
   constexpr int CPR = DK / EPC;                   // chunks per row
   extern __shared__ __align__(16) char smem[];
   char* sK = smem;
   char* sV = smem + S::kKV;
   __shared__ int64_t s_pos[kDKeys];
-  __shared__ float s_q[G][DK];
+  __shared__ __align__(16) float s_q[G][DK];
   __shared__ float s_p[G][kDKeys];
   __shared__ float s_m[G], s_l[G];
-  __shared__ int s_n, s_last;
+  __shared__ int s_last;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int s = blockIdx.x, g = blockIdx.y;
   const T* Q = static_cast<const T*>(a.Q);
   const char* Kh = static_cast<const char*>(a.K) + (int64_t)g * a.n_cap * DK * sizeof(T);
   const char* Vh = static_cast<const char*>(a.V) + (int64_t)g * a.n_cap * DK * sizeof(T);
 
+  // Launched as a programmatic dependent of the select kernel: the query rows are
+  // read before waiting for it; the kept leaves, the appended K/V row and the
+  // re-armed counter after.
+  for (int x = tid; x < G * DK; x += kDT) {
+    const int h = x / DK, dim = x % DK;
+    s_q[h][dim] = to_f32(Q[((int64_t)g * G + h) * DK + dim]) * a.scale_log2;
+  }
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // key positions of this split
   if (tid < kDKeys) {
     int64_t p = -1;
@@ -87,10 +96,6 @@ __global__ void __launch_bounds__(kDT) k_dec_attn(DecAttnArgs a) {
       if (j < a.tail_end) p = j;
     }
     s_pos[tid] = (p >= 0 && p < a.n_cap) ? p : -1;
-  }
-  for (int x = tid; x < G * DK; x += kDT) {
-    const int h = x / DK, dim = x % DK;
-    s_q[h][dim] = to_f32(Q[((int64_t)g * G + h) * DK + dim]) * a.scale_log2;
   }
   __syncthreads();
   // all K and V rows of the split in flight at once (absent keys: zero rows)
@@ -108,20 +113,34 @@ __global__ void __launch_bounds__(kDT) k_dec_attn(DecAttnArgs a) {
   }
   cp_async_wait_all();
   __syncthreads();
-  // scores: thread = (key, heads hg, hg + 2, ...)
+  // scores: two threads per key (halves of the row), every head of the group
   {
-    const int k = tid % kDKeys, hg = tid / kDKeys;
-    const bool valid = s_pos[k] >= 0;
-    for (int h = hg; h < G; h += kDT / kDKeys) {
-      float acc = 0.f;
-#pragma unroll 4
-      for (int c = 0; c < CPR; ++c) {
-        float kv[EPC];
-        unpack<EPC>(*reinterpret_cast<const uint4*>(sK + k * S::kRowBytes + c * 16), (const T*)nullptr, kv);
+    const int k = tid >> 1, hh = tid & 1;
+    float acc[G];
 #pragma unroll
-        for (int e = 0; e < EPC; ++e) acc = fmaf(s_q[h][c * EPC + e], kv[e], acc);
+    for (int h = 0; h < G; ++h) acc[h] = 0.f;
+#pragma unroll 4
+    for (int cc = 0; cc < CPR / 2; ++cc) {
+      const int c = hh * (CPR / 2) + cc;
+      float kv[EPC];
+      unpack<EPC>(*reinterpret_cast<const uint4*>(sK + k * S::kRowBytes + c * 16), (const T*)nullptr, kv);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+#pragma unroll
+        for (int e4 = 0; e4 < EPC / 4; ++e4) {
+          const float4 q4 = *reinterpret_cast<const float4*>(&s_q[h][c * EPC + 4 * e4]);
+          acc[h] = fmaf(q4.x, kv[4 * e4], acc[h]);
+          acc[h] = fmaf(q4.y, kv[4 * e4 + 1], acc[h]);
+          acc[h] = fmaf(q4.z, kv[4 * e4 + 2], acc[h]);
+          acc[h] = fmaf(q4.w, kv[4 * e4 + 3], acc[h]);
+        }
       }
-      s_p[h][k] = valid ? acc : -INFINITY;
+    }
+    const bool valid = s_pos[k] >= 0;
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float v = acc[h] + __shfl_xor_sync(0xffffffffu, acc[h], 1);
+      if (hh == 0) s_p[h][k] = valid ? v : -INFINITY;
     }
   }
   __syncthreads();
@@ -140,18 +159,46 @@ __global__ void __launch_bounds__(kDT) k_dec_attn(DecAttnArgs a) {
     if (lane == 0) { s_m[h] = m; s_l[h] = l; }
   }
   __syncthreads();
-  // unnormalised output of the split: thread = (head, dim) pairs
-  float* part = a.part + ((int64_t)g * a.nsplit + s) * G * (DK + 2);
-  for (int x = tid; x < G * DK; x += kDT) {
-    const int h = x / DK, dim = x % DK;
-    float o = 0.f;
-    if (s_l[h] > 0.f) {
-#pragma unroll 8
-      for (int k = 0; k < kDKeys; ++k)
-        o = fmaf(s_p[h][k], to_f32(*reinterpret_cast<const T*>(sV + k * S::kRowBytes + dim * sizeof(T))), o);
+  // unnormalised output: thread = (pair of dims, slice of the keys), every head;
+  // the key slices are summed through shared memory (the K tile is free now)
+  {
+    constexpr int DP = DK / 2, KS = kDT / DP, KPS = kDKeys / KS;
+    const int dp = tid % DP, ks = tid / DP;
+    float o[G][2];
+#pragma unroll
+    for (int h = 0; h < G; ++h) o[h][0] = o[h][1] = 0.f;
+#pragma unroll 4
+    for (int kk = 0; kk < KPS; ++kk) {
+      const int k = ks * KPS + kk;
+      float v2[2];
+      load2_generic(reinterpret_cast<const T*>(sV + k * S::kRowBytes) + 2 * dp, v2);
+#pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float pk = s_p[h][k];
+        o[h][0] = fmaf(pk, v2[0], o[h][0]);
+        o[h][1] = fmaf(pk, v2[1], o[h][1]);
+      }
     }
-    part[h * (DK + 2) + dim] = o;
-    if (dim == 0) { part[h * (DK + 2) + DK] = s_m[h]; part[h * (DK + 2) + DK + 1] = s_l[h]; }
+    float* s_red = reinterpret_cast<float*>(sK);      // [KS][G][DK]
+#pragma unroll
+    for (int h = 0; h < G; ++h) {
+      s_red[(ks * G + h) * DK + 2 * dp] = o[h][0];
+      s_red[(ks * G + h) * DK + 2 * dp + 1] = o[h][1];
+    }
+  }
+  __syncthreads();
+  float* part = a.part + ((int64_t)g * a.nsplit + s) * G * kPS;
+  {
+    constexpr int KS = kDT / (DK / 2);
+    const float* s_red = reinterpret_cast<const float*>(sK);
+    for (int x = tid; x < G * DK; x += kDT) {
+      const int h = x / DK, dim = x % DK;
+      float o = 0.f;
+#pragma unroll
+      for (int q = 0; q < KS; ++q) o += s_red[(q * G + h) * DK + dim];
+      part[h * kPS + dim] = s_l[h] > 0.f ? o : 0.f;
+      if (dim == 0) { part[h * kPS + DK] = s_m[h]; part[h * kPS + DK + 1] = s_l[h]; }
+    }
   }
   // arrival: the last CTA of the group merges every split
   __threadfence();
@@ -160,29 +207,64 @@ __global__ void __launch_bounds__(kDT) k_dec_attn(DecAttnArgs a) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  const float* pg = a.part + (int64_t)g * a.nsplit * G * (DK + 2);
-  for (int x = tid; x < G * DK; x += kDT) {
-    const int h = x / DK, dim = x % DK;
+  // merge: (max, sum) of every (split, head) in one round of loads, per-head weights
+  // by one warp per head, then the outputs with every split's partial in flight
+  const float* pg = a.part + (int64_t)g * a.nsplit * G * kPS;
+  float* s_w = reinterpret_cast<float*>(sK);          // [nsplit][G] (max, then weight; sum)
+  for (int x = tid; x < a.nsplit * G; x += kDT) {
+    const float* pp = pg + (int64_t)x * kPS;
+    const float m = __ldcg(&pp[DK]), l = __ldcg(&pp[DK + 1]);
+    s_w[2 * x] = l > 0.f ? m : -INFINITY;
+    s_w[2 * x + 1] = l;
+  }
+  __syncthreads();
+  for (int h = warp; h < G; h += kDT / 32) {
     float M = -INFINITY;
-    for (int q = 0; q < a.nsplit; ++q) {
-      const float* pp = pg + ((int64_t)q * G + h) * (DK + 2);
-      if (__ldcg(&pp[DK + 1]) > 0.f) M = fmaxf(M, __ldcg(&pp[DK]));
+    for (int q = lane; q < a.nsplit; q += 32) M = fmaxf(M, s_w[2 * (q * G + h)]);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.f;
+    for (int q = lane; q < a.nsplit; q += 32) {
+      const int x = q * G + h;
+      const float f = M == -INFINITY || s_w[2 * x + 1] <= 0.f ? 0.f : exp2f(s_w[2 * x] - M);
+      L = fmaf(s_w[2 * x + 1], f, L);
+      s_w[2 * x] = f;
     }
-    float L = 0.f, o = 0.f;
-    if (M != -INFINITY) {
-      for (int q = 0; q < a.nsplit; ++q) {
-        const float* pp = pg + ((int64_t)q * G + h) * (DK + 2);
-        const float l = __ldcg(&pp[DK + 1]);
-        if (l > 0.f) {
-          const float f = exp2f(__ldcg(&pp[DK]) - M);
-          L = fmaf(l, f, L);
-          o = fmaf(__ldcg(&pp[dim]), f, o);
-        }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (lane == 0) { s_m[h] = M; s_l[h] = L; }
+  }
+  __syncthreads();
+  for (int x = tid; x < G * DK / 4; x += kDT) {     // (head, 4 dims)
+    const int h = x / (DK / 4), d4 = x % (DK / 4);
+    float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int q0 = 0; q0 < a.nsplit; q0 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int qq = 0; qq < 16; ++qq) {
+        const int q = q0 + qq;
+        v[qq] = q < a.nsplit ? __ldcg(reinterpret_cast<const float4*>(pg + ((int64_t)q * G + h) * kPS) + d4)
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int qq = 0; qq < 16; ++qq) {
+        const int q = q0 + qq;
+        const float f = q < a.nsplit ? s_w[2 * (q * G + h)] : 0.f;
+        o.x = fmaf(v[qq].x, f, o.x);
+        o.y = fmaf(v[qq].y, f, o.y);
+        o.z = fmaf(v[qq].z, f, o.z);
+        o.w = fmaf(v[qq].w, f, o.w);
       }
     }
+    const float L = s_l[h];
+    const float inv = L > 0.f ? 1.f / L : 0.f;
     const int64_t row = (int64_t)g * G + h;
-    static_cast<T*>(a.O)[row * DK + dim] = from_f32<T>(L > 0.f ? o / L : 0.f);
-    if (dim == 0) a.LSE[row] = L > 0.f ? (M + log2f(L)) * kLn2f : -INFINITY;
+    T* Or = static_cast<T*>(a.O) + row * DK + 4 * d4;
+    Or[0] = from_f32<T>(o.x * inv);
+    Or[1] = from_f32<T>(o.y * inv);
+    Or[2] = from_f32<T>(o.z * inv);
+    Or[3] = from_f32<T>(o.w * inv);
+    if (d4 == 0) a.LSE[row] = L > 0.f ? (s_m[h] + log2f(L)) * kLn2f : -INFINITY;
   }
   if (tid == 0) a.cnt[g] = 0;   // re-armed for the next call on this workspace
 }
@@ -196,7 +278,14 @@ cudaError_t launch_dec(const DecAttnArgs& a, int d, int G, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(k_dec_attn<T, DD, GG>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                          (int)smem);                                                 \
     if (e != cudaSuccess) return e;                                                                  \
-    k_dec_attn<T, DD, GG><<<grid, kDT, smem, st>>>(a);                                               \
+    cudaLaunchConfig_t cfg = {};                                                                     \
+    cudaLaunchAttribute attr[1];                                                                     \
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;                                 \
+    attr[0].val.programmaticStreamSerializationAllowed = 1;                                          \
+    cfg.gridDim = grid; cfg.blockDim = dim3(kDT); cfg.dynamicSmemBytes = smem; cfg.stream = st;      \
+    cfg.attrs = attr; cfg.numAttrs = 1;                                                              \
+    e = cudaLaunchKernelEx(&cfg, k_dec_attn<T, DD, GG>, a);                                          \
+    if (e != cudaSuccess) return e;                                                                  \
     return cudaGetLastError();                                                                       \
   }
   LSA_DEC(64, 1) LSA_DEC(64, 2) LSA_DEC(64, 4) LSA_DEC(64, 8)
@@ -206,6 +295,12 @@ cudaError_t launch_dec(const DecAttnArgs& a, int d, int G, cudaStream_t st) {
 }
 
 }  // namespace
+
+int dec_max_splits(int dtype, int d, int G) {
+  const size_t bytes = dtype == LSA_BF16 ? (d == 64 ? DecSmem<__nv_bfloat16, 64>::kKV : DecSmem<__nv_bfloat16, 128>::kKV)
+                                         : (d == 64 ? DecSmem<float, 64>::kKV : DecSmem<float, 128>::kKV);
+  return (int)(bytes / (2 * sizeof(float) * G));   // the merge keeps (max, weight) per (split, head) in the K tile
+}
 
 int dec_splits(int B, int leaf, int64_t tail_len) {
   const int spl = (leaf + kDKeys - 1) / kDKeys;

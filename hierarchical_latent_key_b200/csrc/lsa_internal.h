@@ -124,16 +124,20 @@ struct DecAttnArgs {
   const int32_t* leaf_index;  // [Hkv][n_tree]
   void* O;                    // [Hq][d]
   float* LSE;                 // [Hq]
-  float* part;                // [Hkv][nsplit][G][d + 2]
+  float* part;                // [Hkv][nsplit][G][d + 4] (d outputs, max, sum, 2 pad)
   int32_t* cnt;               // [Hkv], zero on entry, re-zeroed by the last CTA
   int64_t n_cap, n_tree, tail_begin, tail_end;
   int32_t Hq, Hkv, B, leaf, spl, nsplit;
   float scale_log2;
 };
 int dec_splits(int B, int leaf, int64_t tail_len);
+int dec_max_splits(int dtype, int d, int G);
 cudaError_t run_dec_attn(const DecAttnArgs& a, int dtype, int d, int G, cudaStream_t st);
 // flat search: every leaf of the last level scored, the best beam[levels - 1] kept
 cudaError_t run_select_flat(const SelectArgs& a, int dtype, cudaStream_t st);
+// flat search on the tensor cores (bf16 inputs, r = 64, at most 32 kept leaves)
+bool select_flat_tc_supported(const SelectArgs& a, int dtype);
+cudaError_t run_select_flat_tc(const SelectArgs& a, cudaStream_t st);
 
 struct AttnArgs {
   const void* Q;

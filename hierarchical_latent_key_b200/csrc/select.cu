@@ -99,6 +99,58 @@ __device__ __forceinline__ int key_slot(int i) {
   return ln * E + (e ^ (ln % E));
 }
 
+// Keep the best B (<= 64) of the keys v held by one warp (E per lane, element
+// index lane * E + e): writes their node ids to next[0..B) in key order and returns
+// how many are real candidates.  s_key: shared scratch of >= 64 keys that no lane
+// of the warp still needs.
+template <int E>
+__device__ __forceinline__ int warp_keep_best(unsigned long long (&v)[E], int B, unsigned long long* s_key,
+                                              int32_t* next) {
+  const int lane = threadIdx.x & 31;
+  if constexpr (E >= 8) {
+    // Threshold first: the B-th largest of the lanes' two largest keys is a lower
+    // bound of the B-th largest key overall (those 64 are keys of the level), so
+    // every kept key is >= tau.  Keys are distinct, so sorting the keys >= tau
+    // gives exactly the first B of the full order; when more than 64 pass, the
+    // full sort runs instead.
+    unsigned long long smp[2] = {0ull, 0ull};
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const unsigned long long x = v[e];
+      const bool top = x > smp[0];
+      smp[1] = top ? smp[0] : (x > smp[1] ? x : smp[1]);
+      smp[0] = top ? x : smp[0];
+    }
+    warp_sort_desc<2>(smp);
+    const unsigned long long tau = __shfl_sync(0xffffffffu, ((B - 1) & 1) ? smp[1] : smp[0], (B - 1) >> 1);
+    int c = 0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) c += (v[e] != 0ull && v[e] >= tau);
+    int inc = c;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, inc, d);
+      if (lane >= d) inc += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, inc, 31);
+    if (total <= 64) {
+      __syncwarp();                       // every lane has read its keys: s_key is free
+      int o = inc - c;
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if (v[e] != 0ull && v[e] >= tau) s_key[o++] = v[e];
+      __syncwarp();
+      unsigned long long w[2];
+      w[0] = 2 * lane < total ? s_key[2 * lane] : 0ull;
+      w[1] = 2 * lane + 1 < total ? s_key[2 * lane + 1] : 0ull;
+      warp_sort_desc<2>(w);
+      return emit_kept<2>(w, B, next);
+    }
+  }
+  warp_sort_desc<E>(v);
+  return emit_kept<E>(v, B, next);
+}
+
 // Centroid rows are scored by groups of LPR lanes; each lane holds F float4
 // pieces of the latent query, so one warp-wide load covers 32 / LPR whole rows.
 template <int R>
@@ -167,93 +219,97 @@ __device__ __forceinline__ int level_pass(const SelectArgs& a, int l, int ncand,
     const int i = lane * E + e;
     v[e] = i < ncand ? s_key[key_slot<E>(i)] : 0ull;
   }
-  const int B = a.beam[l];
-  if constexpr (E >= 8) {
-    // Threshold first: the B-th largest of the lanes' two largest keys is a lower
-    // bound of the B-th largest key overall (those 64 are keys of the level), so
-    // every kept key is >= tau.  Keys are distinct, so sorting the keys >= tau
-    // gives exactly the first B of the full order; when more than 64 pass, the
-    // full sort runs instead.
-    unsigned long long smp[2] = {0ull, 0ull};
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const unsigned long long x = v[e];
-      const bool top = x > smp[0];
-      smp[1] = top ? smp[0] : (x > smp[1] ? x : smp[1]);
-      smp[0] = top ? x : smp[0];
-    }
-    warp_sort_desc<2>(smp);
-    const unsigned long long tau = __shfl_sync(0xffffffffu, ((B - 1) & 1) ? smp[1] : smp[0], (B - 1) >> 1);
-    int c = 0;
-#pragma unroll
-    for (int e = 0; e < E; ++e) c += (v[e] != 0ull && v[e] >= tau);
-    int inc = c;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, inc, d);
-      if (lane >= d) inc += y;
-    }
-    const int total = __shfl_sync(0xffffffffu, inc, 31);
-    if (total <= 64) {
-      __syncwarp();                       // every lane has read its keys: s_key is free
-      int o = inc - c;
-#pragma unroll
-      for (int e = 0; e < E; ++e)
-        if (v[e] != 0ull && v[e] >= tau) s_key[o++] = v[e];
-      __syncwarp();
-      unsigned long long w[2];
-      w[0] = 2 * lane < total ? s_key[2 * lane] : 0ull;
-      w[1] = 2 * lane + 1 < total ? s_key[2 * lane + 1] : 0ull;
-      warp_sort_desc<2>(w);
-      return emit_kept<2>(w, B, next);
-    }
-  }
-  warp_sort_desc<E>(v);
-  return emit_kept<E>(v, B, next);
+  return warp_keep_best<E>(v, a.beam[l], s_key, next);
 }
 
-// Latent query of (t, g), computed by one warp: the group query (mean of the G
-// query heads) times W[g] (Wg: global or shared memory).  A lane owns columns (2 kp, 2 kp + 1) over the rows
-// j = js, js + JS, ...; the JS row slices are summed by shuffles.  Both select
-// kernels use this routine, so a query's latent (and its walk) does not depend
-// on the batch it is selected in.
+// Latent arithmetic shared by every select kernel, so a query's latent (and its
+// walk) does not depend on the kernel or the batch it is selected in: the group
+// query q (mean of the G query heads, summed in head order) times W[g]; column c
+// is the fixed pairwise sum of kLatParts partial sums, partial p running
+// sequentially over the rows [p DK / kLatParts, (p + 1) DK / kLatParts).
+constexpr int kLatParts = 8;
+
+template <typename T, int R, int DK>
+__device__ __forceinline__ float latent_partial(const float* q, const T* Wg, int c, int p) {
+  constexpr int RPP = DK / kLatParts;
+  float acc = 0.f;
+#pragma unroll 4
+  for (int jj = 0; jj < RPP; ++jj) {
+    const int j = p * RPP + jj;
+    acc = fmaf(q[j], to_f32(Wg[(int64_t)j * R + c]), acc);
+  }
+  return acc;
+}
+__device__ __forceinline__ float latent_combine(const float (&pp)[kLatParts]) {
+  return ((pp[0] + pp[1]) + (pp[2] + pp[3])) + ((pp[4] + pp[5]) + (pp[6] + pp[7]));
+}
+template <typename T, int DK>
+__device__ __forceinline__ float group_mean(const SelectArgs& a, int64_t t, int g, int j) {
+  const T* Q = static_cast<const T*>(a.Q);
+  float sum = 0.f;
+  for (int i = 0; i < a.G; ++i) sum += to_f32(Q[(t * a.Hq + (int64_t)g * a.G + i) * DK + j]);
+  return sum / (float)a.G;
+}
+
+// The latent of (t, g) computed by one warp (Wg: global or shared memory).
 template <typename T, int R, int DK>
 __device__ __forceinline__ void latent_query(const SelectArgs& a, int64_t t, int g, const T* Wg, float* s_q,
                                              float* s_lat) {
+  constexpr int RPP = DK / kLatParts;
   const int lane = threadIdx.x & 31;
-  const T* Q = static_cast<const T*>(a.Q);
-  for (int j = lane; j < DK; j += 32) {
-    float sum = 0.f;
-    for (int i = 0; i < a.G; ++i) sum += to_f32(Q[(t * a.Hq + (int64_t)g * a.G + i) * DK + j]);
-    s_q[j] = sum / (float)a.G;
-  }
+  for (int j = lane; j < DK; j += 32) s_q[j] = group_mean<T, DK>(a, t, g, j);
   __syncwarp();
-  constexpr int JS = 64 / R;
-  const int kp = lane % (R / 2), js = lane / (R / 2);
-  const T* W = Wg + 2 * kp;
-  float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-  for (int j = js; j < DK; j += JS) {
-    float w[2];
-    load2_generic(W + (int64_t)j * R, w);
-    const float qj = s_q[j];
-    acc0 = fmaf(qj, w[0], acc0);
-    acc1 = fmaf(qj, w[1], acc1);
-  }
-#pragma unroll
-  for (int o = R / 2; o < 32; o <<= 1) {
-    acc0 += __shfl_xor_sync(0xffffffffu, acc0, o);
-    acc1 += __shfl_xor_sync(0xffffffffu, acc1, o);
-  }
-  if (js == 0) {
-    s_lat[2 * kp] = acc0;
-    s_lat[2 * kp + 1] = acc1;
+  // lane: columns 2 c2 and 2 c2 + 1 (one 2-element load per row); per column the
+  // same partial sums and pairwise order as latent_partial / latent_combine
+  for (int c2 = lane; c2 < R / 2; c2 += 32) {
+    auto part = [&](int p, float& x0, float& x1) {
+      x0 = 0.f;
+      x1 = 0.f;
+#pragma unroll 4
+      for (int jj = 0; jj < RPP; ++jj) {
+        const int j = p * RPP + jj;
+        float w[2];
+        load2_generic(Wg + (int64_t)j * R + 2 * c2, w);
+        x0 = fmaf(s_q[j], w[0], x0);
+        x1 = fmaf(s_q[j], w[1], x1);
+      }
+    };
+    float a0, a1, b0, b1, lo0, lo1, hi0, hi1, u0, u1;
+    part(0, a0, a1); part(1, b0, b1); lo0 = a0 + b0; lo1 = a1 + b1;
+    part(2, a0, a1); part(3, b0, b1); u0 = a0 + b0; u1 = a1 + b1; lo0 = lo0 + u0; lo1 = lo1 + u1;
+    part(4, a0, a1); part(5, b0, b1); hi0 = a0 + b0; hi1 = a1 + b1;
+    part(6, a0, a1); part(7, b0, b1); u0 = a0 + b0; u1 = a1 + b1; hi0 = hi0 + u0; hi1 = hi1 + u1;
+    const float v0 = lo0 + hi0, v1 = lo1 + hi1;
+    s_lat[2 * c2] = v0;
+    s_lat[2 * c2 + 1] = v1;
     if (a.qlat_out) {
-      a.qlat_out[(t * a.Hkv + g) * R + 2 * kp] = acc0;
-      a.qlat_out[(t * a.Hkv + g) * R + 2 * kp + 1] = acc1;
+      a.qlat_out[(t * a.Hkv + g) * R + 2 * c2] = v0;
+      a.qlat_out[(t * a.Hkv + g) * R + 2 * c2 + 1] = v1;
     }
   }
   __syncwarp();
+}
+
+// The same latent computed by a whole CTA of NT >= max(DK, R * kLatParts) threads
+// (one partial sum per thread); every thread of the CTA must call it.
+template <typename T, int R, int DK, int NT>
+__device__ __forceinline__ void latent_query_cta(const SelectArgs& a, int64_t t, int g, const T* Wg, float* s_q,
+                                                 float (*s_part)[R], float* s_lat) {
+  static_assert(NT >= DK && NT >= R * kLatParts, "");
+  const int tid = threadIdx.x;
+  if (tid < DK) s_q[tid] = group_mean<T, DK>(a, t, g, tid);
+  __syncthreads();
+  if (tid < R * kLatParts) s_part[tid / R][tid % R] = latent_partial<T, R, DK>(s_q, Wg, tid % R, tid / R);
+  __syncthreads();
+  if (tid < R) {
+    float pp[kLatParts];
+#pragma unroll
+    for (int p = 0; p < kLatParts; ++p) pp[p] = s_part[p][tid];
+    const float v = latent_combine(pp);
+    s_lat[tid] = v;
+    if (a.qlat_out) a.qlat_out[(t * a.Hkv + g) * R + tid] = v;
+  }
+  __syncthreads();
 }
 
 // One warp per (query t, KV group g), kSelWarps queries of one group per CTA.
@@ -322,10 +378,6 @@ __global__ void __launch_bounds__(kSelWarps * 32, 3) k_select(SelectArgs a) {
   }
 }
 
-__device__ __forceinline__ void prefetch_l2(const void* p) {
-  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
-}
-
 // Small batches (decode): one CTA of kWideWarps warps per (query t, KV group g),
 // so a level's candidates are scored in one or two memory round trips.  Each
 // warp sorts a chunk of 32 keys; chunk lists are then merged pairwise keeping
@@ -339,12 +391,17 @@ __global__ void __launch_bounds__(kWideWarps * 32) k_select_wide(SelectArgs a) {
   __shared__ unsigned long long s_key[32 * kWideWarps];
   __shared__ __align__(16) T s_w[DK * R];
   __shared__ float s_q[DK];
+  __shared__ float s_part[kLatParts][R];
   __shared__ __align__(16) float s_lat[R];
   __shared__ int32_t s_kept[2][LSA_MAX_BEAM];
   __shared__ int s_valid;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = blockIdx.y;
   const int64_t t = blockIdx.x;
+  // a kernel launched as this one's programmatic dependent (the decode step's
+  // attention) may start now; it waits for this grid to finish before it reads
+  // anything written here
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   if (t == 0) {   // decode step: this head's new key and value rows, the attention's counter
     const int chunks = a.app_row_bytes / 16;
     if (a.app_K && tid < 2 * chunks) {
@@ -358,18 +415,18 @@ __global__ void __launch_bounds__(kWideWarps * 32) k_select_wide(SelectArgs a) {
     }
     if (a.zero_cnt && tid == 0) a.zero_cnt[g] = 0;
   }
-  {  // W[g] staged by the whole CTA in one memory round trip; the top level's rows requested meanwhile
+  {  // W[g] staged by the whole CTA in one memory round trip; the top level's rows are
+     // requested into L2 meanwhile (every walk scores all of them next)
     constexpr int VEC = 16 / sizeof(T);
     const T* W = static_cast<const T*>(a.W) + (int64_t)g * DK * R;
     const char* top = a.tree + a.off_c[0] + (int64_t)g * a.nodes[0] * R * sizeof(float);
-    const int top_lines = (int)((a.nodes[0] * R * (int64_t)sizeof(float) + 127) / 128);
-    for (int x = tid; x < top_lines; x += NT) prefetch_l2(top + (int64_t)x * 128);
+    const int64_t top_lines = (a.nodes[0] * R * (int64_t)sizeof(float) + 127) / 128;
+    for (int64_t x = tid; x < top_lines; x += NT) asm volatile("prefetch.global.L2 [%0];" ::"l"(top + x * 128));
     for (int i = tid * VEC; i < DK * R; i += NT * VEC)
       *reinterpret_cast<uint4*>(&s_w[i]) = __ldg(reinterpret_cast<const uint4*>(W + i));
   }
   __syncthreads();
-  if (warp == 0) latent_query<T, R, DK>(a, t, g, s_w, s_q, s_lat);
-  __syncthreads();
+  latent_query_cta<T, R, DK, NT>(a, t, g, s_w, s_q, s_part, s_lat);
   float4 lat[RS::F];
 #pragma unroll
   for (int f = 0; f < RS::F; ++f) lat[f] = reinterpret_cast<const float4*>(s_lat)[f * RS::LPR + lane % RS::LPR];
@@ -426,27 +483,6 @@ __global__ void __launch_bounds__(kWideWarps * 32) k_select_wide(SelectArgs a) {
           }
           s_key[c] = key;
         }
-      }
-    }
-    // the next level's candidates are children of this level's kept nodes: bring the
-    // children of every candidate into L2 while the keys are sorted (a decode walk is a
-    // chain of dependent reads; this turns the next level's DRAM round trip into an L2 hit)
-    if (l + 1 < a.levels) {
-      const int b1 = a.branching[l + 1];
-      const char* nxt = a.tree + a.off_c[l + 1] + (int64_t)g * a.nodes[l + 1] * R * sizeof(float);
-      const int lines = (b1 * R * (int)sizeof(float) + 127) / 128;   // one candidate's children, 128-B lines
-      for (int x = tid; x < ncand * lines; x += NT) {
-        const int c = x / lines, ln = x % lines;
-        const int64_t id = l == 0 ? c : (int64_t)kept[c / b] * b + (c % b);
-        prefetch_l2(nxt + (id * b1 * R * (int64_t)sizeof(float)) + ln * 128);
-      }
-    } else if (a.leaves_out) {   // last level: the leaf_index slices the attention reads next
-      const char* li = reinterpret_cast<const char*>(a.tree + a.off_leaf) + (int64_t)g * a.n_tree * 4;
-      const int lines = (a.leaf * 4 + 127) / 128;
-      for (int x = tid; x < ncand * lines; x += NT) {
-        const int c = x / lines, ln = x % lines;
-        const int64_t id = l == 0 ? c : (int64_t)kept[c / b] * b + (c % b);
-        prefetch_l2(li + id * a.leaf * 4 + ln * 128);
       }
     }
     __syncthreads();
@@ -716,6 +752,7 @@ static cudaError_t launch_flat(const SelectArgs& a, cudaStream_t st) {
 
 cudaError_t run_select_flat(const SelectArgs& a, int dtype, cudaStream_t st) {
   if (a.T == 0) return cudaSuccess;
+  if (select_flat_tc_supported(a, dtype)) return run_select_flat_tc(a, st);
   return dtype == LSA_BF16 ? launch_flat<__nv_bfloat16>(a, st) : launch_flat<float>(a, st);
 }
 

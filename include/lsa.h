@@ -449,6 +449,9 @@ int lsa_kv_append(void *K, void *V, int32_t n_heads, int64_t n_cap, int32_t d, i
  * Two kernel launches; no host synchronisation.  Requires n_tree - 1 <= pos <
  * n_cap and n_tree <= tail_begin <= pos + 1.  leaves_out (optional, device,
  * [n_heads][beam[levels-1]]) receives the kept leaf ids (-1 pads).
+ * The kept leaves' keys and the tail are attended in chunks of 64 keys, one CTA
+ * each; one call handles up to 17408 / (8 G) chunks at d = 128 bf16 (544 at G = 4)
+ * and returns LSA_ERR_SHAPE beyond that.
  * workspace: lsa_decode_step_workspace_bytes(tree, Hq, d, beam, tail_len_max)
  * bytes with tail_len_max >= pos + 1 - tail_begin; calls that share a workspace
  * must not overlap on the GPU. */

@@ -81,6 +81,15 @@ def test_flat_decode_geometry(lsa):
     print("near-ties", _run(lsa, cfg, 32))
 
 
+def test_flat_ragged_leaves(lsa):
+    """960 leaves per head (the last 128-leaf tile of the tensor-core kernel is half full),
+    two query heads per group, 200 causal queries (a partial query tile)."""
+    cfg = configs.get("prefill_1m").scaled(n=8 * 8 * 5 * 3 * 64, branching=(8, 8, 5, 3), beam=(4, 16, 16, 7),
+                                           Hkv=3, Hq=6, T=200, comps=128)
+    for B in (7, 32):
+        print("near-ties", _run(lsa, cfg, B, seed=11))
+
+
 def test_flat_fp32_small(lsa):
     """fp32, d = 64, r = 16, 256 leaves, no positions; a partial last tile is not possible here,
     so a tree of 16 x 12 leaves (192) gives one."""
