@@ -395,6 +395,13 @@ int lsa_select_flat(const lsa_tree_desc* tree, const void* tree_mem, const void*
   a.T = T; a.Hq = Hq; a.Hkv = tree->n_heads; a.G = Hq / tree->n_heads; a.d = d; a.r = tree->r;
   a.levels = tree->levels; a.leaf = tree->leaf_size; a.beam_max = n_leaves; a.n_tree = tree->n_tree;
   a.off_leaf = tree->off_leaf_index;
+  {   // a prime that does not divide the leaf count: i -> i * p mod n_leaves is a bijection
+    const int64_t NL = tree->nodes[L];
+    const int64_t primes[] = {1000003, 999983, 40503, 7919};
+    a.flat_perm = 1;
+    for (int64_t p : primes)
+      if (NL % p != 0) { a.flat_perm = p % NL == 0 ? 1 : p; break; }
+  }
   cudaError_t e = lsa::run_select_flat(a, dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lsa_select_flat");
   return ok();

@@ -32,7 +32,8 @@ namespace lsa {
 
 namespace {
 
-constexpr int kFT = 128;               // threads = queries per CTA = TMEM lanes
+constexpr int kFT = 128;               // queries per CTA = TMEM lanes
+constexpr int kFTh = 2 * kFT;          // threads: two per query (halves of every leaf tile)
 constexpr int kFN = 128;               // leaves per tile (MMA N)
 constexpr int kFR = 64;                // latent dimension of this path
 constexpr int kFMaxB = 32;             // longest kept list of this path
@@ -45,8 +46,8 @@ struct FlatTcSmem {
   static constexpr uint32_t kB = 3 * kTileB;
   static constexpr uint32_t kW = kB + 6 * kTileB;                 // [64 rows x DK] bf16, K-major
   static constexpr uint32_t kList = kW + kFR * DK * 2;
-  static constexpr uint32_t kMpos = kList + kFMaxB * kFT * 8;
-  static constexpr size_t kBytes = 1024 + kMpos + 2 * kFN * 4;
+  static constexpr uint32_t kMpos = kList + kFMaxB * kFT * 8;   // list region: fp32 row staging, then the lists
+  static constexpr size_t kBytes = 1024 + kMpos + 4 * kFN * 4;   // min positions, then leaf ids, per buffer
 };
 
 // Exact three-way bf16 split of an fp32 value.
@@ -85,8 +86,22 @@ __device__ __forceinline__ void store_split8(char* base, uint32_t stride, int r,
     *reinterpret_cast<uint4*>(base + i * stride + off) = make_uint4(w[i][0], w[i][1], w[i][2], w[i][3]);
 }
 
+// v[i] for a run-time i, by a tree of selects (no local-memory indexing).
+__device__ __forceinline__ float pick32(const float (&v)[32], int i) {
+  float a16[16], a8[8], a4[4], a2[2];
+#pragma unroll
+  for (int k = 0; k < 16; ++k) a16[k] = (i & 16) ? v[k + 16] : v[k];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) a8[k] = (i & 8) ? a16[k + 8] : a16[k];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) a4[k] = (i & 4) ? a8[k + 4] : a8[k];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) a2[k] = (i & 2) ? a4[k + 2] : a4[k];
+  return (i & 1) ? a2[1] : a2[0];
+}
+
 template <int DK>
-__global__ void __launch_bounds__(kFT, 1) k_select_flat_tc(SelectArgs a) {
+__global__ void __launch_bounds__(kFTh, 1) k_select_flat_tc(SelectArgs a) {
   using S = FlatTcSmem<DK>;
   constexpr int NH = DK / 64;                      // 64-column halves of a query / W^T row
   extern __shared__ char smem_raw[];
@@ -95,9 +110,9 @@ __global__ void __launch_bounds__(kFT, 1) k_select_flat_tc(SelectArgs a) {
   __shared__ int s_bad;
   char* base = align1024(smem_raw);
   const uint32_t sbase = smem_u32(base);
-  unsigned long long* list = reinterpret_cast<unsigned long long*>(base + S::kList);   // [B][128]
-  int32_t* s_mpos = reinterpret_cast<int32_t*>(base + S::kMpos);                      // [2][128]
+  int32_t* s_mpos = reinterpret_cast<int32_t*>(base + S::kMpos);   // [2][128] min positions, [2][128] leaf ids
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int row = tid & (kFT - 1), hf = tid / kFT;   // query row (TMEM lane) and half of the columns
   const int g = blockIdx.y;
   const int64_t t0 = (int64_t)blockIdx.x * kFT;
   const int L = a.levels - 1;
@@ -116,7 +131,7 @@ __global__ void __launch_bounds__(kFT, 1) k_select_flat_tc(SelectArgs a) {
   alloc_tmem(&s_taddr, 2 * kFN);
 
   // ---- prologue: the group queries, split in three, and W^T into shared memory ----
-  for (int x = tid; x < kFT * (DK / 8); x += kFT) {
+  for (int x = tid; x < kFT * (DK / 8); x += kFTh) {
     const int r = x / (DK / 8), c = x % (DK / 8);
     const int64_t t = t0 + r;
     float q[8];
@@ -139,7 +154,7 @@ __global__ void __launch_bounds__(kFT, 1) k_select_flat_tc(SelectArgs a) {
     // split i of half (c / 8) at tile (i * NH + c / 8) of the B region
     store_split8(base + S::kB + (c >> 3) * kTileB, NH * kTileB, r, c & 7, q);
   }
-  for (int e = tid; e < kFR * DK; e += kFT) {       // W^T: row = latent column, K-major over d
+  for (int e = tid; e < kFR * DK; e += kFTh) {      // W^T: row = latent column, K-major over d
     const int c = e % kFR, j = e / kFR;
     *reinterpret_cast<__nv_bfloat16*>(base + S::kW + (j >> 6) * (kFR * 128) + tile_off(c, (j & 63) >> 3) +
                                       (j & 7) * 2) = W[e];
@@ -149,7 +164,7 @@ __global__ void __launch_bounds__(kFT, 1) k_select_flat_tc(SelectArgs a) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_taddr;
-  const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+  const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
   bool ok = true;
   if (tid == 0) {   // latent [128 x 64] = sum_i Qbar_i . W, fp32 in TMEM columns [0, 64)
     constexpr uint32_t id_lat = idesc_bf16(128, kFR, false, false);
@@ -167,55 +182,69 @@ __global__ void __launch_bounds__(kFT, 1) k_select_flat_tc(SelectArgs a) {
   }
   ok = __syncthreads_and(mbar_wait(smem_u32(&s_mbar[2]), 0));
   tc_fence_after();
-  const int64_t t = t0 + tid;
+  const int64_t t = t0 + row;
   const int64_t qpos = t < a.T ? (a.q_pos ? (int64_t)a.q_pos[t] : (int64_t)LLONG_MAX) : -1;
-  if (ok) {   // this thread's latent: split into the three A tiles (row tid)
-    float lat[kFR];
-    tmem_ld32(tmem + lane_base, *reinterpret_cast<float(*)[32]>(&lat[0]));
-    tmem_ld32(tmem + lane_base + 32, *reinterpret_cast<float(*)[32]>(&lat[32]));
+  if (ok) {   // this thread's half of its query's latent: split into the three A tiles
+    float lat[32];
+    tmem_ld32(tmem + lane_base + hf * 32, lat);
     if (a.qlat_out && t < a.T) {
-      float* qo = a.qlat_out + (t * a.Hkv + g) * kFR;
+      float* qo = a.qlat_out + (t * a.Hkv + g) * kFR + hf * 32;
 #pragma unroll
-      for (int c = 0; c < kFR; c += 4) *reinterpret_cast<float4*>(qo + c) = make_float4(lat[c], lat[c + 1], lat[c + 2], lat[c + 3]);
+      for (int c = 0; c < 32; c += 4) *reinterpret_cast<float4*>(qo + c) = make_float4(lat[c], lat[c + 1], lat[c + 2], lat[c + 3]);
     }
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
+    for (int c = 0; c < 4; ++c) {
       float x[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) x[e] = lat[c * 8 + e];
-      store_split8(base + S::kA, kTileB, tid, c, x);
+      store_split8(base + S::kA, kTileB, row, hf * 4 + c, x);
     }
   }
 
   // ---- main loop over tiles of kFN leaves ----
   const int ntile = (int)ceil_div(NL, kFN);
-  for (int i = 0; i < B; ++i) list[i * kFT + tid] = 0ull;
-  unsigned long long tau = 0ull;      // smallest kept key once the list is full
-  int nkept = 0;
-  bool bad = false;
-  float crow[kFR];                    // fp32 centroid row of leaf tid of the next tile
-  int32_t cmp = 0;
-  auto load_row = [&](int j) {
-    const int64_t l = min64((int64_t)j * kFN + tid, NL - 1);
-    const float4* src = reinterpret_cast<const float4*>(cent + l * kFR);
+  // the best 32 keys of this thread's query, sorted descending (0 = empty), in registers
+  unsigned long long top[kFMaxB];
 #pragma unroll
-    for (int f = 0; f < kFR / 4; ++f) {
-      const float4 v = __ldg(src + f);
-      crow[4 * f] = v.x; crow[4 * f + 1] = v.y; crow[4 * f + 2] = v.z; crow[4 * f + 3] = v.w;
+  for (int i = 0; i < kFMaxB; ++i) top[i] = 0ull;
+  unsigned long long tau = 0ull;      // top[31]: a key must beat it to enter
+  bool bad = false;
+  int32_t cmp = 0, cleaf = -1;
+  // fp32 centroid rows are staged with cp.async in the list region (row tid, its 16-byte
+  // chunks XOR-swizzled by the row so that the row reads spread over the banks)
+  char* stage = base + S::kList + row * (kFR * 4);
+  auto stage_off = [&](int f) { return (uint32_t)((f ^ (row & 15)) << 4); };
+  // tile j holds the leaves (i * perm) mod NL for i in [j kFN, (j + 1) kFN): neighbouring
+  // leaves score alike, and a scan in tree order would raise each query's threshold slowly
+  auto load_row = [&](int j) {
+    const int64_t i = (int64_t)j * kFN + row;
+    const int64_t l = i < NL ? (i * a.flat_perm) % NL : 0;
+    cleaf = i < NL ? (int32_t)l : -1;
+    const float* src = cent + l * kFR;
+#pragma unroll
+    for (int ff = 0; ff < kFR / 8; ++ff) {   // this half's 8 of the row's 16 chunks
+      const int f = hf * (kFR / 8) + ff;
+      cp_async16(smem_u32(stage + stage_off(f)), src + 4 * f);
     }
+    cp_async_commit();
     cmp = __ldg(&mpos[l]);
   };
   auto store_row = [&](int j) {
     const int buf = j & 1;
     char* bt = base + S::kB + buf * 3 * kTileB;
+    cp_async_wait_prev_n<0>();
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      float x[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = crow[c * 8 + e];
-      store_split8(bt, kTileB, tid, c, x);
+    for (int cc = 0; cc < 4; ++cc) {
+      const int c = hf * 4 + cc;
+      const float4 u = *reinterpret_cast<const float4*>(stage + stage_off(2 * c));
+      const float4 v = *reinterpret_cast<const float4*>(stage + stage_off(2 * c + 1));
+      const float x[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
+      store_split8(bt, kTileB, row, c, x);
     }
-    s_mpos[buf * kFN + tid] = cmp;
+    if (hf == 0) {
+      s_mpos[buf * kFN + row] = cmp;
+      s_mpos[(2 + buf) * kFN + row] = cleaf;
+    }
   };
   auto issue = [&](int j) {           // one thread: the six products of tile j
     const int buf = j & 1;
@@ -257,56 +286,81 @@ __global__ void __launch_bounds__(kFT, 1) k_select_flat_tc(SelectArgs a) {
     tc_fence_after();
     if (!ok) break;
     const int buf = j & 1;
-    const int64_t L0 = (int64_t)j * kFN;
 #pragma unroll 1
-    for (int part = 0; part < kFN / 32; ++part) {
+    for (int part = hf * 2; part < hf * 2 + 2; ++part) {   // this half's 64 columns
       float sc[32];
       tmem_ld32(tmem + buf * kFN + lane_base + part * 32, sc);   // every lane: .sync.aligned
-      if (qpos < 0) continue;
-#pragma unroll 4
+      // candidates against the threshold at the start of the part (a later insert only
+      // raises it, and a key below the current threshold leaves the list unchanged)
+      uint32_t mask = 0u;
+#pragma unroll
       for (int i = 0; i < 32; ++i) {
         const int l = part * 32 + i;
-        const int64_t leaf = L0 + l;
-        if (leaf >= NL || (int64_t)s_mpos[buf * kFN + l] > qpos) continue;
-        if (isnan(sc[i])) {
-          bad = true;
-          continue;
-        }
+        const int32_t leaf = s_mpos[(2 + buf) * kFN + l];
+        const bool elig = qpos >= 0 && leaf >= 0 && (int64_t)s_mpos[buf * kFN + l] <= qpos;
+        const bool nan = isnan(sc[i]);
+        bad |= elig && nan;
         const unsigned long long key =
             ((unsigned long long)orderable(sc[i]) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)leaf);
-        if (key > tau) {
-          int k = nkept < B ? nkept : B - 1;
-          while (k > 0) {
-            const unsigned long long prev = list[(k - 1) * kFT + tid];
-            if (prev > key) break;
-            list[k * kFT + tid] = prev;
-            --k;
-          }
-          list[k * kFT + tid] = key;
-          if (nkept < B) ++nkept;
-          if (nkept == B) tau = list[(B - 1) * kFT + tid];
+        mask |= (elig && !nan && key > tau) ? (1u << i) : 0u;
+      }
+      // one pending candidate per lane per pass through the insertion network: the warp
+      // makes as many passes as its busiest lane has candidates (key 0 changes nothing)
+      while (__any_sync(0xffffffffu, mask != 0u)) {
+        unsigned long long key = 0ull;
+        if (mask) {
+          const int i = __ffs(mask) - 1;
+          mask &= mask - 1u;
+          const int32_t leaf = s_mpos[(2 + buf) * kFN + part * 32 + i];
+          key = ((unsigned long long)orderable(pick32(sc, i)) << 32) |
+                (unsigned long long)(0xffffffffu - (uint32_t)leaf);
         }
+#pragma unroll
+        for (int k = kFMaxB - 1; k > 0; --k) top[k] = top[k] > key ? top[k] : (top[k - 1] > key ? key : top[k - 1]);
+        top[0] = top[0] > key ? top[0] : key;
+        tau = top[kFMaxB - 1];
       }
     }
     tc_fence_before();
+    __syncthreads();   // this tile's leaf ids and min positions are rewritten next iteration
   }
+  cp_async_drain();    // nothing in flight into the staging rows (a timed-out loop may leave one)
+  __syncthreads();     // every product has completed: the B tiles are free
+  // each half's best 32 (B region, [2][32][128]), merged per query into the list region
+  unsigned long long* halves = reinterpret_cast<unsigned long long*>(base + S::kB);
+#pragma unroll
+  for (int i = 0; i < kFMaxB; ++i) halves[(hf * kFMaxB + i) * kFT + row] = top[i];
+  __syncthreads();
+  unsigned long long* list = reinterpret_cast<unsigned long long*>(base + S::kList);   // [32][128]
   __shared__ int32_t s_nk[kFT];
-  s_nk[tid] = qpos >= 0 ? nkept : 0;
+  if (hf == 0) {
+    int ia = 0, ib = 0, nkept = 0;
+    for (int i = 0; i < kFMaxB; ++i) {
+      const unsigned long long x = halves[ia * kFT + row], y = halves[(kFMaxB + ib) * kFT + row];
+      const unsigned long long v = x > y ? x : y;
+      if (x > y) ++ia; else ++ib;
+      list[i * kFT + row] = v;
+      nkept += (i < B && v != 0ull);
+    }
+    s_nk[row] = qpos >= 0 ? nkept : 0;
+  }
   if (bad) s_bad = 1;
   if (!ok && tid == 0) set_status(a.status, LSA_ERR_TIMEOUT);
   __syncthreads();
   if (s_bad && tid == 0) set_status(a.status, LSA_ERR_NONFINITE);
   // outputs: kept leaves in key order (-1 pads), then their keys
-  if (qpos >= 0 && a.leaves_out)
+  if (hf == 0 && qpos >= 0 && a.leaves_out) {
+    const int nkept = s_nk[row];
     for (int i = 0; i < B; ++i)
       a.leaves_out[((int64_t)g * a.T + t) * B + i] =
-          i < nkept ? (int32_t)(0xffffffffu - (uint32_t)(list[i * kFT + tid] & 0xffffffffull)) : -1;
+          i < nkept ? (int32_t)(0xffffffffu - (uint32_t)(list[i * kFT + row] & 0xffffffffull)) : -1;
+  }
   if (a.idx_out) {
     const int lane = tid & 31;
     const int leafn = a.leaf;
     const int64_t K_sel = (int64_t)B * leafn;
     const int32_t* li = reinterpret_cast<const int32_t*>(a.tree + a.off_leaf) + (int64_t)g * a.n_tree;
-    for (int r = warp; r < kFT; r += kFT / 32) {
+    for (int r = warp; r < kFT; r += kFTh / 32) {
       const int64_t tr = t0 + r;
       if (tr >= a.T) break;
       const int nk = s_nk[r];
@@ -346,7 +400,7 @@ cudaError_t run_select_flat_tc(const SelectArgs& a, cudaStream_t st) {
     cudaError_t e = cudaFuncSetAttribute(k_select_flat_tc<DD>, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
                                          (int)smem);                                                          \
     if (e != cudaSuccess) return e;                                                                           \
-    k_select_flat_tc<DD><<<grid, kFT, smem, st>>>(a);                                                         \
+    k_select_flat_tc<DD><<<grid, kFTh, smem, st>>>(a);                                                         \
     return cudaGetLastError();                                                                                \
   }
   LSA_FLAT_TC(64) LSA_FLAT_TC(128)

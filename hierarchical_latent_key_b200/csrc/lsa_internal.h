@@ -110,6 +110,9 @@ struct SelectArgs {
   int64_t app_pos, app_ncap;
   int32_t app_row_bytes;
   int32_t* zero_cnt;
+  // flat search on the tensor cores: leaves are scanned in the order i -> (i * perm) mod
+  // n_leaves (perm coprime with n_leaves), so a query's running threshold rises fast
+  int64_t flat_perm;
 };
 cudaError_t run_select(const SelectArgs& a, int dtype, cudaStream_t st);
 
