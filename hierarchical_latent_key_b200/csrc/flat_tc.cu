@@ -47,7 +47,7 @@ struct FlatTcSmem {
   static constexpr uint32_t kW = kB + 6 * kTileB;                 // [64 rows x DK] bf16, K-major
   static constexpr uint32_t kList = kW + kFR * DK * 2;
   static constexpr uint32_t kMpos = kList + kFMaxB * kFT * 8;   // list region: fp32 row staging, then the lists
-  static constexpr size_t kBytes = 1024 + kMpos + 4 * kFN * 4;   // min positions, then leaf ids, per buffer
+  static constexpr size_t kBytes = 1024 + kMpos + 2 * kFN * 8;   // (min position, leaf id) per column and buffer
 };
 
 // Exact three-way bf16 split of an fp32 value.
@@ -110,7 +110,7 @@ __global__ void __launch_bounds__(kFTh, 1) k_select_flat_tc(SelectArgs a) {
   __shared__ int s_bad;
   char* base = align1024(smem_raw);
   const uint32_t sbase = smem_u32(base);
-  int32_t* s_mpos = reinterpret_cast<int32_t*>(base + S::kMpos);   // [2][128] min positions, [2][128] leaf ids
+  int2* s_ml = reinterpret_cast<int2*>(base + S::kMpos);   // [2][128] (min position, leaf id or -1)
   const int tid = threadIdx.x, warp = tid >> 5;
   const int row = tid & (kFT - 1), hf = tid / kFT;   // query row (TMEM lane) and half of the columns
   const int g = blockIdx.y;
@@ -184,6 +184,9 @@ __global__ void __launch_bounds__(kFTh, 1) k_select_flat_tc(SelectArgs a) {
   tc_fence_after();
   const int64_t t = t0 + row;
   const int64_t qpos = t < a.T ? (a.q_pos ? (int64_t)a.q_pos[t] : (int64_t)LLONG_MAX) : -1;
+  // the same test as min position <= qpos, in 32 bits (every position fits an int32)
+  const int32_t qlim = (int32_t)min64(qpos, (int64_t)INT32_MAX);
+  const bool qok = qpos >= 0;
   if (ok) {   // this thread's half of its query's latent: split into the three A tiles
     float lat[32];
     tmem_ld32(tmem + lane_base + hf * 32, lat);
@@ -241,10 +244,7 @@ __global__ void __launch_bounds__(kFTh, 1) k_select_flat_tc(SelectArgs a) {
       const float x[8] = {u.x, u.y, u.z, u.w, v.x, v.y, v.z, v.w};
       store_split8(bt, kTileB, row, c, x);
     }
-    if (hf == 0) {
-      s_mpos[buf * kFN + row] = cmp;
-      s_mpos[(2 + buf) * kFN + row] = cleaf;
-    }
+    if (hf == 0) s_ml[buf * kFN + row] = make_int2(cmp, cleaf);
   };
   auto issue = [&](int j) {           // one thread: the six products of tile j
     const int buf = j & 1;
@@ -295,9 +295,9 @@ __global__ void __launch_bounds__(kFTh, 1) k_select_flat_tc(SelectArgs a) {
       uint32_t mask = 0u;
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const int l = part * 32 + i;
-        const int32_t leaf = s_mpos[(2 + buf) * kFN + l];
-        const bool elig = qpos >= 0 && leaf >= 0 && (int64_t)s_mpos[buf * kFN + l] <= qpos;
+        const int2 ml = s_ml[buf * kFN + part * 32 + i];   // one 8-byte broadcast read
+        const int32_t leaf = ml.y;
+        const bool elig = qok && leaf >= 0 && ml.x <= qlim;
         const bool nan = isnan(sc[i]);
         bad |= elig && nan;
         const unsigned long long key =
@@ -311,7 +311,7 @@ __global__ void __launch_bounds__(kFTh, 1) k_select_flat_tc(SelectArgs a) {
         if (mask) {
           const int i = __ffs(mask) - 1;
           mask &= mask - 1u;
-          const int32_t leaf = s_mpos[(2 + buf) * kFN + part * 32 + i];
+          const int32_t leaf = s_ml[buf * kFN + part * 32 + i].y;
           key = ((unsigned long long)orderable(pick32(sc, i)) << 32) |
                 (unsigned long long)(0xffffffffu - (uint32_t)leaf);
         }

@@ -838,35 +838,42 @@ __global__ void __launch_bounds__(kTL) k_tl_band(BandArgs a) {
 //
 // Persistent CTAs (one per SM), each walking a contiguous range of chunks with
 // four warp roles joined by mbarriers:
-//   warps 2-3 and 6-7 (two loader groups, alternate chunks): chunk metadata
-//     into shared memory and 16-byte cp.async copies of the chunk's Q rows and
-//     the leaf's K and V rows into one of kPipeStages stages (128B-swizzled
-//     tiles), after an L2 prefetch of the K/V rows two chunks earlier;
-//   warp 11 (one lane, MMA): S = Q.K^T into one of kPipeBufs TMEM buffers, and
+//   warps 8 and 11, 9 and 14 (two loader groups, alternate chunks): chunk
+//     metadata into shared memory and 16-byte cp.async copies of the chunk's Q
+//     rows and the leaf's K and V rows into one of kPipeStages stages
+//     (128B-swizzled tiles), after an L2 prefetch of the K/V rows two chunks
+//     earlier;
+//   warp 10 (one lane, MMA): S = Q.K^T into one of kPipeBufs TMEM buffers, and
 //     once P is in shared memory, O = P.V over the same columns;
-//   warps 0-1 and 12-13 (P, alternate chunks, one TMEM lane per row): P and
+//   warps 0-1 and 2-3 (P, even and odd chunks, one TMEM lane per row): P and
 //     the (m, l) statistics from S;
-//   warps 4-5 and 8-9 (epilogue, alternate chunks, same lanes): O from TMEM to
-//     the partial outputs.
+//   warps 4-5 and 6-7 (epilogue, even and odd chunks, same lanes): O from TMEM
+//     to the partial outputs.
+// A warp reaches only the TMEM lane quarter (warp mod 4), so the rows of even
+// chunks sit in lanes 0-63 and those of odd chunks in lanes 64-127: their M = 128
+// products read the Q (then P) tile from 8 KB below the stage, which puts the
+// chunk's 64 rows in tile rows 64-127.  The softmax and epilogue work of the two
+// parities then runs on all four SM sub-partitions instead of two.
 // Every wait is bounded; on a timeout the CTA records LSA_ERR_TIMEOUT, stops
 // its roles, waits for its copies and MMAs in flight and frees TMEM.
 
 constexpr int kPipeStages = 4;
 constexpr int kPipeBufs = 4;                       // TMEM buffers of 128 columns
-constexpr int kChunkRows = 64;                     // rows of a chunk (TMEM lanes 0-63)
+constexpr int kChunkRows = 64;                     // rows of a chunk (TMEM lanes 0-63 or 64-127)
 constexpr int kPipeLoaders = 64;                   // threads of a loader group (warps 2-3, 6-7)
-constexpr int kPipeThreads = 14 * 32;
+constexpr int kPipeThreads = 15 * 32;              // warps 12 and 13 have no role
 // Stage: Q/P tile [0, 16 KB), K [16, 32 KB), V [32, 48 KB).  The M = 128 products
 // read 128 tile rows; rows 64-127 fall on the next 8 KB of the same stage and
 // belong to no chunk row (their results are never used).
 constexpr uint32_t kStageBytes = 49152;
 constexpr uint32_t kQHalf = kChunkRows * 128;     // bytes between the two 64-column halves of Q
+// odd chunks use odd stages, whose tiles have a whole stage below them to read from
+static_assert(kPipeStages % 2 == 0 && kPipeBufs % 2 == 0 && kQHalf <= kStageBytes, "chunk parity layout");
 
 struct PipeMeta {
   int32_t ent[kPipeStages][kChunkRows];
-  int32_t qpos[kPipeStages][kChunkRows];
-  int32_t pos[kPipeStages][kLeafKeys];
-  int32_t qrow[kPipeStages][kChunkRows];           // global Q row of each tile row (loaders only)
+  int32_t lpos[2][2][kLeafKeys];                   // per loader group and iteration parity: key positions
+  int32_t lqrow[2][2][kChunkRows];                 // and the global Q row of each tile row (loaders only)
   int32_t nvis[kPipeStages][kChunkRows];           // visible keys of each entry: [vlo, nvis)
   int32_t vlo[kPipeStages][kChunkRows];
   int32_t info[kPipeStages][2];                    // head, entries
@@ -941,10 +948,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
     set_status(a.status, LSA_ERR_TIMEOUT);
   };
 
-  if (warp == 2 || warp == 3 || warp == 6 || warp == 7) {
+  if (warp == 8 || warp == 9 || warp == 11 || warp == 14) {
     // ---- loaders: two groups of 64 threads take alternate chunks (and stages);
-    // in a group, lanes (j & 15) x rows (j >> 4) + 4 i copy 16-byte pieces ----
-    const int lt = ((warp & 1) | ((warp >> 1) & 2)) * 32 + lane;
+    // in a group, lanes (j & 15) x rows (j >> 4) + 4 i copy 16-byte pieces.  The
+    // warps of a group sit on different SM sub-partitions. ----
+    const int lt = (warp == 8 ? 0 : warp == 11 ? 1 : warp == 9 ? 2 : 3) * 32 + lane;
     const int group = lt >> 6, j = lt & 63;
     // descriptors come 32 at a time (one per lane) and are broadcast by shuffles;
     // a chunk's metadata is fetched two group iterations before its copies
@@ -1002,17 +1010,23 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       }
       if (k + 4 < N) fetch(k + 4, n2);
       const int s = k % kPipeStages;
-      const bool ok = k < kPipeStages || mbar_wait(smem_u32(&M.sempty[s]), ((k / kPipeStages) - 1) & 1);
       const uint32_t st = sbase + s * kStageBytes;
-      // row addresses through shared memory, so that 16 lanes copy one 256-B row
+      // row addresses through the group's own shared buffers (alternating by
+      // iteration), so that 16 lanes copy one 256-B row; everything that does not
+      // touch the stage is done before waiting for it
       const int n_rows = cur.ne * a.G;
-      if (ok) {
-        M.pos[s][j] = cur.pos;
-        if (j < n_rows) M.qrow[s][j] = (cur.qent >> 6) * a.Hq + cur.g * a.G + j % a.G;
-      }
-      if (loaders_any(!ok || *abort_flag != 0, group)) {   // also the barrier before the copies read them
-        if (!ok) fail();
-        break;
+      int32_t* lpos = M.lpos[group][(k >> 1) & 1];
+      int32_t* lqrow = M.lqrow[group][(k >> 1) & 1];
+      lpos[j] = cur.pos;
+      lqrow[j] = j < n_rows ? (cur.qent >> 6) * a.Hq + cur.g * a.G + j % a.G : -1;
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + group), "n"(kPipeLoaders) : "memory");
+      // visible keys of entry j: position <= q_pos, outside the sink [0, n_sink)
+      // and the window (q_pos - window, q_pos], whose keys the dense part attends
+      int nvis = 0, vlo = 0;
+      if (j < a.epc && cur.ev >= 0) {
+        const int hi = visible_prefix(lpos, (int64_t)cur.eq - a.window);
+        vlo = a.n_sink > 0 ? visible_prefix(lpos, (int64_t)a.n_sink - 1) : 0;
+        nvis = hi > vlo ? hi : vlo;
       }
       const int c = j & 15, rg = j >> 4;
       const int64_t kv_base = (int64_t)cur.g * a.n_cap;
@@ -1021,8 +1035,13 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       int32_t kpos[16], qr[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        kpos[i] = M.pos[s][rg + 4 * i];
-        qr[i] = rg + 4 * i < n_rows ? M.qrow[s][rg + 4 * i] : -1;
+        kpos[i] = lpos[rg + 4 * i];
+        qr[i] = lqrow[rg + 4 * i];
+      }
+      const bool ok = k < kPipeStages || mbar_wait(smem_u32(&M.sempty[s]), ((k / kPipeStages) - 1) & 1);
+      if (loaders_any(!ok || *abort_flag != 0, group)) {   // every thread of the group agrees
+        if (!ok) fail();
+        break;
       }
 #pragma unroll
       for (int i = 0; i < 16; ++i) {   // K and V rows rg, rg + 4, ..., chunk c
@@ -1038,13 +1057,8 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       cp_async_arrive(bar);
       if (j < a.epc) {
         M.ent[s][j] = cur.ev;
-        M.qpos[s][j] = cur.eq;
-        // visible: position <= q_pos, outside the sink [0, n_sink) and the window
-        // (q_pos - window, q_pos], whose keys the dense part attends instead
-        const int hi = cur.ev >= 0 ? visible_prefix(M.pos[s], (int64_t)cur.eq - a.window) : 0;
-        const int lo = cur.ev >= 0 && a.n_sink > 0 ? visible_prefix(M.pos[s], (int64_t)a.n_sink - 1) : 0;
-        M.nvis[s][j] = hi > lo ? hi : lo;
-        M.vlo[s][j] = lo;
+        M.nvis[s][j] = nvis;
+        M.vlo[s][j] = vlo;
       }
       if (j == 0) {
         M.info[s][0] = cur.g;
@@ -1055,7 +1069,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       n1 = n2;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");   // nothing in flight when the CTA exits
-  } else if (warp == 11) {
+  } else if (warp == 10) {
     // ---- MMA issuer ----
     if (lane == 0) {
       constexpr uint32_t id_qk = idesc_bf16(128, 64, false, false);
@@ -1064,7 +1078,9 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
         const int s = k % kPipeStages, b = k % kPipeBufs;
         fence_async_smem();    // the loaders' cp.async writes, seen through the barrier, before the MMA reads
         tc_fence_after();
-        const uint32_t sA = sbase + s * kStageBytes, sK = sA + 16384;
+        // odd chunks: tile rows 64-127 are the chunk's rows (the 8 KB below the stage
+        // feed rows 0-63, whose results are never read)
+        const uint32_t sA = sbase + s * kStageBytes - (k & 1) * kQHalf, sK = sbase + s * kStageBytes + 16384;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t koff = (uint32_t)((kk & 3) * 32);
@@ -1076,7 +1092,7 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       auto pv = [&](int k) {
         const int s = k % kPipeStages, b = k % kPipeBufs;
         tc_fence_after();
-        const uint32_t sP = sbase + s * kStageBytes, sV = sP + 32768;
+        const uint32_t sP = sbase + s * kStageBytes - (k & 1) * kQHalf, sV = sbase + s * kStageBytes + 32768;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
           tc_mma(tmem + b * 128, sdesc_sw128(sP + kk * 32, 16, 1024),
@@ -1121,10 +1137,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       if (!mbar_wait(smem_u32(&M.done), 0)) fail();
     }
     __syncwarp();
-  } else if (warp < 2 || warp == 12 || warp == 13) {
-    // ---- P: two warp pairs take alternate chunks; row r = TMEM lane r ----
+  } else if (warp < 4) {
+    // ---- P: warps 0-1 take the even chunks (TMEM lanes 0-63), warps 2-3 the odd
+    // ones (lanes 64-127); r = the row within the chunk ----
     const int r = (warp & 1) * 32 + lane;
-    const int pgrp = warp >= 12 ? 1 : 0;
+    const int pgrp = warp >> 1;
     const int e = r / a.G, hh = r % a.G;
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
     bool ok = true;
@@ -1188,10 +1205,11 @@ __global__ void __launch_bounds__(kPipeThreads, 1) k_tl_pipe(TreeAttnArgs a) {
       mbar_arrive(smem_u32(&M.pready[s]));
     }
     if (!ok && lane == 0) fail();
-  } else if (warp == 4 || warp == 5 || warp == 8 || warp == 9) {
-    // ---- epilogue: two warp pairs take alternate chunks; row r = TMEM lane r ----
-    const int r = (warp & 3) * 32 + lane;
-    const int egrp = warp >= 8 ? 1 : 0;
+  } else if (warp < 8) {
+    // ---- epilogue: warps 4-5 take the even chunks, warps 6-7 the odd ones (the
+    // TMEM lanes of their P warps); r = the row within the chunk ----
+    const int r = (warp & 1) * 32 + lane;
+    const int egrp = (warp >> 1) & 1;
     bool ok = true;
     for (int k = egrp; k < N; k += 2) {
       if (aborted()) break;
