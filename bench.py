@@ -145,13 +145,17 @@ class Prefill:
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         need = lsa.lsa_tree_attn_workspace_bytes(self.tree.desc, T, Hq, d, self.Q.dtype, cfg.beam[-1])
         self.ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        need = lsa.lsa_select_batched_workspace_bytes(self.tree.desc, T, cfg.beam)
+        self.sel_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
         self.scale = 1.0 / math.sqrt(d)
         self.units = T
-        self.launches_per_step = 1 + 7      # select; tree attention: 3 list + 2 tensor-core passes + 2
+        # batched select: latent + top level, then scan, fill, score and rank per level;
+        # tree attention: 3 list + 2 tensor-core passes + 2
+        self.launches_per_step = 1 + 4 * (len(cfg.beam) - 1) + 7
 
     def select(self, Q=None):
-        self.lsa.lsa_select(self.tree.desc, self.tree.mem, self.Q if Q is None else Q, self.W, self.cfg.beam,
-                            self.q_pos, None, self.leaves, status=self.status)
+        self.lsa.lsa_select_batched(self.tree.desc, self.tree.mem, self.Q if Q is None else Q, self.W, self.cfg.beam,
+                                    self.q_pos, None, self.leaves, workspace=self.sel_ws, status=self.status)
 
     def attend(self, Q=None, O=None, LSE=None):
         self.lsa.lsa_tree_attn(self.tree.desc, self.tree.mem, self.Q if Q is None else Q, self.K, self.V,
@@ -298,6 +302,8 @@ class Train:
         self.attn_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
         need = lsa.lsa_tree_attn_bwd_workspace_bytes(self.desc, T, Hq, d, self.Q.dtype, cfg.beam[-1])
         self.bwd_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+        need = lsa.lsa_select_batched_workspace_bytes(self.desc, T, cfg.beam)
+        self.sel_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
         self.status = torch.zeros(1, dtype=torch.int32, device=dev)
         self.scale = 1.0 / math.sqrt(d)
         self.seed = seed
@@ -307,8 +313,8 @@ class Train:
         return (
             ("build", lambda: L.lsa_build_tree(self.desc, self.tree_mem, self.K, self.W, c.iters, self.seed,
                                               self.build_ws, None, self.status)),
-            ("select", lambda: L.lsa_select(self.desc, self.tree_mem, self.Q, self.W, c.beam, self.q_pos, None,
-                                            self.leaves, status=self.status)),
+            ("select", lambda: L.lsa_select_batched(self.desc, self.tree_mem, self.Q, self.W, c.beam, self.q_pos,
+                                                    None, self.leaves, workspace=self.sel_ws, status=self.status)),
             ("forward", lambda: L.lsa_tree_attn(self.desc, self.tree_mem, self.Q, self.K, self.V, self.leaves,
                                                 self.q_pos, True, self.scale, self.O, self.LSE, self.attn_ws,
                                                 self.status)),

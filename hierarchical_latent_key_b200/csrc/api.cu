@@ -315,9 +315,11 @@ static int beam_checks(const lsa_tree_desc* tree, const int32_t* beam, lsa::Sele
   return LSA_OK;
 }
 
-int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq, int32_t d,
-               int32_t dtype, const void* W, const int32_t* beam, const int32_t* q_pos, int32_t* idx_out,
-               int32_t* leaves_out, float* qlat_out, int32_t* beam_out, int32_t* status, void* stream) {
+// Arguments of lsa_select and lsa_select_batched (same checks); *empty when T == 0.
+static int select_setup(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
+                        int32_t d, int32_t dtype, const void* W, const int32_t* beam, const int32_t* q_pos,
+                        int32_t* idx_out, int32_t* leaves_out, float* qlat_out, int32_t* beam_out, int32_t* status,
+                        lsa::SelectArgs& a, bool* empty) {
   int rc = check_desc(tree);
   if (rc != LSA_OK) return rc;
   if (!beam) return fail(LSA_ERR_INVALID_ARG, "beam must be non-NULL");
@@ -326,21 +328,69 @@ int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, i
   if (d != 64 && d != 128) return fail(LSA_ERR_SHAPE, "d must be 64 or 128 (got %d)", d);
   if (Hq < tree->n_heads || Hq % tree->n_heads) return fail(LSA_ERR_SHAPE, "Hq (%d) must be a multiple of n_heads (%d)", Hq, tree->n_heads);
   if (Hq / tree->n_heads > 64) return fail(LSA_ERR_SHAPE, "more than 64 query heads per group");
-  lsa::SelectArgs a;
   memset(&a, 0, sizeof(a));
   int beam_max = 0;
   if ((rc = beam_checks(tree, beam, a, &beam_max)) != LSA_OK) return rc;
-  if (T == 0) return ok();
+  a.T = T; a.Hq = Hq; a.Hkv = tree->n_heads; a.G = Hq / tree->n_heads; a.d = d; a.r = tree->r;
+  a.levels = tree->levels; a.leaf = tree->leaf_size; a.beam_max = beam_max; a.n_tree = tree->n_tree;
+  a.off_leaf = tree->off_leaf_index;
+  *empty = T == 0;
+  if (T == 0) return LSA_OK;
   if (!tree_mem || !Q || !W) return fail(LSA_ERR_INVALID_ARG, "tree_mem, Q and W must be non-NULL");
   if (!idx_out && !leaves_out) return fail(LSA_ERR_INVALID_ARG, "give idx_out, leaves_out or both");
   a.Q = Q; a.W = W; a.tree = static_cast<const char*>(tree_mem); a.q_pos = q_pos; a.idx_out = idx_out;
   a.leaves_out = leaves_out;
   a.qlat_out = qlat_out; a.beam_out = beam_out; a.status = status;
-  a.T = T; a.Hq = Hq; a.Hkv = tree->n_heads; a.G = Hq / tree->n_heads; a.d = d; a.r = tree->r;
-  a.levels = tree->levels; a.leaf = tree->leaf_size; a.beam_max = beam_max; a.n_tree = tree->n_tree;
-  a.off_leaf = tree->off_leaf_index;
+  return LSA_OK;
+}
+
+int lsa_select(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq, int32_t d,
+               int32_t dtype, const void* W, const int32_t* beam, const int32_t* q_pos, int32_t* idx_out,
+               int32_t* leaves_out, float* qlat_out, int32_t* beam_out, int32_t* status, void* stream) {
+  lsa::SelectArgs a;
+  bool empty = false;
+  int rc = select_setup(tree, tree_mem, Q, T, Hq, d, dtype, W, beam, q_pos, idx_out, leaves_out, qlat_out, beam_out,
+                        status, a, &empty);
+  if (rc != LSA_OK) return rc;
+  if (empty) return ok();
   cudaError_t e = lsa::run_select(a, dtype, static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "lsa_select");
+  return ok();
+}
+
+// the batched schedule packs (query, rank) into 32 bits: query * 32 + rank
+static constexpr int32_t kBatchedMaxT = 1 << 26;
+
+int lsa_select_batched_workspace_bytes(const lsa_tree_desc* tree, int32_t T, const int32_t* beam, size_t* bytes) {
+  int rc = check_desc(tree);
+  if (rc != LSA_OK) return rc;
+  if (!bytes) return fail(LSA_ERR_INVALID_ARG, "bytes must be non-NULL");
+  if (T < 0 || T > kBatchedMaxT) return fail(LSA_ERR_SHAPE, "T must be in [0, 2^26] (got %d)", T);
+  lsa::SelectArgs a;
+  memset(&a, 0, sizeof(a));
+  int beam_max = 0;
+  if ((rc = beam_checks(tree, beam, a, &beam_max)) != LSA_OK) return rc;
+  a.T = T; a.Hkv = tree->n_heads; a.r = tree->r; a.levels = tree->levels;
+  *bytes = lsa::select_nodes_workspace_bytes(a);
+  return ok();
+}
+
+int lsa_select_batched(const lsa_tree_desc* tree, const void* tree_mem, const void* Q, int32_t T, int32_t Hq,
+                       int32_t d, int32_t dtype, const void* W, const int32_t* beam, const int32_t* q_pos,
+                       int32_t* idx_out, int32_t* leaves_out, float* qlat_out, int32_t* beam_out, void* workspace,
+                       size_t workspace_bytes, int32_t* status, void* stream) {
+  lsa::SelectArgs a;
+  bool empty = false;
+  int rc = select_setup(tree, tree_mem, Q, T, Hq, d, dtype, W, beam, q_pos, idx_out, leaves_out, qlat_out, beam_out,
+                        status, a, &empty);
+  if (rc != LSA_OK) return rc;
+  if (T > kBatchedMaxT) return fail(LSA_ERR_SHAPE, "T must be <= 2^26 (got %d)", T);
+  if (empty) return ok();
+  const size_t need = lsa::select_nodes_workspace_bytes(a);
+  if (need > 0 && (!workspace || workspace_bytes < need))
+    return fail(LSA_ERR_WORKSPACE, "workspace of %zu bytes needed (got %zu)", need, workspace_bytes);
+  cudaError_t e = lsa::run_select_nodes(a, dtype, workspace, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lsa_select_batched");
   return ok();
 }
 

@@ -115,6 +115,11 @@ struct SelectArgs {
   int64_t flat_perm;
 };
 cudaError_t run_select(const SelectArgs& a, int dtype, cudaStream_t st);
+// The same search scheduled level by level over (walk, parent) pairs grouped by
+// parent, for large batches; kept lists and outputs equal run_select's bit for bit.
+// ws: select_nodes_workspace_bytes(a) bytes of device memory (a.levels >= 2).
+size_t select_nodes_workspace_bytes(const SelectArgs& a);
+cudaError_t run_select_nodes(const SelectArgs& a, int dtype, void* ws, cudaStream_t st);
 
 // Decode attention (decode.cu): one query token, keys = the kept leaves of every
 // KV group (leaf_index slices) + the tail [tail_begin, tail_end), split into

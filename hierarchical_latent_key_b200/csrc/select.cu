@@ -22,6 +22,7 @@
 
 #include "lsa_common.cuh"
 #include "lsa_internal.h"
+#include "tc_sm100.cuh"
 
 namespace lsa {
 
@@ -550,6 +551,584 @@ static cudaError_t launch_select(const SelectArgs& a, cudaStream_t st) {
   LSA_SEL(16, 64) LSA_SEL(32, 64) LSA_SEL(64, 64) LSA_SEL(16, 128) LSA_SEL(32, 128) LSA_SEL(64, 128)
 #undef LSA_SEL
   return cudaErrorInvalidValue;
+}
+
+// ---- node-major schedule for large batches ------------------------------------
+//
+// The same search, with the same arithmetic, as k_select, reordered for many
+// queries.  At prefill every upper-level node is kept by hundreds of (query,
+// group) walks, and a walk-by-walk schedule reads the node's children from L2
+// once per walk.  Here every level after the first is one pass over the (walk,
+// kept parent) pairs grouped by parent (a counting sort, like the attention's
+// leaf lists): consecutive threads score the children of one parent, so those
+// centroid rows are read once into L1 and then served from there.  Each score
+// goes to the walk's candidate list at the slot the walk-by-walk kernel uses
+// (rank of the parent x branching + child), and a warp per walk keeps the best
+// beam[l] with the same ranking code.  A score is the fp32 expression of
+// level_pass: four sequential FMA chains, chain s over the float4 pieces
+// 4 f + s of the row, then (s0 + s1) + (s2 + s3), which is what its lane-group
+// butterfly computes; so every kept list equals k_select's bit for bit.
+struct NodeSel {
+  SelectArgs a;
+  float* lat;                 // [Hkv][T][r] latent queries
+  int32_t* kept;              // [2][Hkv][T][32] kept node ids by level parity, -1 padded
+  int32_t* nkept;             // [Hkv][T] number of real nodes kept at the last ranked level
+  int32_t* cnt[2];            // [Hkv][max_par] walks per kept node, by level parity
+  int32_t* off;               // [Hkv][max_par + 1] first grouped entry of each parent
+  uint32_t* ent;              // [Hkv][T * 32] walk * 32 + rank of the parent, grouped by parent
+  int32_t* epar;              // [Hkv][T * 32] the parent of each grouped entry
+  unsigned long long* cand;   // [Hkv][T][cstride] candidate keys of the level being ranked
+  int64_t max_par, cstride;
+};
+
+// Level l's kept nodes of walk (g, t), next[0, valid) in rank order: beam_out;
+// then either the lists and parent counts for level l + 1 or, on the last level,
+// the outputs (as k_select writes them).  Called by a whole warp.
+__device__ __forceinline__ void sn_emit(const NodeSel& s, int l, int g, int64_t t, const int32_t* next, int valid) {
+  const SelectArgs& a = s.a;
+  const int lane = threadIdx.x & 31;
+  if (a.beam_out && lane < a.beam_max)
+    a.beam_out[(((int64_t)l * a.Hkv + g) * a.T + t) * a.beam_max + lane] = lane < valid ? next[lane] : -1;
+  if (l + 1 < a.levels) {
+    s.kept[(((int64_t)(l & 1) * a.Hkv + g) * a.T + t) * LSA_MAX_BEAM + lane] = lane < valid ? next[lane] : -1;
+    if (lane == 0) s.nkept[(int64_t)g * a.T + t] = valid;
+    if (lane < valid) atomicAdd(&s.cnt[l & 1][(int64_t)g * s.max_par + next[lane]], 1);
+    return;
+  }
+  const int leaf = a.leaf;
+  const int B = a.beam[l];
+  if (a.leaves_out && lane < B) a.leaves_out[((int64_t)g * a.T + t) * B + lane] = lane < valid ? next[lane] : -1;
+  if (a.idx_out) {
+    const int64_t K_sel = (int64_t)B * leaf;
+    const int32_t* li = reinterpret_cast<const int32_t*>(a.tree + a.off_leaf) + (int64_t)g * a.n_tree;
+    int32_t* out = a.idx_out + ((int64_t)g * a.T + t) * K_sel;
+    for (int64_t i = lane; i < K_sel; i += 32) {
+      const int k = (int)(i / leaf), q = (int)(i % leaf);
+      out[i] = k < valid ? __ldg(&li[(int64_t)next[k] * leaf + q]) : -1;
+    }
+  }
+}
+
+// Latents of kSnLatQ queries of one group per CTA: W[g] and the group means
+// (transposed) in shared memory; a thread computes 4 queries x 4 columns, so two
+// 16-byte shared loads feed 16 FMAs.  Per (query, column) the arithmetic is
+// latent_query's: group mean summed in head order, kLatParts sequential partial
+// sums, combined ((p0 + p1) + (p2 + p3)) + ((p4 + p5) + (p6 + p7)).
+constexpr int kSnLatQ = 32;
+template <typename T, int R, int DK>
+__global__ void __launch_bounds__(128) k_sn_latent(NodeSel s) {
+  const SelectArgs& a = s.a;
+  constexpr int RPP = DK / kLatParts;
+  static_assert(kLatParts == 8, "the combine below is written for 8 partial sums");
+  __shared__ __align__(16) float s_w[DK * R];
+  __shared__ __align__(16) float s_qt[DK][kSnLatQ];
+  const int g = blockIdx.y, tid = threadIdx.x;
+  const int64_t t0 = (int64_t)blockIdx.x * kSnLatQ;
+  const T* Wg = static_cast<const T*>(a.W) + (int64_t)g * DK * R;
+  // every load of the two staging loops is independent of the others (4 elements each)
+#pragma unroll
+  for (int k = 0; k < DK * R / 4 / 128; ++k) {
+    const int i = (k * 128 + tid) * 4;
+    float v[4];
+    load4(Wg + i, v);
+    *reinterpret_cast<float4*>(&s_w[i]) = make_float4(v[0], v[1], v[2], v[3]);
+  }
+  const T* Q = static_cast<const T*>(a.Q);
+#pragma unroll
+  for (int k = 0; k < kSnLatQ * DK / 4 / 128; ++k) {
+    const int i = k * 128 + tid;
+    const int q = i % kSnLatQ, j = (i / kSnLatQ) * 4;   // a warp: 32 queries, one j block
+    const int64_t t = t0 + q;
+    float m[4] = {0.f, 0.f, 0.f, 0.f};
+    if (t < a.T) {   // group mean as group_mean: heads summed in order, then / G
+      for (int h = 0; h < a.G; ++h) {
+        float v[4];
+        load4(Q + (t * a.Hq + (int64_t)g * a.G + h) * DK + j, v);
+#pragma unroll
+        for (int x = 0; x < 4; ++x) m[x] += v[x];
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x) m[x] = m[x] / (float)a.G;
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) s_qt[j + x][q] = m[x];
+  }
+  __syncthreads();
+  for (int blk = tid; blk < (R / 4) * (kSnLatQ / 4); blk += 128) {
+    const int c0 = (blk % (R / 4)) * 4, q0 = (blk / (R / 4)) * 4;
+    float lo[4][4], hi[4][4], pr[4][4], cur[4][4];
+    for (int p = 0; p < kLatParts; ++p) {
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) cur[x][y] = 0.f;
+#pragma unroll 4
+      for (int jj = 0; jj < RPP; ++jj) {
+        const int j = p * RPP + jj;
+        const float4 qv = *reinterpret_cast<const float4*>(&s_qt[j][q0]);
+        const float4 wv = *reinterpret_cast<const float4*>(&s_w[j * R + c0]);
+        const float qa[4] = {qv.x, qv.y, qv.z, qv.w}, wa[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+        for (int x = 0; x < 4; ++x)
+#pragma unroll
+          for (int y = 0; y < 4; ++y) cur[x][y] = fmaf(qa[x], wa[y], cur[x][y]);
+      }
+      // pairwise tree: pr = p_even; then (p_even + p_odd) folded into lo / hi
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) {
+          if ((p & 1) == 0) {
+            pr[x][y] = cur[x][y];
+          } else {
+            const float pair = pr[x][y] + cur[x][y];
+            if (p == 1) lo[x][y] = pair;
+            else if (p == 3) lo[x][y] = lo[x][y] + pair;
+            else if (p == 5) hi[x][y] = pair;
+            else hi[x][y] = hi[x][y] + pair;
+          }
+        }
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+      const int64_t t = t0 + q0 + x;
+      if (t >= a.T) break;
+      const float4 v = make_float4(lo[x][0] + hi[x][0], lo[x][1] + hi[x][1], lo[x][2] + hi[x][2],
+                                   lo[x][3] + hi[x][3]);
+      *reinterpret_cast<float4*>(s.lat + ((int64_t)g * a.T + t) * R + c0) = v;
+      if (a.qlat_out) *reinterpret_cast<float4*>(a.qlat_out + (t * a.Hkv + g) * R + c0) = v;
+    }
+  }
+}
+
+// Level 0, one warp per walk (level_pass as in k_select, on the stored latent).
+template <int R>
+__global__ void __launch_bounds__(kSelWarps * 32) k_sn_top(NodeSel s) {
+  using RS = RowSplit<R>;
+  const SelectArgs& a = s.a;
+  __shared__ unsigned long long s_key[kSelWarps][32 * kSelMaxE];
+  __shared__ int32_t s_next[kSelWarps][LSA_MAX_BEAM];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = blockIdx.y;
+  const int64_t t = (int64_t)blockIdx.x * kSelWarps + warp;
+  if (t >= a.T) return;
+  const float4* lq = reinterpret_cast<const float4*>(s.lat + ((int64_t)g * a.T + t) * R);
+  float4 lat[RS::F];
+#pragma unroll
+  for (int f = 0; f < RS::F; ++f) lat[f] = lq[f * RS::LPR + lane % RS::LPR];
+  const int64_t qpos = a.q_pos ? (int64_t)a.q_pos[t] : (int64_t)LLONG_MAX;
+  const bool all_eligible = qpos >= a.n_tree - 1;
+  const int ncand = (int)a.nodes[0];
+  const float* cent = reinterpret_cast<const float*>(a.tree + a.off_c[0]) + (int64_t)g * a.nodes[0] * R;
+  const int32_t* mpos = reinterpret_cast<const int32_t*>(a.tree + a.off_m[0]) + (int64_t)g * a.nodes[0];
+  bool bad = false;
+  int valid;
+#define LSA_LEVEL0(EE) \
+  level_pass<R, EE>(a, 0, ncand, cent, mpos, all_eligible, qpos, lat, nullptr, a.branching[0], s_key[warp], s_next[warp], bad)
+  if (ncand <= 32) valid = LSA_LEVEL0(1);
+  else if (ncand <= 64) valid = LSA_LEVEL0(2);
+  else if (ncand <= 128) valid = LSA_LEVEL0(4);
+  else if (ncand <= 256) valid = LSA_LEVEL0(8);
+  else valid = LSA_LEVEL0(16);
+#undef LSA_LEVEL0
+  __syncwarp();
+  if (__any_sync(0xffffffffu, bad) && lane == 0) set_status(a.status, LSA_ERR_NONFINITE);
+  sn_emit(s, 0, g, t, s_next[warp], valid);
+}
+
+// Per group: off = exclusive prefix sum of cnt over np parents (off[np] = total),
+// cnt reset to 0 (the fill's cursors), and the next level's counts zeroed.
+__global__ void __launch_bounds__(1024) k_sn_scan(int32_t* cnt, int32_t* cnt_next, int32_t* off, int64_t max_par,
+                                                  int64_t np, int64_t n_next) {
+  __shared__ int32_t s_warp[32];
+  const int g = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t* c = cnt + (int64_t)g * max_par;
+  int32_t* o = off + (int64_t)g * (max_par + 1);
+  const int64_t per = ceil_div(np, (int64_t)1024);
+  const int64_t lo = min64((int64_t)tid * per, np), hi = min64(lo + per, np);
+  int32_t sum = 0;
+  for (int64_t i = lo; i < hi; ++i) sum += c[i];
+  int32_t inc = sum;
+#pragma unroll
+  for (int d = 1; d < 32; d <<= 1) {
+    const int32_t y = __shfl_up_sync(0xffffffffu, inc, d);
+    if (lane >= d) inc += y;
+  }
+  if (lane == 31) s_warp[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = s_warp[lane];
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+      const int32_t y = __shfl_up_sync(0xffffffffu, w, d);
+      if (lane >= d) w += y;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  int32_t run = inc - sum + (warp ? s_warp[warp - 1] : 0);
+  for (int64_t i = lo; i < hi; ++i) {
+    o[i] = run;
+    run += c[i];
+    c[i] = 0;
+  }
+  if (tid == 1023) o[np] = s_warp[31];
+  int32_t* cn = cnt_next + (int64_t)g * max_par;
+  for (int64_t i = tid; i < n_next; i += 1024) cn[i] = 0;
+}
+
+// (walk, rank) pairs of level l - 1's kept lists grouped by parent: a CTA takes
+// kSnFillWalks walks, counts its pairs per parent in shared memory, reserves one
+// range per parent it met with a single global atomic, then places its pairs (the
+// order inside a parent's range is arbitrary; nothing depends on it).  Above
+// kSnFillPar parents every pair reserves its slot with its own atomic.
+constexpr int kSnFillWalks = 128;
+constexpr int kSnFillPar = 4096;
+__global__ void __launch_bounds__(256) k_sn_fill(NodeSel s, int l) {
+  const SelectArgs& a = s.a;
+  __shared__ int32_t s_h[kSnFillPar];
+  const int g = blockIdx.y, tid = threadIdx.x;
+  const int Bp = a.beam[l - 1];
+  const int64_t np = a.nodes[l - 1];
+  const int64_t w0 = (int64_t)blockIdx.x * kSnFillWalks;
+  const int64_t nw = min64(kSnFillWalks, a.T - w0);
+  const int32_t* kept = s.kept + (((int64_t)((l - 1) & 1) * a.Hkv + g) * a.T + w0) * LSA_MAX_BEAM;
+  const int32_t* off = s.off + (int64_t)g * (s.max_par + 1);
+  int32_t* cur = s.cnt[(l - 1) & 1] + (int64_t)g * s.max_par;
+  uint32_t* ent = s.ent + (int64_t)g * a.T * LSA_MAX_BEAM;
+  int32_t* epar = s.epar + (int64_t)g * a.T * LSA_MAX_BEAM;
+  const int64_t ne = nw * Bp;
+  if (np > kSnFillPar) {
+    for (int64_t i = tid; i < ne; i += 256) {
+      const int64_t w = i / Bp;
+      const int rank = (int)(i % Bp);
+      const int32_t p = kept[w * LSA_MAX_BEAM + rank];
+      if (p < 0) continue;
+      const int64_t pos = off[p] + atomicAdd(&cur[p], 1);
+      ent[pos] = (uint32_t)((w0 + w) * LSA_MAX_BEAM + rank);
+      epar[pos] = p;
+    }
+    return;
+  }
+  for (int64_t p = tid; p < np; p += 256) s_h[p] = 0;
+  __syncthreads();
+  for (int64_t i = tid; i < ne; i += 256) {
+    const int32_t p = kept[(i / Bp) * LSA_MAX_BEAM + i % Bp];
+    if (p >= 0) atomicAdd(&s_h[p], 1);
+  }
+  __syncthreads();
+  for (int64_t p = tid; p < np; p += 256) {
+    const int32_t c = s_h[p];
+    s_h[p] = c > 0 ? off[p] + atomicAdd(&cur[p], c) : 0;
+  }
+  __syncthreads();
+  for (int64_t i = tid; i < ne; i += 256) {
+    const int64_t w = i / Bp;
+    const int rank = (int)(i % Bp);
+    const int32_t p = kept[w * LSA_MAX_BEAM + rank];
+    if (p < 0) continue;
+    const int32_t pos = atomicAdd(&s_h[p], 1);
+    ent[pos] = (uint32_t)((w0 + w) * LSA_MAX_BEAM + rank);
+    epar[pos] = p;
+  }
+}
+
+// Children j0 + 4 c + jl (c < CPL) of one entry: level_pass's score (four FMA
+// chains, chain = float4 piece index mod 4, pieces in order, then (s0 + s1) +
+// (s2 + s3)) and key, written to out[j].  An index past b reads child b - 1 and is
+// dropped.  Returns whether a score was NaN.
+template <int R, int CPL>
+__device__ __forceinline__ bool score_children(const float4* q, const float* rows, int stride,
+                                               const int32_t* mp, int64_t id0, int b, int j0, int jl,
+                                               bool all_eligible, int64_t qpos, unsigned long long* out) {
+  const float4* r4[CPL];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    const int j = min(j0 + 4 * c + jl, b - 1);
+    r4[c] = reinterpret_cast<const float4*>(rows + (int64_t)j * stride);
+  }
+  float acc[CPL][4];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c)
+#pragma unroll
+    for (int h = 0; h < 4; ++h) acc[c][h] = 0.f;
+#pragma unroll
+  for (int k = 0; k < R / 4; ++k) {
+    const float4 w = q[k];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const float4 x = r4[c][k];
+      float& y = acc[c][k & 3];
+      y = fmaf(w.x, x.x, y);
+      y = fmaf(w.y, x.y, y);
+      y = fmaf(w.z, x.z, y);
+      y = fmaf(w.w, x.w, y);
+    }
+  }
+  bool bad = false;
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    const int j = j0 + 4 * c + jl;
+    if (j < b) {
+      unsigned long long key = 0ull;
+      if (all_eligible || (int64_t)mp[j] <= qpos) {
+        const float sc = (acc[c][0] + acc[c][1]) + (acc[c][2] + acc[c][3]);
+        if (isnan(sc)) bad = true;
+        else key = ((unsigned long long)orderable(sc) << 32) | (unsigned long long)(0xffffffffu - (uint32_t)(id0 + j));
+      }
+      out[j] = key;
+    }
+  }
+  return bad;
+}
+
+// Level l: a CTA takes `chunk` consecutive grouped entries; their parents form a
+// contiguous id range whose children are contiguous rows of the level, staged in
+// shared memory when they fit (they do unless the parents have very few walks
+// each).  A warp scores 8 entries at a time, 4 lanes per entry: lane jl takes the
+// children jl, jl + 4, ... (CPL = ceil(b / 4) of them, up to 4 at a time), and the
+// 4 lanes of an entry store consecutive keys.  The entries' latents reach a
+// per-warp double buffer with cp.async (each lane copies a quarter): the next
+// group's copies and the entries of the group after it are in flight while the
+// current group is scored.
+constexpr int kSnChunk = 512;   // entries per CTA at most (the host may pick fewer)
+constexpr int kSnRows = 128;    // staged child rows
+template <int R>
+struct SnScoreSmem {
+  static constexpr int RP = R + 4;   // row stride in floats: the 8 rows a warp reads at once hit different banks
+  static constexpr size_t kRows = 0;
+  static constexpr size_t kLat = kRows + (size_t)kSnRows * RP * 4;
+  static constexpr size_t kMp = kLat + (size_t)8 * 2 * 8 * RP * 4;
+  static constexpr size_t kBytes = kMp + (size_t)kSnRows * 4;
+};
+template <int R, int CPL>
+__global__ void __launch_bounds__(256, 2) k_sn_score(NodeSel s, int l, int chunk) {
+  using S = SnScoreSmem<R>;
+  constexpr int RP = S::RP;
+  constexpr int QP = R / 16;  // latent pieces (float4) a lane copies
+  const SelectArgs& a = s.a;
+  extern __shared__ __align__(16) char sn_smem[];
+  float* s_row = reinterpret_cast<float*>(sn_smem + S::kRows);
+  int32_t* s_mp = reinterpret_cast<int32_t*>(sn_smem + S::kMp);
+  const int g = blockIdx.y, tid = threadIdx.x;
+  const int64_t n = s.off[(int64_t)g * (s.max_par + 1) + a.nodes[l - 1]];
+  const int64_t e0 = (int64_t)blockIdx.x * chunk;
+  if (e0 >= n) return;
+  const int64_t e1 = min64(e0 + chunk, n);
+  const uint32_t* ent = s.ent + (int64_t)g * a.T * LSA_MAX_BEAM;
+  const int32_t* epar = s.epar + (int64_t)g * a.T * LSA_MAX_BEAM;
+  const int b = a.branching[l];
+  const int64_t pa = epar[e0], pb = epar[e1 - 1];
+  const int64_t nrows = (pb - pa + 1) * b;
+  const bool staged = nrows <= kSnRows;
+  const float* cent = reinterpret_cast<const float*>(a.tree + a.off_c[l]) + (int64_t)g * a.nodes[l] * R;
+  const int32_t* mpos = reinterpret_cast<const int32_t*>(a.tree + a.off_m[l]) + (int64_t)g * a.nodes[l];
+  if (staged) {   // rows pa*b .. pa*b + nrows - 1, contiguous in the level
+    const float4* src = reinterpret_cast<const float4*>(cent + pa * b * R);
+    for (int i = tid; i < nrows * (R / 4); i += 256)
+      reinterpret_cast<float4*>(s_row)[(i / (R / 4)) * (RP / 4) + i % (R / 4)] = __ldg(&src[i]);
+    for (int i = tid; i < nrows; i += 256) s_mp[i] = __ldg(&mpos[pa * b + i]);
+  }
+  __syncthreads();
+  const int lane = tid & 31, warp = tid >> 5, jl = lane & 3, el = lane >> 2;
+  const int stride = staged ? RP : R;
+  const float* lat = s.lat + (int64_t)g * a.T * R;
+  float* wl = reinterpret_cast<float*>(sn_smem + S::kLat) + warp * 2 * 8 * RP;   // [2][8][RP]
+  bool bad = false;
+  // group k of this warp: entries e0 + (warp + 8 k) * 8 + el
+  auto entry_of = [&](int64_t i, int64_t& t, int& rank, int64_t& p) {
+    t = -1; rank = 0; p = 0;
+    if (i < e1) {
+      const uint32_t e = ent[i];
+      p = epar[i];
+      t = e / LSA_MAX_BEAM;
+      rank = (int)(e % LSA_MAX_BEAM);
+    }
+  };
+  // this lane's quarter of walk t's latent into buffer buf, entry slot el
+  auto copy_lat = [&](int64_t t, int buf) {
+    if (t >= 0) {
+#pragma unroll
+      for (int k = 0; k < QP; ++k)
+        cp_async16(smem_u32(wl + (buf * 8 + el) * RP + (k * 4 + jl) * 4), lat + t * R + (k * 4 + jl) * 4);
+    }
+    cp_async_commit();
+  };
+  auto pos_of = [&](int64_t t) { return t >= 0 && a.q_pos ? (int64_t)a.q_pos[t] : (int64_t)LLONG_MAX; };
+  int64_t i = e0 + warp * 8 + el;
+  int64_t t_c, p_c, t_n, p_n;
+  int r_c, r_n;
+  entry_of(i, t_c, r_c, p_c);
+  copy_lat(t_c, 0);
+  int64_t qp_c = pos_of(t_c);
+  entry_of(i + 64, t_n, r_n, p_n);
+  for (int buf = 0; i - el < e1; i += 64, buf ^= 1) {
+    // in flight while this group is scored: the next group's latents and position,
+    // the entries of the group after it
+    copy_lat(t_n, buf ^ 1);
+    const int64_t qp_n = pos_of(t_n);
+    int64_t t_f, p_f;
+    int r_f;
+    entry_of(i + 128, t_f, r_f, p_f);
+    cp_async_wait_prev();   // this lane's copies of the current group have landed
+    __syncwarp();
+    if (t_c >= 0) {
+      const bool all_eligible = qp_c >= a.n_tree - 1;
+      const float* rows = staged ? s_row + (p_c - pa) * b * RP : cent + p_c * b * R;
+      const int32_t* mp = staged ? s_mp + (p_c - pa) * b : mpos + p_c * b;
+      unsigned long long* out = s.cand + ((int64_t)g * a.T + t_c) * s.cstride + (int64_t)r_c * b;
+      const float4* q = reinterpret_cast<const float4*>(wl + (buf * 8 + el) * RP);
+      for (int j0 = 0; j0 < b; j0 += 4 * CPL)
+        bad |= score_children<R, CPL>(q, rows, stride, mp, p_c * b, b, j0, jl, all_eligible, qp_c, out);
+    }
+    __syncwarp();   // this buffer is refilled two groups later
+    t_c = t_n; r_c = r_n; p_c = p_n; qp_c = qp_n;
+    t_n = t_f; r_n = r_f; p_n = p_f;
+  }
+  cp_async_drain();
+  if (bad) set_status(a.status, LSA_ERR_NONFINITE);
+}
+
+// Level l: one warp per walk keeps the best beam[l] of its candidate list.
+template <int E>
+__global__ void __launch_bounds__(kSelWarps * 32) k_sn_rank(NodeSel s, int l) {
+  const SelectArgs& a = s.a;
+  __shared__ unsigned long long s_key[kSelWarps][64];
+  __shared__ int32_t s_next[kSelWarps][LSA_MAX_BEAM];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = blockIdx.y;
+  const int64_t t = (int64_t)blockIdx.x * kSelWarps + warp;
+  if (t >= a.T) return;
+  const int ncand = s.nkept[(int64_t)g * a.T + t] * a.branching[l];
+  const unsigned long long* cl = s.cand + ((int64_t)g * a.T + t) * s.cstride;
+  // candidate e * 32 + lane in register e: coalesced loads, and a lane's keys come
+  // from different parents, so the threshold of warp_keep_best (the beam-th best of
+  // the lanes' two best keys) usually leaves at most 64 keys to sort.  The kept set
+  // and its order depend only on the keys, not on where they sit.
+  unsigned long long v[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int i = e * 32 + lane;
+    v[e] = i < ncand ? cl[i] : 0ull;
+  }
+  const int valid = warp_keep_best<E>(v, a.beam[l], s_key[warp], s_next[warp]);
+  __syncwarp();
+  sn_emit(s, l, g, t, s_next[warp], valid);
+}
+
+// Workspace regions (256-byte aligned) of the node-major schedule.
+struct NodeSelLayout {
+  size_t lat, kept, nkept, cnt0, cnt1, off, ent, epar, cand, bytes;
+  int64_t max_par, cstride;
+};
+static NodeSelLayout node_sel_layout(const SelectArgs& a) {
+  NodeSelLayout L{};
+  L.max_par = 1;
+  L.cstride = 1;
+  for (int l = 1; l < a.levels; ++l) {
+    L.max_par = a.nodes[l - 1] > L.max_par ? a.nodes[l - 1] : L.max_par;
+    const int64_t c = (int64_t)a.beam[l - 1] * a.branching[l];
+    L.cstride = c > L.cstride ? c : L.cstride;
+  }
+  const int64_t HT = (int64_t)a.Hkv * a.T;
+  size_t o = 0;
+  auto take = [&](size_t n) { const size_t r = o; o += (n + 255) & ~(size_t)255; return r; };
+  L.lat = take((size_t)HT * a.r * 4);
+  L.kept = take((size_t)2 * HT * LSA_MAX_BEAM * 4);
+  L.nkept = take((size_t)HT * 4);
+  L.cnt0 = take((size_t)a.Hkv * L.max_par * 4);
+  L.cnt1 = take((size_t)a.Hkv * L.max_par * 4);
+  L.off = take((size_t)a.Hkv * (L.max_par + 1) * 4);
+  L.ent = take((size_t)HT * LSA_MAX_BEAM * 4);
+  L.epar = take((size_t)HT * LSA_MAX_BEAM * 4);
+  L.cand = take((size_t)HT * L.cstride * 8);
+  L.bytes = o;
+  return L;
+}
+
+size_t select_nodes_workspace_bytes(const SelectArgs& a) {
+  if (a.levels < 2 || a.T == 0) return 0;
+  return node_sel_layout(a).bytes;
+}
+
+template <typename T>
+static cudaError_t launch_select_nodes(const SelectArgs& a, void* ws, cudaStream_t st) {
+  const NodeSelLayout L = node_sel_layout(a);
+  char* w = static_cast<char*>(ws);
+  NodeSel s;
+  s.a = a;
+  s.lat = reinterpret_cast<float*>(w + L.lat);
+  s.kept = reinterpret_cast<int32_t*>(w + L.kept);
+  s.nkept = reinterpret_cast<int32_t*>(w + L.nkept);
+  s.cnt[0] = reinterpret_cast<int32_t*>(w + L.cnt0);
+  s.cnt[1] = reinterpret_cast<int32_t*>(w + L.cnt1);
+  s.off = reinterpret_cast<int32_t*>(w + L.off);
+  s.ent = reinterpret_cast<uint32_t*>(w + L.ent);
+  s.epar = reinterpret_cast<int32_t*>(w + L.epar);
+  s.cand = reinterpret_cast<unsigned long long*>(w + L.cand);
+  s.max_par = L.max_par;
+  s.cstride = L.cstride;
+  cudaError_t e = cudaMemsetAsync(s.cnt[0], 0, (size_t)a.Hkv * L.max_par * 4, st);
+  if (e != cudaSuccess) return e;
+  const dim3 gw((unsigned)ceil_div(a.T, kSelWarps), (unsigned)a.Hkv);
+  const dim3 gl((unsigned)ceil_div(a.T, kSnLatQ), (unsigned)a.Hkv);
+  bool launched = false;
+#define LSA_SN(RR, DD)                                                   \
+  if (a.r == RR && a.d == DD) {                                          \
+    k_sn_latent<T, RR, DD><<<gl, 128, 0, st>>>(s);                       \
+    k_sn_top<RR><<<gw, kSelWarps * 32, 0, st>>>(s);                      \
+    launched = true;                                                     \
+  }
+  LSA_SN(16, 64) LSA_SN(32, 64) LSA_SN(64, 64) LSA_SN(16, 128) LSA_SN(32, 128) LSA_SN(64, 128)
+#undef LSA_SN
+  if (!launched) return cudaErrorInvalidValue;
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  for (int l = 1; l < a.levels; ++l) {
+    const int64_t n_next = l + 1 < a.levels ? a.nodes[l] : 0;
+    k_sn_scan<<<(unsigned)a.Hkv, 1024, 0, st>>>(s.cnt[(l - 1) & 1], s.cnt[l & 1], s.off, s.max_par, a.nodes[l - 1],
+                                                n_next);
+    k_sn_fill<<<dim3((unsigned)ceil_div(a.T, kSnFillWalks), (unsigned)a.Hkv), 256, 0, st>>>(s, l);
+    // entries per CTA: the chunk's parents (about chunk / walks-per-parent + 1 of them)
+    // should have their children fit the staged rows
+    const int64_t per_par = ceil_div(a.T * a.beam[l - 1], a.nodes[l - 1]);
+    int chunk = kSnChunk;
+    while (chunk > 128 && (chunk / per_par + 2) * a.branching[l] > kSnRows) chunk >>= 1;
+    const dim3 gs((unsigned)ceil_div(a.T * a.beam[l - 1], chunk), (unsigned)a.Hkv);
+    // children per lane: ceil(b / 4), at most 4 per pass (larger branchings take several)
+    const int cpl = (a.branching[l] + 3) / 4;
+#define LSA_SNS1(RR, CC)                                                                          \
+  {                                                                                               \
+    const int sm = (int)SnScoreSmem<RR>::kBytes;                                                  \
+    if ((e = cudaFuncSetAttribute(k_sn_score<RR, CC>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                  sm)) != cudaSuccess)                                            \
+      return e;                                                                                   \
+    k_sn_score<RR, CC><<<gs, 256, sm, st>>>(s, l, chunk);                                         \
+  }
+#define LSA_SNS(RR)                                     \
+  if (a.r == RR) {                                      \
+    if (cpl == 1) LSA_SNS1(RR, 1)                       \
+    else if (cpl == 2) LSA_SNS1(RR, 2)                  \
+    else if (cpl == 3) LSA_SNS1(RR, 3)                  \
+    else LSA_SNS1(RR, 4)                                \
+  }
+    LSA_SNS(16) LSA_SNS(32) LSA_SNS(64)
+#undef LSA_SNS
+#undef LSA_SNS1
+    const int64_t nc = (int64_t)a.beam[l - 1] * a.branching[l];
+    if (nc <= 32) k_sn_rank<1><<<gw, kSelWarps * 32, 0, st>>>(s, l);
+    else if (nc <= 64) k_sn_rank<2><<<gw, kSelWarps * 32, 0, st>>>(s, l);
+    else if (nc <= 128) k_sn_rank<4><<<gw, kSelWarps * 32, 0, st>>>(s, l);
+    else if (nc <= 256) k_sn_rank<8><<<gw, kSelWarps * 32, 0, st>>>(s, l);
+    else k_sn_rank<16><<<gw, kSelWarps * 32, 0, st>>>(s, l);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t run_select_nodes(const SelectArgs& a, int dtype, void* ws, cudaStream_t st) {
+  if (a.T == 0) return cudaSuccess;
+  if (a.levels < 2) return run_select(a, dtype, st);
+  return dtype == LSA_BF16 ? launch_select_nodes<__nv_bfloat16>(a, ws, st) : launch_select_nodes<float>(a, ws, st);
 }
 
 // ---- flat search: every leaf centroid scored ----------------------------------

@@ -60,6 +60,8 @@ def _load():
         "lsa_tree_append_workspace_bytes": (ctypes.c_int, [D, i32, ctypes.POINTER(ctypes.c_size_t)]),
         "lsa_tree_append": (ctypes.c_int, [D, P, D, P, P, i64, i32, i32, P, i32, u64, P, sz, P, P, P]),
         "lsa_select": (ctypes.c_int, [D, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, P, P]),
+        "lsa_select_batched_workspace_bytes": (ctypes.c_int, [D, i32, P, ctypes.POINTER(sz)]),
+        "lsa_select_batched": (ctypes.c_int, [D, P, P, i32, i32, i32, i32, P, P, P, P, P, P, P, P, sz, P, P]),
         "lsa_tree_attn_workspace_bytes": (ctypes.c_int, [D, i32, i32, i32, i32, i32, ctypes.POINTER(sz)]),
         "lsa_tree_attn": (ctypes.c_int, [D, P, P, i32, i32, P, P, i64, i32, i32, P, i32, P, i32, f32, P, P, P, sz,
                                          P, P]),
@@ -199,6 +201,27 @@ def lsa_select(desc, tree_mem, Q, W, beam, q_pos, idx_out, leaves_out=None, qlat
     _raise(_lib.lsa_select(ctypes.byref(desc), _ptr(tree_mem), _ptr(Q), T, Hq, d, _dtype(Q), _ptr(W),
                            ctypes.cast(bm, ctypes.c_void_p), _ptr(q_pos), _ptr(idx_out), _ptr(leaves_out),
                            _ptr(qlat_out), _ptr(beam_out), _ptr(status), _stream(stream, Q)), "lsa_select")
+
+
+def lsa_select_batched_workspace_bytes(desc, T, beam) -> int:
+    bm = (ctypes.c_int32 * max(MAX_LEVELS, len(beam)))(*beam)
+    n = ctypes.c_size_t()
+    _raise(_lib.lsa_select_batched_workspace_bytes(ctypes.byref(desc), T, ctypes.cast(bm, ctypes.c_void_p),
+                                                   ctypes.byref(n)), "lsa_select_batched_workspace_bytes")
+    return int(n.value)
+
+
+def lsa_select_batched(desc, tree_mem, Q, W, beam, q_pos, idx_out, leaves_out=None, qlat_out=None, beam_out=None,
+                       workspace=None, status=None, stream=None):
+    """As lsa_select, scheduled for large batches; workspace: device bytes of
+    lsa_select_batched_workspace_bytes(desc, T, beam)."""
+    bm = (ctypes.c_int32 * max(MAX_LEVELS, len(beam)))(*beam)
+    T, Hq, d = Q.shape
+    ws_n = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _raise(_lib.lsa_select_batched(ctypes.byref(desc), _ptr(tree_mem), _ptr(Q), T, Hq, d, _dtype(Q), _ptr(W),
+                                   ctypes.cast(bm, ctypes.c_void_p), _ptr(q_pos), _ptr(idx_out), _ptr(leaves_out),
+                                   _ptr(qlat_out), _ptr(beam_out), _ptr(workspace), ws_n, _ptr(status),
+                                   _stream(stream, Q)), "lsa_select_batched")
 
 
 def lsa_tree_attn_workspace_bytes(desc, T, Hq, d, dtype, n_leaves) -> int:
@@ -474,8 +497,10 @@ def tree_append(tree: Tree, K, W, iters, seed, trace=False, workspace=None, stat
     return (t, tr) if trace else t
 
 
-def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, leaves=False, status=None, check=True):
-    """Returns idx (and, when asked, leaves, query latents, per-level beams, in that order)."""
+def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, leaves=False, status=None, check=True,
+           batched=False):
+    """Returns idx (and, when asked, leaves, query latents, per-level beams, in that order).
+    batched: run lsa_select_batched (same results, scheduled for large batches)."""
     T = Q.shape[0]
     d = tree.desc
     K_sel = beam[-1] * d.leaf_size
@@ -484,9 +509,14 @@ def select(tree: Tree, Q, W, beam, q_pos=None, qlat=False, beams=False, leaves=F
     ql = torch.empty(T, d.n_heads, d.r, dtype=torch.float32, device=Q.device) if qlat else None
     bo = torch.empty(d.levels, d.n_heads, T, max(beam), dtype=torch.int32, device=Q.device) if beams else None
     st = _new_status(Q.device) if status is None else status
-    lsa_select(d, tree.mem, Q, W, beam, q_pos, idx, lv, ql, bo, st)
+    if batched:
+        n = lsa_select_batched_workspace_bytes(d, T, beam)
+        ws = torch.empty(max(n, 1), dtype=torch.uint8, device=Q.device)
+        lsa_select_batched(d, tree.mem, Q, W, beam, q_pos, idx, lv, ql, bo, ws, st)
+    else:
+        lsa_select(d, tree.mem, Q, W, beam, q_pos, idx, lv, ql, bo, st)
     if check:
-        check_status(st, "lsa_select")
+        check_status(st, "lsa_select_batched" if batched else "lsa_select")
     out = [idx]
     if leaves:
         out.append(lv)

@@ -215,6 +215,26 @@ int lsa_select(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, i
                const int32_t *q_pos, int32_t *idx_out, int32_t *leaves_out, float *qlat_out,
                int32_t *beam_out, int32_t *status, void *stream);
 
+/* The same hierarchical search as lsa_select, scheduled for large query batches
+ * (prefill, training): after the top level, every level scores the children of a
+ * kept node for all the walks that kept it together (the (query, group, parent)
+ * triples are grouped by parent first), then ranks each walk's candidates.  The
+ * scores are the same fp32 expressions, so every output (idx_out, leaves_out,
+ * qlat_out, beam_out, status) equals lsa_select's bit for bit.  Arguments as
+ * lsa_select, plus:
+ *  workspace: device memory of lsa_select_batched_workspace_bytes(tree, T, beam)
+ *             bytes (NULL allowed when that is 0); contents need no initialisation
+ *             and are scratch afterwards.  Not shared between concurrent calls.
+ * T must be <= 2^26.  Errors as lsa_select; LSA_ERR_WORKSPACE if the workspace is
+ * missing or too small.  With one level it runs lsa_select's kernel. */
+int lsa_select_batched_workspace_bytes(const lsa_tree_desc *tree, int32_t T, const int32_t *beam,
+                                       size_t *bytes /* host */);
+int lsa_select_batched(const lsa_tree_desc *tree, const void *tree_mem, const void *Q, int32_t T,
+                       int32_t Hq, int32_t d, int32_t dtype, const void *W, const int32_t *beam,
+                       const int32_t *q_pos, int32_t *idx_out, int32_t *leaves_out,
+                       float *qlat_out, int32_t *beam_out, void *workspace,
+                       size_t workspace_bytes, int32_t *status, void *stream);
+
 /* Flat search (bdtechtalks.com, "Latent sparse attention", section "How latent
  * sparse attention works": the first of the two search strategies compares the
  * query with all cluster centroids).  Arguments and outputs as lsa_select with a

@@ -227,3 +227,34 @@ def test_decode_step_rejects(lsa):
     assert call(nt + 3, nt, Vr=None) == lsa.LSA_ERR_INVALID_ARG
     assert call(nt + 3, nt, Hq=12) == lsa.LSA_ERR_SHAPE
     assert call(nt + 3, nt, ws=16) == lsa.LSA_ERR_WORKSPACE
+
+
+def test_select_batched_rejects(lsa):
+    """Host-side checks of the batched search: workspace sizes (growing with T, 0 for no
+    queries), the batch limit, a missing or short workspace, and a bad beam."""
+    L = lsa._lib
+    P = ctypes.c_void_p(16)
+    d = lsa.lsa_tree_describe(8, 64, (16, 16, 16, 4), 64)
+    beam = (ctypes.c_int32 * 4)(8, 32, 32, 32)
+    n = ctypes.c_size_t()
+    sizes = []
+    for T in (0, 1, 4096, 1 << 26):
+        assert L.lsa_select_batched_workspace_bytes(ctypes.byref(d), T, beam, ctypes.byref(n)) == lsa.LSA_OK
+        sizes.append(n.value)
+    assert sizes[0] == 0 and 0 < sizes[1] < sizes[2] < sizes[3]
+    # 4096 queries x 8 groups: the candidate lists alone hold 512 keys of 8 bytes per walk
+    assert sizes[2] >= 4096 * 8 * 512 * 8
+    assert L.lsa_select_batched_workspace_bytes(ctypes.byref(d), (1 << 26) + 1, beam, ctypes.byref(n)) == \
+        lsa.LSA_ERR_SHAPE
+    assert L.lsa_select_batched_workspace_bytes(ctypes.byref(d), 16, beam, None) == lsa.LSA_ERR_INVALID_ARG
+    bad = (ctypes.c_int32 * 4)(8, 32, 33, 32)
+    assert L.lsa_select_batched_workspace_bytes(ctypes.byref(d), 16, bad, ctypes.byref(n)) == lsa.LSA_ERR_SHAPE
+
+    def call(T, ws, ws_bytes):
+        return L.lsa_select_batched(ctypes.byref(d), P, P, T, 32, 128, lsa.LSA_BF16, P, beam, None, P, None, None,
+                                    None, ws, ws_bytes, None, None)
+    assert L.lsa_select_batched_workspace_bytes(ctypes.byref(d), 64, beam, ctypes.byref(n)) == lsa.LSA_OK
+    assert call(64, None, 0) == lsa.LSA_ERR_WORKSPACE
+    assert call(64, P, n.value - 1) == lsa.LSA_ERR_WORKSPACE
+    assert call((1 << 26) + 1, P, 1 << 40) == lsa.LSA_ERR_SHAPE
+    assert call(0, None, 0) == lsa.LSA_OK

@@ -99,8 +99,13 @@ def test_prefill_1m_full(lsa):
     case = cfg.case(DEV)
     tree, trace = lsa.build_tree(case.K, case.W, cfg.branching, cfg.leaf, cfg.iters, cfg.seed, trace=True)
     idx, leaves, beams = lsa.select(tree, case.Q, case.W, cfg.beam, case.q_pos, beams=True, leaves=True)
+    # the batched schedule (the one bench.py times) returns the same lists bit for bit
+    idx_b, leaves_b, beams_b = lsa.select(tree, case.Q, case.W, cfg.beam, case.q_pos, beams=True, leaves=True,
+                                          batched=True)
     O, LSE = lsa.tree_attn(tree, case.Q, case.K, case.V, leaves, case.q_pos, causal=True)
     torch.cuda.synchronize()
+    assert torch.equal(idx_b, idx) and torch.equal(leaves_b, leaves) and torch.equal(beams_b, beams)
+    del idx_b, leaves_b, beams_b
     rng = np.random.default_rng(1)
     qp = case.q_pos.cpu().numpy()
     rows = np.sort(rng.choice(cfg.T, 48, replace=False))
