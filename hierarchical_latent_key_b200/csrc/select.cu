@@ -893,16 +893,17 @@ __device__ __forceinline__ bool score_children(const float4* q, const float* row
 // current group is scored.
 constexpr int kSnChunk = 512;   // entries per CTA at most (the host may pick fewer)
 constexpr int kSnRows = 128;    // staged child rows
+constexpr int kSnWarps = 4;     // warps per CTA (three CTAs per SM: registers for the whole step, no spills)
 template <int R>
 struct SnScoreSmem {
   static constexpr int RP = R + 4;   // row stride in floats: the 8 rows a warp reads at once hit different banks
   static constexpr size_t kRows = 0;
   static constexpr size_t kLat = kRows + (size_t)kSnRows * RP * 4;
-  static constexpr size_t kMp = kLat + (size_t)8 * 2 * 8 * RP * 4;
+  static constexpr size_t kMp = kLat + (size_t)kSnWarps * 2 * 8 * RP * 4;
   static constexpr size_t kBytes = kMp + (size_t)kSnRows * 4;
 };
 template <int R, int CPL>
-__global__ void __launch_bounds__(256, 2) k_sn_score(NodeSel s, int l, int chunk) {
+__global__ void __launch_bounds__(kSnWarps * 32, 3) k_sn_score(NodeSel s, int l, int chunk) {
   using S = SnScoreSmem<R>;
   constexpr int RP = S::RP;
   constexpr int QP = R / 16;  // latent pieces (float4) a lane copies
@@ -925,17 +926,17 @@ __global__ void __launch_bounds__(256, 2) k_sn_score(NodeSel s, int l, int chunk
   const int32_t* mpos = reinterpret_cast<const int32_t*>(a.tree + a.off_m[l]) + (int64_t)g * a.nodes[l];
   if (staged) {   // rows pa*b .. pa*b + nrows - 1, contiguous in the level
     const float4* src = reinterpret_cast<const float4*>(cent + pa * b * R);
-    for (int i = tid; i < nrows * (R / 4); i += 256)
+    for (int i = tid; i < nrows * (R / 4); i += kSnWarps * 32)
       reinterpret_cast<float4*>(s_row)[(i / (R / 4)) * (RP / 4) + i % (R / 4)] = __ldg(&src[i]);
-    for (int i = tid; i < nrows; i += 256) s_mp[i] = __ldg(&mpos[pa * b + i]);
+    for (int i = tid; i < nrows; i += kSnWarps * 32) s_mp[i] = __ldg(&mpos[pa * b + i]);
   }
   __syncthreads();
   const int lane = tid & 31, warp = tid >> 5, jl = lane & 3, el = lane >> 2;
-  const int stride = staged ? RP : R;
+  constexpr int kStep = kSnWarps * 8;   // entries per CTA round
   const float* lat = s.lat + (int64_t)g * a.T * R;
   float* wl = reinterpret_cast<float*>(sn_smem + S::kLat) + warp * 2 * 8 * RP;   // [2][8][RP]
   bool bad = false;
-  // group k of this warp: entries e0 + (warp + 8 k) * 8 + el
+  // group k of this warp: entries e0 + (warp + kSnWarps k) * 8 + el
   auto entry_of = [&](int64_t i, int64_t& t, int& rank, int64_t& p) {
     t = -1; rank = 0; p = 0;
     if (i < e1) {
@@ -961,25 +962,32 @@ __global__ void __launch_bounds__(256, 2) k_sn_score(NodeSel s, int l, int chunk
   entry_of(i, t_c, r_c, p_c);
   copy_lat(t_c, 0);
   int64_t qp_c = pos_of(t_c);
-  entry_of(i + 64, t_n, r_n, p_n);
-  for (int buf = 0; i - el < e1; i += 64, buf ^= 1) {
+  entry_of(i + kStep, t_n, r_n, p_n);
+  for (int buf = 0; i - el < e1; i += kStep, buf ^= 1) {
     // in flight while this group is scored: the next group's latents and position,
     // the entries of the group after it
     copy_lat(t_n, buf ^ 1);
     const int64_t qp_n = pos_of(t_n);
     int64_t t_f, p_f;
     int r_f;
-    entry_of(i + 128, t_f, r_f, p_f);
+    entry_of(i + 2 * kStep, t_f, r_f, p_f);
     cp_async_wait_prev();   // this lane's copies of the current group have landed
     __syncwarp();
     if (t_c >= 0) {
       const bool all_eligible = qp_c >= a.n_tree - 1;
-      const float* rows = staged ? s_row + (p_c - pa) * b * RP : cent + p_c * b * R;
-      const int32_t* mp = staged ? s_mp + (p_c - pa) * b : mpos + p_c * b;
       unsigned long long* out = s.cand + ((int64_t)g * a.T + t_c) * s.cstride + (int64_t)r_c * b;
       const float4* q = reinterpret_cast<const float4*>(wl + (buf * 8 + el) * RP);
-      for (int j0 = 0; j0 < b; j0 += 4 * CPL)
-        bad |= score_children<R, CPL>(q, rows, stride, mp, p_c * b, b, j0, jl, all_eligible, qp_c, out);
+      // two call sites, so that the staged rows are read with shared-memory loads
+      if (staged) {
+        const int64_t loc = (p_c - pa) * b;
+        for (int j0 = 0; j0 < b; j0 += 4 * CPL)
+          bad |= score_children<R, CPL>(q, s_row + loc * RP, RP, s_mp + loc, p_c * b, b, j0, jl, all_eligible,
+                                        qp_c, out);
+      } else {
+        for (int j0 = 0; j0 < b; j0 += 4 * CPL)
+          bad |= score_children<R, CPL>(q, cent + p_c * b * R, R, mpos + p_c * b, p_c * b, b, j0, jl, all_eligible,
+                                        qp_c, out);
+      }
     }
     __syncwarp();   // this buffer is refilled two groups later
     t_c = t_n; r_c = r_n; p_c = p_n; qp_c = qp_n;
@@ -1102,7 +1110,7 @@ static cudaError_t launch_select_nodes(const SelectArgs& a, void* ws, cudaStream
     if ((e = cudaFuncSetAttribute(k_sn_score<RR, CC>, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                   sm)) != cudaSuccess)                                            \
       return e;                                                                                   \
-    k_sn_score<RR, CC><<<gs, 256, sm, st>>>(s, l, chunk);                                         \
+    k_sn_score<RR, CC><<<gs, kSnWarps * 32, sm, st>>>(s, l, chunk);                               \
   }
 #define LSA_SNS(RR)                                     \
   if (a.r == RR) {                                      \
