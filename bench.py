@@ -492,10 +492,10 @@ def time_steps(w, steps, warmup, flush, stream):
 SINK, WINDOW = 16, 512   # sink tokens and recent window of the sink/window measurement
 # DRAM bytes read + written per lsa_tree_attn call of the prefill_1m step, from single-pass ncu
 # captures of the full workload (dram__bytes_read.sum + dram__bytes_write.sum, one launch each,
-# after three warm-up steps): k_tl_pipe 4,900,205,312 + 1,175,268,096 and k_tl_combine
-# 1,111,534,848 + 34,631,680; the five leaf- and chunk-list kernels add about 12 MB and are left out.
+# the first call of the warm-up steps): k_tl_pipe 4,914,926,080 + 1,172,362,496 and k_tl_combine
+# 1,111,510,528 + 31,419,904; the five leaf- and chunk-list kernels add about 12 MB and are left out.
 # To be taken again whenever one of those kernels changes.
-TREE_ATTN_TRAFFIC_BYTES = 4_900_205_312 + 1_175_268_096 + 1_111_534_848 + 34_631_680
+TREE_ATTN_TRAFFIC_BYTES = 4_914_926_080 + 1_172_362_496 + 1_111_510_528 + 31_419_904
 POOL = 4                 # keys per block of the pooled index
 
 
