@@ -108,7 +108,7 @@ template <int E>
 __device__ __forceinline__ int warp_keep_best(unsigned long long (&v)[E], int B, unsigned long long* s_key,
                                               int32_t* next) {
   const int lane = threadIdx.x & 31;
-  if constexpr (E >= 8) {
+  if constexpr (E >= 4) {
     // Threshold first: the B-th largest of the lanes' two largest keys is a lower
     // bound of the B-th largest key overall (those 64 are keys of the level), so
     // every kept key is >= tau.  Keys are distinct, so sorting the keys >= tau
@@ -746,8 +746,15 @@ __global__ void __launch_bounds__(1024) k_sn_scan(int32_t* cnt, int32_t* cnt_nex
   int32_t* o = off + (int64_t)g * (max_par + 1);
   const int64_t per = ceil_div(np, (int64_t)1024);
   const int64_t lo = min64((int64_t)tid * per, np), hi = min64(lo + per, np);
+  constexpr int kBlk = 8;   // a block's loads are all issued before the first is used
   int32_t sum = 0;
-  for (int64_t i = lo; i < hi; ++i) sum += c[i];
+  for (int64_t b0 = lo; b0 < hi; b0 += kBlk) {
+    int32_t v[kBlk];
+#pragma unroll
+    for (int k = 0; k < kBlk; ++k) v[k] = b0 + k < hi ? c[b0 + k] : 0;
+#pragma unroll
+    for (int k = 0; k < kBlk; ++k) sum += v[k];
+  }
   int32_t inc = sum;
 #pragma unroll
   for (int d = 1; d < 32; d <<= 1) {
@@ -767,10 +774,17 @@ __global__ void __launch_bounds__(1024) k_sn_scan(int32_t* cnt, int32_t* cnt_nex
   }
   __syncthreads();
   int32_t run = inc - sum + (warp ? s_warp[warp - 1] : 0);
-  for (int64_t i = lo; i < hi; ++i) {
-    o[i] = run;
-    run += c[i];
-    c[i] = 0;
+  for (int64_t b0 = lo; b0 < hi; b0 += kBlk) {
+    int32_t v[kBlk];
+#pragma unroll
+    for (int k = 0; k < kBlk; ++k) v[k] = b0 + k < hi ? c[b0 + k] : 0;
+#pragma unroll
+    for (int k = 0; k < kBlk; ++k)
+      if (b0 + k < hi) {
+        o[b0 + k] = run;
+        run += v[k];
+        c[b0 + k] = 0;
+      }
   }
   if (tid == 1023) o[np] = s_warp[31];
   int32_t* cn = cnt_next + (int64_t)g * max_par;
@@ -810,25 +824,32 @@ __global__ void __launch_bounds__(256) k_sn_fill(NodeSel s, int l) {
     }
     return;
   }
+  // this thread's pairs i = tid + 256 k, their parents read at once and kept in registers
+  constexpr int kPer = kSnFillWalks * LSA_MAX_BEAM / 256;
+  int32_t pv[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int64_t i = tid + 256 * k;
+    pv[k] = i < ne ? kept[(i / Bp) * LSA_MAX_BEAM + i % Bp] : -1;
+  }
   for (int64_t p = tid; p < np; p += 256) s_h[p] = 0;
   __syncthreads();
-  for (int64_t i = tid; i < ne; i += 256) {
-    const int32_t p = kept[(i / Bp) * LSA_MAX_BEAM + i % Bp];
-    if (p >= 0) atomicAdd(&s_h[p], 1);
-  }
+#pragma unroll
+  for (int k = 0; k < kPer; ++k)
+    if (pv[k] >= 0) atomicAdd(&s_h[pv[k]], 1);
   __syncthreads();
   for (int64_t p = tid; p < np; p += 256) {
     const int32_t c = s_h[p];
     s_h[p] = c > 0 ? off[p] + atomicAdd(&cur[p], c) : 0;
   }
   __syncthreads();
-  for (int64_t i = tid; i < ne; i += 256) {
-    const int64_t w = i / Bp;
-    const int rank = (int)(i % Bp);
-    const int32_t p = kept[w * LSA_MAX_BEAM + rank];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int64_t i = tid + 256 * k;
+    const int32_t p = pv[k];
     if (p < 0) continue;
     const int32_t pos = atomicAdd(&s_h[p], 1);
-    ent[pos] = (uint32_t)((w0 + w) * LSA_MAX_BEAM + rank);
+    ent[pos] = (uint32_t)((w0 + i / Bp) * LSA_MAX_BEAM + i % Bp);
     epar[pos] = p;
   }
 }

@@ -77,15 +77,26 @@ __global__ void k_tl_count(TreeAttnArgs a) {
   if (leaf >= 0 && leaf < a.NL) atomicAdd(&a.cnt[g * a.NL + leaf], 1);
 }
 
+// A thread's range of a single-CTA scan is read kScanBlk elements at a time, every
+// load of a block issued before the first is used (a one-by-one loop would wait
+// out one memory round trip per element).
+constexpr int kScanBlk = 16;
+
 __global__ void __launch_bounds__(1024) k_tl_scan(TreeAttnArgs a) {
   __shared__ int32_t s_warp[32];
   const int64_t g = blockIdx.x;
   int32_t* c = a.cnt + g * a.NL;
   int32_t* o = a.off + g * (a.NL + 1);
   const int64_t per = ceil_div(a.NL, 1024);
-  const int64_t lo = threadIdx.x * per, hi = min64(a.NL, lo + per);
+  const int64_t lo = min64(threadIdx.x * per, a.NL), hi = min64(a.NL, lo + per);
   int32_t s = 0;
-  for (int64_t i = lo; i < hi; ++i) s += c[i];
+  for (int64_t b0 = lo; b0 < hi; b0 += kScanBlk) {
+    int32_t v[kScanBlk];
+#pragma unroll
+    for (int k = 0; k < kScanBlk; ++k) v[k] = b0 + k < hi ? c[b0 + k] : 0;
+#pragma unroll
+    for (int k = 0; k < kScanBlk; ++k) s += v[k];
+  }
   // block exclusive scan of the per-thread sums
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t inc = s;
@@ -107,12 +118,19 @@ __global__ void __launch_bounds__(1024) k_tl_scan(TreeAttnArgs a) {
   }
   __syncthreads();
   int32_t run = inc - s + (warp ? s_warp[warp - 1] : 0);
-  for (int64_t i = lo; i < hi; ++i) {
-    o[i] = run;
-    run += c[i];
-    c[i] = 0;  // becomes the fill cursor
+  for (int64_t b0 = lo; b0 < hi; b0 += kScanBlk) {
+    int32_t v[kScanBlk];
+#pragma unroll
+    for (int k = 0; k < kScanBlk; ++k) v[k] = b0 + k < hi ? c[b0 + k] : 0;
+#pragma unroll
+    for (int k = 0; k < kScanBlk; ++k)
+      if (b0 + k < hi) {
+        o[b0 + k] = run;
+        run += v[k];
+        c[b0 + k] = 0;  // becomes the fill cursor
+      }
   }
-  if (threadIdx.x == 1023) o[a.NL] = run;
+  if (threadIdx.x == 1023) o[a.NL] = s_warp[31];
 }
 
 __global__ void k_tl_fill(TreeAttnArgs a) {
@@ -135,9 +153,22 @@ __global__ void __launch_bounds__(1024) k_tl_cscan(TreeAttnArgs a) {
   const int32_t* o = a.off + g * (a.NL + 1);
   int32_t* c = a.coff + g * a.NL;
   const int64_t per = ceil_div(a.NL, 1024);
-  const int64_t lo = threadIdx.x * per, hi = min64(a.NL, lo + per);
+  const int64_t lo = min64(threadIdx.x * per, a.NL), hi = min64(a.NL, lo + per);
+  // chunks of leaf i: ceil((o[i + 1] - o[i]) / epc), blocks of kScanBlk leaves read at once
+  auto chunks_of = [&](int64_t b0, int32_t (&v)[kScanBlk]) {
+    int32_t e[kScanBlk + 1];
+#pragma unroll
+    for (int k = 0; k <= kScanBlk; ++k) e[k] = b0 + k <= hi ? o[b0 + k] : 0;
+#pragma unroll
+    for (int k = 0; k < kScanBlk; ++k) v[k] = b0 + k < hi ? (e[k + 1] - e[k] + a.epc - 1) / a.epc : 0;
+  };
   int32_t s = 0;
-  for (int64_t i = lo; i < hi; ++i) s += (o[i + 1] - o[i] + a.epc - 1) / a.epc;
+  for (int64_t b0 = lo; b0 < hi; b0 += kScanBlk) {
+    int32_t v[kScanBlk];
+    chunks_of(b0, v);
+#pragma unroll
+    for (int k = 0; k < kScanBlk; ++k) s += v[k];
+  }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t inc = s;
 #pragma unroll
@@ -158,11 +189,17 @@ __global__ void __launch_bounds__(1024) k_tl_cscan(TreeAttnArgs a) {
   }
   __syncthreads();
   int32_t run = inc - s + (warp ? s_warp[warp - 1] : 0);
-  for (int64_t i = lo; i < hi; ++i) {
-    c[i] = run;
-    run += (o[i + 1] - o[i] + a.epc - 1) / a.epc;
+  for (int64_t b0 = lo; b0 < hi; b0 += kScanBlk) {
+    int32_t v[kScanBlk];
+    chunks_of(b0, v);
+#pragma unroll
+    for (int k = 0; k < kScanBlk; ++k)
+      if (b0 + k < hi) {
+        c[b0 + k] = run;
+        run += v[k];
+      }
   }
-  if (threadIdx.x == 1023) a.ctotal[g] = run;
+  if (threadIdx.x == 1023) a.ctotal[g] = s_warp[31];
 }
 
 __global__ void k_tl_chunks(TreeAttnArgs a) {
