@@ -114,6 +114,8 @@ struct SelectArgs {
   // n_leaves (perm coprime with n_leaves), so a query's running threshold rises fast
   int64_t flat_perm;
 };
+// Streaming multiprocessors of the current device (cached per device; 148 if unknown).
+int sm_count();
 cudaError_t run_select(const SelectArgs& a, int dtype, cudaStream_t st);
 // The same search scheduled level by level over (walk, parent) pairs grouped by
 // parent, for large batches; kept lists and outputs equal run_select's bit for bit.

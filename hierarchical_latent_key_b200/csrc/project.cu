@@ -171,6 +171,8 @@ __global__ void __launch_bounds__(kPT, 1)
   free_tmem(tmem, kTmemCols);
 }
 
+}  // namespace
+
 int sm_count() {
   static int count[128] = {};
   int dev = 0;
@@ -182,8 +184,6 @@ int sm_count() {
   }
   return count[dev];
 }
-
-}  // namespace
 
 bool project_tc_supported(int dtype, int r, int d) {
   return dtype == LSA_BF16 && (r == 16 || r == 32 || r == 64) && (d == 64 || d == 128);

@@ -1122,6 +1122,10 @@ static cudaError_t launch_select_nodes(const SelectArgs& a, void* ws, cudaStream
     const int64_t per_par = ceil_div(a.T * a.beam[l - 1], a.nodes[l - 1]);
     int chunk = kSnChunk;
     while (chunk > 128 && (chunk / per_par + 2) * a.branching[l] > kSnRows) chunk >>= 1;
+    // and enough CTAs for about four waves of three per SM (a last partial wave of
+    // one or two leaves most SMs idle)
+    const int64_t pairs = a.T * a.beam[l - 1] * a.Hkv;
+    while (chunk > 128 && pairs / chunk < 4 * 3 * (int64_t)sm_count()) chunk >>= 1;
     const dim3 gs((unsigned)ceil_div(a.T * a.beam[l - 1], chunk), (unsigned)a.Hkv);
     // children per lane: ceil(b / 4), at most 4 per pass (larger branchings take several)
     const int cpl = (a.branching[l] + 3) / 4;
