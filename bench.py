@@ -149,9 +149,9 @@ class Prefill:
         self.sel_ws = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
         self.scale = 1.0 / math.sqrt(d)
         self.units = T
-        # batched select: latent + top level, then scan, fill, score and rank per level;
+        # batched select: latents, top level, then scan, fill, score and rank per level;
         # tree attention: 3 list + 2 tensor-core passes + 2
-        self.launches_per_step = 1 + 4 * (len(cfg.beam) - 1) + 7
+        self.launches_per_step = 2 + 4 * (len(cfg.beam) - 1) + 7
 
     def select(self, Q=None):
         self.lsa.lsa_select_batched(self.tree.desc, self.tree.mem, self.Q if Q is None else Q, self.W, self.cfg.beam,
