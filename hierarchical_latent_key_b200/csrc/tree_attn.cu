@@ -82,6 +82,21 @@ __global__ void k_tl_count(TreeAttnArgs a) {
 // out one memory round trip per element).
 constexpr int kScanBlk = 16;
 
+// Elements [b0, b0 + kScanBlk) of p below hi (0 past it): a full, 16-byte aligned
+// block is read with four unconditional 16-byte loads.
+__device__ __forceinline__ void load_blk(const int32_t* p, int64_t b0, int64_t hi, int32_t (&v)[kScanBlk]) {
+  if (b0 + kScanBlk <= hi && ((reinterpret_cast<uintptr_t>(p + b0) & 15) == 0)) {
+#pragma unroll
+    for (int k = 0; k < kScanBlk / 4; ++k) {
+      const int4 x = reinterpret_cast<const int4*>(p + b0)[k];
+      v[4 * k] = x.x; v[4 * k + 1] = x.y; v[4 * k + 2] = x.z; v[4 * k + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < kScanBlk; ++k) v[k] = b0 + k < hi ? p[b0 + k] : 0;
+  }
+}
+
 __global__ void __launch_bounds__(1024) k_tl_scan(TreeAttnArgs a) {
   __shared__ int32_t s_warp[32];
   const int64_t g = blockIdx.x;
@@ -92,8 +107,7 @@ __global__ void __launch_bounds__(1024) k_tl_scan(TreeAttnArgs a) {
   int32_t s = 0;
   for (int64_t b0 = lo; b0 < hi; b0 += kScanBlk) {
     int32_t v[kScanBlk];
-#pragma unroll
-    for (int k = 0; k < kScanBlk; ++k) v[k] = b0 + k < hi ? c[b0 + k] : 0;
+    load_blk(c, b0, hi, v);
 #pragma unroll
     for (int k = 0; k < kScanBlk; ++k) s += v[k];
   }
@@ -120,8 +134,7 @@ __global__ void __launch_bounds__(1024) k_tl_scan(TreeAttnArgs a) {
   int32_t run = inc - s + (warp ? s_warp[warp - 1] : 0);
   for (int64_t b0 = lo; b0 < hi; b0 += kScanBlk) {
     int32_t v[kScanBlk];
-#pragma unroll
-    for (int k = 0; k < kScanBlk; ++k) v[k] = b0 + k < hi ? c[b0 + k] : 0;
+    load_blk(c, b0, hi, v);
 #pragma unroll
     for (int k = 0; k < kScanBlk; ++k)
       if (b0 + k < hi) {
@@ -156,11 +169,14 @@ __global__ void __launch_bounds__(1024) k_tl_cscan(TreeAttnArgs a) {
   const int64_t lo = min64(threadIdx.x * per, a.NL), hi = min64(a.NL, lo + per);
   // chunks of leaf i: ceil((o[i + 1] - o[i]) / epc), blocks of kScanBlk leaves read at once
   auto chunks_of = [&](int64_t b0, int32_t (&v)[kScanBlk]) {
-    int32_t e[kScanBlk + 1];
+    int32_t e[kScanBlk];
+    load_blk(o, b0, hi + 1, e);   // o[b0 .. min(b0 + kScanBlk, hi + 1)): o has NL + 1 entries
+    const int32_t last = b0 + kScanBlk <= hi ? o[b0 + kScanBlk] : 0;
 #pragma unroll
-    for (int k = 0; k <= kScanBlk; ++k) e[k] = b0 + k <= hi ? o[b0 + k] : 0;
-#pragma unroll
-    for (int k = 0; k < kScanBlk; ++k) v[k] = b0 + k < hi ? (e[k + 1] - e[k] + a.epc - 1) / a.epc : 0;
+    for (int k = 0; k < kScanBlk; ++k) {
+      const int32_t next = k + 1 < kScanBlk ? e[k + 1] : last;
+      v[k] = b0 + k < hi ? (next - e[k] + a.epc - 1) / a.epc : 0;
+    }
   };
   int32_t s = 0;
   for (int64_t b0 = lo; b0 < hi; b0 += kScanBlk) {
